@@ -1,0 +1,202 @@
+/*
+ * psi_verify.h - C ABI of the Psi-Spec verify step on NVIDIA B200 (sm_100a).
+ *
+ * The verify step of the Psi-Spec sampler: the frozen AR path has scored a
+ * block of B drafted tokens (B+1 logit rows, the last one being the bonus
+ * row), the diffusion-LoRA draft supplied B logit rows and the drafted ids.
+ * Per sequence the step keeps the longest prefix of drafted tokens that
+ * passes speculative rejection sampling, then emits one correction token
+ * (drawn from the residual at the first rejection) or one bonus token (drawn
+ * from the bonus row when every draft passed).
+ *
+ * Sources (page title, section):
+ *  [P1] "Uno / Psi-Spec - 같은 모델 안에서 초안 뽑고 AR로 도장 찍기"
+ *       (lanes-ecd.pages.dev): "어디서 왔나" (the Leviathan et al. 2023
+ *       draft -> verify -> correct rule), "Psi-Spec이 한 스텝에서 하는 일"
+ *       (longest consecutive accepted prefix; lossless).
+ *  [P3] "Uno Psi-Spec 是什麼？Diffusion-Augmented LLM 如何保留 AR 分布、
+ *       一次驗證多個 Token" (alphalab.site): "Uno Psi-Spec 怎麼運作？完整走一次
+ *       四個 Token" (steps 3-4: rejection rule, longest accepted prefix,
+ *       residual correction; bonus token from the block-end logits; TPF
+ *       bound), "Linear 與 Tree sampler" (tree verify), "想跑 Uno：先確認官方
+ *       程式需要的環境" (temperature and top-p on the run card).
+ *
+ * Conventions shared by every entry point:
+ *  - All array arguments are DEVICE pointers owned by the caller.  The
+ *    library allocates nothing and keeps no state between calls.
+ *  - Calls are asynchronous on `stream` (NULL = the legacy default stream).
+ *  - Argument errors are detected on the host before any launch and
+ *    returned as a psi_status; nothing is launched in that case.
+ *  - Data errors found on the device (an id outside [0, V), a bad parent
+ *    index, a NaN or +inf logit) are OR-ed into *dev_status (a caller-owned
+ *    device uint32 that the caller zeroes; NULL = not reported).  The
+ *    kernels always run to completion: they never trap, spin or hang.
+ *  - Logits are bfloat16 or float32, row-major; `*_row_stride` is the
+ *    distance between consecutive rows in ELEMENTS (>= V).  Rows whose
+ *    start is 16-byte aligned take the bulk-copy path, others a plain-load
+ *    path; both give the same results.
+ *  - Randomness: the acceptance uniform of row i and the correction/bonus
+ *    uniform of the emitting row are a counter-based hash of
+ *    (seed, sequence id, step, row, purpose), so a step replays exactly from
+ *    its counters and results do not depend on batch composition.
+ */
+#ifndef PSI_VERIFY_H
+#define PSI_VERIFY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st *psi_stream_t; /* same type as cudaStream_t */
+
+typedef enum psi_status {
+  PSI_OK = 0,
+  PSI_ERR_INVALID_ARG = 1, /* null pointer, size or parameter out of range */
+  PSI_ERR_MISALIGNED = 2,  /* pointer not aligned to its element type */
+  PSI_ERR_UNSUPPORTED = 3, /* valid but beyond this build (e.g. V too large) */
+  PSI_ERR_CUDA = 4,        /* a CUDA launch or query failed */
+  PSI_ERR_WORKSPACE = 5,   /* workspace NULL or smaller than the query says */
+  PSI_ERR_TIMEOUT = 6      /* reserved: no kernel here waits on anything */
+} psi_status;
+
+typedef enum psi_dtype { PSI_DTYPE_F32 = 0, PSI_DTYPE_BF16 = 1 } psi_dtype;
+
+/* Bits OR-ed into *dev_status by the kernels. */
+#define PSI_DEV_BAD_TOKEN_ID 1u /* drafted or node id outside [0, V): treated
+                                   as rejected / unmatched */
+#define PSI_DEV_BAD_PARENT 2u   /* parent index >= own index or < -1: node
+                                   unmatched */
+#define PSI_DEV_NONFINITE 4u    /* a NaN or +inf logit was read (-inf is a
+                                   valid logit: probability zero) */
+#define PSI_DEV_TIMEOUT 8u      /* a bounded wait inside a kernel gave up;
+                                   never expected; outputs are then invalid */
+
+/* RNG purposes (the last hash input). */
+#define PSI_PURPOSE_ACCEPT 0u /* u_i of the acceptance test of row i */
+#define PSI_PURPOSE_RESID 1u  /* u' of the correction / bonus draw */
+
+/* Largest supported block and vocabulary. */
+#define PSI_MAX_B 32
+#define PSI_MAX_V 393216
+#define PSI_MAX_TREE_NODES 4096
+
+/* Workspace needed by psi_verify_linear for these sizes (bytes, a multiple
+ * of 256; 0 on invalid sizes).  The workspace needs no initialisation. */
+size_t psi_verify_linear_workspace_bytes(int32_t N, int32_t B, int32_t V,
+                                         psi_dtype dtype, float temperature,
+                                         float top_p);
+
+/*
+ * psi_verify_linear - linear (single-path) verify of N sequences.
+ *
+ * [P1] "Psi-Spec이 한 스텝에서 하는 일"; [P3] "完整走一次四個 Token" steps
+ * 3-4 and the bonus paragraph; temperature / top-p: [P3] run card.
+ *
+ * For T > 0, per sequence n and row i:
+ *   p_i = softmax(ar[n][i] / T), q_i = softmax(draft[n][i] / T); with
+ *   top_p < 1 each is cut to its smallest descending-probability set of mass
+ *   >= top_p (keeping every token tied with the last one admitted) and
+ *   renormalised.  Draft x_i is accepted iff u_i * q_i(x_i) < p_i(x_i) with
+ *   u_i = U(seed, seq, step, i, ACCEPT).  L = first rejected row (B if none).
+ *   If L < B the correction is the inverse-CDF draw, in vocabulary order,
+ *   from max(0, p_L - q_L) at u' = U(seed, seq, step, L, RESID) (from p_L
+ *   itself if that residual is all zero, which needs q_L(x_L) = 0); if
+ *   L == B the bonus token is drawn from p_B the same way.
+ * For T == 0 (greedy): a_i = argmax of ar[n][i] (lowest index on ties);
+ *   accept while x_i == a_i; emit a_L.  draft_logits may be NULL and top_p
+ *   is ignored.
+ *
+ * ar_logits     [N][B+1] rows of V logits (row B = bonus row), stride
+ *               ar_row_stride elements.
+ * draft_logits  [N][B] rows, stride draft_row_stride (ignored if T == 0).
+ * draft_ids     int32 [N][B].
+ * seq_ids       uint64 [N] sequence ids for the RNG, or NULL (= n).
+ * out_tokens    int32 [N][B+1]: x_0..x_{L-1}, then the emitted token, then -1.
+ * out_n_emitted int32 [N]: L + 1, in 1..B+1.
+ * out_p_draft, out_q_draft  float [N][B] or NULL: p_i(x_i), q_i(x_i) after
+ *               top-p (T > 0 only; not written when T == 0).
+ * Limits: 1 <= N, 1 <= B <= PSI_MAX_B, 1 <= V <= PSI_MAX_V, T >= 0 and
+ *   finite, 0 < top_p <= 1.
+ */
+psi_status psi_verify_linear(const void *ar_logits, int64_t ar_row_stride,
+                             const void *draft_logits,
+                             int64_t draft_row_stride, psi_dtype dtype,
+                             const int32_t *draft_ids, int32_t N, int32_t B,
+                             int32_t V, float temperature, float top_p,
+                             uint64_t seed, const uint64_t *seq_ids,
+                             uint64_t step, int32_t *out_tokens,
+                             int32_t *out_n_emitted, float *out_p_draft,
+                             float *out_q_draft, uint32_t *dev_status,
+                             void *workspace, size_t workspace_bytes,
+                             psi_stream_t stream);
+
+/* Workspace needed by psi_verify_tree_greedy (bytes; 0 on invalid sizes). */
+size_t psi_verify_tree_greedy_workspace_bytes(int32_t N, int32_t M, int32_t V,
+                                              psi_dtype dtype);
+
+/*
+ * psi_verify_tree_greedy - greedy (T = 0) verify of a draft tree per sequence.
+ *
+ * [P3] "Linear 與 Tree sampler": several high-probability candidates per
+ * position pruned to a finite prefix tree and verified in one pass.
+ *
+ * ar_logits    [N][M+1] rows (row 0 = root, row k+1 = node k).
+ * node_tokens  int32 [N][M]; parents int32 [N][M] (-1 = child of the root;
+ *              otherwise 0 <= parent < own index).
+ * Node k is matched iff node_tokens[k] == argmax(row of its parent) and its
+ * parent is matched (or is the root).  The deepest matched node (lowest
+ * index among equals) ends the accepted path; the bonus token is the
+ * argmax of that node's own row (root row when nothing matched).
+ * out_path_nodes int32 [N][M]: node indices root-side first, then -1.
+ * out_path_len   int32 [N]: number of accepted nodes (0..M).
+ * out_tokens     int32 [N][M+1]: accepted tokens, then the bonus, then -1.
+ * Limits: 1 <= N, 1 <= M <= PSI_MAX_TREE_NODES, 1 <= V <= PSI_MAX_V.
+ */
+psi_status psi_verify_tree_greedy(const void *ar_logits, int64_t ar_row_stride,
+                                  psi_dtype dtype, const int32_t *node_tokens,
+                                  const int32_t *parents, int32_t N, int32_t M,
+                                  int32_t V, int32_t *out_path_nodes,
+                                  int32_t *out_path_len, int32_t *out_tokens,
+                                  uint32_t *dev_status, void *workspace,
+                                  size_t workspace_bytes, psi_stream_t stream);
+
+/*
+ * psi_rng_uniforms - the uniforms the verify step draws, for inspection and
+ * replay: out[s][r] = U(seed, seq_ids ? seq_ids[s] : s, step, r, purpose),
+ * a float in [0, 1 - 2^-24] with 24 significant bits.
+ * U is the top 24 bits of h = f(f(f(f(f(seed) ^ seq) ^ step) ^ row) ^
+ * purpose), f being the SplitMix64 output function (Steele, Lea & Flood,
+ * OOPSLA 2014).  out: float [n_seq][n_rows] device memory.
+ */
+psi_status psi_rng_uniforms(uint64_t seed, const uint64_t *seq_ids,
+                            int32_t n_seq, uint64_t step, int32_t n_rows,
+                            uint32_t purpose, float *out, psi_stream_t stream);
+
+/*
+ * psi_profile_main_kernel - instrumentation for roofline measurements (no
+ * counterpart on the pages).  After this call, every verify call made from
+ * the same host thread records `before` on its stream immediately before
+ * launching its main kernel (the per-row kernel that reads the logits) and
+ * `after` immediately after it, so that cudaEventElapsedTime(before, after)
+ * is that kernel's duration.  The events are caller-created cudaEvent_t
+ * handles, owned by the caller; psi_profile_main_kernel(NULL, NULL) stops
+ * recording.  Returns PSI_ERR_INVALID_ARG if exactly one event is NULL.
+ */
+struct CUevent_st;
+typedef struct CUevent_st *psi_event_t; /* same type as cudaEvent_t */
+psi_status psi_profile_main_kernel(psi_event_t before, psi_event_t after);
+
+/* Human-readable name of a status code (static string). */
+const char *psi_status_string(psi_status status);
+
+/* Detail of the last host-side error on this thread (static buffer). */
+const char *psi_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PSI_VERIFY_H */

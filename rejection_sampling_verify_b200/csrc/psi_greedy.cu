@@ -1,0 +1,312 @@
+// psi_greedy.cu - greedy (temperature 0) verify kernels.
+//
+//  row_argmax_kernel   argmax of every AR row, lowest index on ties.  Rows
+//                      are split into chunks handled by separate CTAs; each
+//                      CTA streams its chunk with 16-byte non-allocating
+//                      loads (the data is consumed once, so it goes straight
+//                      to registers) and writes one packed (key, ~index)
+//                      word.  HBM-bound: 2 bytes per bf16 logit, no exp.
+//  greedy_emit_kernel  linear rule: accept while x_i == argmax_i, emit the
+//                      argmax of the first mismatching row (or the bonus row).
+//  tree_walk_kernel    tree rule: node matched when its token is its parent
+//                      row's argmax and its parent is matched; deepest
+//                      matched node ends the path.
+//
+// Sources: "Uno Psi-Spec 是什麼？..." (alphalab.site), section "Linear 與 Tree
+// sampler" (tree verify); greedy linear verify is the temperature-0 case of
+// the section "Uno Psi-Spec 怎麼運作？完整走一次四個 Token".
+#include "psi_internal.h"
+
+namespace psi {
+
+// Packed argmax word: order-preserving key in the high half, complemented
+// index in the low half, so the unsigned maximum is the largest value and,
+// among equal values, the lowest index.  0 never wins against a real element.
+__device__ __forceinline__ uint64_t pack_argmax(uint32_t key, uint32_t idx) {
+  return ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - idx);
+}
+
+// Running (value, index) maximum of one thread.  Values are compared as
+// floats: -0 == +0, NaN never wins (it only raises the status bit).
+struct RunMax {
+  float val = -INFINITY;
+  uint32_t idx = 0xFFFFFFFFu;
+  bool bad = false;
+};
+
+template <typename Bits>
+__device__ __forceinline__ void scan_scalar(uint32_t b, uint32_t idx, RunMax &rm) {
+  rm.bad |= Elem<Bits>::bad(b);
+  const float x = Elem<Bits>::to_float(b);
+  if (x > rm.val || rm.idx == 0xFFFFFFFFu && !(x != x) && x == rm.val) {
+    rm.val = x;
+    rm.idx = idx;
+  }
+}
+
+// One 16-byte vector whose first element has index `base`.  Each thread
+// visits its indices in increasing order, so "strictly greater" keeps the
+// lowest index among equal values.
+template <typename Bits>
+__device__ __forceinline__ void scan_vec(const uint4 &w, uint32_t base, RunMax &rm) {
+  constexpr int VEC = Elem<Bits>::kVec;
+  float vm;
+  if constexpr (sizeof(Bits) == 2) {
+    // packed bf16x2 maxima; the _nan form lets a NaN through so it is seen
+    const __nv_bfloat162 m = __hmax2_nan(
+        __hmax2_nan(*reinterpret_cast<const __nv_bfloat162 *>(&w.x),
+                    *reinterpret_cast<const __nv_bfloat162 *>(&w.y)),
+        __hmax2_nan(*reinterpret_cast<const __nv_bfloat162 *>(&w.z),
+                    *reinterpret_cast<const __nv_bfloat162 *>(&w.w)));
+    vm = __bfloat162float(__hmax_nan(__low2bfloat16(m), __high2bfloat16(m)));
+  } else {
+    const float a = __uint_as_float(w.x), b = __uint_as_float(w.y);
+    const float c = __uint_as_float(w.z), d = __uint_as_float(w.w);
+    vm = (a != a || b != b || c != c || d != d) ? NAN : fmaxf(fmaxf(a, b), fmaxf(c, d));
+  }
+  if (!(vm < INFINITY)) {  // a NaN or +inf is in this vector: exact path
+#pragma unroll
+    for (int k = 0; k < VEC; ++k) scan_scalar<Bits>(vec_elem<Bits>(w, k), base + k, rm);
+    return;
+  }
+  if (vm > rm.val || (rm.idx == 0xFFFFFFFFu && vm == rm.val)) {
+    uint32_t first = base;
+#pragma unroll
+    for (int k = VEC - 1; k >= 0; --k)
+      if (Elem<Bits>::to_float(vec_elem<Bits>(w, k)) == vm) first = base + k;
+    rm.val = vm;
+    rm.idx = first;
+  }
+}
+
+template <typename Bits>
+__device__ __forceinline__ uint32_t float_key(float v) {
+  if constexpr (sizeof(Bits) == 2)
+    return Elem<Bits>::key(__float_as_uint(v) >> 16);
+  else
+    return Elem<Bits>::key(__float_as_uint(v));
+}
+
+// grid: rows * splits CTAs; CTA (row, s) covers [s*chunk, min(V, (s+1)*chunk)).
+template <typename Bits>
+__global__ void __launch_bounds__(kThreads) row_argmax_kernel(
+    const Bits *__restrict__ logits, int64_t row_stride, int32_t V, int32_t splits,
+    int32_t chunk, uint64_t *__restrict__ partial, uint32_t *dev_status) {
+  constexpr int VEC = Elem<Bits>::kVec;
+  const int64_t row = blockIdx.x / splits;
+  const int32_t s = blockIdx.x % splits;
+  const Bits *r = logits + row * row_stride;
+  const int32_t c0 = s * chunk;
+  const int32_t c1 = min(V, c0 + chunk);
+
+  RunMax rm;
+
+  // 16-byte aligned middle part [a0, a1), scalar head and tail.
+  const uintptr_t addr0 = reinterpret_cast<uintptr_t>(r + c0);
+  int32_t a0 = c0 + (int32_t)(((16u - (addr0 & 15u)) & 15u) / sizeof(Bits));
+  if ((addr0 % sizeof(Bits)) != 0 || a0 > c1) a0 = c1;  // cannot vectorise
+  const int32_t nvec = (c1 - a0) / VEC;
+  const int32_t a1 = a0 + nvec * VEC;
+
+  for (int32_t v = c0 + threadIdx.x; v < a0; v += kThreads) scan_scalar<Bits>(r[v], v, rm);
+
+  const uint4 *vp = reinterpret_cast<const uint4 *>(r + a0);
+  constexpr int U = 4;  // vectors in flight per thread
+  int32_t j = threadIdx.x;
+  for (; j + (U - 1) * kThreads < nvec; j += U * kThreads) {
+    uint4 w[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) w[u] = ldg_stream(vp + j + u * kThreads);
+#pragma unroll
+    for (int u = 0; u < U; ++u) scan_vec<Bits>(w[u], (uint32_t)(a0 + (j + u * kThreads) * VEC), rm);
+  }
+  for (; j < nvec; j += kThreads) scan_vec<Bits>(ldg_stream(vp + j), (uint32_t)(a0 + j * VEC), rm);
+
+  for (int32_t v = a1 + threadIdx.x; v < c1; v += kThreads) scan_scalar<Bits>(r[v], v, rm);
+
+  // A chunk made only of -inf/NaN reports its first index with the key of
+  // -inf, so an all -inf row resolves to index 0 like everywhere else.
+  uint64_t packed = 0;
+  if (rm.idx != 0xFFFFFFFFu) packed = pack_argmax(float_key<Bits>(rm.val), rm.idx);
+  else if (c0 < c1) packed = pack_argmax(float_key<Bits>(-INFINITY), (uint32_t)c0);
+  packed = warp_max_u64(packed);
+  __shared__ uint64_t red[kWarps];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) red[warp] = packed;
+  const bool any_bad = __syncthreads_or(rm.bad);
+  if (warp == 0) {
+    uint64_t x = lane < kWarps ? red[lane] : 0ull;
+    x = warp_max_u64(x);
+    if (lane == 0) {
+      partial[blockIdx.x] = x;
+      if (any_bad && dev_status) atomicOr(dev_status, PSI_DEV_NONFINITE);
+    }
+  }
+}
+
+__device__ __forceinline__ int32_t argmax_of(const uint64_t *partial, int64_t row,
+                                             int32_t splits) {
+  uint64_t best = 0;
+  for (int32_t s = 0; s < splits; ++s) {
+    const uint64_t w = partial[row * splits + s];
+    best = w > best ? w : best;
+  }
+  return (int32_t)(0xFFFFFFFFu - (uint32_t)best);
+}
+
+// One thread per sequence.
+__global__ void __launch_bounds__(128) greedy_emit_kernel(
+    const uint64_t *__restrict__ partial, int32_t splits, const int32_t *__restrict__ ids,
+    int32_t N, int32_t B, int32_t V, int32_t *__restrict__ out_tokens,
+    int32_t *__restrict__ out_n, uint32_t *dev_status) {
+  const int32_t n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  const int64_t row0 = (int64_t)n * (B + 1);
+  int32_t L = B;
+  bool bad_id = false;
+  for (int32_t i = 0; i < B; ++i) {
+    const int32_t x = ids[(int64_t)n * B + i];
+    bad_id |= (x < 0 || x >= V);
+    if (L == B && x != argmax_of(partial, row0 + i, splits)) L = i;
+  }
+  int32_t *tok = out_tokens + (int64_t)n * (B + 1);
+  for (int32_t i = 0; i < L; ++i) tok[i] = ids[(int64_t)n * B + i];
+  tok[L] = argmax_of(partial, row0 + L, splits);
+  for (int32_t i = L + 1; i <= B; ++i) tok[i] = -1;
+  out_n[n] = L + 1;
+  if (bad_id && dev_status) atomicOr(dev_status, PSI_DEV_BAD_TOKEN_ID);
+}
+
+// One CTA per sequence: argmaxes and node data staged in shared memory, then
+// one thread walks the nodes in index order (parents precede children).
+__global__ void __launch_bounds__(kThreads) tree_walk_kernel(
+    const uint64_t *__restrict__ partial, int32_t splits,
+    const int32_t *__restrict__ node_tokens, const int32_t *__restrict__ parents,
+    int32_t M, int32_t V, int32_t *__restrict__ out_path_nodes,
+    int32_t *__restrict__ out_path_len, int32_t *__restrict__ out_tokens,
+    uint32_t *dev_status) {
+  extern __shared__ int32_t sm[];
+  int32_t *am = sm;              // [M+1]
+  int32_t *tok = am + (M + 1);   // [M]
+  int32_t *par = tok + M;        // [M]
+  int32_t *depth = par + M;      // [M], 0 = unmatched
+  int32_t *path = depth + M;     // [M+1]
+  __shared__ int32_t s_best, s_len;
+
+  const int64_t n = blockIdx.x;
+  for (int32_t j = threadIdx.x; j <= M; j += blockDim.x)
+    am[j] = argmax_of(partial, n * (M + 1) + j, splits);
+  for (int32_t k = threadIdx.x; k < M; k += blockDim.x) {
+    tok[k] = node_tokens[n * M + k];
+    par[k] = parents[n * M + k];
+  }
+  __syncthreads();
+
+  if (threadIdx.x == 0) {
+    uint32_t status = 0;
+    int32_t best = -1, best_depth = 0;
+    for (int32_t k = 0; k < M; ++k) {
+      depth[k] = 0;
+      const int32_t p = par[k];
+      if (p < -1 || p >= k) {
+        status |= PSI_DEV_BAD_PARENT;
+        continue;
+      }
+      const int32_t t = tok[k];
+      if (t < 0 || t >= V) {
+        status |= PSI_DEV_BAD_TOKEN_ID;
+        continue;
+      }
+      const int32_t pd = (p < 0) ? 0 : depth[p];
+      if ((p < 0 || pd > 0) && t == am[p + 1]) {
+        depth[k] = pd + 1;
+        if (depth[k] > best_depth) {
+          best_depth = depth[k];
+          best = k;
+        }
+      }
+    }
+    int32_t d = best_depth;
+    for (int32_t k = best; k >= 0; k = par[k]) path[--d] = k;
+    s_best = best;
+    s_len = best_depth;
+    if (status && dev_status) atomicOr(dev_status, status);
+  }
+  __syncthreads();
+  const int32_t len = s_len;
+  for (int32_t k = threadIdx.x; k < M; k += blockDim.x)
+    out_path_nodes[n * M + k] = k < len ? path[k] : -1;
+  for (int32_t k = threadIdx.x; k <= M; k += blockDim.x) {
+    int32_t v = -1;
+    if (k < len) v = tok[path[k]];
+    else if (k == len) v = am[s_best + 1];
+    out_tokens[n * (M + 1) + k] = v;
+  }
+  if (threadIdx.x == 0) out_path_len[n] = len;
+}
+
+// ---------------------------------------------------------------------------
+// Host launchers.
+// ---------------------------------------------------------------------------
+ArgmaxPlan plan_argmax(int64_t rows, int32_t V, int elem_bytes) {
+  ArgmaxPlan p;
+  const int vec = 16 / elem_bytes;
+  // Aim for at least ~8 waves of CTAs over the SMs, but keep chunks >= 16 KB.
+  const int64_t want_ctas = 148LL * 8 * 4;
+  int64_t splits = (want_ctas + rows - 1) / rows;
+  const int64_t min_chunk = 16384 / elem_bytes;
+  const int64_t max_splits = (V + min_chunk - 1) / min_chunk;
+  if (splits > max_splits) splits = max_splits;
+  if (splits < 1) splits = 1;
+  int64_t chunk = (V + splits - 1) / splits;
+  chunk = (chunk + vec - 1) / vec * vec;
+  splits = (V + chunk - 1) / chunk;
+  p.splits = (int32_t)splits;
+  p.chunk = (int32_t)chunk;
+  return p;
+}
+
+cudaError_t launch_row_argmax(const void *logits, int64_t row_stride, psi_dtype dtype,
+                              int64_t rows, int32_t V, const ArgmaxPlan &plan,
+                              uint64_t *partial, uint32_t *dev_status, cudaStream_t stream) {
+  const int64_t grid = rows * plan.splits;
+  if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+  if (dtype == PSI_DTYPE_BF16)
+    row_argmax_kernel<uint16_t><<<(unsigned)grid, kThreads, 0, stream>>>(
+        static_cast<const uint16_t *>(logits), row_stride, V, plan.splits, plan.chunk, partial,
+        dev_status);
+  else
+    row_argmax_kernel<uint32_t><<<(unsigned)grid, kThreads, 0, stream>>>(
+        static_cast<const uint32_t *>(logits), row_stride, V, plan.splits, plan.chunk, partial,
+        dev_status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_greedy_emit(const uint64_t *partial, int32_t splits, const int32_t *ids,
+                               int32_t N, int32_t B, int32_t V, int32_t *out_tokens,
+                               int32_t *out_n, uint32_t *dev_status, cudaStream_t stream) {
+  greedy_emit_kernel<<<(N + 127) / 128, 128, 0, stream>>>(partial, splits, ids, N, B, V,
+                                                          out_tokens, out_n, dev_status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tree_walk(const uint64_t *partial, int32_t splits, const int32_t *node_tokens,
+                             const int32_t *parents, int32_t N, int32_t M, int32_t V,
+                             int32_t *out_path_nodes, int32_t *out_path_len,
+                             int32_t *out_tokens, uint32_t *dev_status, cudaStream_t stream) {
+  const size_t smem = sizeof(int32_t) * (size_t)(5 * M + 2);
+  static bool configured = false;  // opt in to >48 KB once (only large M needs it)
+  if (smem > 48 * 1024 && !configured) {
+    cudaError_t e = cudaFuncSetAttribute(tree_walk_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(5 * PSI_MAX_TREE_NODES + 2) * 4);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  tree_walk_kernel<<<N, kThreads, smem, stream>>>(partial, splits, node_tokens, parents, M, V,
+                                                  out_path_nodes, out_path_len, out_tokens,
+                                                  dev_status);
+  return cudaGetLastError();
+}
+
+}  // namespace psi

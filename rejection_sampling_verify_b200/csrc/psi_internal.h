@@ -1,0 +1,86 @@
+// psi_internal.h - declarations shared by the library's translation units
+// (launch plans and launchers).  Not part of the public ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "psi_device.cuh"
+#include "psi_verify.h"
+
+namespace psi {
+
+// ---- greedy paths ----------------------------------------------------------
+struct ArgmaxPlan {
+  int32_t splits = 1;  // CTAs per row
+  int32_t chunk = 0;   // elements per CTA (multiple of the 16-byte vector)
+};
+
+ArgmaxPlan plan_argmax(int64_t rows, int32_t V, int elem_bytes);
+
+cudaError_t launch_row_argmax(const void *logits, int64_t row_stride, psi_dtype dtype,
+                              int64_t rows, int32_t V, const ArgmaxPlan &plan,
+                              uint64_t *partial, uint32_t *dev_status, cudaStream_t stream);
+
+cudaError_t launch_greedy_emit(const uint64_t *partial, int32_t splits, const int32_t *ids,
+                               int32_t N, int32_t B, int32_t V, int32_t *out_tokens,
+                               int32_t *out_n, uint32_t *dev_status, cudaStream_t stream);
+
+cudaError_t launch_tree_walk(const uint64_t *partial, int32_t splits, const int32_t *node_tokens,
+                             const int32_t *parents, int32_t N, int32_t M, int32_t V,
+                             int32_t *out_path_nodes, int32_t *out_path_len,
+                             int32_t *out_tokens, uint32_t *dev_status, cudaStream_t stream);
+
+// ---- sampled linear path -----------------------------------------------------
+// Per (sequence, row) record written by the unit kernel, read by the emit
+// kernel.
+struct UnitRecord {
+  int32_t accept;  // row i < B: draft accepted
+  int32_t token;   // correction (rejected row) or bonus (row B), else -1
+};
+
+struct SampledPlan {
+  int32_t cluster = 1;   // CTAs per (sequence, row) unit
+  int32_t slice = 0;     // vocabulary elements per CTA (multiple of the vector)
+  int32_t nvec_pad = 0;  // 16-byte vectors per row buffer (multiple of 32)
+  size_t smem = 0;       // dynamic shared memory per CTA
+};
+
+// Returns false if V does not fit the shared-memory-resident design.
+bool plan_sampled(int32_t V, int elem_bytes, SampledPlan *plan);
+
+struct SampledArgs {
+  const void *ar;
+  int64_t ar_stride;
+  const void *draft;
+  int64_t draft_stride;
+  const int32_t *ids;
+  int32_t N, B, V;
+  float temperature;
+  float top_p;
+  uint64_t seed;
+  const uint64_t *seq_ids;
+  uint64_t step;
+  int32_t *out_tokens;
+  int32_t *out_n;
+  float *out_p;
+  float *out_q;
+  uint32_t *dev_status;
+  UnitRecord *records;  // workspace [N][B+1]
+};
+
+// Optional events recorded around the main kernel launch (instrumentation).
+struct KernelEvents {
+  cudaEvent_t before = nullptr;
+  cudaEvent_t after = nullptr;
+};
+
+cudaError_t launch_sampled(const SampledArgs &a, psi_dtype dtype, const SampledPlan &plan,
+                           const KernelEvents &ev, cudaStream_t stream);
+
+cudaError_t launch_rng_uniforms(uint64_t seed, const uint64_t *seq_ids, int32_t n_seq,
+                                uint64_t step, int32_t n_rows, uint32_t purpose, float *out,
+                                cudaStream_t stream);
+
+}  // namespace psi

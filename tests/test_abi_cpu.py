@@ -1,0 +1,127 @@
+"""CPU checks of the C ABI (no GPU needed): the library loads, exports every
+function the public header declares, and rejects bad arguments on the host
+before launching anything."""
+import os
+import re
+
+import pytest
+
+import rejection_sampling_verify_b200 as psi
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "psi_verify.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(psi_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_function():
+    lib = psi.load_library()
+    names = declared_functions()
+    assert len(names) >= 7, names
+    for name in names:
+        assert hasattr(lib, name), name
+    assert sorted(psi.EXPORTED) == names
+
+
+def test_header_constants_match_binding():
+    text = open(HEADER).read()
+    consts = dict(re.findall(r"#define\s+(PSI_[A-Z_]+)\s+(\d+)u?", text))
+    for k, v in consts.items():
+        assert getattr(psi, k) == int(v), k
+    enums = dict(re.findall(r"\b(PSI_[A-Z_0-9]+)\s*=\s*(\d+)", text))
+    for k, v in enums.items():
+        assert getattr(psi, k) == int(v), k
+
+
+def test_status_strings():
+    for code in range(7):
+        assert psi.psi_status_string(code).startswith("PSI_")
+    assert psi.psi_status_string(99) == "PSI_ERR_UNKNOWN"
+
+
+def test_workspace_queries():
+    ws = psi.psi_verify_linear_workspace_bytes(256, 8, 151936, psi.PSI_DTYPE_BF16, 0.7, 0.95)
+    assert ws >= 256 * 9 * 8 and ws % 256 == 0
+    wg = psi.psi_verify_linear_workspace_bytes(1024, 16, 151936, psi.PSI_DTYPE_BF16, 0.0, 1.0)
+    assert wg >= 1024 * 17 * 8 and wg % 256 == 0
+    assert psi.psi_verify_linear_workspace_bytes(0, 8, 10, 1, 1.0, 1.0) == 0
+    assert psi.psi_verify_linear_workspace_bytes(1, 33, 10, 1, 1.0, 1.0) == 0
+    assert psi.psi_verify_linear_workspace_bytes(1, 8, psi.PSI_MAX_V + 1, 1, 1.0, 1.0) == 0
+    assert psi.psi_verify_linear_workspace_bytes(1, 8, psi.PSI_MAX_V // 2 + 1, 0, 1.0, 1.0) == 0
+    assert psi.psi_verify_tree_greedy_workspace_bytes(16, 64, 151936, 1) > 0
+    assert psi.psi_verify_tree_greedy_workspace_bytes(16, psi.PSI_MAX_TREE_NODES + 1, 10, 1) == 0
+
+
+FAKE = 0x10000  # a 64 KB-aligned fake device address: never dereferenced
+
+
+def _linear(**over):
+    args = dict(ar_logits=FAKE, ar_row_stride=100, draft_logits=FAKE, draft_row_stride=100,
+                dtype=psi.PSI_DTYPE_BF16, draft_ids=FAKE, N=2, B=4, V=100, temperature=1.0,
+                top_p=1.0, seed=0, seq_ids=None, step=0, out_tokens=FAKE, out_n_emitted=FAKE,
+                out_p_draft=None, out_q_draft=None, dev_status=None, workspace=FAKE,
+                workspace_bytes=1 << 20, stream=None)
+    args.update(over)
+    return psi.psi_verify_linear(**args)
+
+
+@pytest.mark.parametrize("over,want", [
+    (dict(N=0), psi.PSI_ERR_INVALID_ARG),
+    (dict(B=0), psi.PSI_ERR_INVALID_ARG),
+    (dict(B=33), psi.PSI_ERR_INVALID_ARG),
+    (dict(V=0), psi.PSI_ERR_INVALID_ARG),
+    (dict(V=psi.PSI_MAX_V + 1, ar_row_stride=psi.PSI_MAX_V + 1,
+          draft_row_stride=psi.PSI_MAX_V + 1), psi.PSI_ERR_UNSUPPORTED),
+    (dict(temperature=-0.5), psi.PSI_ERR_INVALID_ARG),
+    (dict(temperature=float("nan")), psi.PSI_ERR_INVALID_ARG),
+    (dict(temperature=float("inf")), psi.PSI_ERR_INVALID_ARG),
+    (dict(top_p=0.0), psi.PSI_ERR_INVALID_ARG),
+    (dict(top_p=1.5), psi.PSI_ERR_INVALID_ARG),
+    (dict(top_p=float("nan")), psi.PSI_ERR_INVALID_ARG),
+    (dict(ar_logits=None), psi.PSI_ERR_INVALID_ARG),
+    (dict(draft_logits=None), psi.PSI_ERR_INVALID_ARG),
+    (dict(draft_ids=None), psi.PSI_ERR_INVALID_ARG),
+    (dict(out_tokens=None), psi.PSI_ERR_INVALID_ARG),
+    (dict(ar_row_stride=99), psi.PSI_ERR_INVALID_ARG),
+    (dict(dtype=7), psi.PSI_ERR_INVALID_ARG),
+    (dict(ar_logits=FAKE + 1), psi.PSI_ERR_MISALIGNED),
+    (dict(draft_ids=FAKE + 2), psi.PSI_ERR_MISALIGNED),
+    (dict(seq_ids=FAKE + 4), psi.PSI_ERR_MISALIGNED),
+    (dict(workspace=None), psi.PSI_ERR_WORKSPACE),
+    (dict(workspace_bytes=8), psi.PSI_ERR_WORKSPACE),
+])
+def test_linear_rejects_bad_arguments_before_launch(over, want):
+    assert _linear(**over) == want
+    assert psi.psi_last_error()
+
+
+def test_greedy_allows_null_draft():
+    # greedy with a null draft pointer passes validation up to the workspace
+    assert _linear(temperature=0.0, draft_logits=None, workspace=None) == psi.PSI_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("over,want", [
+    (dict(N=0), psi.PSI_ERR_INVALID_ARG),
+    (dict(M=0), psi.PSI_ERR_INVALID_ARG),
+    (dict(M=psi.PSI_MAX_TREE_NODES + 1), psi.PSI_ERR_INVALID_ARG),
+    (dict(parents=None), psi.PSI_ERR_INVALID_ARG),
+    (dict(node_tokens=FAKE + 1), psi.PSI_ERR_MISALIGNED),
+    (dict(workspace_bytes=0), psi.PSI_ERR_WORKSPACE),
+])
+def test_tree_rejects_bad_arguments_before_launch(over, want):
+    args = dict(ar_logits=FAKE, ar_row_stride=50, dtype=psi.PSI_DTYPE_BF16, node_tokens=FAKE,
+                parents=FAKE, N=2, M=8, V=50, out_path_nodes=FAKE, out_path_len=FAKE,
+                out_tokens=FAKE, dev_status=None, workspace=FAKE, workspace_bytes=1 << 20,
+                stream=None)
+    args.update(over)
+    assert psi.psi_verify_tree_greedy(**args) == want
+
+
+def test_rng_rejects_bad_arguments():
+    assert psi.psi_rng_uniforms(0, None, 0, 0, 4, 0, FAKE, None) == psi.PSI_ERR_INVALID_ARG
+    assert psi.psi_rng_uniforms(0, None, 4, 0, 4, 0, None, None) == psi.PSI_ERR_INVALID_ARG
+    assert psi.psi_rng_uniforms(0, None, 4, 0, 4, 0, FAKE + 2, None) == psi.PSI_ERR_MISALIGNED
