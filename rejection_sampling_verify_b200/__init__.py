@@ -230,16 +230,16 @@ def verify_linear(ar, draft, ids, temperature: float, top_p: float = 1.0, seed: 
             torch.empty(N, B, dtype=torch.float32, device=dev) if want_probs and not greedy else None,
             torch.zeros(1, dtype=torch.int32, device=dev))
     ws_bytes = psi_verify_linear_workspace_bytes(N, B, V, code, float(temperature), float(top_p))
-    if ws_bytes == 0:
-        raise PsiError(PSI_ERR_INVALID_ARG, "psi_verify_linear_workspace_bytes")
-    if workspace is None or workspace.numel() < ws_bytes:
+    if ws_bytes == 0:  # invalid sizes: let the ABI report the precise status
+        workspace = None
+    elif workspace is None or workspace.numel() < ws_bytes:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     st = psi_verify_linear(
         _ptr(ar), ar_stride, None if greedy else _ptr(draft), dr_stride, code, _ptr(ids), N, B,
         V, float(temperature), float(top_p), int(seed) & (2**64 - 1),
         _ptr(seq_ids), int(step) & (2**64 - 1), _ptr(out.tokens), _ptr(out.n_emitted),
         _ptr(out.p_draft), _ptr(out.q_draft), _ptr(out.status), _ptr(workspace),
-        workspace.numel(), _stream(stream))
+        0 if workspace is None else workspace.numel(), _stream(stream))
     _check(st, "psi_verify_linear")
     return out
 
@@ -270,14 +270,14 @@ def verify_tree_greedy(ar, node_tokens, parents, workspace=None, stream=None,
                          torch.empty(N, M + 1, dtype=torch.int32, device=dev),
                          torch.zeros(1, dtype=torch.int32, device=dev))
     ws_bytes = psi_verify_tree_greedy_workspace_bytes(N, M, V, code)
-    if ws_bytes == 0:
-        raise PsiError(PSI_ERR_INVALID_ARG, "psi_verify_tree_greedy_workspace_bytes")
-    if workspace is None or workspace.numel() < ws_bytes:
+    if ws_bytes == 0:  # invalid sizes: let the ABI report the precise status
+        workspace = None
+    elif workspace is None or workspace.numel() < ws_bytes:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     st = psi_verify_tree_greedy(_ptr(ar), stride, code, _ptr(node_tokens), _ptr(parents), N, M,
                                 V, _ptr(out.path_nodes), _ptr(out.path_len), _ptr(out.tokens),
-                                _ptr(out.status), _ptr(workspace), workspace.numel(),
-                                _stream(stream))
+                                _ptr(out.status), _ptr(workspace),
+                                0 if workspace is None else workspace.numel(), _stream(stream))
     _check(st, "psi_verify_tree_greedy")
     return out
 

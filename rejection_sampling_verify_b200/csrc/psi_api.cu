@@ -96,7 +96,8 @@ size_t psi_verify_linear_workspace_bytes(int32_t N, int32_t B, int32_t V, psi_dt
     const psi::ArgmaxPlan plan = psi::plan_argmax(rows, V, elem_bytes(dtype));
     return round256(sizeof(uint64_t) * (size_t)rows * plan.splits);
   }
-  return round256(sizeof(psi::UnitRecord) * (size_t)rows);
+  (void)rows;
+  return round256(psi::fast_layout(N, B).total);
 }
 
 psi_status psi_verify_linear(const void *ar_logits, int64_t ar_row_stride,
@@ -175,7 +176,15 @@ psi_status psi_verify_linear(const void *ar_logits, int64_t ar_row_stride,
   a.out_q = out_q_draft;
   a.dev_status = dev_status;
   a.records = static_cast<psi::UnitRecord *>(workspace);
-  e = psi::launch_sampled(a, dtype, plan, g_events, stream);
+  // Streaming path when every row starts on a 16-byte boundary (TMA bulk
+  // copies); otherwise one cluster per unit with plain loads.
+  const bool rows_aligned = aligned_to(ar_logits, 16) && aligned_to(draft_logits, 16) &&
+                            ((size_t)ar_row_stride * es) % 16 == 0 &&
+                            ((size_t)draft_row_stride * es) % 16 == 0;
+  if (rows_aligned)
+    e = psi::launch_sampled_fast(a, dtype, plan, workspace, g_events, stream);
+  else
+    e = psi::launch_sampled(a, dtype, plan, g_events, stream);
   if (e != cudaSuccess) return cuda_fail(e, "sampled verify launch");
   return PSI_OK;
 }

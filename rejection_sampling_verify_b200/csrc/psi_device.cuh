@@ -100,11 +100,13 @@ struct Elem<uint32_t> {
 // Element k (0..kVec-1) of a 16-byte vector.
 template <typename Bits>
 __device__ __forceinline__ uint32_t vec_elem(const uint4 &v, int k) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  // selects rather than an indexed array, so a run-time k stays in registers
+  const int q = sizeof(Bits) == 2 ? (k >> 1) : k;
+  const uint32_t word = q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
   if constexpr (sizeof(Bits) == 2)
-    return (k & 1) ? (w[k >> 1] >> 16) : (w[k >> 1] & 0xFFFFu);
+    return (k & 1) ? (word >> 16) : (word & 0xFFFFu);
   else
-    return w[k];
+    return word;
 }
 
 // Cheap screen for "some element may be NaN/+-inf": true for every vector

@@ -76,8 +76,38 @@ struct KernelEvents {
   cudaEvent_t after = nullptr;
 };
 
+// General path: one cluster per unit for every unit, then the emit kernel.
 cudaError_t launch_sampled(const SampledArgs &a, psi_dtype dtype, const SampledPlan &plan,
                            const KernelEvents &ev, cudaStream_t stream);
+
+// The cluster kernel over a device-side list of units: full verify of each
+// listed unit (kModeList = 1) or only its correction/bonus draw, written to
+// out_tokens (kModeSample = 2).  `max_clusters` persistent clusters.
+cudaError_t launch_cluster_list(const SampledArgs &a, psi_dtype dtype, const SampledPlan &plan,
+                                int mode, const int32_t *list, const int32_t *count,
+                                int max_clusters, cudaStream_t stream);
+
+// ---- streaming path (rows 16-byte aligned) ------------------------------------
+// Per logit row: statistics written by the row-statistics kernel.
+struct RowRecord {
+  float m;            // row maximum
+  int32_t flags;      // kRowNeedGeneral: the general path must handle the unit
+  double z;           // sum over the row of exp((x - m) / T)
+  double zp;          // normaliser after top-p (z when top-p is off)
+  uint32_t tau_bits;  // top-p threshold logit (raw bits); keep x >= tau
+  int32_t n_nuc;      // nucleus entries stored for this row
+};
+constexpr int32_t kRowNeedGeneral = 1;
+constexpr int32_t kRowNonfinite = 2;
+constexpr int kNucCap = 1024;   // nucleus entries kept per row
+
+struct FastLayout {  // workspace carve-up of the streaming path
+  size_t rec_off, rows_off, nuc_off, counters_off, list_a_off, list_b_off, total;
+};
+FastLayout fast_layout(int32_t N, int32_t B);
+
+cudaError_t launch_sampled_fast(const SampledArgs &a, psi_dtype dtype, const SampledPlan &plan,
+                                void *workspace, const KernelEvents &ev, cudaStream_t stream);
 
 cudaError_t launch_rng_uniforms(uint64_t seed, const uint64_t *seq_ids, int32_t n_seq,
                                 uint64_t step, int32_t n_rows, uint32_t purpose, float *out,

@@ -38,6 +38,9 @@ namespace psi {
 namespace {
 
 constexpr int kBins = 512;                         // radix bins per level (9 bits)
+constexpr int kModeGrid = 0;    // one unit per cluster, units in grid order
+constexpr int kModeList = 1;    // full verify of the units in a device list
+constexpr int kModeSample = 2;  // correction/bonus draw only, token written to the output
 constexpr float kFixScale = 1099511627776.0f;      // 2^40
 constexpr double kFixScaleD = 1099511627776.0;     // 2^40
 constexpr double kFixInv = 1.0 / 1099511627776.0;  // 2^-40
@@ -270,7 +273,9 @@ template <typename Bits>
 __global__ void __launch_bounds__(kThreads) sampled_unit_kernel(SampledArgs a, SampledPlan plan,
                                                                  float coef, double coef64,
                                                                  float w_min, float w_narrow,
-                                                                 int use_top_p) {
+                                                                 int use_top_p, int mode,
+                                                                 const int32_t *work_list,
+                                                                 const int32_t *work_count) {
   constexpr int VEC = Elem<Bits>::kVec;
   extern __shared__ __align__(128) unsigned char dyn_smem[];
   __shared__ Xchg xc;
@@ -286,8 +291,19 @@ __global__ void __launch_bounds__(kThreads) sampled_unit_kernel(SampledArgs a, S
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t rank = cluster_rank();
   const uint32_t C = cluster_size();
-  const int64_t unit = blockIdx.x / C;
   const int32_t B = a.B, V = a.V;
+  if (tid == 0) {
+    mbar_init(&mbar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // kModeGrid: cluster k handles unit k.  kModeList / kModeSample: the
+  // clusters of a small persistent grid walk a device-side list of units.
+  const int64_t n_items = mode == kModeGrid ? (int64_t)a.N * (B + 1) : (int64_t)*work_count;
+  const int64_t first = blockIdx.x / C, stride = gridDim.x / C;
+  uint32_t parity = 0;
+  for (int64_t item = first; item < n_items; item += stride, parity ^= 1u) {
+  const int64_t unit = mode == kModeGrid ? item : (int64_t)work_list[item];
   const int32_t n = (int32_t)(unit / (B + 1));
   const int32_t i = (int32_t)(unit % (B + 1));
   const bool has_q = i < B;
@@ -312,12 +328,7 @@ __global__ void __launch_bounds__(kThreads) sampled_unit_kernel(SampledArgs a, S
   const bool aligned = ((reinterpret_cast<uintptr_t>(row_p + c0) & 15u) == 0) &&
                        (!has_q || (reinterpret_cast<uintptr_t>(row_q + c0) & 15u) == 0);
   const int32_t bulk = aligned ? (len / VEC) * VEC : 0;
-  if (tid == 0) {
-    mbar_init(&mbar, 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-  if (tid == 0 && bulk > 0) {
+  if (tid == 0) {  // completes this item's phase (at once when nothing is copied)
     const uint32_t bytes = (uint32_t)bulk * sizeof(Bits);
     mbar_arrive_expect_tx(&mbar, bytes * (has_q ? 2u : 1u));
     for (uint32_t off = 0; off < bytes; off += 32768u) {
@@ -353,7 +364,7 @@ __global__ void __launch_bounds__(kThreads) sampled_unit_kernel(SampledArgs a, S
     for (int t = tid; t < 2 * kBins; t += kThreads) hist[t] = 0ull;
   __syncthreads();
   bool timed_out = false;
-  if (bulk > 0) timed_out = !mbar_wait_bounded(&mbar, 0);
+  timed_out = !mbar_wait_bounded(&mbar, parity);
 
   const uint4 *vp = reinterpret_cast<const uint4 *>(buf_p);
   const uint4 *vq = reinterpret_cast<const uint4 *>(buf_q);
@@ -573,8 +584,8 @@ __global__ void __launch_bounds__(kThreads) sampled_unit_kernel(SampledArgs a, S
       }
       const float u = uniform24(a.seed, seq, a.step, (uint64_t)i, PSI_PURPOSE_ACCEPT);
       const int accept = (u * q < p) ? 1 : 0;
-      need = !accept;
-      if (rank == 0) {
+      need = (mode == kModeSample) ? 1 : !accept;
+      if (rank == 0 && mode != kModeSample) {
         const int64_t o = (int64_t)n * B + i;
         if (a.out_p) a.out_p[o] = p;
         if (a.out_q) a.out_q[o] = q;
@@ -582,7 +593,7 @@ __global__ void __launch_bounds__(kThreads) sampled_unit_kernel(SampledArgs a, S
         if (accept) a.records[unit].token = -1;
         if (!valid && a.dev_status) atomicOr(a.dev_status, PSI_DEV_BAD_TOKEN_ID);
       }
-    } else if (rank == 0) {
+    } else if (rank == 0 && mode != kModeSample) {
       a.records[unit].accept = 1;  // the bonus row always draws
     }
     bc.need_sample = need;
@@ -771,14 +782,22 @@ __global__ void __launch_bounds__(kThreads) sampled_unit_kernel(SampledArgs a, S
         }
         if (token < 0) token = c0;
       }
-      if (lane == 0) a.records[unit].token = token;
+      if (lane == 0) {
+        if (mode == kModeSample) a.out_tokens[unit] = token;
+        else a.records[unit].token = token;
+      }
     }
   }
-  if (bc.need_sample && bc.w_total <= 0.f && rank == 0 && tid == 0)
-    a.records[unit].token = 0;  // no positive weight anywhere (degenerate row)
+  if (bc.need_sample && bc.w_total <= 0.f && rank == 0 && tid == 0) {
+    // no positive weight anywhere (degenerate row)
+    if (mode == kModeSample) a.out_tokens[unit] = 0;
+    else a.records[unit].token = 0;
+  }
 
   // keep this CTA's shared memory alive until every peer is done reading it
+  // (and the buffers free for the next item)
   cluster_sync();
+  }  // work items
 }
 
 // One thread per sequence: first rejected row -> emitted tokens.
@@ -826,10 +845,31 @@ bool plan_sampled(int32_t V, int elem_bytes, SampledPlan *plan) {
   return true;
 }
 
+struct ClusterParams {
+  float coef;
+  double coef64;
+  float w_min, w_narrow;
+  int use_top_p;
+};
+
+static ClusterParams cluster_params(const SampledArgs &a) {
+  ClusterParams c;
+  c.coef64 = 1.4426950408889634 / (double)a.temperature;  // log2(e) / T
+  c.coef = (float)c.coef64;
+  c.use_top_p = a.top_p < 1.0f ? 1 : 0;
+  // Only e(v) above (1 - top_p) / V can reach the threshold (the mass below
+  // the threshold key exceeds (1 - top_p) * Z >= 1 - top_p and is spread over
+  // at most V tokens); half of it leaves room for rounding.
+  c.w_min = c.use_top_p ? (float)(0.5 * (1.0 - (double)a.top_p) / (double)a.V) : 0.f;
+  c.w_narrow = fmaxf(kNarrowWindow, c.w_min);
+  return c;
+}
+
 template <typename Bits>
-static cudaError_t launch_typed(const SampledArgs &a, const SampledPlan &plan, float coef,
-                                double coef64, float w_min, float w_narrow, int use_top_p,
-                                const KernelEvents &ev, cudaStream_t stream) {
+static cudaError_t launch_cluster_kernel(const SampledArgs &a, const SampledPlan &plan, int mode,
+                                         const int32_t *list, const int32_t *count,
+                                         int64_t n_clusters, const KernelEvents *ev,
+                                         cudaStream_t stream) {
   auto kernel = sampled_unit_kernel<Bits>;
   static int configured_smem = 0;
   if ((int)plan.smem > configured_smem) {
@@ -840,9 +880,9 @@ static cudaError_t launch_typed(const SampledArgs &a, const SampledPlan &plan, f
     if (e != cudaSuccess) return e;
     configured_smem = (int)plan.smem;
   }
-  const int64_t units = (int64_t)a.N * (a.B + 1);
-  const int64_t grid = units * plan.cluster;
-  if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+  const int64_t grid = n_clusters * plan.cluster;
+  if (grid > 0x7FFFFFFFLL || grid < 1) return cudaErrorInvalidConfiguration;
+  const ClusterParams c = cluster_params(a);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -856,28 +896,33 @@ static cudaError_t launch_typed(const SampledArgs &a, const SampledPlan &plan, f
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t e;
-  if (ev.before && (e = cudaEventRecord(ev.before, stream)) != cudaSuccess) return e;
-  e = cudaLaunchKernelEx(&cfg, kernel, a, plan, coef, coef64, w_min, w_narrow, use_top_p);
+  if (ev && ev->before && (e = cudaEventRecord(ev->before, stream)) != cudaSuccess) return e;
+  e = cudaLaunchKernelEx(&cfg, kernel, a, plan, c.coef, c.coef64, c.w_min, c.w_narrow,
+                         c.use_top_p, mode, list, count);
   if (e != cudaSuccess) return e;
-  if (ev.after && (e = cudaEventRecord(ev.after, stream)) != cudaSuccess) return e;
+  if (ev && ev->after && (e = cudaEventRecord(ev->after, stream)) != cudaSuccess) return e;
+  return cudaSuccess;
+}
+
+cudaError_t launch_sampled(const SampledArgs &a, psi_dtype dtype, const SampledPlan &plan,
+                           const KernelEvents &ev, cudaStream_t stream) {
+  const int64_t units = (int64_t)a.N * (a.B + 1);
+  cudaError_t e =
+      dtype == PSI_DTYPE_BF16
+          ? launch_cluster_kernel<uint16_t>(a, plan, kModeGrid, nullptr, nullptr, units, &ev, stream)
+          : launch_cluster_kernel<uint32_t>(a, plan, kModeGrid, nullptr, nullptr, units, &ev, stream);
+  if (e != cudaSuccess) return e;
   sampled_emit_kernel<<<(a.N + 127) / 128, 128, 0, stream>>>(a.records, a.ids, a.N, a.B,
                                                              a.out_tokens, a.out_n);
   return cudaGetLastError();
 }
 
-cudaError_t launch_sampled(const SampledArgs &a, psi_dtype dtype, const SampledPlan &plan,
-                           const KernelEvents &ev, cudaStream_t stream) {
-  const double coef64 = 1.4426950408889634 / (double)a.temperature;  // log2(e) / T
-  const float coef = (float)coef64;
-  const int use_top_p = a.top_p < 1.0f ? 1 : 0;
-  // Only e(v) above (1 - top_p) / V can reach the threshold (the mass below
-  // the threshold key exceeds (1 - top_p) * Z >= 1 - top_p and is spread over
-  // at most V tokens); half of it leaves room for rounding.
-  const float w_min = use_top_p ? (float)(0.5 * (1.0 - (double)a.top_p) / (double)a.V) : 0.f;
-  const float w_narrow = fmaxf(kNarrowWindow, w_min);
+cudaError_t launch_cluster_list(const SampledArgs &a, psi_dtype dtype, const SampledPlan &plan,
+                                int mode, const int32_t *list, const int32_t *count,
+                                int max_clusters, cudaStream_t stream) {
   if (dtype == PSI_DTYPE_BF16)
-    return launch_typed<uint16_t>(a, plan, coef, coef64, w_min, w_narrow, use_top_p, ev, stream);
-  return launch_typed<uint32_t>(a, plan, coef, coef64, w_min, w_narrow, use_top_p, ev, stream);
+    return launch_cluster_kernel<uint16_t>(a, plan, mode, list, count, max_clusters, nullptr, stream);
+  return launch_cluster_kernel<uint32_t>(a, plan, mode, list, count, max_clusters, nullptr, stream);
 }
 
 }  // namespace psi
