@@ -361,7 +361,7 @@ def main():
     peak, peak_kind = hbm_peak()
     achieved = alg / (main_ms / 1000.0) / 1e9
     kernel = "psi_tree_argmax" if is_tree else (
-        "psi_sampled_unit" if cfg.temperature > 0 else "psi_row_argmax")
+        "psi_row_scan" if cfg.temperature > 0 else "psi_row_argmax")
 
     # end to end through the public API with host buffers
     e2e = None
@@ -376,7 +376,10 @@ def main():
                "sample": f"{n} of the {cfg.N} sequences of one step ({dt:.1f} s, single thread)"}
 
     if rank == 0:
-        launches_per_step = 2
+        # our kernels per call: argmax + emit (greedy), argmax + tree walk,
+        # or row_scan, unit, their second passes, two cluster list launches
+        # and fast_emit (sampled); the memset of the list counters is not ours
+        launches_per_step = 2 if (is_tree or cfg.temperature == 0) else 7
         line = {
             "metric": METRIC, "value": value, "unit": "blocks/s", "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,

@@ -181,7 +181,7 @@ psi_status psi_verify_linear(const void *ar_logits, int64_t ar_row_stride,
   const bool rows_aligned = aligned_to(ar_logits, 16) && aligned_to(draft_logits, 16) &&
                             ((size_t)ar_row_stride * es) % 16 == 0 &&
                             ((size_t)draft_row_stride * es) % 16 == 0;
-  if (rows_aligned)
+  if (rows_aligned && psi::fast_path_fits(N, B))
     e = psi::launch_sampled_fast(a, dtype, plan, workspace, g_events, stream);
   else
     e = psi::launch_sampled(a, dtype, plan, g_events, stream);

@@ -8,25 +8,29 @@
 // "想跑 Uno：先確認官方程式需要的環境" (temperature, top-p).
 //
 // Kernels, in launch order:
-//   row_stats      Persistent CTAs stream every logit row ONCE from HBM
-//                  through a 4-stage ring of TMA bulk copies (16 KB each) in
-//                  shared memory.  Per row: maximum m and sum of exponentials
-//                  Z (online, fp32 for the bulk of the row), and with top-p
-//                  the few elements within 2^16 of the running maximum
-//                  ("candidates", typically ~1% of the row) kept in shared
-//                  memory, re-evaluated in double precision at the end of the
-//                  row, and radix-selected on their logit key to find the
-//                  top-p threshold tau, the renormaliser Z' and the nucleus
-//                  (written out, <= 1024 entries).
-//   unit_decide    One CTA per (sequence, row): p(x), q(x), the acceptance
-//                  test, and -- with top-p -- the correction or bonus draw
-//                  over the nucleus only (max(0, p - q) vanishes outside p's
-//                  nucleus), so no logit is read twice.
-//   (cluster kernel, list mode)  units the streaming path cannot handle
-//                  (candidate overflow, a top-p set wider than the window).
-//   fast_emit      First rejected row per sequence; emitted tokens.  Without
-//                  top-p the emitting row's draw needs the whole row again:
-//                  it is queued for the cluster kernel in sample mode.
+//   row_scan   Persistent CTAs stream every logit row ONCE from HBM with
+//              16-byte non-allocating loads (8 per thread in flight, double
+//              buffered in registers).  A row is read in batches of 2048
+//              vectors; inside a batch every thread uses the same reference
+//              (a lower bound of the row maximum, raised between batches), so
+//              all sums are independent of timing.  Elements within the
+//              window below the reference ("candidates", ~0.5% of a row) are
+//              masked out of the fp32 sum of exponentials; the vectors that
+//              hold them are parked in a shared-memory ring and, after the
+//              batch's barrier, split into candidates (to a per-row list in
+//              global memory) and elements that fell below the raised
+//              threshold (a 2^40 fixed-point sum).
+//   unit       One CTA per (sequence, row) unit: finishes the unit's q and p
+//              rows from their candidates (row maximum, Z, the top-p threshold
+//              and renormaliser, p's nucleus), decides the drafted token and
+//              draws the correction or bonus token over p's nucleus.
+//   row_scan / unit, second pass   Rows whose window held less than top_p of
+//              the mass (rescanned with a wider window) or whose candidates
+//              overflowed (rescanned with the exact maximum known).
+//   (cluster kernel, list mode)  Units the second pass could not settle.
+//   fast_emit  First rejected row per sequence; emitted tokens.  Without
+//              top-p the emitting row's draw needs the whole row again: it is
+//              queued for the cluster kernel in sample mode.
 #include <algorithm>
 
 #include "psi_internal.h"
@@ -35,33 +39,42 @@ namespace psi {
 
 namespace {
 
-constexpr int kStages = 4;
-constexpr int kChunkBytes = 16384;
-constexpr int kCandCap = 4096;              // candidate buffer (shared memory)
 constexpr double kFixD = 1099511627776.0;  // 2^40
-// Candidate window, in log2 units below the (running) row maximum: starts at
-// 16 (e > 2^-16 of the maximum) and narrows by 2 down to 12 when the buffer
-// fills; the final window must hold top_p of the mass, else the unit goes to
-// the general path.
-constexpr float kWindowLog2 = 16.f;
-constexpr float kWindowStepLog2 = 2.f;
-constexpr float kWindowMinLog2 = 12.f;
+constexpr float kFixF = 1099511627776.0f;
+constexpr int kInFlight = 8;        // 16-byte loads per thread per batch
+constexpr int kRing = 2048;         // parked vectors (shared memory ring)
 constexpr int kUnitThreads = 256;
+constexpr int kUnitWarps = kUnitThreads / 32;
 constexpr int kListClusters = 16;
+constexpr int32_t kWideBit = int32_t(1) << 30;  // second-pass row entry: wide window
+// Candidate window, in log2 units below the reference.  The first pass uses
+// a narrow window (13 units for top_p <= 0.95, wider as top_p approaches 1);
+// the second pass the wide one.
+constexpr float kWindowBaseLog2 = 13.f;
+constexpr float kWindowWideLog2 = 20.f;
+// Candidates are dropped into the fixed-point sum only while the threshold
+// lies at most this many log2 units above the row's first reference: every
+// dropped term is then below 2^4 (2^44 in 2^40 fixed point), so a row of up
+// to 2^19 elements cannot overflow the 64-bit sum.
+constexpr float kDropGuardLog2 = 4.f;
 
 struct FastArgs {
   SampledArgs s;
-  int64_t rows;          // N*(B+1) AR rows followed by N*B draft rows
-  float coef;            // log2(e) / T
+  int64_t rows;        // N*(B+1) AR rows followed by N*B draft rows
+  float coef;          // log2(e) / T
   double coef64;
-  float win_off;         // initial window width in logit units: 16 / coef
+  float win_narrow;    // window widths in logit units
+  float win_wide;
   int use_top_p;
-  UnitRecord *rec;       // [N*(B+1)]
-  RowRecord *rowrec;     // [rows]
-  uint64_t *nuc;         // [rows][kNucCap]
-  int32_t *counters;     // [0] list A count, [1] list B count
-  int32_t *list_a;       // units for the general path
-  int32_t *list_b;       // units whose draw needs the whole row
+  int pass;            // 1: every row / unit; 2: the listed ones
+  UnitRecord *rec;     // [N*(B+1)]
+  RowRecord *rowrec;   // [rows]
+  uint64_t *cand;      // [rows][kCandCap]: (bits << 32) | vocabulary index
+  int32_t *counters;   // [0] general units, [1] sample-mode units, [2] wide rows, [3] wide units
+  int32_t *list_a;     // units for the general path
+  int32_t *list_b;     // units whose draw needs the whole row
+  int32_t *wide_rows;  // rows for the second scan (| kWideBit: wide window)
+  int32_t *wide_units; // units for the second unit pass
 };
 
 template <typename Bits>
@@ -71,6 +84,7 @@ __device__ __forceinline__ const Bits *row_ptr(const FastArgs &a, int64_t r) {
   return static_cast<const Bits *>(a.s.draft) + (r - nar) * a.s.draft_stride;
 }
 
+// Largest element of a 16-byte vector (NaN if it holds one).
 template <typename Bits>
 __device__ __forceinline__ float raw_vec_max(const uint4 &w) {
   if constexpr (sizeof(Bits) == 2) {
@@ -94,8 +108,8 @@ __device__ __forceinline__ T warp_sum_any(T v) {
   return v;
 }
 
-// Block-wide sum (fixed order), broadcast to every thread.
-template <typename T>
+// Block-wide reductions (fixed order), broadcast to every thread.
+template <typename T, int W>
 __device__ __forceinline__ T block_sum_all(T v, T *scratch) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   v = warp_sum_any(v);
@@ -104,10 +118,11 @@ __device__ __forceinline__ T block_sum_all(T v, T *scratch) {
   __syncthreads();
   T r = T(0);
 #pragma unroll
-  for (int w = 0; w < kWarps; ++w) r += scratch[w];
+  for (int w = 0; w < W; ++w) r += scratch[w];
   return r;
 }
 
+template <int W>
 __device__ __forceinline__ float block_max_all(float v, float *scratch) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   v = warp_max(v);
@@ -116,7 +131,7 @@ __device__ __forceinline__ float block_max_all(float v, float *scratch) {
   __syncthreads();
   float r = -INFINITY;
 #pragma unroll
-  for (int w = 0; w < kWarps; ++w) r = fmaxf(r, scratch[w]);
+  for (int w = 0; w < W; ++w) r = fmaxf(r, scratch[w]);
   return r;
 }
 
@@ -132,446 +147,474 @@ __device__ __forceinline__ uint32_t key_to_bits(uint32_t key) {
     return (key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key;
 }
 
-// Packed fp32 pairs (sm_100 f32x2 instructions).
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-  float2 d;
-  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2,%3};\n\tmov.b64 rb, {%4,%5};\n\t"
-      "mov.b64 rc, {%6,%7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0,%1}, rd;\n\t}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-  return d;
-}
-
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
-  float2 d;
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2,%3};\n\tmov.b64 rb, {%4,%5};\n\t"
-      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0,%1}, rd;\n\t}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return d;
-}
-
-// Block-wide compaction of the candidate buffer: entries with logit > thr
-// stay (packed to the front, in thread order); the others leave the buffer
-// and their mass exp2((x - ref) * coef) is added to zd_t, the thread's
-// dropped-mass accumulator, whose reference zd_ref is moved to `ref` first.
-// An overflowed buffer (count > capacity) stays marked as overflowed.
+// Candidate threshold in the element type: bf16 thresholds are rounded
+// down, so the candidate set can only grow; the streaming sum and the
+// extraction use this same test (x > value).
 template <typename Bits>
-__device__ void compact_candidates(unsigned long long *cand, int *s_cand, int *s_keep, float thr,
-                                   float ref, float coef, float &zd_t, float &zd_ref) {
-  constexpr int PER = kCandCap / kThreads;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (zd_ref != ref) {
-    zd_t = (zd_ref == -INFINITY) ? 0.f : zd_t * fast_exp2((zd_ref - ref) * coef);
-    zd_ref = ref;
-  }
-  const int count = *s_cand;
-  const int n_have = min(count, kCandCap);
-  unsigned long long mine[PER];
-  uint32_t kept = 0u;  // bit t: entry t of this thread stays
-  int keep = 0;
-#pragma unroll
-  for (int t = 0; t < PER; ++t) {
-    const int j = tid * PER + t;
-    mine[t] = 0ull;
-    if (j < n_have) {
-      const unsigned long long e = cand[j];
-      const float x = Elem<Bits>::to_float((uint32_t)(e >> 32));
-      if (x > thr) {
-        mine[t] = e;
-        kept |= 1u << t;
-        ++keep;
-      } else {
-        zd_t += fast_exp2((x - ref) * coef);
-      }
-    }
-  }
-  int incl = keep;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  __syncthreads();  // every entry has been read
-  if (lane == 31) s_keep[warp] = incl;
-  __syncthreads();
-  int off = incl - keep, tot = 0;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) {
-    if (w < warp) off += s_keep[w];
-    tot += s_keep[w];
-  }
-#pragma unroll
-  for (int t = 0; t < PER; ++t)
-    if (kept & (1u << t)) cand[off++] = mine[t];
-  __syncthreads();  // everyone has read the old count and s_keep
-  if (threadIdx.x == 0) *s_cand = (count > kCandCap) ? kCandCap + 1 : tot;
-  __syncthreads();
-}
+struct Threshold {
+  uint32_t pair;  // bf16x2 (both halves) or the f32 bits
+  float value;
+};
 
-// Warp-aggregated append of this lane's candidates (bit e of `mask`: element
-// e of the vector starting at vocabulary index `base`).  Every lane of the
-// warp must call it.  Returns the largest appended logit of this lane.
 template <typename Bits>
-__device__ __forceinline__ float append_candidates(const uint4 &w, uint32_t mask, int32_t base,
-                                                   int *s_cand, unsigned long long *cand) {
-  const int lane = threadIdx.x & 31;
-  const int cnt = __popc(mask);
-  int incl = cnt;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  const int tot = __shfl_sync(0xFFFFFFFFu, incl, 31);
-  int first = 0;
-  if (lane == 31 && tot) first = atomicAdd(s_cand, tot);
-  int pos = __shfl_sync(0xFFFFFFFFu, first, 31) + incl - cnt;
-  float mx = -INFINITY;
-  while (mask) {
-    const int e = __ffs(mask) - 1;
-    mask &= mask - 1;
-    const uint32_t b = vec_elem<Bits>(w, e);
-    mx = fmaxf(mx, Elem<Bits>::to_float(b));
-    if (pos < kCandCap) cand[pos] = ((unsigned long long)b << 32) | (uint32_t)(base + e);
-    ++pos;
-  }
-  return mx;
-}
-
-// The streaming step on one 16-byte vector: elements above the candidate
-// threshold are replaced by -inf (their bit set in the returned mask), the
-// exponentials of the others are added to the two packed accumulators.
-template <typename Bits>
-__device__ __forceinline__ uint32_t stream_vec(uint4 w, float thr, float2 c2, float2 s2,
-                                               float2 &acc_a, float2 &acc_b) {
-  uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-  uint32_t mask = 0u;
+__device__ __forceinline__ Threshold<Bits> make_threshold(float thr) {
+  Threshold<Bits> t;
   if constexpr (sizeof(Bits) == 2) {
-    // thr rounded down to bf16: x > thr implies x > thr_b, so the candidate
-    // set can only grow; sum and append use this same test.
-    const __nv_bfloat162 t2 = __bfloat162bfloat162(__float2bfloat16_rd(thr));
+    const __nv_bfloat16 h = __float2bfloat16_rd(thr);
+    const __nv_bfloat162 h2 = __bfloat162bfloat162(h);
+    t.pair = *reinterpret_cast<const uint32_t *>(&h2);
+    t.value = __bfloat162float(h);
+  } else {
+    t.pair = __float_as_uint(thr);
+    t.value = thr;
+  }
+  return t;
+}
+
+// The streaming step on one 16-byte vector: elements above the threshold
+// are replaced by -inf, the exponentials of the others are added to the two
+// packed accumulators.  Returns nonzero iff the vector holds a candidate.
+template <typename Bits>
+__device__ __forceinline__ uint32_t stream_vec(uint4 w, const Threshold<Bits> &t, float2 c2,
+                                               float2 s2, float2 &acc_a, float2 &acc_b) {
+  uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+  uint32_t any = 0u;
+  if constexpr (sizeof(Bits) == 2) {
+    const __nv_bfloat162 t2 = *reinterpret_cast<const __nv_bfloat162 *>(&t.pair);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const uint32_t m = __hgt2_mask(*reinterpret_cast<const __nv_bfloat162 *>(&ws[q]), t2);
       ws[q] = (ws[q] & ~m) | (0xFF80FF80u & m);
-      mask |= ((m & 1u) | ((m >> 15) & 2u)) << (2 * q);
+      any |= m;
     }
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const float2 x = make_float2(__uint_as_float(ws[q] << 16), __uint_as_float(ws[q] & 0xFFFF0000u));
-      const float2 t = ffma2(x, c2, s2);
-      const float2 e = make_float2(fast_exp2(t.x), fast_exp2(t.y));
-      if (q & 1) acc_b = fadd2(acc_b, e);
-      else acc_a = fadd2(acc_a, e);
+      const float2 u = __ffma2_rn(x, c2, s2);
+      const float2 e = make_float2(fast_exp2(u.x), fast_exp2(u.y));
+      if (q & 1) acc_b = __fadd2_rn(acc_b, e);
+      else acc_a = __fadd2_rn(acc_a, e);
     }
   } else {
 #pragma unroll
     for (int q = 0; q < 4; ++q)
-      if (__uint_as_float(ws[q]) > thr) {
-        mask |= 1u << q;
+      if (__uint_as_float(ws[q]) > t.value) {
+        any = 1u;
         ws[q] = 0xFF800000u;
       }
 #pragma unroll
     for (int q = 0; q < 4; q += 2) {
       const float2 x = make_float2(__uint_as_float(ws[q]), __uint_as_float(ws[q + 1]));
-      const float2 t = ffma2(x, c2, s2);
-      const float2 e = make_float2(fast_exp2(t.x), fast_exp2(t.y));
-      if (q & 2) acc_b = fadd2(acc_b, e);
-      else acc_a = fadd2(acc_a, e);
+      const float2 u = __ffma2_rn(x, c2, s2);
+      const float2 e = make_float2(fast_exp2(u.x), fast_exp2(u.y));
+      if (q & 2) acc_b = __fadd2_rn(acc_b, e);
+      else acc_a = __fadd2_rn(acc_a, e);
     }
   }
-  return mask;
+  return any;
 }
 
+// Appends each lane's candidates (bit q of `mask`: element q of vector `w`,
+// vector index `j` in the row) to the row's list in global memory: one
+// shared-memory atomic per warp.  Every lane of the warp takes part.
 template <typename Bits>
-__device__ __forceinline__ float candidate_threshold_value(float thr) {
-  if constexpr (sizeof(Bits) == 2)
-    return __bfloat162float(__float2bfloat16_rd(thr));
-  else
-    return thr;
-}
-
-// ---------------------------------------------------------------------------
-// row_stats
-// ---------------------------------------------------------------------------
-template <typename Bits>
-__global__ void __launch_bounds__(kThreads, 2) row_stats_kernel(const FastArgs a) {
+__device__ __forceinline__ void append_candidates(uint32_t mask, const uint4 &w, int32_t j,
+                                                  int *s_cand, uint64_t *dst) {
   constexpr int VEC = Elem<Bits>::kVec;
-  constexpr int CH = kChunkBytes / (int)sizeof(Bits);  // elements per chunk
-  constexpr int KEYB = Elem<Bits>::kKeyBits;
-  extern __shared__ __align__(128) unsigned char smem[];
-  Bits *stages = reinterpret_cast<Bits *>(smem);
-  unsigned long long *cand = reinterpret_cast<unsigned long long *>(smem + kStages * kChunkBytes);
-  __shared__ __align__(8) uint64_t mbar[kStages];
-  __shared__ float s_f[kWarps];
+  const int lane = threadIdx.x & 31;
+  const int c = __popc(mask);
+  int incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+  if (total == 0) return;
+  int base = 0;
+  if (lane == 31) base = atomicAdd(s_cand, total);
+  int pos = __shfl_sync(0xFFFFFFFFu, base, 31) + incl - c;
+  while (mask) {
+    const int q = __ffs(mask) - 1;
+    mask &= mask - 1;
+    if (pos < kCandCap)
+      dst[pos] = ((uint64_t)vec_elem<Bits>(w, q) << 32) | (uint32_t)(j * VEC + q);
+    ++pos;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// row_scan
+// ---------------------------------------------------------------------------
+// Each CTA walks its rows (item = blockIdx.x + t * gridDim.x) as one stream
+// of batches g = t * nb + k; the loads of batch g + 1 (the next row's first
+// batch at a row's end) are in flight while batch g is consumed.
+template <typename Bits>
+__global__ void __launch_bounds__(kThreads, 2) row_scan_kernel(const __grid_constant__ FastArgs a) {
+  constexpr int VEC = Elem<Bits>::kVec;
+  constexpr int U = kInFlight;
+  constexpr int BATCH = U * kThreads;  // vectors per batch
+  __shared__ uint4 fring[kRing];       // parked vectors
+  __shared__ int32_t fidx[kRing];      // their vector index in the row
   __shared__ float s_wmax[2][kWarps];
-  __shared__ double s_d[kWarps];
-  __shared__ unsigned long long s_u[kWarps];
-  __shared__ unsigned long long s_bs[2][kWarps];
-  __shared__ int s_cand, s_nuc;
-  __shared__ int s_keep[kWarps];
+  __shared__ float s_red[kWarps];
+  __shared__ double s_zsum[kWarps];
+  __shared__ unsigned long long s_dsum[kWarps];
+  __shared__ int s_fcount[3];          // parked vectors of batch g (counter g % 3)
+  __shared__ int s_cand;               // candidates of the current row
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int32_t V = a.s.V;
-  const int64_t R = a.rows;
-  const int32_t nck = (V + CH - 1) / CH;
-  const int64_t my_rows = ((int64_t)blockIdx.x < R) ? (R - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-  const int64_t total = my_rows * nck;
+  const int32_t nvec = V / VEC;  // whole 16-byte vectors per row
+  const int32_t tail = V - nvec * VEC;
+  const int32_t nb = nvec > 0 ? (nvec + BATCH - 1) / BATCH : 1;
+  const int64_t R = a.pass == 1 ? a.rows : (int64_t)a.counters[2];
+  if ((int64_t)blockIdx.x >= R) return;
+  const int64_t total = ((R - 1 - (int64_t)blockIdx.x) / gridDim.x + 1) * nb;
   const float coef = a.coef;
   const float2 c2 = make_float2(coef, coef);
-  const int max_narrowings = (int)((kWindowLog2 - kWindowMinLog2) / kWindowStepLog2);
-  // Without top-p the "window" is empty: candidates are only the elements
-  // above the running reference (a few per row), summed exactly at the end.
-  const float win0 = a.use_top_p ? a.win_off : 0.f;
+  uint4 neg;
+  neg.x = neg.y = neg.z = neg.w = sizeof(Bits) == 2 ? 0xFF80FF80u : 0xFF800000u;
+  if (tid < 3) s_fcount[tid] = 0;
+  if (tid == 0) s_cand = 0;
 
-  if (blockIdx.x == 0 && tid < 2) a.counters[tid] = 0;  // work lists of this call
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&mbar[s], 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-
-  auto issue = [&](int64_t g) {  // thread 0: start the copy of chunk g
-    if (g >= total) return;
-    const int64_t r = blockIdx.x + (g / nck) * (int64_t)gridDim.x;
-    const int32_t c0 = (int32_t)(g % nck) * CH;
-    const int32_t len = min(CH, V - c0);
-    const uint32_t bytes = (uint32_t)(len / VEC) * VEC * (uint32_t)sizeof(Bits);
-    uint64_t *bar = &mbar[g % kStages];
-    mbar_arrive_expect_tx(bar, bytes);
-    if (bytes) bulk_load(stages + (g % kStages) * CH, row_ptr<Bits>(a, r) + c0, bytes, bar);
+  // row of local index t, and its window (logit units)
+  auto row_entry = [&](int64_t t, float &off) -> int64_t {
+    const int64_t item = (int64_t)blockIdx.x + t * gridDim.x;
+    if (a.pass == 1) {
+      off = a.use_top_p ? a.win_narrow : 0.f;
+      return item;
+    }
+    const int32_t e = a.wide_rows[item];
+    off = !a.use_top_p ? 0.f : (e & kWideBit) ? a.win_wide : a.win_narrow;
+    return (int64_t)(e & ~kWideBit);
   };
-  if (tid == 0)
-    for (int64_t g = 0; g < kStages; ++g) issue(g);
+  auto load = [&](uint4(&buf)[U], int64_t g) {
+    if (g >= total) return;
+    const int64_t t = g / nb;
+    const int32_t k = (int32_t)(g - t * nb);
+    float unused;
+    const uint4 *rv = reinterpret_cast<const uint4 *>(row_ptr<Bits>(a, row_entry(t, unused)));
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int32_t j = k * BATCH + tid + u * kThreads;
+      buf[u] = j < nvec ? ldg_stream(rv + j) : neg;
+    }
+  };
 
-  // m_ref: CTA-uniform lower bound of the row maximum, never below any
-  // non-candidate seen so far.  z_t: this thread's sum of exp2((x - m_ref) *
-  // coef) over non-candidates (each <= 1, so nothing overflows); zd_t: mass
-  // of candidates dropped by a compaction, relative to zd_ref.  off: window
-  // width in logit units.
-  float z_t = 0.f, m_ref = -INFINITY, shift = -INFINITY;
-  float zd_t = 0.f, zd_ref = -INFINITY, off = win0;
-  int narrowed = 0;
-  bool timed_out = false;
-  for (int64_t g = 0; g < total; ++g) {
-    const int64_t r = blockIdx.x + (g / nck) * (int64_t)gridDim.x;
-    const int32_t k = (int32_t)(g % nck);
-    const int32_t c0 = k * CH, len = min(CH, V - c0), nv = len / VEC, tail = len - nv * VEC;
-    const Bits *row = row_ptr<Bits>(a, r);
-    const uint4 *sv = reinterpret_cast<const uint4 *>(stages + (g % kStages) * CH);
+  // per-row state (the same in every thread, except the partial sums)
+  int64_t r = 0;
+  const Bits *row = nullptr;
+  float off = 0.f, ref = -INFINITY, ref0 = -INFINITY, shift = -INFINITY, z_t = 0.f;
+  float2 acc_a = make_float2(0.f, 0.f), acc_b = make_float2(0.f, 0.f);
+  unsigned long long dsum = 0ull;
+  bool lost = false;
+  int fbase = 0, n_prev = 0;  // ring: first slot of the current batch, slots still held
+
+  auto consume = [&](const uint4(&buf)[U], int64_t g) {
+    const int64_t t = g / nb;
+    const int32_t k = (int32_t)(g - t * nb);
     if (k == 0) {
-      z_t = 0.f;
-      zd_t = 0.f;
-      zd_ref = -INFINITY;
-      off = win0;
-      narrowed = 0;
-      if (tid == 0) s_cand = 0;
-      // First reference: the maximum over every chunk of this row already in
-      // the ring (up to kStages * 16 KB of the row).
-      const int32_t in_ring = min(kStages, nck);
-      const int32_t ahead = (total - g < (int64_t)in_ring) ? (int32_t)(total - g) : in_ring;
+      // ---- start of a row: the first reference is the first batch's maximum
+      r = row_entry(t, off);
+      row = row_ptr<Bits>(a, r);
       float mx = -INFINITY;
-      for (int32_t h = 0; h < ahead; ++h) {
-        const int64_t gh = g + h;
-        timed_out |= !mbar_wait_bounded(&mbar[gh % kStages], (uint32_t)((gh / kStages) & 1));
-        const int32_t ch0 = h * CH, chl = min(CH, V - ch0), chv = chl / VEC;
-        const uint4 *hv = reinterpret_cast<const uint4 *>(stages + (gh % kStages) * CH);
-        for (int32_t j = tid; j < chv; j += kThreads) {
-          const float vm = raw_vec_max<Bits>(hv[j]);
-          if (vm == vm) mx = fmaxf(mx, vm);
-        }
-        const int32_t cht = chl - chv * VEC;
-        if (tid < cht) {
-          const float x = Elem<Bits>::to_float(row[ch0 + chv * VEC + tid]);
-          if (x == x) mx = fmaxf(mx, x);
-        }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const float vm = raw_vec_max<Bits>(buf[u]);
+        if (vm == vm) mx = fmaxf(mx, vm);
       }
-      m_ref = block_max_all(mx, s_f);
-      if (!(m_ref < INFINITY)) m_ref = -INFINITY;  // +inf: everything above -inf is a candidate
-      shift = (m_ref == -INFINITY) ? -INFINITY : -m_ref * coef;
+      if (tid < tail) {
+        const float x = Elem<Bits>::to_float(row[(int64_t)nvec * VEC + tid]);
+        if (x == x) mx = fmaxf(mx, x);
+      }
+      ref = block_max_all<kWarps>(mx, s_red);
+      // second pass: the row maximum is known from the first
+      if (a.pass == 2) ref = fmaxf(ref, a.rowrec[r].ref);
+      if (!(ref < INFINITY)) ref = -INFINITY;  // +inf: every finite element is a candidate
+      ref0 = ref;
+      shift = (ref == -INFINITY) ? -INFINITY : -ref * coef;
+      z_t = 0.f;
+      acc_a = acc_b = make_float2(0.f, 0.f);
+      dsum = 0ull;
+      lost = false;
     }
-    timed_out |= !mbar_wait_bounded(&mbar[g % kStages], (uint32_t)((g / kStages) & 1));
-    const float thr = m_ref - off;  // candidate iff x > thr (as rounded for the test)
+    // ---- stream the batch; park the vectors that hold a candidate
+    const Threshold<Bits> th = make_threshold<Bits>(ref - off);
     const float2 s2 = make_float2(shift, shift);
-    float2 acc_a = make_float2(0.f, 0.f), acc_b = make_float2(0.f, 0.f);
+    const int cap = kRing - n_prev;
+    int *cnt = &s_fcount[g % 3];
     float cmx = -INFINITY;
-    uint4 neg;
-    neg.x = neg.y = neg.z = neg.w = sizeof(Bits) == 2 ? 0xFF80FF80u : 0xFF800000u;
-    // Two vectors per lane per iteration; every lane of a warp runs the same
-    // number of iterations (the ballot below needs the whole warp).
-    for (int32_t j0 = warp * 32; j0 < nv; j0 += 2 * kThreads) {
-      const int32_t ja = j0 + lane, jb = j0 + kThreads + lane;
-      const uint4 wa = ja < nv ? sv[ja] : neg;
-      const uint4 wb = jb < nv ? sv[jb] : neg;
-      const uint32_t ma = stream_vec<Bits>(wa, thr, c2, s2, acc_a, acc_b);
-      const uint32_t mb = stream_vec<Bits>(wb, thr, c2, s2, acc_a, acc_b);
-      if (__ballot_sync(0xFFFFFFFFu, (ma | mb) != 0u)) {
-        cmx = fmaxf(cmx, append_candidates<Bits>(wa, ma, c0 + ja * VEC, &s_cand, cand));
-        cmx = fmaxf(cmx, append_candidates<Bits>(wb, mb, c0 + jb * VEC, &s_cand, cand));
-      }
-    }
-    z_t += (acc_a.x + acc_a.y) + (acc_b.x + acc_b.y);
-    if (tid < tail) {  // ragged end of the row (fewer than one vector)
-      const uint32_t b = row[c0 + nv * VEC + tid];
-      const float x = Elem<Bits>::to_float(b);
-      if (x > candidate_threshold_value<Bits>(thr)) {
-        const int slot = atomicAdd(&s_cand, 1);
-        if (slot < kCandCap)
-          cand[slot] = ((unsigned long long)b << 32) | (uint32_t)(c0 + nv * VEC + tid);
-        cmx = fmaxf(cmx, x);
-      } else {
-        z_t += fast_exp2(fmaf(x, coef, shift));
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint32_t h = stream_vec<Bits>(buf[u], th, c2, s2, acc_a, acc_b);
+      const unsigned flagged = __ballot_sync(0xFFFFFFFFu, h != 0u);
+      if (flagged) {
+        const int leader = __ffs(flagged) - 1;
+        int first = 0;
+        if (lane == leader) first = atomicAdd(cnt, __popc(flagged));
+        first = __shfl_sync(0xFFFFFFFFu, first, leader);
+        if (h) {
+          const int idx = first + __popc(flagged & ((1u << lane) - 1u));
+          if (idx < cap) {
+            const int slot = (fbase + idx) & (kRing - 1);
+            fring[slot] = buf[u];
+            fidx[slot] = k * BATCH + tid + u * kThreads;
+          }
+          cmx = fmaxf(cmx, raw_vec_max<Bits>(buf[u]));
+        }
       }
     }
     cmx = warp_max(cmx);
     if (lane == 0) s_wmax[g & 1][warp] = cmx;
-    __syncthreads();  // stage consumed, candidate maxima and count published
-    float m_new = m_ref;
+    __syncthreads();
+    const int n_k = *cnt;
+    if (tid == 0) s_fcount[(g + 2) % 3] = 0;  // batch g - 1's counter: read by all, next used by g + 2
+    // ---- raise the reference (same value in every thread)
+    float nr = ref;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) m_new = fmaxf(m_new, s_wmax[g & 1][w]);
-    if (!(m_new < INFINITY)) m_new = m_ref;  // a +inf candidate: the row is flagged later
-    if (tid == 0) issue(g + kStages);
-    if (m_new > m_ref) {
-      z_t = (m_ref == -INFINITY) ? 0.f : z_t * fast_exp2((m_ref - m_new) * coef);
-      shift = -m_new * coef;
+    for (int w = 0; w < kWarps; ++w) nr = fmaxf(nr, s_wmax[g & 1][w]);
+    if (!(nr < INFINITY)) nr = ref;
+    if (nr > ref) {
+      const float f = (ref == -INFINITY) ? 0.f : fast_exp2((ref - nr) * coef);
+      z_t = (z_t + (acc_a.x + acc_a.y) + (acc_b.x + acc_b.y)) * f;
+      acc_a = acc_b = make_float2(0.f, 0.f);
+      ref = nr;
+      shift = -nr * coef;
     }
-    if (s_cand > kCandCap / 2 &&
-        (m_new > m_ref || (a.use_top_p && narrowed < max_narrowings))) {
-      // Keep the buffer at most half full: drop what fell below the window
-      // (the maximum may have risen), narrowing the window if needed.
-      compact_candidates<Bits>(cand, &s_cand, s_keep, m_new - off, m_new, coef, zd_t, zd_ref);
-      while (a.use_top_p && s_cand > kCandCap / 2 && s_cand <= kCandCap &&
-             narrowed < max_narrowings) {
-        ++narrowed;
-        off = (kWindowLog2 - kWindowStepLog2 * (float)narrowed) / coef;
-        compact_candidates<Bits>(cand, &s_cand, s_keep, m_new - off, m_new, coef, zd_t, zd_ref);
+    // ---- split the parked vectors: candidates above the raised threshold
+    // go to the row's list, the rest of what the batch masked is dropped into
+    // the fixed-point sum (relative to ref0, so the sum is order-free)
+    const int n_in = min(n_k, cap);
+    if (n_k > cap) lost = true;
+    const float th2 = make_threshold<Bits>(ref - off).value;
+    const bool drop = ref0 > -INFINITY && (ref - off - ref0) * coef <= kDropGuardLog2;
+    const float shift0 = -ref0 * coef;
+    uint64_t *dst = a.cand + r * (int64_t)kCandCap;
+    for (int b = warp * 32; b < n_in; b += kThreads) {
+      const int e = b + lane;
+      uint32_t cmask = 0u;
+      uint4 w = neg;
+      int32_t j = 0;
+      if (e < n_in) {
+        const int slot = (fbase + e) & (kRing - 1);
+        w = fring[slot];
+        j = fidx[slot];
+#pragma unroll
+        for (int q = 0; q < VEC; ++q) {
+          const float x = Elem<Bits>::to_float(vec_elem<Bits>(w, q));
+          if (x > th.value) {
+            if (!drop || x > th2) cmask |= 1u << q;
+            else dsum += __float2ull_rn(fast_exp2(fmaf(x, coef, shift0)) * kFixF);
+          }
+        }
       }
+      append_candidates<Bits>(cmask, w, j, &s_cand, dst);
     }
-    m_ref = m_new;
-    if (k != nck - 1) continue;
+    fbase = (fbase + n_in) & (kRing - 1);
+    n_prev = n_in;
 
-    // ---- end of row r ---------------------------------------------------
-    // Every element is either a non-candidate (<= m_ref) or a candidate, so
-    // the row maximum is the larger of m_ref and the largest candidate.
-    float cm = -INFINITY;
-    for (int j = tid; j < min(s_cand, kCandCap); j += kThreads)
-      cm = fmaxf(cm, Elem<Bits>::to_float((uint32_t)(cand[j] >> 32)));
-    const float M = fmaxf(m_ref, block_max_all(cm, s_f));
-    int32_t flags = 0;
-    const bool overflow = s_cand > kCandCap;
-    if (a.use_top_p) {
-      // Candidates below the final window leave the buffer (their mass is
-      // small: fp32 relative to M); the rest are the only elements that can
-      // be at or above the top-p threshold.
-      compact_candidates<Bits>(cand, &s_cand, s_keep, M - off, M, coef, zd_t, zd_ref);
-    }
-    float zl = (m_ref == -INFINITY || !(M < INFINITY)) ? 0.f : z_t * fast_exp2((m_ref - M) * coef);
-    if (z_t != z_t) zl = z_t;  // a NaN logit poisons the sum (flagged below)
-    if (zd_ref != -INFINITY) zl += zd_t * fast_exp2((zd_ref - M) * coef);
-    const double z_light = block_sum_all((double)zl, s_d);
-    const int n_in = min(s_cand, kCandCap);
-    double Z = z_light, zp = z_light;
-    uint32_t tau_bits = Elem<Bits>::kNegInf;
-    int n_nuc = 0;
-    if (!a.use_top_p) {
-      // the few elements that rose above the running reference
-      unsigned long long zc = 0ull;
-      for (int j = tid; j < n_in; j += kThreads)
-        zc += __double2ull_rn(
-            exact_exp2d(Elem<Bits>::to_float((uint32_t)(cand[j] >> 32)), M, a.coef64) * kFixD);
-      Z = z_light + (double)block_sum_all(zc, s_u) / kFixD;
-      zp = Z;
-      if (overflow) flags |= kRowNeedGeneral;
-    } else if (overflow || n_in > kCandCap / 2 || !(M > -INFINITY)) {
-      flags |= kRowNeedGeneral;
-    } else {
-      // Exact masses (2^-40 fixed point, order-independent sums) into the
-      // idle half of the buffer; entries rewritten as (key << 32 | index).
-      unsigned long long *cmass = cand + kCandCap / 2;
-      unsigned long long zin = 0ull;
-      for (int j = tid; j < n_in; j += kThreads) {
-        const unsigned long long e = cand[j];
-        const uint32_t b = (uint32_t)(e >> 32);
-        const unsigned long long fx =
-            __double2ull_rn(exact_exp2d(Elem<Bits>::to_float(b), M, a.coef64) * kFixD);
-        cmass[j] = fx;
-        zin += fx;
-        cand[j] = ((unsigned long long)Elem<Bits>::key(b) << 32) | (e & 0xFFFFFFFFull);
+    if (k == nb - 1) {
+      // ---- end of the row: ragged end, sums, row record
+      if (tid < tail) {
+        const uint32_t bits = row[(int64_t)nvec * VEC + tid];
+        const float x = Elem<Bits>::to_float(bits);
+        if (x > th2) {
+          const int slot = atomicAdd(&s_cand, 1);
+          if (slot < kCandCap) dst[slot] = ((uint64_t)bits << 32) | (uint32_t)(nvec * VEC + tid);
+        } else {
+          z_t += fast_exp2(fmaf(x, coef, shift));
+        }
       }
-      zin = block_sum_all(zin, s_u);  // (its barriers also publish cmass / cand)
-      Z = z_light + (double)zin / kFixD;
-      zp = Z;
-      const unsigned long long target = (unsigned long long)ceil((double)a.s.top_p * Z * kFixD);
-      if (zin < target) {
-        flags |= kRowNeedGeneral;  // the window holds less than top_p of the mass
-      } else {
-        // Top-p threshold: the largest key t whose suffix mass S(t) reaches
-        // top_p of the total; binary search, one barrier per step.
-        uint64_t lo = 0, hi = 1ull << KEYB;
-        unsigned long long s_lo = zin;
-        int par = 0;
-        while (hi - lo > 1) {
-          const uint64_t mid = (lo + hi) >> 1;
-          unsigned long long part = 0ull;
-          for (int j = tid; j < n_in; j += kThreads)
-            if ((cand[j] >> 32) >= mid) part += cmass[j];
-          part = warp_sum_any(part);
-          if (lane == 0) s_bs[par][warp] = part;
-          __syncthreads();
-          unsigned long long S = 0ull;
+      z_t += (acc_a.x + acc_a.y) + (acc_b.x + acc_b.y);
+      const double zs = warp_sum_any((double)z_t);
+      const unsigned long long ds = warp_sum_any(dsum);
+      if (lane == 0) {
+        s_zsum[warp] = zs;
+        s_dsum[warp] = ds;
+      }
+      __syncthreads();
+      if (tid == 0) {
+        double zt = 0.0;
+        unsigned long long zd = 0ull;
 #pragma unroll
-          for (int w = 0; w < kWarps; ++w) S += s_bs[par][w];
-          par ^= 1;
-          if (S >= target) {
-            lo = mid;
-            s_lo = S;
-          } else {
-            hi = mid;
-          }
+        for (int w = 0; w < kWarps; ++w) {
+          zt += s_zsum[w];
+          zd += s_dsum[w];
         }
-        zp = (double)s_lo / kFixD;
-        tau_bits = key_to_bits<Bits>((uint32_t)lo);
-        // the nucleus: every candidate with key >= tau, as (bits << 32 | index)
-        if (tid == 0) s_nuc = 0;
-        __syncthreads();
-        uint64_t *nuc = a.nuc + r * (int64_t)kNucCap;
-        for (int j = tid; j < n_in; j += kThreads) {
-          const unsigned long long e = cand[j];
-          const uint32_t key = (uint32_t)(e >> 32);
-          if (key >= (uint32_t)lo) {
-            const int slot = atomicAdd(&s_nuc, 1);
-            if (slot < kNucCap)
-              nuc[slot] = ((unsigned long long)key_to_bits<Bits>(key) << 32) | (e & 0xFFFFFFFFull);
-          }
-        }
-        __syncthreads();
-        n_nuc = s_nuc;
-        if (n_nuc > kNucCap) flags |= kRowNeedGeneral;
+        RowRecord rec;
+        rec.ref = ref;
+        rec.ref0 = ref0;
+        rec.n_cand = s_cand;
+        rec.flags = lost ? kRowLost : 0;
+        rec.zt = zt;
+        rec.zd = zd;
+        a.rowrec[r] = rec;
+        s_cand = 0;  // (the next row appends only after its first barrier)
       }
     }
-    if (M == -INFINITY || !(fabsf(M * coef) < INFINITY) || !(Z < INFINITY)) flags |= kRowNonfinite;
-    if (tid == 0) {
-      RowRecord rec;
-      rec.m = M;
-      rec.flags = flags;
-      rec.z = Z;
-      rec.zp = zp;
-      rec.tau_bits = tau_bits;
-      rec.n_nuc = n_nuc;
-      a.rowrec[r] = rec;
-    }
-    __syncthreads();  // candidate buffer and counters free for the next row
+  };
+
+  uint4 b0[U], b1[U];
+  load(b0, 0);
+  for (int64_t g = 0; g < total; g += 2) {
+    load(b1, g + 1);
+    consume(b0, g);
+    if (g + 1 >= total) break;
+    load(b0, g + 2);
+    consume(b1, g + 1);
   }
-  // (NaN / +inf logits surface as non-finite row statistics, reported by
-  // unit_decide; a bounded wait that gave up is reported here.)
-  const bool any_timeout = __syncthreads_or(timed_out);
-  if (tid == 0 && any_timeout && a.s.dev_status) atomicOr(a.s.dev_status, PSI_DEV_TIMEOUT);
 }
 
 // ---------------------------------------------------------------------------
-// unit_decide
+// unit
 // ---------------------------------------------------------------------------
+// Statistics of one finished row (the same in every thread).
+struct RowFinal {
+  float m;            // row maximum
+  double zp;          // normaliser after top-p (Z without top-p)
+  uint32_t tau_bits;  // top-p threshold (raw bits): keep x >= tau
+  int n_nuc;          // nucleus entries left in UnitShared::ms (when asked for)
+  int status;         // kFin* bits
+};
+constexpr int kFinOverflow = 1;   // candidates lost: rescan with the exact maximum
+constexpr int kFinCoverage = 2;   // the window holds less than top_p: rescan wider
+constexpr int kFinNonfinite = 4;  // NaN / +inf logit, or no finite logit
+
+struct UnitShared {
+  unsigned long long kc[kCandCap];  // (key << 32) | index; later the draw weights (double)
+  unsigned long long ms[kCandCap];  // 2^40 fixed-point masses; later the nucleus (index << 32 | bits)
+  double d[kUnitWarps];
+  unsigned long long u[kUnitWarps];
+  unsigned long long bs[2][kUnitWarps];
+  float f[kUnitWarps];
+  uint32_t k2[2][kUnitWarps];
+  int n;
+  int need;
+};
+
+// Row maximum, Z, top-p threshold tau and renormaliser Z' of row r from its
+// record and candidate list, and (want_nuc) p's nucleus: every candidate
+// with x >= tau.  The top-p threshold is the largest logit key t whose
+// suffix mass S(t) (all x with key >= t) reaches top_p * Z; only candidates
+// can be at or above it (the window holds at least top_p of the mass).
+template <typename Bits>
+__device__ __noinline__ RowFinal finish_row(const FastArgs &a, int64_t r, UnitShared *sh,
+                                            bool want_nuc) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  RowFinal out;
+  out.m = -INFINITY;
+  out.zp = 0.0;
+  out.tau_bits = Elem<Bits>::kNegInf;
+  out.n_nuc = 0;
+  out.status = 0;
+  const RowRecord rs = a.rowrec[r];
+  if (rs.n_cand > kCandCap || (rs.flags & kRowLost)) {
+    out.status = kFinOverflow;
+    return out;
+  }
+  const int n = rs.n_cand;
+  const uint64_t *src = a.cand + r * (int64_t)kCandCap;
+  float cm = -INFINITY;
+  uint32_t kmax = 0u, kmin_inv = 0u;
+  for (int j = tid; j < n; j += kUnitThreads) {
+    const uint64_t e = src[j];
+    const uint32_t b = (uint32_t)(e >> 32);
+    cm = fmaxf(cm, Elem<Bits>::to_float(b));
+    const uint32_t key = Elem<Bits>::key(b);
+    sh->kc[j] = ((unsigned long long)key << 32) | (e & 0xFFFFFFFFull);
+    kmax = max(kmax, key);
+    kmin_inv = max(kmin_inv, ~key);
+  }
+  cm = warp_max(cm);
+  kmax = warp_max_u32(kmax);
+  kmin_inv = warp_max_u32(kmin_inv);
+  __syncthreads();
+  if (lane == 0) {
+    sh->f[warp] = cm;
+    sh->k2[0][warp] = kmax;
+    sh->k2[1][warp] = kmin_inv;
+  }
+  __syncthreads();
+  float M = rs.ref;
+  uint32_t KMAX = 0u, KMIN_INV = 0u;
+#pragma unroll
+  for (int w = 0; w < kUnitWarps; ++w) {
+    M = fmaxf(M, sh->f[w]);
+    KMAX = max(KMAX, sh->k2[0][w]);
+    KMIN_INV = max(KMIN_INV, sh->k2[1][w]);
+  }
+  out.m = M;
+  if (!(M > -INFINITY) || !(fabsf(M * a.coef) < INFINITY) || rs.zt != rs.zt) {
+    out.status = kFinNonfinite;
+    return out;
+  }
+  // exact masses relative to M (2^40 fixed point: order-free sums)
+  unsigned long long zin = 0ull;
+  for (int j = tid; j < n; j += kUnitThreads) {
+    const uint32_t b = key_to_bits<Bits>((uint32_t)(sh->kc[j] >> 32));
+    const unsigned long long fx =
+        __double2ull_rn(exact_exp2d(Elem<Bits>::to_float(b), M, a.coef64) * kFixD);
+    sh->ms[j] = fx;
+    zin += fx;
+  }
+  zin = block_sum_all<unsigned long long, kUnitWarps>(zin, sh->u);
+  double Z = (double)zin / kFixD;
+  if (rs.ref > -INFINITY) Z += rs.zt * exp2(((double)rs.ref - (double)M) * a.coef64);
+  if (rs.zd) Z += (double)rs.zd / kFixD * exp2(((double)rs.ref0 - (double)M) * a.coef64);
+  out.zp = Z;
+  if (!(Z < INFINITY)) {
+    out.status = kFinNonfinite;
+    return out;
+  }
+  if (!a.use_top_p) return out;
+  const unsigned long long target = (unsigned long long)ceil((double)a.s.top_p * Z * kFixD);
+  if (zin < target) {
+    out.status = kFinCoverage;
+    return out;
+  }
+  // binary search over [kmin, kmax]: S(kmin) = zin reaches the target
+  uint64_t lo = ~KMIN_INV, hi = (uint64_t)KMAX + 1;
+  unsigned long long s_lo = zin;
+  int par = 0;
+  while (hi - lo > 1) {
+    const uint64_t mid = (lo + hi) >> 1;
+    unsigned long long part = 0ull;
+    for (int j = tid; j < n; j += kUnitThreads)
+      if ((sh->kc[j] >> 32) >= mid) part += sh->ms[j];
+    part = warp_sum_any(part);
+    if (lane == 0) sh->bs[par][warp] = part;
+    __syncthreads();
+    unsigned long long S = 0ull;
+#pragma unroll
+    for (int w = 0; w < kUnitWarps; ++w) S += sh->bs[par][w];
+    par ^= 1;
+    if (S >= target) {
+      lo = mid;
+      s_lo = S;
+    } else {
+      hi = mid;
+    }
+  }
+  out.zp = (double)s_lo / kFixD;
+  out.tau_bits = key_to_bits<Bits>((uint32_t)lo);
+  if (want_nuc) {
+    __syncthreads();  // every read of the masses is done
+    if (tid == 0) sh->n = 0;
+    __syncthreads();
+    for (int j = tid; j < n; j += kUnitThreads) {
+      const unsigned long long e = sh->kc[j];
+      const uint32_t key = (uint32_t)(e >> 32);
+      if (key >= (uint32_t)lo) {
+        const int slot = atomicAdd(&sh->n, 1);
+        sh->ms[slot] = ((e & 0xFFFFFFFFull) << 32) | key_to_bits<Bits>(key);
+      }
+    }
+    __syncthreads();
+    out.n_nuc = sh->n;
+  }
+  return out;
+}
 
 // In-place ascending bitonic sort of n (a power of two) 64-bit keys.
 __device__ void bitonic_sort(unsigned long long *v, int n) {
@@ -581,10 +624,10 @@ __device__ void bitonic_sort(unsigned long long *v, int n) {
         const int p = t ^ j;
         if (p > t) {
           const bool up = (t & k) == 0;
-          const unsigned long long a = v[t], b = v[p];
-          if ((a > b) == up) {
-            v[t] = b;
-            v[p] = a;
+          const unsigned long long x = v[t], y = v[p];
+          if ((x > y) == up) {
+            v[t] = y;
+            v[p] = x;
           }
         }
       }
@@ -602,7 +645,6 @@ __device__ void block_scan(double *w, int n, double *scratch) {
     run += w[j];
     w[j] = run;
   }
-  // exclusive scan of the per-thread totals
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   double incl = run;
 #pragma unroll
@@ -610,6 +652,7 @@ __device__ void block_scan(double *w, int n, double *scratch) {
     const double v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
     if (lane >= o) incl += v;
   }
+  __syncthreads();
   if (lane == 31) scratch[warp] = incl;
   __syncthreads();
   double off = incl - run;
@@ -619,129 +662,144 @@ __device__ void block_scan(double *w, int n, double *scratch) {
 }
 
 template <typename Bits>
-__global__ void __launch_bounds__(kUnitThreads) unit_decide_kernel(const FastArgs a) {
-  __shared__ unsigned long long ent[kNucCap];
-  __shared__ double wv[kNucCap];
-  __shared__ double scratch[kUnitThreads / 32];
-  __shared__ int s_need;
+__global__ void __launch_bounds__(kUnitThreads) unit_kernel(const __grid_constant__ FastArgs a) {
+  __shared__ UnitShared sh;
   const int tid = threadIdx.x;
   const SampledArgs &s = a.s;
   const int32_t B = s.B, N = s.N, V = s.V;
-  const int64_t unit = blockIdx.x;
-  const int32_t n = (int32_t)(unit / (B + 1)), i = (int32_t)(unit % (B + 1));
-  const bool has_q = i < B;
-  const int64_t rp_idx = unit;
-  const int64_t rq_idx = (int64_t)N * (B + 1) + (int64_t)n * B + i;
-  const RowRecord rp = a.rowrec[rp_idx];
-  RowRecord rq = rp;
-  if (has_q) rq = a.rowrec[rq_idx];
-  const bool general = ((rp.flags | (has_q ? rq.flags : 0)) & kRowNeedGeneral) != 0;
-  if (general) {  // the cluster kernel verifies this unit (records included)
-    if (tid == 0) a.list_a[atomicAdd(&a.counters[0], 1)] = (int32_t)unit;
-    return;
-  }
-  const uint64_t seq = s.seq_ids ? s.seq_ids[n] : (uint64_t)n;
-  const Bits *row_p = static_cast<const Bits *>(s.ar) + unit * s.ar_stride;
-  const Bits *row_q = has_q ? static_cast<const Bits *>(s.draft) + ((int64_t)n * B + i) * s.draft_stride
-                            : nullptr;
-  const float tau_p = Elem<Bits>::to_float(rp.tau_bits);
-  const float tau_q = Elem<Bits>::to_float(rq.tau_bits);
-
-  if (tid == 0) {
-    int need = 1;
-    if (has_q) {
-      const int32_t x = s.ids[(int64_t)n * B + i];
-      double p = 0.0, q = 0.0;
-      const bool valid = x >= 0 && x < V;
-      if (valid) {
-        const float xp = Elem<Bits>::to_float(row_p[x]);
-        const float xq = Elem<Bits>::to_float(row_q[x]);
-        if (xp >= tau_p && rp.zp > 0.0) p = exact_exp2d(xp, rp.m, a.coef64) / rp.zp;
-        if (xq >= tau_q && rq.zp > 0.0) q = exact_exp2d(xq, rq.m, a.coef64) / rq.zp;
+  const int64_t n_items = a.pass == 1 ? (int64_t)N * (B + 1) : (int64_t)a.counters[3];
+  for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const int64_t unit = a.pass == 1 ? item : (int64_t)a.wide_units[item];
+    const int32_t n = (int32_t)(unit / (B + 1)), i = (int32_t)(unit % (B + 1));
+    const bool has_q = i < B;
+    const int64_t rp_idx = unit;
+    const int64_t rq_idx = (int64_t)N * (B + 1) + (int64_t)n * B + i;
+    RowFinal fq;
+    fq.m = -INFINITY;
+    fq.zp = 0.0;
+    fq.tau_bits = 0u;
+    fq.status = 0;
+    if (has_q) fq = finish_row<Bits>(a, rq_idx, &sh, false);
+    const RowFinal fp = finish_row<Bits>(a, rp_idx, &sh, true);
+    const int fail_q = fq.status & (kFinOverflow | kFinCoverage);
+    const int fail_p = fp.status & (kFinOverflow | kFinCoverage);
+    if (fail_q || fail_p) {
+      if (tid == 0) {
+        if (a.pass == 1) {  // rescan the failed rows, then finish the unit again
+          if (fail_q)
+            a.wide_rows[atomicAdd(&a.counters[2], 1)] =
+                (int32_t)rq_idx | ((fail_q & kFinCoverage) ? kWideBit : 0);
+          if (fail_p)
+            a.wide_rows[atomicAdd(&a.counters[2], 1)] =
+                (int32_t)rp_idx | ((fail_p & kFinCoverage) ? kWideBit : 0);
+          a.wide_units[atomicAdd(&a.counters[3], 1)] = (int32_t)unit;
+        } else {  // the general path verifies this unit (records included)
+          a.list_a[atomicAdd(&a.counters[0], 1)] = (int32_t)unit;
+        }
       }
-      const double u = (double)uniform24(s.seed, seq, s.step, (uint64_t)i, PSI_PURPOSE_ACCEPT);
-      const int accept = (u * q < p) ? 1 : 0;
-      need = !accept;
-      if (s.out_p) s.out_p[(int64_t)n * B + i] = (float)p;
-      if (s.out_q) s.out_q[(int64_t)n * B + i] = (float)q;
-      a.rec[unit].accept = accept;
-      if (accept) a.rec[unit].token = -1;
-      if (!valid && s.dev_status) atomicOr(s.dev_status, PSI_DEV_BAD_TOKEN_ID);
-    } else {
-      a.rec[unit].accept = 1;
+      continue;
     }
-    if (((rp.flags | (has_q ? rq.flags : 0)) & kRowNonfinite) && s.dev_status)
-      atomicOr(s.dev_status, PSI_DEV_NONFINITE);
-    s_need = need;
-  }
-  __syncthreads();
-  if (!s_need) return;
-  if (!a.use_top_p) {  // the draw needs whole rows: decided after the emit step
-    if (tid == 0) a.rec[unit].token = -2;
-    return;
-  }
+    const uint64_t seq = s.seq_ids ? s.seq_ids[n] : (uint64_t)n;
+    const Bits *row_p = static_cast<const Bits *>(s.ar) + unit * s.ar_stride;
+    const Bits *row_q = has_q ? static_cast<const Bits *>(s.draft) + ((int64_t)n * B + i) * s.draft_stride
+                              : nullptr;
+    const float tau_p = Elem<Bits>::to_float(fp.tau_bits);
+    const float tau_q = Elem<Bits>::to_float(fq.tau_bits);
 
-  // ---- correction / bonus draw over p's nucleus ----------------------------
-  const int nn = rp.n_nuc;
-  int np2 = 1;
-  while (np2 < nn) np2 <<= 1;
-  const uint64_t *nuc = a.nuc + rp_idx * (int64_t)kNucCap;
-  for (int t = tid; t < np2; t += kUnitThreads) {
-    if (t < nn) {
-      const uint64_t e = nuc[t];  // (bits << 32) | index  ->  (index << 32) | bits
-      ent[t] = ((e & 0xFFFFFFFFull) << 32) | (e >> 32);
-    } else {
-      ent[t] = ~0ull;
-    }
-  }
-  __syncthreads();
-  bitonic_sort(ent, np2);  // vocabulary order
-  for (int pass = 0; pass < 2; ++pass) {
-    const bool p_only = !has_q || pass == 1;
-    for (int t = tid; t < nn; t += kUnitThreads) {
-      const int32_t v = (int32_t)(ent[t] >> 32);
-      const float xp = Elem<Bits>::to_float((uint32_t)(ent[t] & 0xFFFFFFFFull));
-      double w = exact_exp2d(xp, rp.m, a.coef64) / rp.zp;
-      if (!p_only) {
-        const float xq = Elem<Bits>::to_float(row_q[v]);
-        const double q = (xq >= tau_q && rq.zp > 0.0) ? exact_exp2d(xq, rq.m, a.coef64) / rq.zp : 0.0;
-        w = w > q ? w - q : 0.0;
+    // ---- accept / reject the drafted token
+    if (tid == 0) {
+      int need = 1;
+      if (has_q) {
+        const int32_t x = s.ids[(int64_t)n * B + i];
+        double p = 0.0, q = 0.0;
+        const bool valid = x >= 0 && x < V;
+        if (valid) {
+          const float xp = Elem<Bits>::to_float(row_p[x]);
+          const float xq = Elem<Bits>::to_float(row_q[x]);
+          if (xp >= tau_p && fp.zp > 0.0) p = exact_exp2d(xp, fp.m, a.coef64) / fp.zp;
+          if (xq >= tau_q && fq.zp > 0.0) q = exact_exp2d(xq, fq.m, a.coef64) / fq.zp;
+        }
+        const double u = (double)uniform24(s.seed, seq, s.step, (uint64_t)i, PSI_PURPOSE_ACCEPT);
+        const int accept = (u * q < p) ? 1 : 0;
+        need = !accept;
+        if (s.out_p) s.out_p[(int64_t)n * B + i] = (float)p;
+        if (s.out_q) s.out_q[(int64_t)n * B + i] = (float)q;
+        a.rec[unit].accept = accept;
+        if (accept) a.rec[unit].token = -1;
+        if (!valid && s.dev_status) atomicOr(s.dev_status, PSI_DEV_BAD_TOKEN_ID);
+      } else {
+        a.rec[unit].accept = 1;
       }
-      wv[t] = w;
+      if (((fp.status | fq.status) & kFinNonfinite) && s.dev_status)
+        atomicOr(s.dev_status, PSI_DEV_NONFINITE);
+      sh.need = need;
     }
     __syncthreads();
-    block_scan(wv, nn, scratch);
-    const double W = nn > 0 ? wv[nn - 1] : 0.0;
-    if (W > 0.0 || p_only) {
-      if (tid == 0) {
-        int32_t token = 0;
-        if (W > 0.0) {
-          const double u2 = (double)uniform24(s.seed, seq, s.step, (uint64_t)i, PSI_PURPOSE_RESID);
-          const double t = u2 * W;
-          int lo = 0, hi = nn;  // first j with wv[j] > t
-          while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (wv[mid] > t) hi = mid;
-            else lo = mid + 1;
-          }
-          if (lo >= nn) {  // rounding: the last entry with positive weight
-            lo = nn - 1;
-            while (lo > 0 && !(wv[lo] > wv[lo - 1])) --lo;
-          }
-          token = (int32_t)(ent[lo] >> 32);
-        }
-        a.rec[unit].token = token;
-      }
-      break;
+    const int need = sh.need;
+    __syncthreads();  // (sh.need is rewritten by the next unit)
+    if (!need) continue;
+    if (!a.use_top_p) {  // the draw needs whole rows: decided after the emit step
+      if (tid == 0) a.rec[unit].token = -2;
+      continue;
     }
-    __syncthreads();  // residual vanished: draw from p itself
+
+    // ---- correction / bonus draw over p's nucleus, in vocabulary order
+    const int nn = fp.n_nuc;
+    int np2 = 1;
+    while (np2 < nn) np2 <<= 1;
+    unsigned long long *ent = sh.ms;
+    for (int t = nn + tid; t < np2; t += kUnitThreads) ent[t] = ~0ull;
+    __syncthreads();
+    bitonic_sort(ent, np2);
+    double *wv = reinterpret_cast<double *>(sh.kc);
+    for (int pass = 0; pass < 2; ++pass) {
+      const bool p_only = !has_q || pass == 1;
+      for (int t = tid; t < nn; t += kUnitThreads) {
+        const int32_t v = (int32_t)(ent[t] >> 32);
+        const float xp = Elem<Bits>::to_float((uint32_t)(ent[t] & 0xFFFFFFFFull));
+        double w = exact_exp2d(xp, fp.m, a.coef64) / fp.zp;
+        if (!p_only) {
+          const float xq = Elem<Bits>::to_float(row_q[v]);
+          const double q = (xq >= tau_q && fq.zp > 0.0) ? exact_exp2d(xq, fq.m, a.coef64) / fq.zp : 0.0;
+          w = w > q ? w - q : 0.0;
+        }
+        wv[t] = w;
+      }
+      __syncthreads();
+      block_scan(wv, nn, sh.d);
+      const double W = nn > 0 ? wv[nn - 1] : 0.0;
+      if (W > 0.0 || p_only) {
+        if (tid == 0) {
+          int32_t token = 0;
+          if (W > 0.0) {
+            const double u2 = (double)uniform24(s.seed, seq, s.step, (uint64_t)i, PSI_PURPOSE_RESID);
+            const double t = u2 * W;
+            int lo = 0, hi = nn;  // first j with wv[j] > t
+            while (lo < hi) {
+              const int mid = (lo + hi) >> 1;
+              if (wv[mid] > t) hi = mid;
+              else lo = mid + 1;
+            }
+            if (lo >= nn) {  // rounding: the last entry with positive weight
+              lo = nn - 1;
+              while (lo > 0 && !(wv[lo] > wv[lo - 1])) --lo;
+            }
+            token = (int32_t)(ent[lo] >> 32);
+          }
+          a.rec[unit].token = token;
+        }
+        break;
+      }
+      __syncthreads();  // residual vanished: draw from p itself
+    }
+    __syncthreads();  // shared buffers free for the next unit
   }
 }
 
 // ---------------------------------------------------------------------------
 // fast_emit: one thread per sequence.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) fast_emit_kernel(const FastArgs a) {
+__global__ void __launch_bounds__(128) fast_emit_kernel(const __grid_constant__ FastArgs a) {
   const int32_t n = blockIdx.x * blockDim.x + threadIdx.x;
   const SampledArgs &s = a.s;
   if (n >= s.N) return;
@@ -779,23 +837,28 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 template <typename Bits>
 cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, const KernelEvents &ev,
                               cudaStream_t stream) {
-  const size_t smem = (size_t)kStages * kChunkBytes + sizeof(unsigned long long) * kCandCap;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(row_stats_kernel<Bits>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
-  const int64_t grid1 = std::min<int64_t>(fa.rows, (int64_t)sm_count() * 2);
+  const int64_t units = (int64_t)fa.s.N * (fa.s.B + 1);
+  const int64_t persistent = (int64_t)sm_count() * 2;
+  const int64_t grid_scan = std::min<int64_t>(fa.rows, persistent);
   cudaError_t e;
+  // the work-list counters of this call start at zero
+  if ((e = cudaMemsetAsync(fa.counters, 0, 4 * sizeof(int32_t), stream)) != cudaSuccess) return e;
   if (ev.before && (e = cudaEventRecord(ev.before, stream)) != cudaSuccess) return e;
-  row_stats_kernel<Bits><<<(unsigned)grid1, kThreads, smem, stream>>>(fa);
+  row_scan_kernel<Bits><<<(unsigned)grid_scan, kThreads, 0, stream>>>(fa);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (ev.after && (e = cudaEventRecord(ev.after, stream)) != cudaSuccess) return e;
-  const int64_t units = (int64_t)fa.s.N * (fa.s.B + 1);
-  unit_decide_kernel<Bits><<<(unsigned)units, kUnitThreads, 0, stream>>>(fa);
+  unit_kernel<Bits><<<(unsigned)units, kUnitThreads, 0, stream>>>(fa);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  {
+    // second pass over the rows and units the first one could not settle
+    // (usually none: the CTAs find empty lists and exit)
+    FastArgs f2 = fa;
+    f2.pass = 2;
+    row_scan_kernel<Bits><<<(unsigned)grid_scan, kThreads, 0, stream>>>(f2);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    unit_kernel<Bits><<<(unsigned)std::min<int64_t>(units, persistent), kUnitThreads, 0, stream>>>(f2);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   const psi_dtype dt = sizeof(Bits) == 2 ? PSI_DTYPE_BF16 : PSI_DTYPE_F32;
   SampledArgs sa = fa.s;
   sa.records = fa.rec;
@@ -819,16 +882,25 @@ FastLayout fast_layout(int32_t N, int32_t B) {
   off = align256(off + sizeof(UnitRecord) * (size_t)units);
   L.rows_off = off;
   off = align256(off + sizeof(RowRecord) * (size_t)rows);
-  L.nuc_off = off;
-  off = align256(off + sizeof(uint64_t) * (size_t)rows * kNucCap);
+  L.cand_off = off;
+  off = align256(off + sizeof(uint64_t) * (size_t)rows * kCandCap);
   L.counters_off = off;
   off = align256(off + sizeof(int32_t) * 4);
   L.list_a_off = off;
   off = align256(off + sizeof(int32_t) * (size_t)units);
   L.list_b_off = off;
   off = align256(off + sizeof(int32_t) * (size_t)N);
+  L.wide_rows_off = off;
+  off = align256(off + sizeof(int32_t) * (size_t)rows);
+  L.wide_units_off = off;
+  off = align256(off + sizeof(int32_t) * (size_t)units);
   L.total = off;
   return L;
+}
+
+bool fast_path_fits(int32_t N, int32_t B) {
+  // row indices travel in 30 bits of a second-pass list entry
+  return (int64_t)N * (2 * (int64_t)B + 1) < (int64_t(1) << 30);
 }
 
 cudaError_t launch_sampled_fast(const SampledArgs &a, psi_dtype dtype, const SampledPlan &plan,
@@ -840,14 +912,23 @@ cudaError_t launch_sampled_fast(const SampledArgs &a, psi_dtype dtype, const Sam
   fa.rows = (int64_t)a.N * (a.B + 1) + (int64_t)a.N * a.B;
   fa.coef64 = 1.4426950408889634 / (double)a.temperature;
   fa.coef = (float)fa.coef64;
-  fa.win_off = kWindowLog2 / fa.coef;
+  // first-pass window: 13 log2 units for top_p <= 0.95, one more unit for
+  // every halving of the allowed tail mass beyond 5%, at most the wide window
+  double wlog2 = kWindowBaseLog2;
+  if (a.top_p < 1.0f && a.top_p > 0.95f) wlog2 += log2(0.05 / (1.0 - (double)a.top_p));
+  if (wlog2 > kWindowWideLog2) wlog2 = kWindowWideLog2;
+  fa.win_narrow = (float)(wlog2 / fa.coef64);
+  fa.win_wide = (float)(kWindowWideLog2 / fa.coef64);
   fa.use_top_p = a.top_p < 1.0f ? 1 : 0;
+  fa.pass = 1;
   fa.rec = reinterpret_cast<UnitRecord *>(ws + L.rec_off);
   fa.rowrec = reinterpret_cast<RowRecord *>(ws + L.rows_off);
-  fa.nuc = reinterpret_cast<uint64_t *>(ws + L.nuc_off);
+  fa.cand = reinterpret_cast<uint64_t *>(ws + L.cand_off);
   fa.counters = reinterpret_cast<int32_t *>(ws + L.counters_off);
   fa.list_a = reinterpret_cast<int32_t *>(ws + L.list_a_off);
   fa.list_b = reinterpret_cast<int32_t *>(ws + L.list_b_off);
+  fa.wide_rows = reinterpret_cast<int32_t *>(ws + L.wide_rows_off);
+  fa.wide_units = reinterpret_cast<int32_t *>(ws + L.wide_units_off);
   fa.s.records = fa.rec;
   if (dtype == PSI_DTYPE_BF16) return launch_fast_typed<uint16_t>(fa, plan, ev, stream);
   return launch_fast_typed<uint32_t>(fa, plan, ev, stream);

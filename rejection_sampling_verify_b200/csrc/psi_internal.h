@@ -88,23 +88,28 @@ cudaError_t launch_cluster_list(const SampledArgs &a, psi_dtype dtype, const Sam
                                 int max_clusters, cudaStream_t stream);
 
 // ---- streaming path (rows 16-byte aligned) ------------------------------------
-// Per logit row: statistics written by the row-statistics kernel.
+// Per logit row: what the row-scan kernel leaves for the unit kernel.  Every
+// element of the row is counted exactly once: in zt (at or below the
+// threshold of its batch), in zd (a candidate that fell below a later
+// threshold) or in the row's candidate list.
 struct RowRecord {
-  float m;            // row maximum
-  int32_t flags;      // kRowNeedGeneral: the general path must handle the unit
-  double z;           // sum over the row of exp((x - m) / T)
-  double zp;          // normaliser after top-p (z when top-p is off)
-  uint32_t tau_bits;  // top-p threshold logit (raw bits); keep x >= tau
-  int32_t n_nuc;      // nucleus entries stored for this row
+  float ref;        // final running reference: the row maximum, unless the row holds +inf
+  float ref0;       // reference of zd (the first reference of the row)
+  int32_t n_cand;   // candidates appended (more than the capacity: overflow)
+  int32_t flags;    // kRowLost: flagged vectors were dropped (ring overflow)
+  double zt;        // sum of exp2((x - ref) * log2(e) / T) over the non-candidates
+  uint64_t zd;      // 2^40 * sum of exp2((x - ref0) * log2(e) / T) over dropped candidates
 };
-constexpr int32_t kRowNeedGeneral = 1;
-constexpr int32_t kRowNonfinite = 2;
-constexpr int kNucCap = 1024;   // nucleus entries kept per row
+constexpr int32_t kRowLost = 1;
+constexpr int kCandCap = 2048;     // candidates kept per row (global workspace)
 
 struct FastLayout {  // workspace carve-up of the streaming path
-  size_t rec_off, rows_off, nuc_off, counters_off, list_a_off, list_b_off, total;
+  size_t rec_off, rows_off, cand_off, counters_off, list_a_off, list_b_off, wide_rows_off,
+      wide_units_off, total;
 };
 FastLayout fast_layout(int32_t N, int32_t B);
+// False when the streaming path's row indices would not fit its lists.
+bool fast_path_fits(int32_t N, int32_t B);
 
 cudaError_t launch_sampled_fast(const SampledArgs &a, psi_dtype dtype, const SampledPlan &plan,
                                 void *workspace, const KernelEvents &ev, cudaStream_t stream);

@@ -338,3 +338,34 @@ def test_host_argument_errors():
     with pytest.raises(psi.PsiError) as e:
         psi.verify_linear(big, big_d, torch.zeros(1, 1, dtype=torch.int32, device="cuda"), 1.0)
     assert e.value.status == psi.PSI_ERR_UNSUPPORTED
+
+
+def test_sampled_second_pass_rows():
+    """Rows whose top-p mass reaches below the narrow first-pass window (two
+    tokens on top, 1500 tokens 2^-13.5 below them, the rest far below): the
+    streaming path must settle them on its second pass."""
+    g = torch.Generator().manual_seed(21)
+    N, B, V = 3, 3, 20000
+    ar = torch.full((N, B + 1, V), -40.0)
+    for n in range(N):
+        for i in range(B + 1):
+            perm = torch.randperm(V, generator=g)
+            ar[n, i, perm[:2]] = 0.0
+            ar[n, i, perm[2:1502]] = -13.5 * float(np.log(2.0))
+    draft = ar[:, :B] + 0.05 * torch.randn(N, B, V, generator=g)
+    ar, draft = ar.to(torch.bfloat16), draft.to(torch.bfloat16)
+    ids = psi_inputs.gumbel_max(draft, 1.0, g)
+    b = _batch(ar.cuda(), draft.cuda(), ids, 1.0, 0.95)
+    assert_linear_parity(gpu_linear(b, 6, 0), oracle_linear(b, 6, 0))
+
+
+@pytest.mark.parametrize("top_p", [0.9, 1.0])
+def test_sampled_general_units_many_per_cluster(top_p):
+    """Flat rows (i.i.d. N(0, 2^2) logits at T = 1, V = 40000): nearly every
+    element lies within the streaming window, so with top-p every unit goes
+    to the cluster kernel's list mode, more units than the list-mode grid
+    has clusters (several units per cluster); without top-p every emitting
+    row's draw takes the sample mode."""
+    cfg = psi_inputs.LinearConfig("flat", 24, 4, 40000, "f32", 1.0, top_p, 31, 1, "tiny", 1.0)
+    b = psi_inputs.linear_batch(cfg, device="cuda")
+    assert_linear_parity(gpu_linear(b, 3, 1), oracle_linear(b, 3, 1))
