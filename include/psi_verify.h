@@ -134,6 +134,39 @@ psi_status psi_verify_linear(const void *ar_logits, int64_t ar_row_stride,
                              void *workspace, size_t workspace_bytes,
                              psi_stream_t stream);
 
+/*
+ * psi_verify_linear_noalloc - psi_verify_linear for callers that cannot
+ * allocate device memory (no counterpart on the pages: an integration
+ * variant, same arithmetic and results as psi_verify_linear).
+ *
+ * Arguments and results as psi_verify_linear, without the workspace: the
+ * call uses a scratch array of PSI_NOALLOC_SCRATCH_BYTES that the library
+ * holds in device memory (one per device, created with the library's module;
+ * nothing is allocated at run time).  Its address is looked up once per
+ * device, on the first call made with that device current; make that first
+ * call before capturing the stream into a graph, since it issues a
+ * runtime query besides the launches.  The scratch needs no initialisation:
+ * what the verify needs zeroed it clears itself on every call.
+ * Calls that overlap in time on the same device share the scratch and race:
+ * the caller serialises them (one stream, or events between streams).
+ * Returns PSI_ERR_UNSUPPORTED, without launching anything, when
+ * psi_verify_linear_workspace_bytes for these sizes exceeds
+ * PSI_NOALLOC_SCRATCH_BYTES (the sampled path needs about 16.5 KB per logit
+ * row, N * (2B + 1) rows: e.g. N <= 29 at B = 8; the greedy path far less),
+ * and PSI_ERR_CUDA if the scratch address cannot be obtained.
+ */
+#define PSI_NOALLOC_SCRATCH_BYTES 8388608u /* 8 MiB */
+psi_status psi_verify_linear_noalloc(const void *ar_logits, int64_t ar_row_stride,
+                                     const void *draft_logits,
+                                     int64_t draft_row_stride, psi_dtype dtype,
+                                     const int32_t *draft_ids, int32_t N, int32_t B,
+                                     int32_t V, float temperature, float top_p,
+                                     uint64_t seed, const uint64_t *seq_ids,
+                                     uint64_t step, int32_t *out_tokens,
+                                     int32_t *out_n_emitted, float *out_p_draft,
+                                     float *out_q_draft, uint32_t *dev_status,
+                                     psi_stream_t stream);
+
 /* Workspace needed by psi_verify_tree_greedy (bytes; 0 on invalid sizes). */
 size_t psi_verify_tree_greedy_workspace_bytes(int32_t N, int32_t M, int32_t V,
                                               psi_dtype dtype);

@@ -43,10 +43,12 @@ PSI_PURPOSE_RESID = 1
 PSI_MAX_B = 32
 PSI_MAX_V = 393216
 PSI_MAX_TREE_NODES = 4096
+PSI_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 EXPORTED = (
     "psi_verify_linear_workspace_bytes",
     "psi_verify_linear",
+    "psi_verify_linear_noalloc",
     "psi_verify_tree_greedy_workspace_bytes",
     "psi_verify_tree_greedy",
     "psi_rng_uniforms",
@@ -82,6 +84,9 @@ def load_library():
     lib.psi_verify_linear.restype = C.c_int
     lib.psi_verify_linear.argtypes = [vp, i64, vp, i64, C.c_int, vp, i32, i32, i32, f32, f32,
                                       u64, vp, u64, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.psi_verify_linear_noalloc.restype = C.c_int
+    lib.psi_verify_linear_noalloc.argtypes = [vp, i64, vp, i64, C.c_int, vp, i32, i32, i32, f32,
+                                              f32, u64, vp, u64, vp, vp, vp, vp, vp, vp]
     lib.psi_verify_tree_greedy_workspace_bytes.restype = sz
     lib.psi_verify_tree_greedy_workspace_bytes.argtypes = [i32, i32, i32, C.c_int]
     lib.psi_verify_tree_greedy.restype = C.c_int
@@ -122,6 +127,16 @@ def psi_verify_linear(ar_logits, ar_row_stride, draft_logits, draft_row_stride, 
         ar_logits, ar_row_stride, draft_logits, draft_row_stride, dtype, draft_ids, N, B, V,
         temperature, top_p, seed, seq_ids, step, out_tokens, out_n_emitted, out_p_draft,
         out_q_draft, dev_status, workspace, workspace_bytes, stream))
+
+
+def psi_verify_linear_noalloc(ar_logits, ar_row_stride, draft_logits, draft_row_stride, dtype,
+                              draft_ids, N, B, V, temperature, top_p, seed, seq_ids, step,
+                              out_tokens, out_n_emitted, out_p_draft, out_q_draft, dev_status,
+                              stream) -> int:
+    return int(load_library().psi_verify_linear_noalloc(
+        ar_logits, ar_row_stride, draft_logits, draft_row_stride, dtype, draft_ids, N, B, V,
+        temperature, top_p, seed, seq_ids, step, out_tokens, out_n_emitted, out_p_draft,
+        out_q_draft, dev_status, stream))
 
 
 def psi_verify_tree_greedy_workspace_bytes(N, M, V, dtype) -> int:

@@ -2,6 +2,7 @@
 // and the counter-RNG kernel.  Declarations and documentation are in
 // include/psi_verify.h.
 #include <math.h>
+#include <mutex>
 #include <stdarg.h>
 #include <stdio.h>
 #include <string.h>
@@ -256,6 +257,56 @@ psi_status psi_profile_main_kernel(psi_event_t before, psi_event_t after) {
   g_events.before = reinterpret_cast<cudaEvent_t>(before);
   g_events.after = reinterpret_cast<cudaEvent_t>(after);
   return PSI_OK;
+}
+
+// Scratch of psi_verify_linear_noalloc: part of the library's device module
+// (one copy per device), so using it allocates nothing.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PSI_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kNoallocDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kNoallocDevices] = {};
+}  // namespace
+
+psi_status psi_verify_linear_noalloc(const void *ar_logits, int64_t ar_row_stride,
+                                     const void *draft_logits, int64_t draft_row_stride,
+                                     psi_dtype dtype, const int32_t *draft_ids, int32_t N,
+                                     int32_t B, int32_t V, float temperature, float top_p,
+                                     uint64_t seed, const uint64_t *seq_ids, uint64_t step,
+                                     int32_t *out_tokens, int32_t *out_n_emitted,
+                                     float *out_p_draft, float *out_q_draft,
+                                     uint32_t *dev_status, psi_stream_t stream) {
+  const size_t need = psi_verify_linear_workspace_bytes(N, B, V, dtype, temperature, top_p);
+  if (need == 0)  // invalid sizes: psi_verify_linear reports the precise status
+    return psi_verify_linear(ar_logits, ar_row_stride, draft_logits, draft_row_stride, dtype,
+                             draft_ids, N, B, V, temperature, top_p, seed, seq_ids, step,
+                             out_tokens, out_n_emitted, out_p_draft, out_q_draft, dev_status,
+                             nullptr, 0, stream);
+  if (need > (size_t)PSI_NOALLOC_SCRATCH_BYTES)
+    return fail(PSI_ERR_UNSUPPORTED, "these sizes need %zu bytes of scratch, above the %zu held",
+                need, (size_t)PSI_NOALLOC_SCRATCH_BYTES);
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kNoallocDevices)
+    return fail(PSI_ERR_UNSUPPORTED, "device %d above the %d this entry point tracks", dev,
+                kNoallocDevices);
+  void *scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {  // once per device, with that device current
+      void *p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+      g_noalloc_ptr[dev] = p;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  return psi_verify_linear(ar_logits, ar_row_stride, draft_logits, draft_row_stride, dtype,
+                           draft_ids, N, B, V, temperature, top_p, seed, seq_ids, step,
+                           out_tokens, out_n_emitted, out_p_draft, out_q_draft, dev_status,
+                           scratch, (size_t)PSI_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 }  // extern "C"
