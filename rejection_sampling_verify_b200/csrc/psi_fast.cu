@@ -42,7 +42,7 @@ namespace {
 constexpr double kFixD = 1099511627776.0;  // 2^40
 constexpr float kFixF = 1099511627776.0f;
 constexpr int kInFlight = 8;        // 16-byte loads per thread per batch
-constexpr int kRing = 2048;         // parked vectors (shared memory ring)
+constexpr int kRing = 4096;         // parked vectors per row (shared memory)
 constexpr int kUnitThreads = 256;
 constexpr int kUnitWarps = kUnitThreads / 32;
 constexpr int kListClusters = 16;
@@ -52,11 +52,6 @@ constexpr int32_t kWideBit = int32_t(1) << 30;  // second-pass row entry: wide w
 // the second pass the wide one.
 constexpr float kWindowBaseLog2 = 13.f;
 constexpr float kWindowWideLog2 = 20.f;
-// Candidates are dropped into the fixed-point sum only while the threshold
-// lies at most this many log2 units above the row's first reference: every
-// dropped term is then below 2^4 (2^44 in 2^40 fixed point), so a row of up
-// to 2^19 elements cannot overflow the 64-bit sum.
-constexpr float kDropGuardLog2 = 4.f;
 
 struct FastArgs {
   SampledArgs s;
@@ -246,22 +241,77 @@ __device__ __forceinline__ void append_candidates(uint32_t mask, const uint4 &w,
 // ---------------------------------------------------------------------------
 // row_scan
 // ---------------------------------------------------------------------------
+// Running maximum of a 16-byte vector into `vm` (bf16: two lanes; f32: one).
+template <typename Bits>
+__device__ __forceinline__ void vec_max_into(const uint4 &w, uint32_t &vm) {
+  if constexpr (sizeof(Bits) == 2) {
+    __nv_bfloat162 m = *reinterpret_cast<const __nv_bfloat162 *>(&vm);
+    m = __hmax2(m, *reinterpret_cast<const __nv_bfloat162 *>(&w.x));
+    m = __hmax2(m, *reinterpret_cast<const __nv_bfloat162 *>(&w.y));
+    m = __hmax2(m, *reinterpret_cast<const __nv_bfloat162 *>(&w.z));
+    m = __hmax2(m, *reinterpret_cast<const __nv_bfloat162 *>(&w.w));
+    vm = *reinterpret_cast<const uint32_t *>(&m);
+  } else {
+    float m = __uint_as_float(vm);
+    m = fmaxf(fmaxf(m, __uint_as_float(w.x)), fmaxf(__uint_as_float(w.y), __uint_as_float(w.z)));
+    vm = __float_as_uint(fmaxf(m, __uint_as_float(w.w)));
+  }
+}
+
+template <typename Bits>
+__device__ __forceinline__ float vm_to_float(uint32_t vm) {
+  if constexpr (sizeof(Bits) == 2)
+    return fmaxf(__uint_as_float(vm << 16), __uint_as_float(vm & 0xFFFF0000u));
+  else
+    return __uint_as_float(vm);
+}
+
+// Candidate bits of a parked vector: bit q set iff element q > t.
+template <typename Bits>
+__device__ __forceinline__ uint32_t above_bits(const uint4 &w, float t) {
+  uint32_t mask = 0u;
+  if constexpr (sizeof(Bits) == 2) {
+    const __nv_bfloat162 t2 = __float2bfloat162_rn(t);  // t is a bf16 value: exact
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t m = __hgt2_mask(*reinterpret_cast<const __nv_bfloat162 *>(&ws[q]), t2);
+      mask |= ((m & 1u) | ((m >> 15) & 2u)) << (2 * q);
+    }
+  } else {
+    mask = (__uint_as_float(w.x) > t ? 1u : 0u) | (__uint_as_float(w.y) > t ? 2u : 0u) |
+           (__uint_as_float(w.z) > t ? 4u : 0u) | (__uint_as_float(w.w) > t ? 8u : 0u);
+  }
+  return mask;
+}
+
+constexpr int kMaxBatches = 32;  // batches per row
+
 // Each CTA walks its rows (item = blockIdx.x + t * gridDim.x) as one stream
-// of batches g = t * nb + k; the loads of batch g + 1 (the next row's first
-// batch at a row's end) are in flight while batch g is consumed.
+// of batches; the loads of the next batch (the next row's first batch at a
+// row's end) are in flight while a batch is consumed.  Vectors that hold an
+// element above their batch's threshold are parked (with the batch) in a
+// shared-memory ring; at the row's end, with the reference final, their
+// elements above the final threshold become candidates and the others go to
+// the 2^40 fixed-point sum.
 template <typename Bits>
 __global__ void __launch_bounds__(kThreads, 2) row_scan_kernel(const __grid_constant__ FastArgs a) {
   constexpr int VEC = Elem<Bits>::kVec;
   constexpr int U = kInFlight;
   constexpr int BATCH = U * kThreads;  // vectors per batch
-  __shared__ uint4 fring[kRing];       // parked vectors
-  __shared__ int32_t fidx[kRing];      // their vector index in the row
+  constexpr int kMaxVec = (sizeof(Bits) == 2 ? PSI_MAX_V : PSI_MAX_V / 2) / VEC;
+  static_assert((kMaxVec + BATCH - 1) / BATCH <= kMaxBatches, "batch index too wide");
+  static_assert(kMaxVec <= 0xFFFF, "vector index too wide");
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint4 *fring = reinterpret_cast<uint4 *>(smem);                 // [kRing] parked vectors
+  uint32_t *fidx = reinterpret_cast<uint32_t *>(fring + kRing);  // (batch << 16) | vector index
   __shared__ float s_wmax[2][kWarps];
   __shared__ float s_red[kWarps];
+  __shared__ float s_thr[kMaxBatches];  // threshold of each batch of the row
   __shared__ double s_zsum[kWarps];
   __shared__ unsigned long long s_dsum[kWarps];
-  __shared__ int s_fcount[3];          // parked vectors of batch g (counter g % 3)
-  __shared__ int s_cand;               // candidates of the current row
+  __shared__ int s_nflag;               // parked vectors of the current row
+  __shared__ int s_cand;                // candidates of the current row
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int32_t V = a.s.V;
@@ -270,13 +320,15 @@ __global__ void __launch_bounds__(kThreads, 2) row_scan_kernel(const __grid_cons
   const int32_t nb = nvec > 0 ? (nvec + BATCH - 1) / BATCH : 1;
   const int64_t R = a.pass == 1 ? a.rows : (int64_t)a.counters[2];
   if ((int64_t)blockIdx.x >= R) return;
-  const int64_t total = ((R - 1 - (int64_t)blockIdx.x) / gridDim.x + 1) * nb;
+  const int64_t my_rows = (R - 1 - (int64_t)blockIdx.x) / gridDim.x + 1;
   const float coef = a.coef;
   const float2 c2 = make_float2(coef, coef);
   uint4 neg;
   neg.x = neg.y = neg.z = neg.w = sizeof(Bits) == 2 ? 0xFF80FF80u : 0xFF800000u;
-  if (tid < 3) s_fcount[tid] = 0;
-  if (tid == 0) s_cand = 0;
+  if (tid == 0) {
+    s_nflag = 0;
+    s_cand = 0;
+  }
 
   // row of local index t, and its window (logit units)
   auto row_entry = [&](int64_t t, float &off) -> int64_t {
@@ -289,41 +341,48 @@ __global__ void __launch_bounds__(kThreads, 2) row_scan_kernel(const __grid_cons
     off = !a.use_top_p ? 0.f : (e & kWideBit) ? a.win_wide : a.win_narrow;
     return (int64_t)(e & ~kWideBit);
   };
-  auto load = [&](uint4(&buf)[U], int64_t g) {
-    if (g >= total) return;
-    const int64_t t = g / nb;
-    const int32_t k = (int32_t)(g - t * nb);
-    float unused;
-    const uint4 *rv = reinterpret_cast<const uint4 *>(row_ptr<Bits>(a, row_entry(t, unused)));
+
+  // ---- loader: batch lk of local row lt
+  int64_t lt = 0;
+  int32_t lk = 0;
+  float unused_off;
+  const uint4 *lrv = reinterpret_cast<const uint4 *>(row_ptr<Bits>(a, row_entry(0, unused_off)));
+  auto load = [&](uint4(&buf)[U]) {
+    if (lt >= my_rows) return;
+    const int32_t j0 = lk * BATCH + tid;
+    if ((lk + 1) * BATCH <= nvec) {
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int32_t j = k * BATCH + tid + u * kThreads;
-      buf[u] = j < nvec ? ldg_stream(rv + j) : neg;
+      for (int u = 0; u < U; ++u) buf[u] = ldg_stream(lrv + j0 + u * kThreads);
+    } else {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int32_t j = j0 + u * kThreads;
+        buf[u] = j < nvec ? ldg_stream(lrv + j) : neg;
+      }
+    }
+    if (++lk == nb) {
+      lk = 0;
+      if (++lt < my_rows)
+        lrv = reinterpret_cast<const uint4 *>(row_ptr<Bits>(a, row_entry(lt, unused_off)));
     }
   };
 
-  // per-row state (the same in every thread, except the partial sums)
-  int64_t r = 0;
+  // ---- consumer state (the same in every thread, except the partial sums)
+  int64_t ct = 0, r = 0;
+  int32_t ck = 0;
   const Bits *row = nullptr;
-  float off = 0.f, ref = -INFINITY, ref0 = -INFINITY, shift = -INFINITY, z_t = 0.f;
+  float off = 0.f, ref = -INFINITY, shift = -INFINITY, z_t = 0.f;
   float2 acc_a = make_float2(0.f, 0.f), acc_b = make_float2(0.f, 0.f);
-  unsigned long long dsum = 0ull;
-  bool lost = false;
-  int fbase = 0, n_prev = 0;  // ring: first slot of the current batch, slots still held
 
-  auto consume = [&](const uint4(&buf)[U], int64_t g) {
-    const int64_t t = g / nb;
-    const int32_t k = (int32_t)(g - t * nb);
-    if (k == 0) {
-      // ---- start of a row: the first reference is the first batch's maximum
-      r = row_entry(t, off);
+  auto consume = [&](const uint4(&buf)[U]) {
+    if (ck == 0) {
+      // start of a row: the first reference is the first batch's maximum
+      r = row_entry(ct, off);
       row = row_ptr<Bits>(a, r);
-      float mx = -INFINITY;
+      uint32_t vm = sizeof(Bits) == 2 ? 0xFF80FF80u : 0xFF800000u;
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const float vm = raw_vec_max<Bits>(buf[u]);
-        if (vm == vm) mx = fmaxf(mx, vm);
-      }
+      for (int u = 0; u < U; ++u) vec_max_into<Bits>(buf[u], vm);
+      float mx = vm_to_float<Bits>(vm);
       if (tid < tail) {
         const float x = Elem<Bits>::to_float(row[(int64_t)nvec * VEC + tid]);
         if (x == x) mx = fmaxf(mx, x);
@@ -332,48 +391,44 @@ __global__ void __launch_bounds__(kThreads, 2) row_scan_kernel(const __grid_cons
       // second pass: the row maximum is known from the first
       if (a.pass == 2) ref = fmaxf(ref, a.rowrec[r].ref);
       if (!(ref < INFINITY)) ref = -INFINITY;  // +inf: every finite element is a candidate
-      ref0 = ref;
       shift = (ref == -INFINITY) ? -INFINITY : -ref * coef;
       z_t = 0.f;
       acc_a = acc_b = make_float2(0.f, 0.f);
-      dsum = 0ull;
-      lost = false;
     }
-    // ---- stream the batch; park the vectors that hold a candidate
+    // ---- stream the batch
     const Threshold<Bits> th = make_threshold<Bits>(ref - off);
+    if (tid == 0) s_thr[ck] = th.value;
     const float2 s2 = make_float2(shift, shift);
-    const int cap = kRing - n_prev;
-    int *cnt = &s_fcount[g % 3];
-    float cmx = -INFINITY;
+    uint32_t hm = 0u;  // bit u: vector u holds an element above the threshold
+    uint32_t vm = sizeof(Bits) == 2 ? 0xFF80FF80u : 0xFF800000u;
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const uint32_t h = stream_vec<Bits>(buf[u], th, c2, s2, acc_a, acc_b);
-      const unsigned flagged = __ballot_sync(0xFFFFFFFFu, h != 0u);
-      if (flagged) {
-        const int leader = __ffs(flagged) - 1;
-        int first = 0;
-        if (lane == leader) first = atomicAdd(cnt, __popc(flagged));
-        first = __shfl_sync(0xFFFFFFFFu, first, leader);
-        if (h) {
-          const int idx = first + __popc(flagged & ((1u << lane) - 1u));
-          if (idx < cap) {
-            const int slot = (fbase + idx) & (kRing - 1);
-            fring[slot] = buf[u];
-            fidx[slot] = k * BATCH + tid + u * kThreads;
+      hm |= (stream_vec<Bits>(buf[u], th, c2, s2, acc_a, acc_b) != 0u ? 1u : 0u) << u;
+      vec_max_into<Bits>(buf[u], vm);
+    }
+    // ---- park the flagged vectors
+    if (__any_sync(0xFFFFFFFFu, hm != 0u)) {
+      const int c = __popc(hm);
+      int idx = 0;
+      if (c) idx = atomicAdd(&s_nflag, c);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        if ((hm >> u) & 1u) {
+          if (idx < kRing) {
+            fring[idx] = buf[u];
+            fidx[idx] = ((uint32_t)ck << 16) | (uint32_t)(ck * BATCH + tid + u * kThreads);
           }
-          cmx = fmaxf(cmx, raw_vec_max<Bits>(buf[u]));
+          ++idx;
         }
       }
     }
-    cmx = warp_max(cmx);
-    if (lane == 0) s_wmax[g & 1][warp] = cmx;
+    // ---- raise the reference to the batch maximum (same value in every thread)
+    const float cmx = warp_max(vm_to_float<Bits>(vm));
+    if (lane == 0) s_wmax[ck & 1][warp] = cmx;
     __syncthreads();
-    const int n_k = *cnt;
-    if (tid == 0) s_fcount[(g + 2) % 3] = 0;  // batch g - 1's counter: read by all, next used by g + 2
-    // ---- raise the reference (same value in every thread)
     float nr = ref;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) nr = fmaxf(nr, s_wmax[g & 1][w]);
+    for (int w = 0; w < kWarps; ++w) nr = fmaxf(nr, s_wmax[ck & 1][w]);
     if (!(nr < INFINITY)) nr = ref;
     if (nr > ref) {
       const float f = (ref == -INFINITY) ? 0.f : fast_exp2((ref - nr) * coef);
@@ -382,87 +437,88 @@ __global__ void __launch_bounds__(kThreads, 2) row_scan_kernel(const __grid_cons
       ref = nr;
       shift = -nr * coef;
     }
-    // ---- split the parked vectors: candidates above the raised threshold
-    // go to the row's list, the rest of what the batch masked is dropped into
-    // the fixed-point sum (relative to ref0, so the sum is order-free)
-    const int n_in = min(n_k, cap);
-    if (n_k > cap) lost = true;
-    const float th2 = make_threshold<Bits>(ref - off).value;
-    const bool drop = ref0 > -INFINITY && (ref - off - ref0) * coef <= kDropGuardLog2;
-    const float shift0 = -ref0 * coef;
+    if (++ck < nb) return;
+
+    // ---- end of the row: the reference is final
+    ck = 0;
+    ++ct;
+    const float thf = make_threshold<Bits>(ref - off).value;
     uint64_t *dst = a.cand + r * (int64_t)kCandCap;
-    for (int b = warp * 32; b < n_in; b += kThreads) {
-      const int e = b + lane;
+    if (tid < tail) {  // the ragged end (never streamed)
+      const uint32_t bits = row[(int64_t)nvec * VEC + tid];
+      const float x = Elem<Bits>::to_float(bits);
+      if (x > thf) {
+        const int slot = atomicAdd(&s_cand, 1);
+        if (slot < kCandCap) dst[slot] = ((uint64_t)bits << 32) | (uint32_t)(nvec * VEC + tid);
+      } else {
+        z_t += fast_exp2(fmaf(x, coef, shift));
+      }
+    }
+    z_t += (acc_a.x + acc_a.y) + (acc_b.x + acc_b.y);
+    // parked vectors: elements above the final threshold are candidates, the
+    // rest of what their batch masked goes to the fixed-point sum (each term
+    // <= 1: order-free)
+    const int n_flag = s_nflag;
+    const int nf = min(n_flag, kRing);
+    unsigned long long dsum = 0ull;
+    for (int b = 0; b < nf; b += kThreads) {
+      const int e = b + tid;
       uint32_t cmask = 0u;
       uint4 w = neg;
       int32_t j = 0;
-      if (e < n_in) {
-        const int slot = (fbase + e) & (kRing - 1);
-        w = fring[slot];
-        j = fidx[slot];
-#pragma unroll
-        for (int q = 0; q < VEC; ++q) {
+      if (e < nf) {
+        w = fring[e];
+        const uint32_t tag = fidx[e];
+        j = (int32_t)(tag & 0xFFFFu);
+        cmask = above_bits<Bits>(w, thf);
+        uint32_t dmask = above_bits<Bits>(w, s_thr[tag >> 16]) & ~cmask;
+        while (dmask) {
+          const int q = __ffs(dmask) - 1;
+          dmask &= dmask - 1;
           const float x = Elem<Bits>::to_float(vec_elem<Bits>(w, q));
-          if (x > th.value) {
-            if (!drop || x > th2) cmask |= 1u << q;
-            else dsum += __float2ull_rn(fast_exp2(fmaf(x, coef, shift0)) * kFixF);
-          }
+          dsum += __float2ull_rn(fast_exp2(fmaf(x, coef, shift)) * kFixF);
         }
       }
       append_candidates<Bits>(cmask, w, j, &s_cand, dst);
     }
-    fbase = (fbase + n_in) & (kRing - 1);
-    n_prev = n_in;
-
-    if (k == nb - 1) {
-      // ---- end of the row: ragged end, sums, row record
-      if (tid < tail) {
-        const uint32_t bits = row[(int64_t)nvec * VEC + tid];
-        const float x = Elem<Bits>::to_float(bits);
-        if (x > th2) {
-          const int slot = atomicAdd(&s_cand, 1);
-          if (slot < kCandCap) dst[slot] = ((uint64_t)bits << 32) | (uint32_t)(nvec * VEC + tid);
-        } else {
-          z_t += fast_exp2(fmaf(x, coef, shift));
-        }
-      }
-      z_t += (acc_a.x + acc_a.y) + (acc_b.x + acc_b.y);
-      const double zs = warp_sum_any((double)z_t);
-      const unsigned long long ds = warp_sum_any(dsum);
-      if (lane == 0) {
-        s_zsum[warp] = zs;
-        s_dsum[warp] = ds;
-      }
-      __syncthreads();
-      if (tid == 0) {
-        double zt = 0.0;
-        unsigned long long zd = 0ull;
+    const double zs = warp_sum_any((double)z_t);
+    const unsigned long long ds = warp_sum_any(dsum);
+    if (lane == 0) {
+      s_zsum[warp] = zs;
+      s_dsum[warp] = ds;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      double zt = 0.0;
+      unsigned long long zd = 0ull;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-          zt += s_zsum[w];
-          zd += s_dsum[w];
-        }
-        RowRecord rec;
-        rec.ref = ref;
-        rec.ref0 = ref0;
-        rec.n_cand = s_cand;
-        rec.flags = lost ? kRowLost : 0;
-        rec.zt = zt;
-        rec.zd = zd;
-        a.rowrec[r] = rec;
-        s_cand = 0;  // (the next row appends only after its first barrier)
+      for (int w = 0; w < kWarps; ++w) {
+        zt += s_zsum[w];
+        zd += s_dsum[w];
       }
+      RowRecord rec;
+      rec.ref = ref;
+      rec.n_cand = s_cand;
+      rec.flags = n_flag > kRing ? kRowLost : 0;
+      rec.pad = 0;
+      rec.zt = zt;
+      rec.zd = zd;
+      a.rowrec[r] = rec;
+      // (the next row parks and appends only after its first barrier)
+      s_nflag = 0;
+      s_cand = 0;
     }
   };
 
   uint4 b0[U], b1[U];
-  load(b0, 0);
+  const int64_t total = my_rows * nb;
+  load(b0);
   for (int64_t g = 0; g < total; g += 2) {
-    load(b1, g + 1);
-    consume(b0, g);
+    load(b1);
+    consume(b0);
     if (g + 1 >= total) break;
-    load(b0, g + 2);
-    consume(b1, g + 1);
+    load(b0);
+    consume(b1);
   }
 }
 
@@ -560,8 +616,8 @@ __device__ __noinline__ RowFinal finish_row(const FastArgs &a, int64_t r, UnitSh
   }
   zin = block_sum_all<unsigned long long, kUnitWarps>(zin, sh->u);
   double Z = (double)zin / kFixD;
-  if (rs.ref > -INFINITY) Z += rs.zt * exp2(((double)rs.ref - (double)M) * a.coef64);
-  if (rs.zd) Z += (double)rs.zd / kFixD * exp2(((double)rs.ref0 - (double)M) * a.coef64);
+  if (rs.ref > -INFINITY)
+    Z += (rs.zt + (double)rs.zd / kFixD) * exp2(((double)rs.ref - (double)M) * a.coef64);
   out.zp = Z;
   if (!(Z < INFINITY)) {
     out.status = kFinNonfinite;
@@ -834,6 +890,8 @@ int sm_count() {
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
+constexpr size_t kScanSmem = (sizeof(uint4) + sizeof(uint32_t)) * kRing;
+
 template <typename Bits>
 cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, const KernelEvents &ev,
                               cudaStream_t stream) {
@@ -841,10 +899,17 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, const
   const int64_t persistent = (int64_t)sm_count() * 2;
   const int64_t grid_scan = std::min<int64_t>(fa.rows, persistent);
   cudaError_t e;
+  static bool configured = false;
+  if (!configured) {
+    if ((e = cudaFuncSetAttribute(row_scan_kernel<Bits>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kScanSmem)) != cudaSuccess)
+      return e;
+    configured = true;
+  }
   // the work-list counters of this call start at zero
   if ((e = cudaMemsetAsync(fa.counters, 0, 4 * sizeof(int32_t), stream)) != cudaSuccess) return e;
   if (ev.before && (e = cudaEventRecord(ev.before, stream)) != cudaSuccess) return e;
-  row_scan_kernel<Bits><<<(unsigned)grid_scan, kThreads, 0, stream>>>(fa);
+  row_scan_kernel<Bits><<<(unsigned)grid_scan, kThreads, kScanSmem, stream>>>(fa);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (ev.after && (e = cudaEventRecord(ev.after, stream)) != cudaSuccess) return e;
   unit_kernel<Bits><<<(unsigned)units, kUnitThreads, 0, stream>>>(fa);
@@ -854,7 +919,7 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, const
     // (usually none: the CTAs find empty lists and exit)
     FastArgs f2 = fa;
     f2.pass = 2;
-    row_scan_kernel<Bits><<<(unsigned)grid_scan, kThreads, 0, stream>>>(f2);
+    row_scan_kernel<Bits><<<(unsigned)grid_scan, kThreads, kScanSmem, stream>>>(f2);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     unit_kernel<Bits><<<(unsigned)std::min<int64_t>(units, persistent), kUnitThreads, 0, stream>>>(f2);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -90,15 +90,15 @@ cudaError_t launch_cluster_list(const SampledArgs &a, psi_dtype dtype, const Sam
 // ---- streaming path (rows 16-byte aligned) ------------------------------------
 // Per logit row: what the row-scan kernel leaves for the unit kernel.  Every
 // element of the row is counted exactly once: in zt (at or below the
-// threshold of its batch), in zd (a candidate that fell below a later
-// threshold) or in the row's candidate list.
+// threshold of its batch), in zd (above it, but at or below the row's final
+// threshold) or in the row's candidate list (above the final threshold).
 struct RowRecord {
   float ref;        // final running reference: the row maximum, unless the row holds +inf
-  float ref0;       // reference of zd (the first reference of the row)
   int32_t n_cand;   // candidates appended (more than the capacity: overflow)
   int32_t flags;    // kRowLost: flagged vectors were dropped (ring overflow)
-  double zt;        // sum of exp2((x - ref) * log2(e) / T) over the non-candidates
-  uint64_t zd;      // 2^40 * sum of exp2((x - ref0) * log2(e) / T) over dropped candidates
+  int32_t pad;
+  double zt;        // sum of exp2((x - ref) * log2(e) / T) over the unmasked elements
+  uint64_t zd;      // 2^40 * the same sum over masked elements that are not candidates
 };
 constexpr int32_t kRowLost = 1;
 constexpr int kCandCap = 2048;     // candidates kept per row (global workspace)
