@@ -43,8 +43,6 @@ constexpr double kFixD = 1099511627776.0;  // 2^40
 constexpr float kFixF = 1099511627776.0f;
 constexpr int kInFlight = 8;        // 16-byte loads per thread per batch
 constexpr int kRing = 4096;         // parked vectors per row (shared memory)
-constexpr int kUnitThreads = 256;
-constexpr int kUnitWarps = kUnitThreads / 32;
 constexpr int kListClusters = 16;
 constexpr int32_t kWideBit = int32_t(1) << 30;  // second-pass row entry: wide window
 // Candidate window, in log2 units below the reference.  The first pass uses
@@ -65,6 +63,7 @@ struct FastArgs {
   UnitRecord *rec;     // [N*(B+1)]
   RowRecord *rowrec;   // [rows]
   uint64_t *cand;      // [rows][kCandCap]: (bits << 32) | vocabulary index
+  uint32_t *cmass;     // [rows][kCandCap]: masses of rows with more candidates than a warp keeps
   int32_t *counters;   // [0] general units, [1] sample-mode units, [2] wide rows, [3] wide units
   int32_t *list_a;     // units for the general path
   int32_t *list_b;     // units whose draw needs the whole row
@@ -523,46 +522,47 @@ __global__ void __launch_bounds__(kThreads, 2) row_scan_kernel(const __grid_cons
 }
 
 // ---------------------------------------------------------------------------
-// unit
+// unit: one warp per (sequence, row) unit
 // ---------------------------------------------------------------------------
-// Statistics of one finished row (the same in every thread).
+// Statistics of one finished row (the same in every lane).
 struct RowFinal {
   float m;            // row maximum
   double zp;          // normaliser after top-p (Z without top-p)
   uint32_t tau_bits;  // top-p threshold (raw bits): keep x >= tau
-  int n_nuc;          // nucleus entries left in UnitShared::ms (when asked for)
+  uint32_t tau_key;   // its order-preserving key (0 without top-p)
+  int n;              // candidates of the row
   int status;         // kFin* bits
 };
 constexpr int kFinOverflow = 1;   // candidates lost: rescan with the exact maximum
 constexpr int kFinCoverage = 2;   // the window holds less than top_p: rescan wider
 constexpr int kFinNonfinite = 4;  // NaN / +inf logit, or no finite logit
 
-struct UnitShared {
-  unsigned long long kc[kCandCap];  // (key << 32) | index; later the draw weights (double)
-  unsigned long long ms[kCandCap];  // 2^40 fixed-point masses; later the nucleus (index << 32 | bits)
-  double d[kUnitWarps];
-  unsigned long long u[kUnitWarps];
-  unsigned long long bs[2][kUnitWarps];
-  float f[kUnitWarps];
-  uint32_t k2[2][kUnitWarps];
-  int n;
-  int need;
+constexpr int kUnitCtaWarps = 4;   // warps (units) per CTA
+constexpr int kWarpCand = 1024;    // candidates a warp keeps in shared memory
+constexpr double kFix31 = 2147483648.0;  // 2^31: candidate masses (each <= 1) in u32
+
+struct WarpScratch {
+  unsigned long long ent[kWarpCand];  // copy of the candidate list: (bits << 32) | vocabulary index
+  uint32_t mass[kWarpCand];           // 2^31 fixed-point masses; later the draw weights (float)
 };
 
 // Row maximum, Z, top-p threshold tau and renormaliser Z' of row r from its
-// record and candidate list, and (want_nuc) p's nucleus: every candidate
-// with x >= tau.  The top-p threshold is the largest logit key t whose
-// suffix mass S(t) (all x with key >= t) reaches top_p * Z; only candidates
-// can be at or above it (the window holds at least top_p of the mass).
+// record and candidate list.  The top-p threshold is the largest logit key t
+// whose suffix mass S(t) (every x with key >= t) reaches top_p * Z; only
+// candidates can be at or above it when the candidates hold at least top_p
+// of the mass.  Rows with more candidates than the warp's shared memory
+// holds read the global candidate list directly (it stays unchanged: a
+// second pass may finish the row again).
 template <typename Bits>
-__device__ __noinline__ RowFinal finish_row(const FastArgs &a, int64_t r, UnitShared *sh,
-                                            bool want_nuc) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+__device__ RowFinal finish_row(const FastArgs &a, int64_t r, WarpScratch *ws,
+                               unsigned long long *&ent, uint32_t *&mass) {
+  const int lane = threadIdx.x & 31;
   RowFinal out;
   out.m = -INFINITY;
   out.zp = 0.0;
   out.tau_bits = Elem<Bits>::kNegInf;
-  out.n_nuc = 0;
+  out.tau_key = 0u;
+  out.n = 0;
   out.status = 0;
   const RowRecord rs = a.rowrec[r];
   if (rs.n_cand > kCandCap || (rs.flags & kRowLost)) {
@@ -570,52 +570,41 @@ __device__ __noinline__ RowFinal finish_row(const FastArgs &a, int64_t r, UnitSh
     return out;
   }
   const int n = rs.n_cand;
-  const uint64_t *src = a.cand + r * (int64_t)kCandCap;
+  out.n = n;
+  unsigned long long *src = reinterpret_cast<unsigned long long *>(a.cand + r * (int64_t)kCandCap);
+  ent = n <= kWarpCand ? ws->ent : src;
+  mass = n <= kWarpCand ? ws->mass : a.cmass + r * (int64_t)kCandCap;
+  __syncwarp();  // the previous row's readers of the scratch are done
   float cm = -INFINITY;
   uint32_t kmax = 0u, kmin_inv = 0u;
-  for (int j = tid; j < n; j += kUnitThreads) {
-    const uint64_t e = src[j];
+  for (int j = lane; j < n; j += 32) {
+    const unsigned long long e = src[j];
     const uint32_t b = (uint32_t)(e >> 32);
     cm = fmaxf(cm, Elem<Bits>::to_float(b));
     const uint32_t key = Elem<Bits>::key(b);
-    sh->kc[j] = ((unsigned long long)key << 32) | (e & 0xFFFFFFFFull);
+    if (ent != src) ent[j] = e;
     kmax = max(kmax, key);
     kmin_inv = max(kmin_inv, ~key);
   }
-  cm = warp_max(cm);
+  const float M = fmaxf(rs.ref, warp_max(cm));
   kmax = warp_max_u32(kmax);
   kmin_inv = warp_max_u32(kmin_inv);
-  __syncthreads();
-  if (lane == 0) {
-    sh->f[warp] = cm;
-    sh->k2[0][warp] = kmax;
-    sh->k2[1][warp] = kmin_inv;
-  }
-  __syncthreads();
-  float M = rs.ref;
-  uint32_t KMAX = 0u, KMIN_INV = 0u;
-#pragma unroll
-  for (int w = 0; w < kUnitWarps; ++w) {
-    M = fmaxf(M, sh->f[w]);
-    KMAX = max(KMAX, sh->k2[0][w]);
-    KMIN_INV = max(KMIN_INV, sh->k2[1][w]);
-  }
   out.m = M;
   if (!(M > -INFINITY) || !(fabsf(M * a.coef) < INFINITY) || rs.zt != rs.zt) {
     out.status = kFinNonfinite;
     return out;
   }
-  // exact masses relative to M (2^40 fixed point: order-free sums)
+  // exact masses relative to M in 2^31 fixed point (order-free sums)
   unsigned long long zin = 0ull;
-  for (int j = tid; j < n; j += kUnitThreads) {
-    const uint32_t b = key_to_bits<Bits>((uint32_t)(sh->kc[j] >> 32));
-    const unsigned long long fx =
-        __double2ull_rn(exact_exp2d(Elem<Bits>::to_float(b), M, a.coef64) * kFixD);
-    sh->ms[j] = fx;
+  for (int j = lane; j < n; j += 32) {
+    const uint32_t b = (uint32_t)(ent[j] >> 32);
+    const uint32_t fx = __double2uint_rn(exact_exp2d(Elem<Bits>::to_float(b), M, a.coef64) * kFix31);
+    mass[j] = fx;
     zin += fx;
   }
-  zin = block_sum_all<unsigned long long, kUnitWarps>(zin, sh->u);
-  double Z = (double)zin / kFixD;
+  zin = warp_sum_any(zin);
+  __syncwarp();
+  double Z = (double)zin / kFix31;
   if (rs.ref > -INFINITY)
     Z += (rs.zt + (double)rs.zd / kFixD) * exp2(((double)rs.ref - (double)M) * a.coef64);
   out.zp = Z;
@@ -624,123 +613,61 @@ __device__ __noinline__ RowFinal finish_row(const FastArgs &a, int64_t r, UnitSh
     return out;
   }
   if (!a.use_top_p) return out;
-  const unsigned long long target = (unsigned long long)ceil((double)a.s.top_p * Z * kFixD);
+  const unsigned long long target = (unsigned long long)ceil((double)a.s.top_p * Z * kFix31);
   if (zin < target) {
     out.status = kFinCoverage;
     return out;
   }
   // binary search over [kmin, kmax]: S(kmin) = zin reaches the target
-  uint64_t lo = ~KMIN_INV, hi = (uint64_t)KMAX + 1;
+  uint64_t lo = ~kmin_inv, hi = (uint64_t)kmax + 1;
   unsigned long long s_lo = zin;
-  int par = 0;
   while (hi - lo > 1) {
     const uint64_t mid = (lo + hi) >> 1;
     unsigned long long part = 0ull;
-    for (int j = tid; j < n; j += kUnitThreads)
-      if ((sh->kc[j] >> 32) >= mid) part += sh->ms[j];
+    for (int j = lane; j < n; j += 32)
+      if (Elem<Bits>::key((uint32_t)(ent[j] >> 32)) >= mid) part += mass[j];
     part = warp_sum_any(part);
-    if (lane == 0) sh->bs[par][warp] = part;
-    __syncthreads();
-    unsigned long long S = 0ull;
-#pragma unroll
-    for (int w = 0; w < kUnitWarps; ++w) S += sh->bs[par][w];
-    par ^= 1;
-    if (S >= target) {
+    if (part >= target) {
       lo = mid;
-      s_lo = S;
+      s_lo = part;
     } else {
       hi = mid;
     }
   }
-  out.zp = (double)s_lo / kFixD;
+  out.zp = (double)s_lo / kFix31;
+  out.tau_key = (uint32_t)lo;
   out.tau_bits = key_to_bits<Bits>((uint32_t)lo);
-  if (want_nuc) {
-    __syncthreads();  // every read of the masses is done
-    if (tid == 0) sh->n = 0;
-    __syncthreads();
-    for (int j = tid; j < n; j += kUnitThreads) {
-      const unsigned long long e = sh->kc[j];
-      const uint32_t key = (uint32_t)(e >> 32);
-      if (key >= (uint32_t)lo) {
-        const int slot = atomicAdd(&sh->n, 1);
-        sh->ms[slot] = ((e & 0xFFFFFFFFull) << 32) | key_to_bits<Bits>(key);
-      }
-    }
-    __syncthreads();
-    out.n_nuc = sh->n;
-  }
   return out;
 }
 
-// In-place ascending bitonic sort of n (a power of two) 64-bit keys.
-__device__ void bitonic_sort(unsigned long long *v, int n) {
-  for (int k = 2; k <= n; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int t = threadIdx.x; t < n; t += blockDim.x) {
-        const int p = t ^ j;
-        if (p > t) {
-          const bool up = (t & k) == 0;
-          const unsigned long long x = v[t], y = v[p];
-          if ((x > y) == up) {
-            v[t] = y;
-            v[p] = x;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  }
-}
-
-// Inclusive prefix sums of w[0..n) in index order (deterministic), in place.
-__device__ void block_scan(double *w, int n, double *scratch) {
-  const int per = (n + kUnitThreads - 1) / kUnitThreads;
-  const int b0 = threadIdx.x * per, b1 = min(n, b0 + per);
-  double run = 0.0;
-  for (int j = b0; j < b1; ++j) {
-    run += w[j];
-    w[j] = run;
-  }
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  double incl = run;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const double v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  __syncthreads();
-  if (lane == 31) scratch[warp] = incl;
-  __syncthreads();
-  double off = incl - run;
-  for (int w2 = 0; w2 < warp; ++w2) off += scratch[w2];
-  for (int j = b0; j < b1; ++j) w[j] += off;
-  __syncthreads();
-}
-
 template <typename Bits>
-__global__ void __launch_bounds__(kUnitThreads) unit_kernel(const __grid_constant__ FastArgs a) {
-  __shared__ UnitShared sh;
-  const int tid = threadIdx.x;
+__global__ void __launch_bounds__(32 * kUnitCtaWarps) unit_kernel(const __grid_constant__ FastArgs a) {
+  __shared__ WarpScratch scratch[kUnitCtaWarps];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  WarpScratch *ws = &scratch[warp];
   const SampledArgs &s = a.s;
   const int32_t B = s.B, N = s.N, V = s.V;
   const int64_t n_items = a.pass == 1 ? (int64_t)N * (B + 1) : (int64_t)a.counters[3];
-  for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+  for (int64_t item = (int64_t)blockIdx.x * kUnitCtaWarps + warp; item < n_items;
+       item += (int64_t)gridDim.x * kUnitCtaWarps) {
     const int64_t unit = a.pass == 1 ? item : (int64_t)a.wide_units[item];
     const int32_t n = (int32_t)(unit / (B + 1)), i = (int32_t)(unit % (B + 1));
     const bool has_q = i < B;
     const int64_t rp_idx = unit;
     const int64_t rq_idx = (int64_t)N * (B + 1) + (int64_t)n * B + i;
+    unsigned long long *ent = nullptr;
+    uint32_t *mass = nullptr;
     RowFinal fq;
     fq.m = -INFINITY;
     fq.zp = 0.0;
     fq.tau_bits = 0u;
     fq.status = 0;
-    if (has_q) fq = finish_row<Bits>(a, rq_idx, &sh, false);
-    const RowFinal fp = finish_row<Bits>(a, rp_idx, &sh, true);
+    if (has_q) fq = finish_row<Bits>(a, rq_idx, ws, ent, mass);
+    const RowFinal fp = finish_row<Bits>(a, rp_idx, ws, ent, mass);
     const int fail_q = fq.status & (kFinOverflow | kFinCoverage);
     const int fail_p = fp.status & (kFinOverflow | kFinCoverage);
     if (fail_q || fail_p) {
-      if (tid == 0) {
+      if (lane == 0) {
         if (a.pass == 1) {  // rescan the failed rows, then finish the unit again
           if (fail_q)
             a.wide_rows[atomicAdd(&a.counters[2], 1)] =
@@ -762,9 +689,9 @@ __global__ void __launch_bounds__(kUnitThreads) unit_kernel(const __grid_constan
     const float tau_p = Elem<Bits>::to_float(fp.tau_bits);
     const float tau_q = Elem<Bits>::to_float(fq.tau_bits);
 
-    // ---- accept / reject the drafted token
-    if (tid == 0) {
-      int need = 1;
+    // ---- accept / reject the drafted token (lane 0)
+    int need = 1;
+    if (lane == 0) {
       if (has_q) {
         const int32_t x = s.ids[(int64_t)n * B + i];
         double p = 0.0, q = 0.0;
@@ -788,67 +715,63 @@ __global__ void __launch_bounds__(kUnitThreads) unit_kernel(const __grid_constan
       }
       if (((fp.status | fq.status) & kFinNonfinite) && s.dev_status)
         atomicOr(s.dev_status, PSI_DEV_NONFINITE);
-      sh.need = need;
     }
-    __syncthreads();
-    const int need = sh.need;
-    __syncthreads();  // (sh.need is rewritten by the next unit)
+    need = __shfl_sync(0xFFFFFFFFu, need, 0);
     if (!need) continue;
     if (!a.use_top_p) {  // the draw needs whole rows: decided after the emit step
-      if (tid == 0) a.rec[unit].token = -2;
+      if (lane == 0) a.rec[unit].token = -2;
       continue;
     }
 
-    // ---- correction / bonus draw over p's nucleus, in vocabulary order
-    const int nn = fp.n_nuc;
-    int np2 = 1;
-    while (np2 < nn) np2 <<= 1;
-    unsigned long long *ent = sh.ms;
-    for (int t = nn + tid; t < np2; t += kUnitThreads) ent[t] = ~0ull;
-    __syncthreads();
-    bitonic_sort(ent, np2);
-    double *wv = reinterpret_cast<double *>(sh.kc);
+    // ---- correction / bonus draw over p's nucleus (its candidates with key
+    // >= tau), inverse CDF in vocabulary order
+    float *w = reinterpret_cast<float *>(mass);
+    const int nc = (fp.status & kFinNonfinite) ? 0 : fp.n;
+    int32_t token = 0;
     for (int pass = 0; pass < 2; ++pass) {
       const bool p_only = !has_q || pass == 1;
-      for (int t = tid; t < nn; t += kUnitThreads) {
-        const int32_t v = (int32_t)(ent[t] >> 32);
-        const float xp = Elem<Bits>::to_float((uint32_t)(ent[t] & 0xFFFFFFFFull));
-        double w = exact_exp2d(xp, fp.m, a.coef64) / fp.zp;
-        if (!p_only) {
-          const float xq = Elem<Bits>::to_float(row_q[v]);
-          const double q = (xq >= tau_q && fq.zp > 0.0) ? exact_exp2d(xq, fq.m, a.coef64) / fq.zp : 0.0;
-          w = w > q ? w - q : 0.0;
-        }
-        wv[t] = w;
-      }
-      __syncthreads();
-      block_scan(wv, nn, sh.d);
-      const double W = nn > 0 ? wv[nn - 1] : 0.0;
-      if (W > 0.0 || p_only) {
-        if (tid == 0) {
-          int32_t token = 0;
-          if (W > 0.0) {
-            const double u2 = (double)uniform24(s.seed, seq, s.step, (uint64_t)i, PSI_PURPOSE_RESID);
-            const double t = u2 * W;
-            int lo = 0, hi = nn;  // first j with wv[j] > t
-            while (lo < hi) {
-              const int mid = (lo + hi) >> 1;
-              if (wv[mid] > t) hi = mid;
-              else lo = mid + 1;
-            }
-            if (lo >= nn) {  // rounding: the last entry with positive weight
-              lo = nn - 1;
-              while (lo > 0 && !(wv[lo] > wv[lo - 1])) --lo;
-            }
-            token = (int32_t)(ent[lo] >> 32);
+      double part = 0.0;
+      for (int j = lane; j < nc; j += 32) {
+        const unsigned long long e = ent[j];
+        const uint32_t bits = (uint32_t)(e >> 32);
+        float wj = 0.f;
+        if (Elem<Bits>::key(bits) >= fp.tau_key) {
+          const float xp = Elem<Bits>::to_float(bits);
+          double pv = exact_exp2d(xp, fp.m, a.coef64) / fp.zp;
+          if (!p_only) {
+            const float xq = Elem<Bits>::to_float(row_q[(uint32_t)e]);
+            const double qv =
+                (xq >= tau_q && fq.zp > 0.0) ? exact_exp2d(xq, fq.m, a.coef64) / fq.zp : 0.0;
+            pv = pv > qv ? pv - qv : 0.0;
           }
-          a.rec[unit].token = token;
+          wj = (float)pv;
         }
-        break;
+        w[j] = wj;
+        part += (double)wj;
       }
-      __syncthreads();  // residual vanished: draw from p itself
+      const double W = warp_sum_any(part);
+      __syncwarp();
+      if (!(W > 0.0) && !p_only) continue;  // residual vanished: draw from p itself
+      if (W > 0.0) {
+        const double t = (double)uniform24(s.seed, seq, s.step, (uint64_t)i, PSI_PURPOSE_RESID) * W;
+        // smallest X with C(X) = sum of w over entries with index < X above t;
+        // the token is X - 1 (C(V) = W > t)
+        uint32_t lo = 0u, hi = (uint32_t)V;
+        while (hi - lo > 1) {
+          const uint32_t mid = (lo + hi) >> 1;
+          double c = 0.0;
+          for (int j = lane; j < nc; j += 32)
+            if ((uint32_t)ent[j] < mid) c += (double)w[j];
+          c = warp_sum_any(c);
+          if (c > t) hi = mid;
+          else lo = mid;
+        }
+        token = (int32_t)lo;
+      }
+      break;
     }
-    __syncthreads();  // shared buffers free for the next unit
+    if (lane == 0) a.rec[unit].token = token;
+    __syncwarp();  // the scratch is free for the next unit
   }
 }
 
@@ -912,7 +835,8 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, const
   row_scan_kernel<Bits><<<(unsigned)grid_scan, kThreads, kScanSmem, stream>>>(fa);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (ev.after && (e = cudaEventRecord(ev.after, stream)) != cudaSuccess) return e;
-  unit_kernel<Bits><<<(unsigned)units, kUnitThreads, 0, stream>>>(fa);
+  unit_kernel<Bits><<<(unsigned)((units + kUnitCtaWarps - 1) / kUnitCtaWarps), 32 * kUnitCtaWarps, 0,
+                      stream>>>(fa);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   {
     // second pass over the rows and units the first one could not settle
@@ -921,7 +845,8 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, const
     f2.pass = 2;
     row_scan_kernel<Bits><<<(unsigned)grid_scan, kThreads, kScanSmem, stream>>>(f2);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    unit_kernel<Bits><<<(unsigned)std::min<int64_t>(units, persistent), kUnitThreads, 0, stream>>>(f2);
+    unit_kernel<Bits><<<(unsigned)std::min<int64_t>((units + kUnitCtaWarps - 1) / kUnitCtaWarps, persistent),
+                        32 * kUnitCtaWarps, 0, stream>>>(f2);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   const psi_dtype dt = sizeof(Bits) == 2 ? PSI_DTYPE_BF16 : PSI_DTYPE_F32;
@@ -949,6 +874,8 @@ FastLayout fast_layout(int32_t N, int32_t B) {
   off = align256(off + sizeof(RowRecord) * (size_t)rows);
   L.cand_off = off;
   off = align256(off + sizeof(uint64_t) * (size_t)rows * kCandCap);
+  L.cmass_off = off;
+  off = align256(off + sizeof(uint32_t) * (size_t)rows * kCandCap);
   L.counters_off = off;
   off = align256(off + sizeof(int32_t) * 4);
   L.list_a_off = off;
@@ -989,6 +916,7 @@ cudaError_t launch_sampled_fast(const SampledArgs &a, psi_dtype dtype, const Sam
   fa.rec = reinterpret_cast<UnitRecord *>(ws + L.rec_off);
   fa.rowrec = reinterpret_cast<RowRecord *>(ws + L.rows_off);
   fa.cand = reinterpret_cast<uint64_t *>(ws + L.cand_off);
+  fa.cmass = reinterpret_cast<uint32_t *>(ws + L.cmass_off);
   fa.counters = reinterpret_cast<int32_t *>(ws + L.counters_off);
   fa.list_a = reinterpret_cast<int32_t *>(ws + L.list_a_off);
   fa.list_b = reinterpret_cast<int32_t *>(ws + L.list_b_off);
