@@ -218,6 +218,12 @@ __device__ __forceinline__ void bulk_load(void *dst_smem, const void *src, uint3
       : "memory");
 }
 
+// Hint: bring `bytes` of global memory at `src` into L2 (no data returned,
+// no completion to wait for).  src and bytes must be multiples of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // Thread-block clusters.
 // ---------------------------------------------------------------------------

@@ -19,7 +19,7 @@
 //              hold them are parked in a shared-memory ring and, after the
 //              batch's barrier, split into candidates (to a per-row list in
 //              global memory) and elements that fell below the raised
-//              threshold (a 2^40 fixed-point sum).
+//              threshold (a 2^31 fixed-point sum).
 //   unit       One CTA per (sequence, row) unit: finishes the unit's q and p
 //              rows from their candidates (row maximum, Z, the top-p threshold
 //              and renormaliser, p's nucleus), decides the drafted token and
@@ -39,8 +39,7 @@ namespace psi {
 
 namespace {
 
-constexpr double kFixD = 1099511627776.0;  // 2^40
-constexpr float kFixF = 1099511627776.0f;
+constexpr float kFix31F = 2147483648.0f;  // 2^31: dropped masses (each <= 1)
 constexpr int kInFlight = 8;        // 16-byte loads per thread per batch
 constexpr int kRing = 4096;         // parked vectors per row (shared memory)
 constexpr int kListClusters = 16;
@@ -285,6 +284,7 @@ __device__ __forceinline__ uint32_t above_bits(const uint4 &w, float t) {
 }
 
 constexpr int kMaxBatches = 32;  // batches per row
+constexpr int kPrefetch = 3;     // L2 prefetch distance, in batches beyond the register loads
 
 // Each CTA walks its rows (item = blockIdx.x + t * gridDim.x) as one stream
 // of batches; the loads of the next batch (the next row's first batch at a
@@ -292,7 +292,7 @@ constexpr int kMaxBatches = 32;  // batches per row
 // element above their batch's threshold are parked (with the batch) in a
 // shared-memory ring; at the row's end, with the reference final, their
 // elements above the final threshold become candidates and the others go to
-// the 2^40 fixed-point sum.
+// the 2^31 fixed-point sum.
 template <typename Bits>
 __global__ void __launch_bounds__(kThreads, 2) row_scan_kernel(const __grid_constant__ FastArgs a) {
   constexpr int VEC = Elem<Bits>::kVec;
@@ -341,12 +341,32 @@ __global__ void __launch_bounds__(kThreads, 2) row_scan_kernel(const __grid_cons
     return (int64_t)(e & ~kWideBit);
   };
 
-  // ---- loader: batch lk of local row lt
+  // ---- loader: batch lk of local row lt; thread 0 also asks L2 for the
+  // batch kPrefetch batches ahead (pt, pk), so that HBM keeps streaming while
+  // the CTA is busy at a row's end
   int64_t lt = 0;
   int32_t lk = 0;
   float unused_off;
   const uint4 *lrv = reinterpret_cast<const uint4 *>(row_ptr<Bits>(a, row_entry(0, unused_off)));
+  int64_t pt = 0;
+  int32_t pk = 0;
+  const uint4 *prv = lrv;
+  auto advance_prefetch = [&]() {
+    if (pt >= my_rows) return;
+    if (tid == 0 && nvec > 0) {
+      const int32_t v0 = pk * BATCH;
+      const int32_t nv = min(BATCH, nvec - v0);
+      prefetch_l2_bulk(prv + v0, (uint32_t)nv * 16u);
+    }
+    if (++pk == nb) {
+      pk = 0;
+      if (++pt < my_rows)
+        prv = reinterpret_cast<const uint4 *>(row_ptr<Bits>(a, row_entry(pt, unused_off)));
+    }
+  };
+  for (int d = 0; d < kPrefetch; ++d) advance_prefetch();
   auto load = [&](uint4(&buf)[U]) {
+    advance_prefetch();
     if (lt >= my_rows) return;
     const int32_t j0 = lk * BATCH + tid;
     if ((lk + 1) * BATCH <= nvec) {
@@ -475,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 2) row_scan_kernel(const __grid_cons
           const int q = __ffs(dmask) - 1;
           dmask &= dmask - 1;
           const float x = Elem<Bits>::to_float(vec_elem<Bits>(w, q));
-          dsum += __float2ull_rn(fast_exp2(fmaf(x, coef, shift)) * kFixF);
+          dsum += __float2uint_rn(fast_exp2(fmaf(x, coef, shift)) * kFix31F);
         }
       }
       append_candidates<Bits>(cmask, w, j, &s_cand, dst);
@@ -499,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 2) row_scan_kernel(const __grid_cons
       rec.ref = ref;
       rec.n_cand = s_cand;
       rec.flags = n_flag > kRing ? kRowLost : 0;
-      rec.pad = 0;
+      rec.n_parked = n_flag;
       rec.zt = zt;
       rec.zd = zd;
       a.rowrec[r] = rec;
@@ -606,7 +626,7 @@ __device__ RowFinal finish_row(const FastArgs &a, int64_t r, WarpScratch *ws,
   __syncwarp();
   double Z = (double)zin / kFix31;
   if (rs.ref > -INFINITY)
-    Z += (rs.zt + (double)rs.zd / kFixD) * exp2(((double)rs.ref - (double)M) * a.coef64);
+    Z += (rs.zt + (double)rs.zd / kFix31) * exp2(((double)rs.ref - (double)M) * a.coef64);
   out.zp = Z;
   if (!(Z < INFINITY)) {
     out.status = kFinNonfinite;

@@ -96,9 +96,9 @@ struct RowRecord {
   float ref;        // final running reference: the row maximum, unless the row holds +inf
   int32_t n_cand;   // candidates appended (more than the capacity: overflow)
   int32_t flags;    // kRowLost: flagged vectors were dropped (ring overflow)
-  int32_t pad;
+  int32_t n_parked; // vectors parked by the scan (diagnostics)
   double zt;        // sum of exp2((x - ref) * log2(e) / T) over the unmasked elements
-  uint64_t zd;      // 2^40 * the same sum over masked elements that are not candidates
+  uint64_t zd;      // 2^31 * the same sum over masked elements that are not candidates
 };
 constexpr int32_t kRowLost = 1;
 constexpr int kCandCap = 2048;     // candidates kept per row (global workspace)
