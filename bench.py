@@ -418,6 +418,8 @@ def measure_e2e(psi, cfg, batch, seq_ids, ws, K, dev, pg, world):
     if is_tree:
         host = [batch.ar.cpu().pin_memory(), batch.node_tokens.cpu().pin_memory(),
                 batch.parents.cpu().pin_memory()]
+    elif cfg.temperature == 0:  # greedy: the draft logits are not an input
+        host = [batch.ar.cpu().pin_memory(), batch.ids.cpu().pin_memory()]
     else:
         host = [batch.ar.cpu().pin_memory(), batch.draft.cpu().pin_memory(),
                 batch.ids.cpu().pin_memory()]
@@ -433,9 +435,13 @@ def measure_e2e(psi, cfg, batch, seq_ids, ws, K, dev, pg, world):
     def step(k):
         for d, h in zip(dev_bufs, host):
             d.copy_(h, non_blocking=True)
-        b = (psi_inputs.TreeBatch(*dev_bufs, None) if is_tree else
-             psi_inputs.LinearBatch(dev_bufs[0], dev_bufs[1], dev_bufs[2], cfg.temperature,
-                                    cfg.top_p))
+        if is_tree:
+            b = psi_inputs.TreeBatch(*dev_bufs, None)
+        elif cfg.temperature == 0:
+            b = psi_inputs.LinearBatch(dev_bufs[0], None, dev_bufs[1], cfg.temperature, cfg.top_p)
+        else:
+            b = psi_inputs.LinearBatch(dev_bufs[0], dev_bufs[1], dev_bufs[2], cfg.temperature,
+                                       cfg.top_p)
         o = call_verify(psi, cfg, b, k, seq_ids, ws, out)
         res_host[0].copy_(o.tokens, non_blocking=True)
         res_host[1].copy_(o.path_len if is_tree else o.n_emitted, non_blocking=True)
