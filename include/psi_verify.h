@@ -32,9 +32,9 @@
  *    device uint32 that the caller zeroes; NULL = not reported).  The
  *    kernels always run to completion: they never trap, spin or hang.
  *  - Logits are bfloat16 or float32, row-major; `*_row_stride` is the
- *    distance between consecutive rows in ELEMENTS (>= V).  Rows whose
- *    start is 16-byte aligned take the bulk-copy path, others a plain-load
- *    path; both give the same results.
+ *    distance between consecutive rows in ELEMENTS (>= V).  Sampled rows
+ *    whose start is 16-byte aligned take the streaming path, others the
+ *    cluster path; both give the same results.
  *  - Randomness: the acceptance uniform of row i and the correction/bonus
  *    uniform of the emitting row are a counter-based hash of
  *    (seed, sequence id, step, row, purpose), so a step replays exactly from
