@@ -236,6 +236,55 @@ __device__ __forceinline__ void append_candidates(uint32_t mask, const uint4 &w,
   }
 }
 
+// Appends the candidates of two vectors per lane (masks m0, m1) with one
+// warp scan; every lane of the warp takes part.
+template <typename Bits>
+__device__ __forceinline__ void append_candidates2(uint32_t m0, const uint4 &w0, int32_t j0,
+                                                   uint32_t m1, const uint4 &w1, int32_t j1,
+                                                   int *s_cand, uint64_t *dst) {
+  constexpr int VEC = Elem<Bits>::kVec;
+  const int lane = threadIdx.x & 31;
+  const int c = __popc(m0) + __popc(m1);
+  int incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+  if (total == 0) return;
+  int base = 0;
+  if (lane == 31) base = atomicAdd(s_cand, total);
+  int pos = __shfl_sync(0xFFFFFFFFu, base, 31) + incl - c;
+  while (m0) {
+    const int q = __ffs(m0) - 1;
+    m0 &= m0 - 1;
+    if (pos < kCandCap) dst[pos] = ((uint64_t)vec_elem<Bits>(w0, q) << 32) | (uint32_t)(j0 * VEC + q);
+    ++pos;
+  }
+  while (m1) {
+    const int q = __ffs(m1) - 1;
+    m1 &= m1 - 1;
+    if (pos < kCandCap) dst[pos] = ((uint64_t)vec_elem<Bits>(w1, q) << 32) | (uint32_t)(j1 * VEC + q);
+    ++pos;
+  }
+}
+
+// Sum of exp2(x * coef + shift) over the elements of `w` selected by `mask`
+// (fixed order; every selected term <= 1).
+template <typename Bits>
+__device__ __forceinline__ float masked_exp_sum(const uint4 &w, uint32_t mask, float coef,
+                                                float shift) {
+  constexpr int VEC = Elem<Bits>::kVec;
+  float sum = 0.f;
+#pragma unroll
+  for (int q = 0; q < VEC; ++q) {
+    const float e = fast_exp2(fmaf(Elem<Bits>::to_float(vec_elem<Bits>(w, q)), coef, shift));
+    sum += ((mask >> q) & 1u) ? e : 0.f;
+  }
+  return sum;
+}
+
 // ---------------------------------------------------------------------------
 // row_scan
 // ---------------------------------------------------------------------------
@@ -475,30 +524,31 @@ __global__ void __launch_bounds__(kThreads, 2) row_scan_kernel(const __grid_cons
     }
     z_t += (acc_a.x + acc_a.y) + (acc_b.x + acc_b.y);
     // parked vectors: elements above the final threshold are candidates, the
-    // rest of what their batch masked goes to the fixed-point sum (each term
-    // <= 1: order-free)
+    // rest of what their batch masked goes to the 2^31 fixed-point sum (one
+    // rounded fp32 sum per vector, <= 8; at most 4096 of them: order-free,
+    // no overflow)
     const int n_flag = s_nflag;
     const int nf = min(n_flag, kRing);
     unsigned long long dsum = 0ull;
-    for (int b = 0; b < nf; b += kThreads) {
-      const int e = b + tid;
-      uint32_t cmask = 0u;
-      uint4 w = neg;
-      int32_t j = 0;
-      if (e < nf) {
-        w = fring[e];
-        const uint32_t tag = fidx[e];
-        j = (int32_t)(tag & 0xFFFFu);
-        cmask = above_bits<Bits>(w, thf);
-        uint32_t dmask = above_bits<Bits>(w, s_thr[tag >> 16]) & ~cmask;
-        while (dmask) {
-          const int q = __ffs(dmask) - 1;
-          dmask &= dmask - 1;
-          const float x = Elem<Bits>::to_float(vec_elem<Bits>(w, q));
-          dsum += __float2uint_rn(fast_exp2(fmaf(x, coef, shift)) * kFix31F);
+    // two parked vectors per thread per step: more shared-memory loads and
+    // exponentials in flight, one warp scan for both appends
+    for (int b = 0; b < nf; b += 2 * kThreads) {
+      uint32_t cm[2] = {0u, 0u};
+      uint4 w[2] = {neg, neg};
+      int32_t j[2] = {0, 0};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int e = b + h * kThreads + tid;
+        if (e < nf) {
+          w[h] = fring[e];
+          const uint32_t tag = fidx[e];
+          j[h] = (int32_t)(tag & 0xFFFFu);
+          cm[h] = above_bits<Bits>(w[h], thf);
+          const uint32_t dm = above_bits<Bits>(w[h], s_thr[tag >> 16]) & ~cm[h];
+          if (dm) dsum += __float2ull_rn(masked_exp_sum<Bits>(w[h], dm, coef, shift) * kFix31F);
         }
       }
-      append_candidates<Bits>(cmask, w, j, &s_cand, dst);
+      append_candidates2<Bits>(cm[0], w[0], j[0], cm[1], w[1], j[1], &s_cand, dst);
     }
     const double zs = warp_sum_any((double)z_t);
     const unsigned long long ds = warp_sum_any(dsum);
