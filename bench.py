@@ -195,11 +195,49 @@ def make_inputs(cfg, device, rank):
 
 
 def call_verify(psi, cfg, batch, step, seq_ids, ws, out):
+    """One verify step as a server calls it: tokens and counts only (no p / q
+    diagnostics), which lets the sampled path read rows in early-exit rounds."""
     if isinstance(cfg, psi_inputs.TreeConfig):
         return psi.verify_tree_greedy(batch.ar, batch.node_tokens, batch.parents, workspace=ws,
                                       out=out)
     return psi.verify_linear(batch.ar, batch.draft, batch.ids, cfg.temperature, cfg.top_p,
-                             seed=cfg.seed, step=step, seq_ids=seq_ids, workspace=ws, out=out)
+                             seed=cfg.seed, step=step, seq_ids=seq_ids, want_probs=False,
+                             workspace=ws, out=out)
+
+
+def sampled_rounds(cfg):
+    """Position rounds of the sampled path's early exit: [(first, end), ...]."""
+    rs = 3  # PSI_ROUND_POSITIONS
+    return [(i, min(cfg.B + 1, i + rs)) for i in range(0, cfg.B + 1, rs)]
+
+
+def rows_in_round(cfg, r):
+    i0, i1 = r
+    return (i1 - i0) + (min(i1, cfg.B) - i0)  # AR rows + draft rows (none for the bonus row)
+
+
+def main_launch_bytes(cfg) -> int:
+    """Algorithmic bytes of one launch of the timed main kernel: the first
+    round's row scan for the sampled path (every sequence's rows of
+    positions 0..2), the argmax of every AR row for the greedy paths."""
+    if isinstance(cfg, psi_inputs.TreeConfig) or cfg.temperature == 0:
+        return algorithmic_bytes(cfg)
+    es = 4 if cfg.dtype == "f32" else 2
+    return cfg.N * rows_in_round(cfg, sampled_rounds(cfg)[0]) * cfg.V * es
+
+
+def rows_read(cfg, n_emitted) -> int:
+    """Logit rows the sampled path read for these results: a sequence takes
+    part in the rounds up to the one holding its emitting position."""
+    rounds = sampled_rounds(cfg)
+    total = 0
+    for n in n_emitted:
+        L = int(n) - 1
+        for r in rounds:
+            total += rows_in_round(cfg, r)
+            if L < r[1]:
+                break
+    return total
 
 
 def units(cfg) -> int:
@@ -251,7 +289,10 @@ def config_block(cfg, name, world):
         c.update(batch=cfg.N, tree_nodes=cfg.M, vocab=cfg.V, depth=cfg.depth, width=cfg.width)
     else:
         c.update(batch=cfg.N, block=cfg.B, vocab=cfg.V, temperature=cfg.temperature,
-                 top_p=cfg.top_p, logits_dtype=cfg.dtype)
+                 top_p=cfg.top_p, logits_dtype=cfg.dtype,
+                 outputs="tokens and counts (no p/q diagnostics)")
+        if cfg.temperature > 0:
+            c.update(schedule="early-exit rounds of 3 positions; roofline = first round's row scan")
     c.update(global_batch=cfg.N * world, parallelism=f"batch-sharded x{world} (no collective)",
              l2="inputs larger than L2 (no flush needed)",
              inputs="seeded synthetic logits resident in HBM")
@@ -357,7 +398,13 @@ def main():
     ms_per_step = elapsed_ms / K
     blocks = units(cfg) * world * K
     value = blocks / (elapsed_ms / 1000.0)
-    alg = algorithmic_bytes(cfg)
+    alg = main_launch_bytes(cfg)
+    formula = algorithmic_bytes(cfg)
+    es = 4 if getattr(cfg, "dtype", "bf16") == "f32" else 2
+    if is_tree or cfg.temperature == 0:
+        read = formula
+    else:
+        read = rows_read(cfg, out.n_emitted.cpu().numpy()) * cfg.V * es
     peak, peak_kind = hbm_peak()
     achieved = alg / (main_ms / 1000.0) / 1e9
     kernel = "psi_tree_argmax" if is_tree else (
@@ -377,16 +424,19 @@ def main():
 
     if rank == 0:
         # our kernels per call: argmax + emit (greedy), argmax + tree walk,
-        # or row_scan, unit, their second passes, two cluster list launches
-        # and fast_emit (sampled); the memset of the list counters is not ours
-        launches_per_step = 2 if (is_tree or cfg.temperature == 0) else 7
+        # or per early-exit round list building, row scan, unit finish and
+        # their second passes, then two cluster list launches and fast_emit
+        launches_per_step = 2 if (is_tree or cfg.temperature == 0) else \
+            5 * len(sampled_rounds(cfg)) + 3
         line = {
             "metric": METRIC, "value": value, "unit": "blocks/s", "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if getattr(cfg, "dtype", "bf16") == "bf16" else "f32",
             "data": "synthetic", "config": config_block(cfg, name, world),
-            "logits_gbs": alg * world / (elapsed_ms / K / 1000.0) / 1e9,
+            "formula_bytes_per_step": formula * world,
+            "bytes_read_per_step": read * world,
+            "read_gbs": read * world / (elapsed_ms / K / 1000.0) / 1e9,
             "roofline": {"kernel": kernel, "bound": "hbm", "achieved": achieved, "peak": peak,
                          "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
                          "algorithmic_bytes_per_launch": alg, "launch_ms": main_ms,

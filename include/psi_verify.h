@@ -83,6 +83,9 @@ typedef enum psi_dtype { PSI_DTYPE_F32 = 0, PSI_DTYPE_BF16 = 1 } psi_dtype;
 #define PSI_MAX_B 32
 #define PSI_MAX_V 393216
 #define PSI_MAX_TREE_NODES 4096
+/* Positions per early-exit round of the sampled linear verify (see
+ * psi_verify_linear). */
+#define PSI_ROUND_POSITIONS 3
 
 /* Workspace needed by psi_verify_linear for these sizes (bytes, a multiple
  * of 256; 0 on invalid sizes).  The workspace needs no initialisation. */
@@ -119,6 +122,13 @@ size_t psi_verify_linear_workspace_bytes(int32_t N, int32_t B, int32_t V,
  * out_n_emitted int32 [N]: L + 1, in 1..B+1.
  * out_p_draft, out_q_draft  float [N][B] or NULL: p_i(x_i), q_i(x_i) after
  *               top-p (T > 0 only; not written when T == 0).
+ * Early exit (T > 0, both out_p_draft and out_q_draft NULL): rows after a
+ *   sequence's first rejection do not change its result, so positions are
+ *   verified in rounds of PSI_ROUND_POSITIONS (0-2, 3-5, ...) and a sequence
+ *   takes part in a round only if every draft of the earlier rounds was
+ *   accepted.  Tokens and counts are the same as with every row read; the
+ *   status bits then cover the rows that were read.  A caller asking for
+ *   p / q gets every row read.
  * Limits: 1 <= N, 1 <= B <= PSI_MAX_B, 1 <= V <= PSI_MAX_V, T >= 0 and
  *   finite, 0 < top_p <= 1.
  */
@@ -151,8 +161,8 @@ psi_status psi_verify_linear(const void *ar_logits, int64_t ar_row_stride,
  * the caller serialises them (one stream, or events between streams).
  * Returns PSI_ERR_UNSUPPORTED, without launching anything, when
  * psi_verify_linear_workspace_bytes for these sizes exceeds
- * PSI_NOALLOC_SCRATCH_BYTES (the sampled path needs about 24.6 KB per logit
- * row, N * (2B + 1) rows: e.g. N <= 20 at B = 8; the greedy path far less),
+ * PSI_NOALLOC_SCRATCH_BYTES (the sampled path needs about 16.4 KB per logit
+ * row, N * (2B + 1) rows: e.g. N <= 30 at B = 8; the greedy path far less),
  * and PSI_ERR_CUDA if the scratch address cannot be obtained.
  */
 #define PSI_NOALLOC_SCRATCH_BYTES 8388608u /* 8 MiB */

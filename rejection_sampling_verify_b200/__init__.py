@@ -44,6 +44,7 @@ PSI_MAX_B = 32
 PSI_MAX_V = 393216
 PSI_MAX_TREE_NODES = 4096
 PSI_NOALLOC_SCRATCH_BYTES = 8 << 20
+PSI_ROUND_POSITIONS = 3
 
 EXPORTED = (
     "psi_verify_linear_workspace_bytes",

@@ -43,6 +43,7 @@ constexpr float kFix31F = 2147483648.0f;  // 2^31: dropped masses (each <= 1)
 constexpr int kInFlight = 8;        // 16-byte loads per thread per batch
 constexpr int kRing = 4096;         // parked vectors per row (shared memory)
 constexpr int kListClusters = 16;
+constexpr int kCounters = 8;  // work-list counters (see FastArgs::counters)
 constexpr int32_t kWideBit = int32_t(1) << 30;  // second-pass row entry: wide window
 // Candidate window, in log2 units below the reference.  The first pass uses
 // a narrow window (13 units for top_p <= 0.95, wider as top_p approaches 1);
@@ -58,12 +59,19 @@ struct FastArgs {
   float win_narrow;    // window widths in logit units
   float win_wide;
   int use_top_p;
-  int pass;            // 1: every row / unit; 2: the listed ones
+  int pass;            // 1: a first scan / finish; 2: a rescan of rows that failed
+  const int32_t *rlist;   // rows to scan (nullptr: every row); entries may carry kWideBit
+  const int32_t *rcount;  // their number
+  const int32_t *ulist;   // units to finish (nullptr: every unit)
+  const int32_t *ucount;  // their number
+  int32_t *active;        // [N] sequence still verifying (early-exit rounds)
+  int32_t *round_rows;    // rows of the current round
+  int32_t *round_units;   // units of the current round
   UnitRecord *rec;     // [N*(B+1)]
   RowRecord *rowrec;   // [rows]
   uint64_t *cand;      // [rows][kCandCap]: (bits << 32) | vocabulary index
-  uint32_t *cmass;     // [rows][kCandCap]: masses of rows with more candidates than a warp keeps
-  int32_t *counters;   // [0] general units, [1] sample-mode units, [2] wide rows, [3] wide units
+  int32_t *counters;   // [0] general units, [1] sample-mode units, [2] wide rows, [3] wide units,
+                       // [4 + 2k], [5 + 2k] rows and units of round parity k
   int32_t *list_a;     // units for the general path
   int32_t *list_b;     // units whose draw needs the whole row
   int32_t *wide_rows;  // rows for the second scan (| kWideBit: wide window)
@@ -366,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 2) row_scan_kernel(const __grid_cons
   const int32_t nvec = V / VEC;  // whole 16-byte vectors per row
   const int32_t tail = V - nvec * VEC;
   const int32_t nb = nvec > 0 ? (nvec + BATCH - 1) / BATCH : 1;
-  const int64_t R = a.pass == 1 ? a.rows : (int64_t)a.counters[2];
+  const int64_t R = a.rlist ? (int64_t)*a.rcount : a.rows;
   if ((int64_t)blockIdx.x >= R) return;
   const int64_t my_rows = (R - 1 - (int64_t)blockIdx.x) / gridDim.x + 1;
   const float coef = a.coef;
@@ -381,11 +389,11 @@ __global__ void __launch_bounds__(kThreads, 2) row_scan_kernel(const __grid_cons
   // row of local index t, and its window (logit units)
   auto row_entry = [&](int64_t t, float &off) -> int64_t {
     const int64_t item = (int64_t)blockIdx.x + t * gridDim.x;
-    if (a.pass == 1) {
+    if (!a.rlist) {
       off = a.use_top_p ? a.win_narrow : 0.f;
       return item;
     }
-    const int32_t e = a.wide_rows[item];
+    const int32_t e = a.rlist[item];
     off = !a.use_top_p ? 0.f : (e & kWideBit) ? a.win_wide : a.win_narrow;
     return (int64_t)(e & ~kWideBit);
   };
@@ -592,9 +600,9 @@ __global__ void __launch_bounds__(kThreads, 2) row_scan_kernel(const __grid_cons
 }
 
 // ---------------------------------------------------------------------------
-// unit: one warp per (sequence, row) unit
+// unit: one CTA of two warps per (sequence, row) unit
 // ---------------------------------------------------------------------------
-// Statistics of one finished row (the same in every lane).
+// Statistics of one finished row (the same in every lane of its warp).
 struct RowFinal {
   float m;            // row maximum
   double zp;          // normaliser after top-p (Z without top-p)
@@ -607,25 +615,29 @@ constexpr int kFinOverflow = 1;   // candidates lost: rescan with the exact maxi
 constexpr int kFinCoverage = 2;   // the window holds less than top_p: rescan wider
 constexpr int kFinNonfinite = 4;  // NaN / +inf logit, or no finite logit
 
-constexpr int kUnitCtaWarps = 4;   // warps (units) per CTA
-constexpr int kWarpCand = 1024;    // candidates a warp keeps in shared memory
-constexpr double kFix31 = 2147483648.0;  // 2^31: candidate masses (each <= 1) in u32
+constexpr int kLoadChunk = 8;            // global loads per lane in flight together
+constexpr double kFix31 = 2147483648.0;  // 2^31: exact mass sums (each term <= 1) in u32 steps
 
 struct WarpScratch {
-  unsigned long long ent[kWarpCand];  // copy of the candidate list: (bits << 32) | vocabulary index
-  uint32_t mass[kWarpCand];           // 2^31 fixed-point masses; later the draw weights (float)
+  uint32_t key[kCandCap];  // candidate keys (order-preserving image of the logit)
+  uint32_t idx[kCandCap];  // vocabulary indices
+  float w[kCandCap];       // masses exp2((x - M) * log2(e)/T); later the draw weights
 };
 
+// A candidate's mass in 2^31 fixed point: the same function of the fp32 mass
+// wherever it is summed, so every exact sum is order-free.
+__device__ __forceinline__ uint32_t fixed31(float m) { return __float2uint_rn(m * kFix31F); }
+
 // Row maximum, Z, top-p threshold tau and renormaliser Z' of row r from its
-// record and candidate list.  The top-p threshold is the largest logit key t
-// whose suffix mass S(t) (every x with key >= t) reaches top_p * Z; only
-// candidates can be at or above it when the candidates hold at least top_p
-// of the mass.  Rows with more candidates than the warp's shared memory
-// holds read the global candidate list directly (it stays unchanged: a
-// second pass may finish the row again).
+// record and candidate list, by one warp.  The top-p threshold is the largest
+// logit key t whose suffix mass S(t) (every x with key >= t) reaches
+// top_p * Z: a binary search over the candidates' key range with fp32 partial
+// sums (a step may differ from exact arithmetic only within ~1e-7 of the
+// target), then S(tau) exactly in fixed point.  Only candidates can be at or
+// above tau when they hold at least top_p of the mass.  The global candidate
+// list stays unchanged, so a second pass may finish the row again.
 template <typename Bits>
-__device__ RowFinal finish_row(const FastArgs &a, int64_t r, WarpScratch *ws,
-                               unsigned long long *&ent, uint32_t *&mass) {
+__device__ RowFinal finish_row(const FastArgs &a, int64_t r, WarpScratch *ws) {
   const int lane = threadIdx.x & 31;
   RowFinal out;
   out.m = -INFINITY;
@@ -641,20 +653,30 @@ __device__ RowFinal finish_row(const FastArgs &a, int64_t r, WarpScratch *ws,
   }
   const int n = rs.n_cand;
   out.n = n;
-  unsigned long long *src = reinterpret_cast<unsigned long long *>(a.cand + r * (int64_t)kCandCap);
-  ent = n <= kWarpCand ? ws->ent : src;
-  mass = n <= kWarpCand ? ws->mass : a.cmass + r * (int64_t)kCandCap;
-  __syncwarp();  // the previous row's readers of the scratch are done
+  const unsigned long long *src =
+      reinterpret_cast<const unsigned long long *>(a.cand + r * (int64_t)kCandCap);
   float cm = -INFINITY;
   uint32_t kmax = 0u, kmin_inv = 0u;
-  for (int j = lane; j < n; j += 32) {
-    const unsigned long long e = src[j];
-    const uint32_t b = (uint32_t)(e >> 32);
-    cm = fmaxf(cm, Elem<Bits>::to_float(b));
-    const uint32_t key = Elem<Bits>::key(b);
-    if (ent != src) ent[j] = e;
-    kmax = max(kmax, key);
-    kmin_inv = max(kmin_inv, ~key);
+  for (int base = 0; base < n; base += 32 * kLoadChunk) {
+    unsigned long long e[kLoadChunk];
+#pragma unroll
+    for (int c = 0; c < kLoadChunk; ++c) {
+      const int j = base + 32 * c + lane;
+      e[c] = j < n ? __ldcg(src + j) : 0ull;
+    }
+#pragma unroll
+    for (int c = 0; c < kLoadChunk; ++c) {
+      const int j = base + 32 * c + lane;
+      if (j < n) {
+        const uint32_t b = (uint32_t)(e[c] >> 32);
+        cm = fmaxf(cm, Elem<Bits>::to_float(b));
+        const uint32_t key = Elem<Bits>::key(b);
+        ws->key[j] = key;
+        ws->idx[j] = (uint32_t)e[c];
+        kmax = max(kmax, key);
+        kmin_inv = max(kmin_inv, ~key);
+      }
+    }
   }
   const float M = fmaxf(rs.ref, warp_max(cm));
   kmax = warp_max_u32(kmax);
@@ -664,15 +686,12 @@ __device__ RowFinal finish_row(const FastArgs &a, int64_t r, WarpScratch *ws,
     out.status = kFinNonfinite;
     return out;
   }
-  // masses relative to M: fp32 exp2 rounded to 2^31 fixed point (order-free
-  // sums; relative error ~1e-6)
   const float shm = -M * a.coef;
   unsigned long long zin = 0ull;
   for (int j = lane; j < n; j += 32) {
-    const float x = Elem<Bits>::to_float((uint32_t)(ent[j] >> 32));
-    const uint32_t fx = __float2uint_rn(fast_exp2(fmaf(x, a.coef, shm)) * kFix31F);
-    mass[j] = fx;
-    zin += fx;
+    const float m = fast_exp2(fmaf(Elem<Bits>::to_float(key_to_bits<Bits>(ws->key[j])), a.coef, shm));
+    ws->w[j] = m;
+    zin += fixed31(m);
   }
   zin = warp_sum_any(zin);
   __syncwarp();
@@ -685,164 +704,194 @@ __device__ RowFinal finish_row(const FastArgs &a, int64_t r, WarpScratch *ws,
     return out;
   }
   if (!a.use_top_p) return out;
-  const unsigned long long target = (unsigned long long)ceil((double)a.s.top_p * Z * kFix31);
-  if (zin < target) {
+  const double target = (double)a.s.top_p * Z;
+  if ((double)zin / kFix31 < target) {
     out.status = kFinCoverage;
     return out;
   }
-  // binary search over [kmin, kmax]: S(kmin) = zin reaches the target
-  uint64_t lo = ~kmin_inv, hi = (uint64_t)kmax + 1;
-  unsigned long long s_lo = zin;
-  while (hi - lo > 1) {
-    const uint64_t mid = (lo + hi) >> 1;
-    unsigned long long part = 0ull;
+  const float target_f = (float)target;
+  uint32_t lo = ~kmin_inv, hi = kmax + 1u;  // S(lo) >= target
+  while (hi - lo > 1u) {
+    const uint32_t mid = lo + ((hi - lo) >> 1);
+    float part = 0.f;
     for (int j = lane; j < n; j += 32)
-      if (Elem<Bits>::key((uint32_t)(ent[j] >> 32)) >= mid) part += mass[j];
-    part = warp_sum_any(part);
-    if (part >= target) {
-      lo = mid;
-      s_lo = part;
-    } else {
-      hi = mid;
-    }
+      if (ws->key[j] >= mid) part += ws->w[j];
+    part = warp_sum(part);
+    if (part >= target_f) lo = mid;
+    else hi = mid;
   }
+  unsigned long long s_lo = 0ull;
+  for (int j = lane; j < n; j += 32)
+    if (ws->key[j] >= lo) s_lo += fixed31(ws->w[j]);
+  s_lo = warp_sum_any(s_lo);
   out.zp = (double)s_lo / kFix31;
-  out.tau_key = (uint32_t)lo;
-  out.tau_bits = key_to_bits<Bits>((uint32_t)lo);
+  out.tau_key = lo;
+  out.tau_bits = key_to_bits<Bits>(lo);
   return out;
 }
 
+struct UnitShared {
+  WarpScratch ws[2];  // warp 0: the p row, warp 1: the q row
+  RowFinal fq;
+  int need;
+};
+
 template <typename Bits>
-__global__ void __launch_bounds__(32 * kUnitCtaWarps) unit_kernel(const __grid_constant__ FastArgs a) {
-  __shared__ WarpScratch scratch[kUnitCtaWarps];
+__global__ void __launch_bounds__(64) unit_kernel(const __grid_constant__ FastArgs a) {
+  extern __shared__ __align__(16) unsigned char unit_smem[];  // one UnitShared (> 48 KB)
+  UnitShared &sh = *reinterpret_cast<UnitShared *>(unit_smem);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  WarpScratch *ws = &scratch[warp];
   const SampledArgs &s = a.s;
   const int32_t B = s.B, N = s.N, V = s.V;
-  const int64_t n_items = a.pass == 1 ? (int64_t)N * (B + 1) : (int64_t)a.counters[3];
-  for (int64_t item = (int64_t)blockIdx.x * kUnitCtaWarps + warp; item < n_items;
-       item += (int64_t)gridDim.x * kUnitCtaWarps) {
-    const int64_t unit = a.pass == 1 ? item : (int64_t)a.wide_units[item];
+  const int64_t n_items = a.ulist ? (int64_t)*a.ucount : (int64_t)N * (B + 1);
+  for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const int64_t unit = a.ulist ? (int64_t)a.ulist[item] : item;
     const int32_t n = (int32_t)(unit / (B + 1)), i = (int32_t)(unit % (B + 1));
     const bool has_q = i < B;
     const int64_t rp_idx = unit;
     const int64_t rq_idx = (int64_t)N * (B + 1) + (int64_t)n * B + i;
-    unsigned long long *ent = nullptr;
-    uint32_t *mass = nullptr;
-    RowFinal fq;
-    fq.m = -INFINITY;
-    fq.zp = 0.0;
-    fq.tau_bits = 0u;
-    fq.status = 0;
-    if (has_q) fq = finish_row<Bits>(a, rq_idx, ws, ent, mass);
-    const RowFinal fp = finish_row<Bits>(a, rp_idx, ws, ent, mass);
-    const int fail_q = fq.status & (kFinOverflow | kFinCoverage);
-    const int fail_p = fp.status & (kFinOverflow | kFinCoverage);
-    if (fail_q || fail_p) {
-      if (lane == 0) {
-        if (a.pass == 1) {  // rescan the failed rows, then finish the unit again
-          if (fail_q)
-            a.wide_rows[atomicAdd(&a.counters[2], 1)] =
-                (int32_t)rq_idx | ((fail_q & kFinCoverage) ? kWideBit : 0);
-          if (fail_p)
-            a.wide_rows[atomicAdd(&a.counters[2], 1)] =
-                (int32_t)rp_idx | ((fail_p & kFinCoverage) ? kWideBit : 0);
-          a.wide_units[atomicAdd(&a.counters[3], 1)] = (int32_t)unit;
-        } else {  // the general path verifies this unit (records included)
-          a.list_a[atomicAdd(&a.counters[0], 1)] = (int32_t)unit;
-        }
-      }
-      continue;
+    // the two rows in parallel
+    RowFinal fp;
+    if (warp == 0) {
+      fp = finish_row<Bits>(a, rp_idx, &sh.ws[0]);
+    } else if (has_q) {
+      const RowFinal f = finish_row<Bits>(a, rq_idx, &sh.ws[1]);
+      if (lane == 0) sh.fq = f;
+    } else if (lane == 0) {
+      sh.fq.m = -INFINITY;
+      sh.fq.zp = 0.0;
+      sh.fq.tau_bits = 0u;
+      sh.fq.tau_key = 0u;
+      sh.fq.n = 0;
+      sh.fq.status = 0;
     }
-    const uint64_t seq = s.seq_ids ? s.seq_ids[n] : (uint64_t)n;
-    const Bits *row_p = static_cast<const Bits *>(s.ar) + unit * s.ar_stride;
-    const Bits *row_q = has_q ? static_cast<const Bits *>(s.draft) + ((int64_t)n * B + i) * s.draft_stride
-                              : nullptr;
-    const float tau_p = Elem<Bits>::to_float(fp.tau_bits);
-    const float tau_q = Elem<Bits>::to_float(fq.tau_bits);
-
-    // ---- accept / reject the drafted token (lane 0)
-    int need = 1;
-    if (lane == 0) {
-      if (has_q) {
-        const int32_t x = s.ids[(int64_t)n * B + i];
-        double p = 0.0, q = 0.0;
-        const bool valid = x >= 0 && x < V;
-        if (valid) {
-          const float xp = Elem<Bits>::to_float(row_p[x]);
-          const float xq = Elem<Bits>::to_float(row_q[x]);
-          if (xp >= tau_p && fp.zp > 0.0) p = exact_exp2d(xp, fp.m, a.coef64) / fp.zp;
-          if (xq >= tau_q && fq.zp > 0.0) q = exact_exp2d(xq, fq.m, a.coef64) / fq.zp;
-        }
-        const double u = (double)uniform24(s.seed, seq, s.step, (uint64_t)i, PSI_PURPOSE_ACCEPT);
-        const int accept = (u * q < p) ? 1 : 0;
-        need = !accept;
-        if (s.out_p) s.out_p[(int64_t)n * B + i] = (float)p;
-        if (s.out_q) s.out_q[(int64_t)n * B + i] = (float)q;
-        a.rec[unit].accept = accept;
-        if (accept) a.rec[unit].token = -1;
-        if (!valid && s.dev_status) atomicOr(s.dev_status, PSI_DEV_BAD_TOKEN_ID);
-      } else {
-        a.rec[unit].accept = 1;
-      }
-      if (((fp.status | fq.status) & kFinNonfinite) && s.dev_status)
-        atomicOr(s.dev_status, PSI_DEV_NONFINITE);
-    }
-    need = __shfl_sync(0xFFFFFFFFu, need, 0);
-    if (!need) continue;
-    if (!a.use_top_p) {  // the draw needs whole rows: decided after the emit step
-      if (lane == 0) a.rec[unit].token = -2;
-      continue;
-    }
-
-    // ---- correction / bonus draw over p's nucleus (its candidates with key
-    // >= tau), inverse CDF in vocabulary order
-    float *w = reinterpret_cast<float *>(mass);
-    const int nc = (fp.status & kFinNonfinite) ? 0 : fp.n;
-    const float shp = -fp.m * a.coef, inv_zp = fp.zp > 0.0 ? (float)(1.0 / fp.zp) : 0.f;
-    const float shq = -fq.m * a.coef, inv_zq = fq.zp > 0.0 ? (float)(1.0 / fq.zp) : 0.f;
-    int32_t token = 0;
-    for (int pass = 0; pass < 2; ++pass) {
-      const bool p_only = !has_q || pass == 1;
-      double part = 0.0;
-      for (int j = lane; j < nc; j += 32) {
-        const unsigned long long e = ent[j];
-        const uint32_t bits = (uint32_t)(e >> 32);
-        float wj = 0.f;
-        if (Elem<Bits>::key(bits) >= fp.tau_key) {
-          wj = fast_exp2(fmaf(Elem<Bits>::to_float(bits), a.coef, shp)) * inv_zp;
-          if (!p_only) {
-            const float xq = Elem<Bits>::to_float(row_q[(uint32_t)e]);
-            const float qv = xq >= tau_q ? fast_exp2(fmaf(xq, a.coef, shq)) * inv_zq : 0.f;
-            wj = fmaxf(wj - qv, 0.f);
+    __syncthreads();
+    if (warp == 0) {
+      const RowFinal fq = sh.fq;
+      const int fail_q = fq.status & (kFinOverflow | kFinCoverage);
+      const int fail_p = fp.status & (kFinOverflow | kFinCoverage);
+      const uint64_t seq = s.seq_ids ? s.seq_ids[n] : (uint64_t)n;
+      const Bits *row_p = static_cast<const Bits *>(s.ar) + unit * s.ar_stride;
+      const Bits *row_q =
+          has_q ? static_cast<const Bits *>(s.draft) + ((int64_t)n * B + i) * s.draft_stride : nullptr;
+      const float tau_p = Elem<Bits>::to_float(fp.tau_bits);
+      const float tau_q = Elem<Bits>::to_float(fq.tau_bits);
+      int need = 0;
+      if (fail_q || fail_p) {
+        if (lane == 0) {
+          if (a.pass == 1) {  // rescan the failed rows, then finish the unit again
+            if (fail_q)
+              a.wide_rows[atomicAdd(&a.counters[2], 1)] =
+                  (int32_t)rq_idx | ((fail_q & kFinCoverage) ? kWideBit : 0);
+            if (fail_p)
+              a.wide_rows[atomicAdd(&a.counters[2], 1)] =
+                  (int32_t)rp_idx | ((fail_p & kFinCoverage) ? kWideBit : 0);
+            a.wide_units[atomicAdd(&a.counters[3], 1)] = (int32_t)unit;
+          } else {  // the general path verifies this unit (records included)
+            a.list_a[atomicAdd(&a.counters[0], 1)] = (int32_t)unit;
+            a.rec[unit].accept = -1;  // decided at the end; a later round treats it as accepted
           }
         }
-        w[j] = wj;
-        part += (double)wj;
-      }
-      const double W = warp_sum_any(part);
-      __syncwarp();
-      if (!(W > 0.0) && !p_only) continue;  // residual vanished: draw from p itself
-      if (W > 0.0) {
-        const double t = (double)uniform24(s.seed, seq, s.step, (uint64_t)i, PSI_PURPOSE_RESID) * W;
-        // smallest X with C(X) = sum of w over entries with index < X above t;
-        // the token is X - 1 (C(V) = W > t)
-        uint32_t lo = 0u, hi = (uint32_t)V;
-        while (hi - lo > 1) {
-          const uint32_t mid = (lo + hi) >> 1;
-          double c = 0.0;
-          for (int j = lane; j < nc; j += 32)
-            if ((uint32_t)ent[j] < mid) c += (double)w[j];
-          c = warp_sum_any(c);
-          if (c > t) hi = mid;
-          else lo = mid;
+      } else {
+        // ---- accept / reject the drafted token (lane 0, double precision)
+        need = 1;
+        if (lane == 0) {
+          if (has_q) {
+            const int32_t x = s.ids[(int64_t)n * B + i];
+            double p = 0.0, q = 0.0;
+            const bool valid = x >= 0 && x < V;
+            if (valid) {
+              const float xp = Elem<Bits>::to_float(row_p[x]);
+              const float xq = Elem<Bits>::to_float(row_q[x]);
+              if (xp >= tau_p && fp.zp > 0.0) p = exact_exp2d(xp, fp.m, a.coef64) / fp.zp;
+              if (xq >= tau_q && fq.zp > 0.0) q = exact_exp2d(xq, fq.m, a.coef64) / fq.zp;
+            }
+            const double u = (double)uniform24(s.seed, seq, s.step, (uint64_t)i, PSI_PURPOSE_ACCEPT);
+            const int accept = (u * q < p) ? 1 : 0;
+            need = !accept;
+            if (s.out_p) s.out_p[(int64_t)n * B + i] = (float)p;
+            if (s.out_q) s.out_q[(int64_t)n * B + i] = (float)q;
+            a.rec[unit].accept = accept;
+            if (accept) a.rec[unit].token = -1;
+            if (!valid && s.dev_status) atomicOr(s.dev_status, PSI_DEV_BAD_TOKEN_ID);
+          } else {
+            a.rec[unit].accept = 1;
+          }
+          if (((fp.status | fq.status) & kFinNonfinite) && s.dev_status)
+            atomicOr(s.dev_status, PSI_DEV_NONFINITE);
         }
-        token = (int32_t)lo;
+        need = __shfl_sync(0xFFFFFFFFu, need, 0);
+        if (need && !a.use_top_p) {  // the draw needs whole rows: decided after the emit step
+          if (lane == 0) a.rec[unit].token = -2;
+          need = 0;
+        }
       }
-      break;
+      if (need) {
+        // ---- correction / bonus draw over p's nucleus (its candidates with
+        // key >= tau), inverse CDF in vocabulary order
+        WarpScratch *ws = &sh.ws[0];
+        const int nc = (fp.status & kFinNonfinite) ? 0 : fp.n;
+        const float inv_zp = fp.zp > 0.0 ? (float)(1.0 / fp.zp) : 0.f;
+        const float shq = -fq.m * a.coef, inv_zq = fq.zp > 0.0 ? (float)(1.0 / fq.zp) : 0.f;
+        int32_t token = 0;
+        for (int pass = 0; pass < 2; ++pass) {
+          const bool p_only = !has_q || pass == 1;
+          float part = 0.f;
+          for (int base = 0; base < nc; base += 32 * kLoadChunk) {
+            // q logits of this chunk's nucleus entries, loads in flight together
+            uint32_t xqb[kLoadChunk];
+#pragma unroll
+            for (int c = 0; c < kLoadChunk; ++c) {
+              const int j = base + 32 * c + lane;
+              xqb[c] = 0u;
+              if (!p_only && j < nc && ws->key[j] >= fp.tau_key) xqb[c] = row_q[ws->idx[j]];
+            }
+#pragma unroll
+            for (int c = 0; c < kLoadChunk; ++c) {
+              const int j = base + 32 * c + lane;
+              if (j < nc) {
+                float wj = 0.f;
+                if (ws->key[j] >= fp.tau_key) {
+                  // p(v) from the stored mass (pass 0 only: it is overwritten)
+                  wj = (pass == 0 ? ws->w[j] : fast_exp2(fmaf(
+                                                    Elem<Bits>::to_float(key_to_bits<Bits>(ws->key[j])),
+                                                    a.coef, -fp.m * a.coef))) * inv_zp;
+                  if (!p_only) {
+                    const float xq = Elem<Bits>::to_float(xqb[c]);
+                    const float qv = xq >= tau_q ? fast_exp2(fmaf(xq, a.coef, shq)) * inv_zq : 0.f;
+                    wj = fmaxf(wj - qv, 0.f);
+                  }
+                }
+                ws->w[j] = wj;
+                part += wj;
+              }
+            }
+          }
+          const float W = warp_sum(part);
+          __syncwarp();
+          if (!(W > 0.f) && !p_only) continue;  // residual vanished: draw from p itself
+          if (W > 0.f) {
+            const float t = uniform24(s.seed, seq, s.step, (uint64_t)i, PSI_PURPOSE_RESID) * W;
+            // smallest X with C(X) = (weight of entries with index < X) > t;
+            // the token is X - 1 (C(V) = W > t)
+            uint32_t lo = 0u, hi = (uint32_t)V;
+            while (hi - lo > 1u) {
+              const uint32_t mid = (lo + hi) >> 1;
+              float c = 0.f;
+              for (int j = lane; j < nc; j += 32)
+                if (ws->idx[j] < mid) c += ws->w[j];
+              c = warp_sum(c);
+              if (c > t) hi = mid;
+              else lo = mid;
+            }
+            token = (int32_t)lo;
+          }
+          break;
+        }
+        if (lane == 0) a.rec[unit].token = token;
+      }
     }
-    if (lane == 0) a.rec[unit].token = token;
-    __syncwarp();  // the scratch is free for the next unit
+    __syncthreads();  // shared memory free for the next unit
   }
 }
 
@@ -886,39 +935,108 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 constexpr size_t kScanSmem = (sizeof(uint4) + sizeof(uint32_t)) * kRing;
 
+// ---------------------------------------------------------------------------
+// round_advance: one thread per sequence.  Early-exit rounds: round k covers
+// positions [k * PSI_ROUND_POSITIONS, (k + 1) * PSI_ROUND_POSITIONS) of B + 1.
+// A sequence takes part in round k when every drafted token of the earlier
+// rounds was accepted (a unit left to the general path counts as accepted:
+// its rows are then read although a rejection may make them unused).  The
+// kernel lists the round's rows and units, and resets the lists that the
+// round's finish step and the next round fill.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) round_advance_kernel(const __grid_constant__ FastArgs a,
+                                                            int k) {
+  const int32_t n = blockIdx.x * blockDim.x + threadIdx.x;
+  const SampledArgs &s = a.s;
+  const int32_t B = s.B, N = s.N;
+  if (n == 0) {
+    a.counters[2] = 0;  // this round's second-pass lists
+    a.counters[3] = 0;
+    a.counters[4 + 2 * ((k + 1) & 1)] = 0;  // the next round's lists
+    a.counters[5 + 2 * ((k + 1) & 1)] = 0;
+  }
+  if (n >= N) return;
+  const int32_t i0 = k * PSI_ROUND_POSITIONS;
+  const int32_t i1 = min(B + 1, i0 + PSI_ROUND_POSITIONS);
+  int act = 1;
+  if (k > 0) {
+    act = a.active[n];
+    const UnitRecord *r = a.rec + (int64_t)n * (B + 1);
+    for (int32_t i = i0 - PSI_ROUND_POSITIONS; act && i < i0; ++i)
+      if (i < B && r[i].accept == 0) act = 0;
+  }
+  a.active[n] = act;
+  if (!act || i0 >= i1) return;
+  int32_t *rc = a.counters + 4 + 2 * (k & 1);
+  const int32_t nu = i1 - i0;
+  const int32_t nd = min(i1, B) - i0;  // draft rows (the bonus row has none)
+  const int32_t su = atomicAdd(rc + 1, nu);
+  const int32_t sr = atomicAdd(rc, nu + nd);
+  for (int32_t i = i0; i < i1; ++i) {
+    const int32_t unit = n * (B + 1) + i;
+    a.round_units[su + (i - i0)] = unit;
+    a.round_rows[sr + (i - i0)] = unit;  // the AR row has the unit's index
+  }
+  for (int32_t i = i0; i < i0 + nd; ++i)
+    a.round_rows[sr + nu + (i - i0)] = N * (B + 1) + n * B + i;
+}
+
 template <typename Bits>
-cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, const KernelEvents &ev,
-                              cudaStream_t stream) {
+cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool early_exit,
+                              const KernelEvents &ev, cudaStream_t stream) {
   const int64_t units = (int64_t)fa.s.N * (fa.s.B + 1);
   const int64_t persistent = (int64_t)sm_count() * 2;
   const int64_t grid_scan = std::min<int64_t>(fa.rows, persistent);
+  const int64_t grid_unit = units;
   cudaError_t e;
   static bool configured = false;
   if (!configured) {
     if ((e = cudaFuncSetAttribute(row_scan_kernel<Bits>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kScanSmem)) != cudaSuccess)
       return e;
+    if ((e = cudaFuncSetAttribute(unit_kernel<Bits>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)sizeof(UnitShared))) != cudaSuccess)
+      return e;
     configured = true;
   }
   // the work-list counters of this call start at zero
-  if ((e = cudaMemsetAsync(fa.counters, 0, 4 * sizeof(int32_t), stream)) != cudaSuccess) return e;
-  if (ev.before && (e = cudaEventRecord(ev.before, stream)) != cudaSuccess) return e;
-  row_scan_kernel<Bits><<<(unsigned)grid_scan, kThreads, kScanSmem, stream>>>(fa);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (ev.after && (e = cudaEventRecord(ev.after, stream)) != cudaSuccess) return e;
-  unit_kernel<Bits><<<(unsigned)((units + kUnitCtaWarps - 1) / kUnitCtaWarps), 32 * kUnitCtaWarps, 0,
-                      stream>>>(fa);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  {
-    // second pass over the rows and units the first one could not settle
-    // (usually none: the CTAs find empty lists and exit)
-    FastArgs f2 = fa;
-    f2.pass = 2;
-    row_scan_kernel<Bits><<<(unsigned)grid_scan, kThreads, kScanSmem, stream>>>(f2);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    unit_kernel<Bits><<<(unsigned)std::min<int64_t>((units + kUnitCtaWarps - 1) / kUnitCtaWarps, persistent),
-                        32 * kUnitCtaWarps, 0, stream>>>(f2);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(fa.counters, 0, kCounters * sizeof(int32_t), stream)) != cudaSuccess)
+    return e;
+  // rows / units of one pass (first scan or rescan), then finish them
+  auto scan_and_finish = [&](const FastArgs &f, bool timed) -> cudaError_t {
+    cudaError_t err;
+    if (timed && ev.before && (err = cudaEventRecord(ev.before, stream)) != cudaSuccess) return err;
+    row_scan_kernel<Bits><<<(unsigned)grid_scan, kThreads, kScanSmem, stream>>>(f);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (timed && ev.after && (err = cudaEventRecord(ev.after, stream)) != cudaSuccess) return err;
+    const int64_t g = f.pass == 1 ? grid_unit : std::min<int64_t>(grid_unit, persistent);
+    unit_kernel<Bits><<<(unsigned)g, 64, sizeof(UnitShared), stream>>>(f);
+    return cudaGetLastError();
+  };
+  // the second pass over the rows and units a first pass could not settle
+  // (usually none: the CTAs find empty lists and exit)
+  FastArgs f2 = fa;
+  f2.pass = 2;
+  f2.rlist = fa.wide_rows;
+  f2.rcount = fa.counters + 2;
+  f2.ulist = fa.wide_units;
+  f2.ucount = fa.counters + 3;
+  if (!early_exit) {
+    if ((e = scan_and_finish(fa, true)) != cudaSuccess) return e;
+    if ((e = scan_and_finish(f2, false)) != cudaSuccess) return e;
+  } else {
+    const int rounds = (fa.s.B + 1 + PSI_ROUND_POSITIONS - 1) / PSI_ROUND_POSITIONS;
+    for (int k = 0; k < rounds; ++k) {
+      round_advance_kernel<<<(fa.s.N + 127) / 128, 128, 0, stream>>>(fa, k);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      FastArgs f1 = fa;
+      f1.rlist = fa.round_rows;
+      f1.rcount = fa.counters + 4 + 2 * (k & 1);
+      f1.ulist = fa.round_units;
+      f1.ucount = fa.counters + 5 + 2 * (k & 1);
+      if ((e = scan_and_finish(f1, k == 0)) != cudaSuccess) return e;
+      if ((e = scan_and_finish(f2, false)) != cudaSuccess) return e;
+    }
   }
   const psi_dtype dt = sizeof(Bits) == 2 ? PSI_DTYPE_BF16 : PSI_DTYPE_F32;
   SampledArgs sa = fa.s;
@@ -945,10 +1063,8 @@ FastLayout fast_layout(int32_t N, int32_t B) {
   off = align256(off + sizeof(RowRecord) * (size_t)rows);
   L.cand_off = off;
   off = align256(off + sizeof(uint64_t) * (size_t)rows * kCandCap);
-  L.cmass_off = off;
-  off = align256(off + sizeof(uint32_t) * (size_t)rows * kCandCap);
   L.counters_off = off;
-  off = align256(off + sizeof(int32_t) * 4);
+  off = align256(off + sizeof(int32_t) * kCounters);
   L.list_a_off = off;
   off = align256(off + sizeof(int32_t) * (size_t)units);
   L.list_b_off = off;
@@ -957,6 +1073,12 @@ FastLayout fast_layout(int32_t N, int32_t B) {
   off = align256(off + sizeof(int32_t) * (size_t)rows);
   L.wide_units_off = off;
   off = align256(off + sizeof(int32_t) * (size_t)units);
+  L.round_rows_off = off;
+  off = align256(off + sizeof(int32_t) * (size_t)rows);
+  L.round_units_off = off;
+  off = align256(off + sizeof(int32_t) * (size_t)units);
+  L.active_off = off;
+  off = align256(off + sizeof(int32_t) * (size_t)N);
   L.total = off;
   return L;
 }
@@ -987,15 +1109,24 @@ cudaError_t launch_sampled_fast(const SampledArgs &a, psi_dtype dtype, const Sam
   fa.rec = reinterpret_cast<UnitRecord *>(ws + L.rec_off);
   fa.rowrec = reinterpret_cast<RowRecord *>(ws + L.rows_off);
   fa.cand = reinterpret_cast<uint64_t *>(ws + L.cand_off);
-  fa.cmass = reinterpret_cast<uint32_t *>(ws + L.cmass_off);
   fa.counters = reinterpret_cast<int32_t *>(ws + L.counters_off);
   fa.list_a = reinterpret_cast<int32_t *>(ws + L.list_a_off);
   fa.list_b = reinterpret_cast<int32_t *>(ws + L.list_b_off);
   fa.wide_rows = reinterpret_cast<int32_t *>(ws + L.wide_rows_off);
   fa.wide_units = reinterpret_cast<int32_t *>(ws + L.wide_units_off);
+  fa.round_rows = reinterpret_cast<int32_t *>(ws + L.round_rows_off);
+  fa.round_units = reinterpret_cast<int32_t *>(ws + L.round_units_off);
+  fa.active = reinterpret_cast<int32_t *>(ws + L.active_off);
+  fa.rlist = nullptr;
+  fa.rcount = nullptr;
+  fa.ulist = nullptr;
+  fa.ucount = nullptr;
   fa.s.records = fa.rec;
-  if (dtype == PSI_DTYPE_BF16) return launch_fast_typed<uint16_t>(fa, plan, ev, stream);
-  return launch_fast_typed<uint32_t>(fa, plan, ev, stream);
+  // without p / q outputs only the rows up to each sequence's first rejection
+  // matter: verify in early-exit rounds
+  const bool early_exit = a.out_p == nullptr && a.out_q == nullptr;
+  if (dtype == PSI_DTYPE_BF16) return launch_fast_typed<uint16_t>(fa, plan, early_exit, ev, stream);
+  return launch_fast_typed<uint32_t>(fa, plan, early_exit, ev, stream);
 }
 
 }  // namespace psi

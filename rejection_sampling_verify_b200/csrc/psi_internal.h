@@ -104,8 +104,8 @@ constexpr int32_t kRowLost = 1;
 constexpr int kCandCap = 2048;     // candidates kept per row (global workspace)
 
 struct FastLayout {  // workspace carve-up of the streaming path
-  size_t rec_off, rows_off, cand_off, cmass_off, counters_off, list_a_off, list_b_off, wide_rows_off,
-      wide_units_off, total;
+  size_t rec_off, rows_off, cand_off, counters_off, list_a_off, list_b_off, wide_rows_off,
+      wide_units_off, round_rows_off, round_units_off, active_off, total;
 };
 FastLayout fast_layout(int32_t N, int32_t B);
 // False when the streaming path's row indices would not fit its lists.

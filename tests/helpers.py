@@ -18,14 +18,14 @@ NEAR_TIE = 1e-5
 
 
 def gpu_linear(batch: psi_inputs.LinearBatch, seed: int, step: int, seq_ids=None,
-               device="cuda"):
+               device="cuda", want_probs: bool = True):
     import rejection_sampling_verify_b200 as psi
     ar = batch.ar.to(device)
     draft = batch.draft.to(device) if batch.draft is not None else None
     ids = batch.ids.to(device)
     sid = None if seq_ids is None else torch.as_tensor(np.asarray(seq_ids, dtype=np.uint64).view(np.int64), device=device)
     r = psi.verify_linear(ar, draft, ids, batch.temperature, batch.top_p, seed=seed, step=step,
-                          seq_ids=sid)
+                          seq_ids=sid, want_probs=want_probs)
     torch.cuda.synchronize()
     out = dict(tokens=r.tokens.cpu().numpy(), n_emitted=r.n_emitted.cpu().numpy(),
                status=int(r.status.item()) & 0xFFFFFFFF)
