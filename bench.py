@@ -206,28 +206,31 @@ def call_verify(psi, cfg, batch, step, seq_ids, ws, out):
 
 
 def sampled_rounds(cfg):
-    """Position rounds of the sampled path's early exit: [(first, end), ...]."""
-    rs = 3  # PSI_ROUND_POSITIONS
+    """Position rounds of the linear paths' early exit: [(first, end), ...];
+    one round of every position below PSI_EARLY_EXIT_MIN_N sequences."""
+    rs = 3 if cfg.N >= 64 else cfg.B + 1  # PSI_ROUND_POSITIONS, PSI_EARLY_EXIT_MIN_N
     return [(i, min(cfg.B + 1, i + rs)) for i in range(0, cfg.B + 1, rs)]
 
 
 def rows_in_round(cfg, r):
+    """AR rows of the round's positions, plus draft rows when T > 0 (none for
+    the bonus row)."""
     i0, i1 = r
-    return (i1 - i0) + (min(i1, cfg.B) - i0)  # AR rows + draft rows (none for the bonus row)
+    return (i1 - i0) + ((min(i1, cfg.B) - i0) if cfg.temperature > 0 else 0)
 
 
 def main_launch_bytes(cfg) -> int:
     """Algorithmic bytes of one launch of the timed main kernel: the first
-    round's row scan for the sampled path (every sequence's rows of
-    positions 0..2), the argmax of every AR row for the greedy paths."""
-    if isinstance(cfg, psi_inputs.TreeConfig) or cfg.temperature == 0:
+    round's row scan (sampled) or argmax (greedy linear) over every
+    sequence's rows of positions 0..2; the argmax of every tree row."""
+    if isinstance(cfg, psi_inputs.TreeConfig):
         return algorithmic_bytes(cfg)
     es = 4 if cfg.dtype == "f32" else 2
     return cfg.N * rows_in_round(cfg, sampled_rounds(cfg)[0]) * cfg.V * es
 
 
 def rows_read(cfg, n_emitted) -> int:
-    """Logit rows the sampled path read for these results: a sequence takes
+    """Logit rows the linear paths read for these results: a sequence takes
     part in the rounds up to the one holding its emitting position."""
     rounds = sampled_rounds(cfg)
     total = 0
@@ -291,8 +294,8 @@ def config_block(cfg, name, world):
         c.update(batch=cfg.N, block=cfg.B, vocab=cfg.V, temperature=cfg.temperature,
                  top_p=cfg.top_p, logits_dtype=cfg.dtype,
                  outputs="tokens and counts (no p/q diagnostics)")
-        if cfg.temperature > 0:
-            c.update(schedule="early-exit rounds of 3 positions; roofline = first round's row scan")
+        c.update(schedule=("early-exit rounds of 3 positions; roofline = the first round's main kernel"
+                           if cfg.N >= 64 else "one pass over every row"))
     c.update(global_batch=cfg.N * world, parallelism=f"batch-sharded x{world} (no collective)",
              l2="inputs larger than L2 (no flush needed)",
              inputs="seeded synthetic logits resident in HBM")
@@ -401,7 +404,7 @@ def main():
     alg = main_launch_bytes(cfg)
     formula = algorithmic_bytes(cfg)
     es = 4 if getattr(cfg, "dtype", "bf16") == "f32" else 2
-    if is_tree or cfg.temperature == 0:
+    if is_tree:
         read = formula
     else:
         read = rows_read(cfg, out.n_emitted.cpu().numpy()) * cfg.V * es
@@ -423,11 +426,19 @@ def main():
                "sample": f"{n} of the {cfg.N} sequences of one step ({dt:.1f} s, single thread)"}
 
     if rank == 0:
-        # our kernels per call: argmax + emit (greedy), argmax + tree walk,
-        # or per early-exit round list building, row scan, unit finish and
-        # their second passes, then two cluster list launches and fast_emit
-        launches_per_step = 2 if (is_tree or cfg.temperature == 0) else \
-            5 * len(sampled_rounds(cfg)) + 3
+        # our kernels per call: argmax + tree walk; greedy linear: per
+        # early-exit round list building and argmax, then emit; sampled: per
+        # round list building, row scan, unit finish and their second passes,
+        # then two cluster list launches and fast_emit
+        rounds = 0 if is_tree else len(sampled_rounds(cfg))
+        if is_tree or (cfg.temperature == 0 and cfg.N < 64):
+            launches_per_step = 2
+        elif cfg.temperature == 0:  # per round: list building and argmax; then emit
+            launches_per_step = 2 * rounds + 1
+        elif cfg.N < 64:  # one pass: row scan, unit, their second passes, lists, emit
+            launches_per_step = 7
+        else:
+            launches_per_step = 5 * rounds + 3
         line = {
             "metric": METRIC, "value": value, "unit": "blocks/s", "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,

@@ -86,6 +86,9 @@ typedef enum psi_dtype { PSI_DTYPE_F32 = 0, PSI_DTYPE_BF16 = 1 } psi_dtype;
 /* Positions per early-exit round of the sampled linear verify (see
  * psi_verify_linear). */
 #define PSI_ROUND_POSITIONS 3
+/* Smallest batch that takes the early-exit rounds (smaller batches are
+ * latency-bound: one pass over every row is faster). */
+#define PSI_EARLY_EXIT_MIN_N 64
 
 /* Workspace needed by psi_verify_linear for these sizes (bytes, a multiple
  * of 256; 0 on invalid sizes).  The workspace needs no initialisation. */
@@ -122,13 +125,15 @@ size_t psi_verify_linear_workspace_bytes(int32_t N, int32_t B, int32_t V,
  * out_n_emitted int32 [N]: L + 1, in 1..B+1.
  * out_p_draft, out_q_draft  float [N][B] or NULL: p_i(x_i), q_i(x_i) after
  *               top-p (T > 0 only; not written when T == 0).
- * Early exit (T > 0, both out_p_draft and out_q_draft NULL): rows after a
- *   sequence's first rejection do not change its result, so positions are
- *   verified in rounds of PSI_ROUND_POSITIONS (0-2, 3-5, ...) and a sequence
- *   takes part in a round only if every draft of the earlier rounds was
- *   accepted.  Tokens and counts are the same as with every row read; the
- *   status bits then cover the rows that were read.  A caller asking for
- *   p / q gets every row read.
+ * Early exit (both out_p_draft and out_q_draft NULL, N >= PSI_EARLY_EXIT_MIN_N,
+ *   any T): rows after a
+ *   sequence's first rejection (or greedy mismatch) do not change its
+ *   result, so positions are verified in rounds of PSI_ROUND_POSITIONS
+ *   (0-2, 3-5, ...) and a sequence takes part in a round only if every
+ *   draft of the earlier rounds was accepted.  Tokens and counts are the
+ *   same as with every row read; the NONFINITE status bit then covers the
+ *   rows that were read.  A caller passing p / q buffers (for T == 0 they
+ *   are not written) gets every row read.
  * Limits: 1 <= N, 1 <= B <= PSI_MAX_B, 1 <= V <= PSI_MAX_V, T >= 0 and
  *   finite, 0 < top_p <= 1.
  */

@@ -93,9 +93,11 @@ size_t psi_verify_linear_workspace_bytes(int32_t N, int32_t B, int32_t V, psi_dt
     return 0;
   if (!(temperature >= 0.f) || !isfinite(temperature)) return 0;
   const int64_t rows = (int64_t)N * (B + 1);
-  if (temperature == 0.f) {
+  if (temperature == 0.f) {  // the every-row plan or the early-exit rounds, whichever is larger
     const psi::ArgmaxPlan plan = psi::plan_argmax(rows, V, elem_bytes(dtype));
-    return round256(sizeof(uint64_t) * (size_t)rows * plan.splits);
+    const size_t full = round256(sizeof(uint64_t) * (size_t)rows * plan.splits);
+    const size_t rounds = round256(psi::greedy_layout(N, B, V, elem_bytes(dtype)).total);
+    return full > rounds ? full : rounds;
   }
   (void)rows;
   return round256(psi::fast_layout(N, B).total);
@@ -139,6 +141,14 @@ psi_status psi_verify_linear(const void *ar_logits, int64_t ar_row_stride,
 
   const int64_t rows = (int64_t)N * (B + 1);
   cudaError_t e;
+  if (greedy && !out_p_draft && !out_q_draft && N >= PSI_EARLY_EXIT_MIN_N) {
+    // tokens only: rows after a sequence's first mismatch are never read
+    e = psi::launch_greedy_early_exit(ar_logits, ar_row_stride, dtype, draft_ids, N, B, V,
+                                      workspace, out_tokens, out_n_emitted, dev_status, g_events,
+                                      stream);
+    if (e != cudaSuccess) return cuda_fail(e, "greedy verify launch");
+    return PSI_OK;
+  }
   if (greedy) {
     const psi::ArgmaxPlan plan = psi::plan_argmax(rows, V, (int)es);
     uint64_t *partial = static_cast<uint64_t *>(workspace);

@@ -1124,7 +1124,7 @@ cudaError_t launch_sampled_fast(const SampledArgs &a, psi_dtype dtype, const Sam
   fa.s.records = fa.rec;
   // without p / q outputs only the rows up to each sequence's first rejection
   // matter: verify in early-exit rounds
-  const bool early_exit = a.out_p == nullptr && a.out_q == nullptr;
+  const bool early_exit = a.out_p == nullptr && a.out_q == nullptr && a.N >= PSI_EARLY_EXIT_MIN_N;
   if (dtype == PSI_DTYPE_BF16) return launch_fast_typed<uint16_t>(fa, plan, early_exit, ev, stream);
   return launch_fast_typed<uint32_t>(fa, plan, early_exit, ev, stream);
 }

@@ -15,6 +15,8 @@
 // Sources: "Uno Psi-Spec 是什麼？..." (alphalab.site), section "Linear 與 Tree
 // sampler" (tree verify); greedy linear verify is the temperature-0 case of
 // the section "Uno Psi-Spec 怎麼運作？完整走一次四個 Token".
+#include <algorithm>
+
 #include "psi_internal.h"
 
 namespace psi {
@@ -87,14 +89,19 @@ __device__ __forceinline__ uint32_t float_key(float v) {
     return Elem<Bits>::key(__float_as_uint(v));
 }
 
-// grid: rows * splits CTAs; CTA (row, s) covers [s*chunk, min(V, (s+1)*chunk)).
+// grid: rows * splits CTAs; CTA (item, s) covers [s*chunk, min(V, (s+1)*chunk))
+// of row `item`, or of row rlist[item] for the first *rcount items when a
+// row list is given (the other CTAs exit).
 template <typename Bits>
 __global__ void __launch_bounds__(kThreads) row_argmax_kernel(
     const Bits *__restrict__ logits, int64_t row_stride, int32_t V, int32_t splits,
-    int32_t chunk, uint64_t *__restrict__ partial, uint32_t *dev_status) {
+    int32_t chunk, uint64_t *__restrict__ partial, uint32_t *dev_status,
+    const int32_t *__restrict__ rlist, const int32_t *__restrict__ rcount) {
   constexpr int VEC = Elem<Bits>::kVec;
-  const int64_t row = blockIdx.x / splits;
+  const int64_t item = blockIdx.x / splits;
   const int32_t s = blockIdx.x % splits;
+  if (rlist && item >= *rcount) return;
+  const int64_t row = rlist ? (int64_t)rlist[item] : item;
   const Bits *r = logits + row * row_stride;
   const int32_t c0 = s * chunk;
   const int32_t c1 = min(V, c0 + chunk);
@@ -138,7 +145,7 @@ __global__ void __launch_bounds__(kThreads) row_argmax_kernel(
     uint64_t x = lane < kWarps ? red[lane] : 0ull;
     x = warp_max_u64(x);
     if (lane == 0) {
-      partial[blockIdx.x] = x;
+      partial[row * splits + s] = x;
       if (any_bad && dev_status) atomicOr(dev_status, PSI_DEV_NONFINITE);
     }
   }
@@ -248,6 +255,8 @@ __global__ void __launch_bounds__(kThreads) tree_walk_kernel(
 // ---------------------------------------------------------------------------
 // Host launchers.
 // ---------------------------------------------------------------------------
+size_t round_up256(size_t x) { return (x + 255) / 256 * 256; }
+
 ArgmaxPlan plan_argmax(int64_t rows, int32_t V, int elem_bytes) {
   ArgmaxPlan p;
   const int vec = 16 / elem_bytes;
@@ -274,12 +283,89 @@ cudaError_t launch_row_argmax(const void *logits, int64_t row_stride, psi_dtype 
   if (dtype == PSI_DTYPE_BF16)
     row_argmax_kernel<uint16_t><<<(unsigned)grid, kThreads, 0, stream>>>(
         static_cast<const uint16_t *>(logits), row_stride, V, plan.splits, plan.chunk, partial,
-        dev_status);
+        dev_status, nullptr, nullptr);
   else
     row_argmax_kernel<uint32_t><<<(unsigned)grid, kThreads, 0, stream>>>(
         static_cast<const uint32_t *>(logits), row_stride, V, plan.splits, plan.chunk, partial,
-        dev_status);
+        dev_status, nullptr, nullptr);
   return cudaGetLastError();
+}
+
+GreedyLayout greedy_layout(int32_t N, int32_t B, int32_t V, int elem_bytes) {
+  GreedyLayout L;
+  const int64_t rows = (int64_t)N * (B + 1);
+  L.plan = plan_argmax((int64_t)N * std::min(B + 1, PSI_ROUND_POSITIONS), V, elem_bytes);
+  size_t off = 0;
+  L.partial_off = off;
+  off = round_up256(off + sizeof(uint64_t) * (size_t)rows * L.plan.splits);
+  L.rows_off = off;
+  off = round_up256(off + sizeof(int32_t) * (size_t)N * PSI_ROUND_POSITIONS);
+  L.counters_off = off;
+  off = round_up256(off + sizeof(int32_t) * 4);
+  L.active_off = off;
+  off = round_up256(off + sizeof(int32_t) * (size_t)N);
+  L.total = off;
+  return L;
+}
+
+// One thread per sequence: the AR rows of early-exit round k (positions
+// [k * PSI_ROUND_POSITIONS, ...) of B + 1).  A sequence takes part when
+// every draft of the earlier rounds matched its row's argmax.
+__global__ void __launch_bounds__(128) greedy_advance_kernel(
+    const uint64_t *__restrict__ partial, int32_t splits, const int32_t *__restrict__ ids,
+    int32_t N, int32_t B, int k, int32_t *active, int32_t *round_rows, int32_t *counters) {
+  const int32_t n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n == 0) counters[(k + 1) & 1] = 0;  // the next round's list
+  if (n >= N) return;
+  const int32_t i0 = k * PSI_ROUND_POSITIONS;
+  const int32_t i1 = min(B + 1, i0 + PSI_ROUND_POSITIONS);
+  const int64_t row0 = (int64_t)n * (B + 1);
+  int act = 1;
+  if (k > 0) {
+    act = active[n];
+    for (int32_t i = i0 - PSI_ROUND_POSITIONS; act && i < i0; ++i)
+      if (i < B && ids[(int64_t)n * B + i] != argmax_of(partial, row0 + i, splits)) act = 0;
+  }
+  active[n] = act;
+  if (!act || i0 >= i1) return;
+  const int32_t at = atomicAdd(&counters[k & 1], i1 - i0);
+  for (int32_t i = i0; i < i1; ++i) round_rows[at + (i - i0)] = (int32_t)(row0 + i);
+}
+
+cudaError_t launch_greedy_early_exit(const void *logits, int64_t row_stride, psi_dtype dtype,
+                                     const int32_t *ids, int32_t N, int32_t B, int32_t V,
+                                     void *workspace, int32_t *out_tokens, int32_t *out_n,
+                                     uint32_t *dev_status, const KernelEvents &ev,
+                                     cudaStream_t stream) {
+  const GreedyLayout L = greedy_layout(N, B, V, dtype == PSI_DTYPE_F32 ? 4 : 2);
+  char *ws = static_cast<char *>(workspace);
+  uint64_t *partial = reinterpret_cast<uint64_t *>(ws + L.partial_off);
+  int32_t *rows = reinterpret_cast<int32_t *>(ws + L.rows_off);
+  int32_t *counters = reinterpret_cast<int32_t *>(ws + L.counters_off);
+  int32_t *active = reinterpret_cast<int32_t *>(ws + L.active_off);
+  const int64_t grid = (int64_t)N * std::min(B + 1, PSI_ROUND_POSITIONS) * L.plan.splits;
+  if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(counters, 0, 4 * sizeof(int32_t), stream)) != cudaSuccess) return e;
+  const int rounds = (B + 1 + PSI_ROUND_POSITIONS - 1) / PSI_ROUND_POSITIONS;
+  for (int k = 0; k < rounds; ++k) {
+    greedy_advance_kernel<<<(N + 127) / 128, 128, 0, stream>>>(partial, L.plan.splits, ids, N, B,
+                                                               k, active, rows, counters);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (k == 0 && ev.before && (e = cudaEventRecord(ev.before, stream)) != cudaSuccess) return e;
+    if (dtype == PSI_DTYPE_BF16)
+      row_argmax_kernel<uint16_t><<<(unsigned)grid, kThreads, 0, stream>>>(
+          static_cast<const uint16_t *>(logits), row_stride, V, L.plan.splits, L.plan.chunk,
+          partial, dev_status, rows, counters + (k & 1));
+    else
+      row_argmax_kernel<uint32_t><<<(unsigned)grid, kThreads, 0, stream>>>(
+          static_cast<const uint32_t *>(logits), row_stride, V, L.plan.splits, L.plan.chunk,
+          partial, dev_status, rows, counters + (k & 1));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (k == 0 && ev.after && (e = cudaEventRecord(ev.after, stream)) != cudaSuccess) return e;
+  }
+  return launch_greedy_emit(partial, L.plan.splits, ids, N, B, V, out_tokens, out_n, dev_status,
+                            stream);
 }
 
 cudaError_t launch_greedy_emit(const uint64_t *partial, int32_t splits, const int32_t *ids,

@@ -27,6 +27,20 @@ cudaError_t launch_greedy_emit(const uint64_t *partial, int32_t splits, const in
                                int32_t N, int32_t B, int32_t V, int32_t *out_tokens,
                                int32_t *out_n, uint32_t *dev_status, cudaStream_t stream);
 
+// Greedy linear verify in early-exit rounds (rows of positions after a
+// sequence's first mismatch are not read); workspace carve-up.
+struct GreedyLayout {
+  ArgmaxPlan plan;
+  size_t partial_off, rows_off, counters_off, active_off, total;
+};
+GreedyLayout greedy_layout(int32_t N, int32_t B, int32_t V, int elem_bytes);
+struct KernelEvents;
+cudaError_t launch_greedy_early_exit(const void *logits, int64_t row_stride, psi_dtype dtype,
+                                     const int32_t *ids, int32_t N, int32_t B, int32_t V,
+                                     void *workspace, int32_t *out_tokens, int32_t *out_n,
+                                     uint32_t *dev_status, const KernelEvents &ev,
+                                     cudaStream_t stream);
+
 cudaError_t launch_tree_walk(const uint64_t *partial, int32_t splits, const int32_t *node_tokens,
                              const int32_t *parents, int32_t N, int32_t M, int32_t V,
                              int32_t *out_path_nodes, int32_t *out_path_len,

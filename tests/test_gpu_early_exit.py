@@ -1,6 +1,6 @@
-"""Early-exit rounds of the sampled linear verify (no p / q outputs requested):
-tokens and counts must equal the oracle's and, exactly, the GPU's own
-every-row results on the same inputs."""
+"""Early-exit rounds of the linear verify (no p / q outputs requested, batch
+large enough): tokens and counts must equal the oracle's and, exactly, the
+GPU's own every-row results on the same inputs."""
 import numpy as np
 import pytest
 import torch
@@ -17,40 +17,51 @@ def _batch(ar, draft, ids, T, top_p):
     return psi_inputs.LinearBatch(ar, draft, ids, T, top_p)
 
 
-def _check(b, seed, step, seq_ids=None, oracle_rows=None):
-    early = gpu_linear(b, seed, step, seq_ids=seq_ids, want_probs=False)
-    full = gpu_linear(b, seed, step, seq_ids=seq_ids, want_probs=True)
+MIN_N = 64  # PSI_EARLY_EXIT_MIN_N
+
+
+def _check(b, seed, step, oracle_pick=8):
+    """Early exit against the every-row run (all sequences, exactly) and the
+    oracle (the first `oracle_pick` sequences, or all if None)."""
+    assert b.ar.shape[0] >= MIN_N
+    early = gpu_linear(b, seed, step, want_probs=False)
+    full = gpu_linear(b, seed, step, want_probs=True)
     assert np.array_equal(early["tokens"], full["tokens"])
     assert np.array_equal(early["n_emitted"], full["n_emitted"])
     assert early["status"] == full["status"]
-    if oracle_rows is None:
-        assert_linear_parity(early, oracle_linear(b, seed, step, seq_ids=seq_ids))
+    pick = np.arange(b.ar.shape[0] if oracle_pick is None else oracle_pick)
+    sub = _batch(b.ar[pick].cpu(), b.draft[pick].cpu(), b.ids[pick].cpu(), b.temperature,
+                 b.top_p)
+    o = oracle_linear(sub, seed, step, seq_ids=pick.astype(np.uint64))
+    gs = {k: (v[pick] if isinstance(v, np.ndarray) else v) for k, v in early.items()}
+    gs["status"] = early["status"] if oracle_pick is None else o["status"]
+    assert_linear_parity(gs, o)
     return early
 
 
 @pytest.mark.parametrize("index", range(3))
 def test_early_exit_nucleus_recipe(index):
     cfg = CFG["large_batch_nucleus"]
-    b = psi_inputs.linear_batch(cfg, device="cuda", N=16, index=index)
+    b = psi_inputs.linear_batch(cfg, device="cuda", N=MIN_N, index=index)
     g = _check(b, cfg.seed, index)
     # some sequences stop in the first round, some run past it
-    assert g["n_emitted"].min() <= 3 and g["n_emitted"].max() >= 1
+    assert g["n_emitted"].min() <= 3 and g["n_emitted"].max() > 3
 
 
 @pytest.mark.parametrize("B", [1, 2, 3, 4, 5, 8, 32])
 @pytest.mark.parametrize("top_p", [1.0, 0.8])
 def test_early_exit_block_sizes(B, top_p):
     rng = torch.Generator().manual_seed(100 + B)
-    N, V = 6, 5003
+    N, V = MIN_N, 5003
     ar = (1.2 * torch.randn(N, B + 1, V, generator=rng)).to(torch.bfloat16)
     draft = (ar[:, :B].float() + 0.2 * torch.randn(N, B, V, generator=rng)).to(torch.bfloat16)
     ids = psi_inputs.gumbel_max(draft, 1.0, rng)
-    _check(_batch(ar, draft, ids, 1.0, top_p), 9, B)
+    _check(_batch(ar, draft, ids, 1.0, top_p), 9, B, oracle_pick=None)
 
 
 def test_early_exit_single_stream_recipe():
     cfg = CFG["single_stream"]
-    b = psi_inputs.linear_batch(cfg, device="cuda", index=1)
+    b = psi_inputs.linear_batch(cfg, device="cuda", N=MIN_N, index=1)
     _check(b, cfg.seed, 4)
 
 
@@ -64,13 +75,13 @@ def test_early_exit_tiny_recipe_many_sequences():
                    axis=1).astype(np.int32)
     b = _batch(base.ar.expand(n, -1, -1).contiguous(), base.draft.expand(n, -1, -1).contiguous(),
                torch.tensor(ids), cfg.temperature, cfg.top_p)
-    _check(b, cfg.seed, 2)
+    _check(b, cfg.seed, 2, oracle_pick=None)
 
 
 def test_early_exit_rescanned_and_general_units():
     # rows whose top-p mass reaches below the first window (second scan)
     g = torch.Generator().manual_seed(21)
-    N, B, V = 3, 3, 20000
+    N, B, V = MIN_N, 3, 20000
     ar = torch.full((N, B + 1, V), -40.0)
     for n in range(N):
         for i in range(B + 1):
@@ -83,7 +94,8 @@ def test_early_exit_rescanned_and_general_units():
     _check(_batch(ar.cuda(), draft.cuda(), ids, 1.0, 0.95), 6, 0)
     # flat rows: every unit goes to the general path
     for top_p in (0.9, 1.0):
-        cfg = psi_inputs.LinearConfig("flat", 24, 4, 40000, "f32", 1.0, top_p, 31, 1, "tiny", 1.0)
+        cfg = psi_inputs.LinearConfig("flat", MIN_N, 4, 40000, "f32", 1.0, top_p, 31, 1, "tiny",
+                                      1.0)
         _check(psi_inputs.linear_batch(cfg, device="cuda"), 3, 1)
 
 
@@ -92,21 +104,68 @@ def test_early_exit_full_size_sampled():
     a sample checked against the oracle one by one."""
     cfg = CFG["large_batch_nucleus"]
     b = psi_inputs.linear_batch(cfg, device="cuda")
-    g = _check(b, cfg.seed, 7, oracle_rows=False)
-    pick = np.array([1, 64, 200, 255])
-    sub = _batch(b.ar[pick].cpu(), b.draft[pick].cpu(), b.ids[pick].cpu(), cfg.temperature,
-                 cfg.top_p)
-    o = oracle_linear(sub, cfg.seed, 7, seq_ids=pick.astype(np.uint64))
-    gs = {k: (v[pick] if isinstance(v, np.ndarray) else v) for k, v in g.items()}
-    gs["status"] = 0
-    assert_linear_parity(gs, o)
+    g = _check(b, cfg.seed, 7, oracle_pick=4)
     assert g["status"] == 0
+
+
+def test_small_batches_read_every_row():
+    """Below PSI_EARLY_EXIT_MIN_N sequences the tokens-only call is the
+    every-row pass (same results either way)."""
+    cfg = CFG["single_stream"]
+    b = psi_inputs.linear_batch(cfg, device="cuda", index=2)
+    early = gpu_linear(b, cfg.seed, 1, want_probs=False)
+    full = gpu_linear(b, cfg.seed, 1, want_probs=True)
+    assert np.array_equal(early["tokens"], full["tokens"])
+    assert_linear_parity(early, oracle_linear(b, cfg.seed, 1))
 
 
 def test_early_exit_deterministic():
     cfg = CFG["large_batch_nucleus"]
-    b = psi_inputs.linear_batch(cfg, device="cuda", N=32, index=5)
+    b = psi_inputs.linear_batch(cfg, device="cuda", N=MIN_N, index=5)
     r1 = gpu_linear(b, 1, 2, want_probs=False)
     r2 = gpu_linear(b, 1, 2, want_probs=False)
     assert np.array_equal(r1["tokens"], r2["tokens"])
     assert np.array_equal(r1["n_emitted"], r2["n_emitted"])
+
+
+def _greedy_raw(b, with_pq):
+    """Greedy verify through the C ABI; with_pq passes p / q buffers (which
+    T = 0 never writes) to ask for every row to be read."""
+    import rejection_sampling_verify_b200 as psi
+    N, B1, V = b.ar.shape
+    B = B1 - 1
+    code = psi.PSI_DTYPE_BF16 if b.ar.dtype == torch.bfloat16 else psi.PSI_DTYPE_F32
+    tok = torch.empty(N, B + 1, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(N, dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    pq = torch.zeros(2, N, B, device="cuda") if with_pq else None
+    ws_bytes = psi.psi_verify_linear_workspace_bytes(N, B, V, code, 0.0, 1.0)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    ids = b.ids.to("cuda")
+    r = psi.psi_verify_linear(b.ar.data_ptr(), V, 0, V, code, ids.data_ptr(), N, B, V, 0.0, 1.0,
+                              0, 0, 0, tok.data_ptr(), cnt.data_ptr(),
+                              pq[0].data_ptr() if with_pq else 0,
+                              pq[1].data_ptr() if with_pq else 0, st.data_ptr(), ws.data_ptr(),
+                              ws_bytes, 0)
+    assert r == psi.PSI_OK, psi.psi_last_error()
+    torch.cuda.synchronize()
+    return tok.cpu().numpy(), cnt.cpu().numpy(), int(st.item())
+
+
+@pytest.mark.parametrize("B", [1, 2, 3, 5, 16, 32])
+def test_greedy_early_exit_equals_every_row(B):
+    b = psi_inputs.linear_batch(psi_inputs.LinearConfig("g", MIN_N, B, 30011, "bf16", 0.0, 1.0,
+                                                        B, 1, "zipf", 0.6), device="cuda")
+    early, full = _greedy_raw(b, False), _greedy_raw(b, True)
+    for x, y in zip(early, full):
+        assert np.array_equal(x, y)
+    o = oracle_linear(b, 0, 0)
+    assert np.array_equal(early[0], o["tokens"]) and np.array_equal(early[1], o["n_emitted"])
+
+
+def test_greedy_early_exit_full_size():
+    cfg = CFG["max_batch_greedy"]
+    b = psi_inputs.linear_batch(cfg, device="cuda")
+    early, full = _greedy_raw(b, False), _greedy_raw(b, True)
+    for x, y in zip(early, full):
+        assert np.array_equal(x, y)
