@@ -450,14 +450,19 @@ __global__ void __launch_bounds__(kThreads, 2) row_scan_kernel(const __grid_cons
   float off = 0.f, ref = -INFINITY, shift = -INFINITY, z_t = 0.f;
   float2 acc_a = make_float2(0.f, 0.f), acc_b = make_float2(0.f, 0.f);
 
-  auto consume = [&](const uint4(&buf)[U]) {
+  auto consume = [&](const uint4(&buf)[U], const uint4(&nxt)[U]) {
     if (ck == 0) {
-      // start of a row: the first reference is the first batch's maximum
+      // start of a row: the first reference is the maximum of its first two
+      // batches (the second one's loads are already in flight)
       r = row_entry(ct, off);
       row = row_ptr<Bits>(a, r);
       uint32_t vm = sizeof(Bits) == 2 ? 0xFF80FF80u : 0xFF800000u;
 #pragma unroll
       for (int u = 0; u < U; ++u) vec_max_into<Bits>(buf[u], vm);
+      if (nb > 1) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) vec_max_into<Bits>(nxt[u], vm);
+      }
       float mx = vm_to_float<Bits>(vm);
       if (tid < tail) {
         const float x = Elem<Bits>::to_float(row[(int64_t)nvec * VEC + tid]);
@@ -592,10 +597,10 @@ __global__ void __launch_bounds__(kThreads, 2) row_scan_kernel(const __grid_cons
   load(b0);
   for (int64_t g = 0; g < total; g += 2) {
     load(b1);
-    consume(b0);
+    consume(b0, b1);
     if (g + 1 >= total) break;
     load(b0);
-    consume(b1);
+    consume(b1, b0);
   }
 }
 
