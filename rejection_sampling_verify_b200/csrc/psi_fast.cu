@@ -620,13 +620,17 @@ constexpr int kFinOverflow = 1;   // candidates lost: rescan with the exact maxi
 constexpr int kFinCoverage = 2;   // the window holds less than top_p: rescan wider
 constexpr int kFinNonfinite = 4;  // NaN / +inf logit, or no finite logit
 
-constexpr int kLoadChunk = 8;            // global loads per lane in flight together
+constexpr int kLoadChunk = 16;           // global loads per lane in flight together
+constexpr int kQChunk = 16;              // q loads per lane in flight together
+constexpr int kRegCand = 16;             // candidates per lane a search keeps in registers
 constexpr double kFix31 = 2147483648.0;  // 2^31: exact mass sums (each term <= 1) in u32 steps
 
 struct WarpScratch {
-  uint32_t key[kCandCap];  // candidate keys (order-preserving image of the logit)
-  uint32_t idx[kCandCap];  // vocabulary indices
-  float w[kCandCap];       // masses exp2((x - M) * log2(e)/T); later the draw weights
+  uint32_t key[kCandCap];  // candidate keys (order-preserving image of the logit); later the
+                           // nucleus masses
+  uint32_t idx[kCandCap];  // vocabulary indices; later the nucleus indices
+  uint32_t m[kCandCap];    // 2^31 fixed-point masses exp2((x - M) * log2(e)/T); later the
+                           // draw weights
 };
 
 // A candidate's mass in 2^31 fixed point: the same function of the fp32 mass
@@ -694,9 +698,10 @@ __device__ RowFinal finish_row(const FastArgs &a, int64_t r, WarpScratch *ws) {
   const float shm = -M * a.coef;
   unsigned long long zin = 0ull;
   for (int j = lane; j < n; j += 32) {
-    const float m = fast_exp2(fmaf(Elem<Bits>::to_float(key_to_bits<Bits>(ws->key[j])), a.coef, shm));
-    ws->w[j] = m;
-    zin += fixed31(m);
+    const uint32_t m =
+        fixed31(fast_exp2(fmaf(Elem<Bits>::to_float(key_to_bits<Bits>(ws->key[j])), a.coef, shm)));
+    ws->m[j] = m;
+    zin += m;
   }
   zin = warp_sum_any(zin);
   __syncwarp();
@@ -709,26 +714,51 @@ __device__ RowFinal finish_row(const FastArgs &a, int64_t r, WarpScratch *ws) {
     return out;
   }
   if (!a.use_top_p) return out;
-  const double target = (double)a.s.top_p * Z;
-  if ((double)zin / kFix31 < target) {
+  const unsigned long long target = (unsigned long long)ceil((double)a.s.top_p * Z * kFix31);
+  if (zin < target) {
     out.status = kFinCoverage;
     return out;
   }
-  const float target_f = (float)target;
-  uint32_t lo = ~kmin_inv, hi = kmax + 1u;  // S(lo) >= target
-  while (hi - lo > 1u) {
-    const uint32_t mid = lo + ((hi - lo) >> 1);
-    float part = 0.f;
-    for (int j = lane; j < n; j += 32)
-      if (ws->key[j] >= mid) part += ws->w[j];
-    part = warp_sum(part);
-    if (part >= target_f) lo = mid;
-    else hi = mid;
+  // binary search over [kmin, kmax] with exact integer sums (order-free):
+  // S(kmin) = zin reaches the target
+  uint32_t lo = ~kmin_inv, hi = kmax + 1u;
+  unsigned long long s_lo = zin;
+  if (n <= 32 * kRegCand) {
+    uint32_t kr[kRegCand], mr[kRegCand];  // the row's candidates in registers
+#pragma unroll
+    for (int c = 0; c < kRegCand; ++c) {
+      const int j = lane + 32 * c;
+      kr[c] = j < n ? ws->key[j] : 0u;
+      mr[c] = j < n ? ws->m[j] : 0u;
+    }
+    while (hi - lo > 1u) {
+      const uint32_t mid = lo + ((hi - lo) >> 1);
+      unsigned long long part = 0ull;
+#pragma unroll
+      for (int c = 0; c < kRegCand; ++c) part += kr[c] >= mid ? mr[c] : 0u;
+      part = warp_sum_any(part);
+      if (part >= target) {
+        lo = mid;
+        s_lo = part;
+      } else {
+        hi = mid;
+      }
+    }
+  } else {
+    while (hi - lo > 1u) {
+      const uint32_t mid = lo + ((hi - lo) >> 1);
+      unsigned long long part = 0ull;
+      for (int j = lane; j < n; j += 32)
+        if (ws->key[j] >= mid) part += ws->m[j];
+      part = warp_sum_any(part);
+      if (part >= target) {
+        lo = mid;
+        s_lo = part;
+      } else {
+        hi = mid;
+      }
+    }
   }
-  unsigned long long s_lo = 0ull;
-  for (int j = lane; j < n; j += 32)
-    if (ws->key[j] >= lo) s_lo += fixed31(ws->w[j]);
-  s_lo = warp_sum_any(s_lo);
   out.zp = (double)s_lo / kFix31;
   out.tau_key = lo;
   out.tau_bits = key_to_bits<Bits>(lo);
@@ -833,61 +863,99 @@ __global__ void __launch_bounds__(64) unit_kernel(const __grid_constant__ FastAr
       }
       if (need) {
         // ---- correction / bonus draw over p's nucleus (its candidates with
-        // key >= tau), inverse CDF in vocabulary order
+        // key >= tau), inverse CDF in vocabulary order, exact integer sums
         WarpScratch *ws = &sh.ws[0];
         const int nc = (fp.status & kFinNonfinite) ? 0 : fp.n;
         const float inv_zp = fp.zp > 0.0 ? (float)(1.0 / fp.zp) : 0.f;
         const float shq = -fq.m * a.coef, inv_zq = fq.zp > 0.0 ? (float)(1.0 / fq.zp) : 0.f;
+        // compact the nucleus to the front, in candidate order: index in
+        // idx[], mass in key[] (reads of a group precede its writes, which
+        // land at or before the group)
+        const unsigned below = (1u << lane) - 1u;
+        int nn = 0;
+        for (int base = 0; base < nc; base += 32) {
+          const int j = base + lane;
+          const bool in = j < nc && ws->key[j] >= fp.tau_key;
+          uint32_t v = 0u, m = 0u;
+          if (in) {
+            v = ws->idx[j];
+            m = ws->m[j];
+          }
+          const unsigned bal = __ballot_sync(0xFFFFFFFFu, in);
+          __syncwarp();
+          if (in) {
+            const int d = nn + __popc(bal & below);
+            ws->idx[d] = v;
+            ws->key[d] = m;
+          }
+          nn += __popc(bal);
+        }
+        __syncwarp();
         int32_t token = 0;
         for (int pass = 0; pass < 2; ++pass) {
           const bool p_only = !has_q || pass == 1;
-          float part = 0.f;
-          for (int base = 0; base < nc; base += 32 * kLoadChunk) {
-            // q logits of this chunk's nucleus entries, loads in flight together
-            uint32_t xqb[kLoadChunk];
+          unsigned long long part = 0ull;
+          for (int base = 0; base < nn; base += 32 * kQChunk) {
+            uint32_t xqb[kQChunk];  // q logits of the chunk, loads in flight together
 #pragma unroll
-            for (int c = 0; c < kLoadChunk; ++c) {
+            for (int c = 0; c < kQChunk; ++c) {
               const int j = base + 32 * c + lane;
-              xqb[c] = 0u;
-              if (!p_only && j < nc && ws->key[j] >= fp.tau_key) xqb[c] = row_q[ws->idx[j]];
+              xqb[c] = (!p_only && j < nn) ? (uint32_t)row_q[ws->idx[j]] : 0u;
             }
 #pragma unroll
-            for (int c = 0; c < kLoadChunk; ++c) {
+            for (int c = 0; c < kQChunk; ++c) {
               const int j = base + 32 * c + lane;
-              if (j < nc) {
-                float wj = 0.f;
-                if (ws->key[j] >= fp.tau_key) {
-                  // p(v) from the stored mass (pass 0 only: it is overwritten)
-                  wj = (pass == 0 ? ws->w[j] : fast_exp2(fmaf(
-                                                    Elem<Bits>::to_float(key_to_bits<Bits>(ws->key[j])),
-                                                    a.coef, -fp.m * a.coef))) * inv_zp;
-                  if (!p_only) {
-                    const float xq = Elem<Bits>::to_float(xqb[c]);
-                    const float qv = xq >= tau_q ? fast_exp2(fmaf(xq, a.coef, shq)) * inv_zq : 0.f;
-                    wj = fmaxf(wj - qv, 0.f);
-                  }
+              if (j < nn) {
+                float pv = (float)ws->key[j] * (1.f / kFix31F) * inv_zp;
+                if (!p_only) {
+                  const float xq = Elem<Bits>::to_float(xqb[c]);
+                  const float qv = xq >= tau_q ? fast_exp2(fmaf(xq, a.coef, shq)) * inv_zq : 0.f;
+                  pv = fmaxf(pv - qv, 0.f);
                 }
-                ws->w[j] = wj;
+                const uint32_t wj = fixed31(fminf(pv, 1.f));
+                ws->m[j] = wj;
                 part += wj;
               }
             }
           }
-          const float W = warp_sum(part);
+          const unsigned long long W = warp_sum_any(part);
           __syncwarp();
-          if (!(W > 0.f) && !p_only) continue;  // residual vanished: draw from p itself
-          if (W > 0.f) {
-            const float t = uniform24(s.seed, seq, s.step, (uint64_t)i, PSI_PURPOSE_RESID) * W;
+          if (W == 0ull && !p_only) continue;  // residual vanished: draw from p itself
+          if (W > 0ull) {
+            // t = floor(u' * W) exactly (u' = k / 2^24)
+            const float u2 = uniform24(s.seed, seq, s.step, (uint64_t)i, PSI_PURPOSE_RESID);
+            const unsigned long long k = (unsigned long long)(u2 * 16777216.0f);
+            const unsigned long long t = (__umul64hi(k, W) << 40) | ((k * W) >> 24);
             // smallest X with C(X) = (weight of entries with index < X) > t;
             // the token is X - 1 (C(V) = W > t)
             uint32_t lo = 0u, hi = (uint32_t)V;
-            while (hi - lo > 1u) {
-              const uint32_t mid = (lo + hi) >> 1;
-              float c = 0.f;
-              for (int j = lane; j < nc; j += 32)
-                if (ws->idx[j] < mid) c += ws->w[j];
-              c = warp_sum(c);
-              if (c > t) hi = mid;
-              else lo = mid;
+            if (nn <= 32 * kRegCand) {
+              uint32_t ir[kRegCand], wr[kRegCand];
+#pragma unroll
+              for (int c = 0; c < kRegCand; ++c) {
+                const int j = lane + 32 * c;
+                ir[c] = j < nn ? ws->idx[j] : 0xFFFFFFFFu;
+                wr[c] = j < nn ? ws->m[j] : 0u;
+              }
+              while (hi - lo > 1u) {
+                const uint32_t mid = (lo + hi) >> 1;
+                unsigned long long c = 0ull;
+#pragma unroll
+                for (int q = 0; q < kRegCand; ++q) c += ir[q] < mid ? wr[q] : 0u;
+                c = warp_sum_any(c);
+                if (c > t) hi = mid;
+                else lo = mid;
+              }
+            } else {
+              while (hi - lo > 1u) {
+                const uint32_t mid = (lo + hi) >> 1;
+                unsigned long long c = 0ull;
+                for (int j = lane; j < nn; j += 32)
+                  if (ws->idx[j] < mid) c += ws->m[j];
+                c = warp_sum_any(c);
+                if (c > t) hi = mid;
+                else lo = mid;
+              }
             }
             token = (int32_t)lo;
           }
