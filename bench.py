@@ -206,10 +206,16 @@ def call_verify(psi, cfg, batch, step, seq_ids, ws, out):
 
 
 def sampled_rounds(cfg):
-    """Position rounds of the linear paths' early exit: [(first, end), ...];
-    one round of every position below PSI_EARLY_EXIT_MIN_N sequences."""
-    rs = 3 if cfg.N >= 64 else cfg.B + 1  # PSI_ROUND_POSITIONS, PSI_EARLY_EXIT_MIN_N
-    return [(i, min(cfg.B + 1, i + rs)) for i in range(0, cfg.B + 1, rs)]
+    """Position rounds of the linear paths' early exit: [(first, end), ...]
+    (the schedule of include/psi_verify.h); one round of every position
+    below PSI_EARLY_EXIT_MIN_N sequences."""
+    import rejection_sampling_verify_b200 as psi
+    if cfg.N < psi.PSI_EARLY_EXIT_MIN_N:
+        return [(0, cfg.B + 1)]
+    short = psi.PSI_GREEDY_SHORT_ROUNDS if cfg.temperature == 0 else psi.PSI_SAMPLED_SHORT_ROUNDS
+    rs = psi.PSI_ROUND_POSITIONS
+    begins = [min(k * rs, cfg.B + 1) for k in range(short + 1)] + [cfg.B + 1]
+    return [(a, b) for a, b in zip(begins, begins[1:]) if a < b]
 
 
 def rows_in_round(cfg, r):
@@ -294,8 +300,8 @@ def config_block(cfg, name, world):
         c.update(batch=cfg.N, block=cfg.B, vocab=cfg.V, temperature=cfg.temperature,
                  top_p=cfg.top_p, logits_dtype=cfg.dtype,
                  outputs="tokens and counts (no p/q diagnostics)")
-        c.update(schedule=("early-exit rounds of 3 positions; roofline = the first round's main kernel"
-                           if cfg.N >= 64 else "one pass over every row"))
+        c.update(schedule=(f"early-exit rounds {sampled_rounds(cfg)}; roofline = the first round's "
+                           "main kernel" if cfg.N >= 64 else "one pass over every row"))
     c.update(global_batch=cfg.N * world, parallelism=f"batch-sharded x{world} (no collective)",
              l2="inputs larger than L2 (no flush needed)",
              inputs="seeded synthetic logits resident in HBM")

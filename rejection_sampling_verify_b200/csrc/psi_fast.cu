@@ -1010,7 +1010,7 @@ constexpr size_t kScanSmem = (sizeof(uint4) + sizeof(uint32_t)) * kRing;
 
 // ---------------------------------------------------------------------------
 // round_advance: one thread per sequence.  Early-exit rounds: round k covers
-// positions [k * PSI_ROUND_POSITIONS, (k + 1) * PSI_ROUND_POSITIONS) of B + 1.
+// positions [round_begin(k), round_begin(k + 1)) of B + 1.
 // A sequence takes part in round k when every drafted token of the earlier
 // rounds was accepted (a unit left to the general path counts as accepted:
 // its rows are then read although a rejection may make them unused).  The
@@ -1029,13 +1029,13 @@ __global__ void __launch_bounds__(128) round_advance_kernel(const __grid_constan
     a.counters[5 + 2 * ((k + 1) & 1)] = 0;
   }
   if (n >= N) return;
-  const int32_t i0 = k * PSI_ROUND_POSITIONS;
-  const int32_t i1 = min(B + 1, i0 + PSI_ROUND_POSITIONS);
+  const int32_t i0 = round_begin(k, B, PSI_SAMPLED_SHORT_ROUNDS);
+  const int32_t i1 = round_begin(k + 1, B, PSI_SAMPLED_SHORT_ROUNDS);
   int act = 1;
   if (k > 0) {
     act = a.active[n];
     const UnitRecord *r = a.rec + (int64_t)n * (B + 1);
-    for (int32_t i = i0 - PSI_ROUND_POSITIONS; act && i < i0; ++i)
+    for (int32_t i = round_begin(k - 1, B, PSI_SAMPLED_SHORT_ROUNDS); act && i < i0; ++i)
       if (i < B && r[i].accept == 0) act = 0;
   }
   a.active[n] = act;
@@ -1098,7 +1098,7 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
     if ((e = scan_and_finish(fa, true)) != cudaSuccess) return e;
     if ((e = scan_and_finish(f2, false)) != cudaSuccess) return e;
   } else {
-    const int rounds = (fa.s.B + 1 + PSI_ROUND_POSITIONS - 1) / PSI_ROUND_POSITIONS;
+    const int rounds = round_count(fa.s.B, PSI_SAMPLED_SHORT_ROUNDS);
     for (int k = 0; k < rounds; ++k) {
       round_advance_kernel<<<(fa.s.N + 127) / 128, 128, 0, stream>>>(fa, k);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -299,7 +299,7 @@ GreedyLayout greedy_layout(int32_t N, int32_t B, int32_t V, int elem_bytes) {
   L.partial_off = off;
   off = round_up256(off + sizeof(uint64_t) * (size_t)rows * L.plan.splits);
   L.rows_off = off;
-  off = round_up256(off + sizeof(int32_t) * (size_t)N * PSI_ROUND_POSITIONS);
+  off = round_up256(off + sizeof(int32_t) * (size_t)N * (B + 1));
   L.counters_off = off;
   off = round_up256(off + sizeof(int32_t) * 4);
   L.active_off = off;
@@ -309,7 +309,7 @@ GreedyLayout greedy_layout(int32_t N, int32_t B, int32_t V, int elem_bytes) {
 }
 
 // One thread per sequence: the AR rows of early-exit round k (positions
-// [k * PSI_ROUND_POSITIONS, ...) of B + 1).  A sequence takes part when
+// [round_begin(k), round_begin(k + 1)) of B + 1).  A sequence takes part when
 // every draft of the earlier rounds matched its row's argmax.
 __global__ void __launch_bounds__(128) greedy_advance_kernel(
     const uint64_t *__restrict__ partial, int32_t splits, const int32_t *__restrict__ ids,
@@ -317,13 +317,13 @@ __global__ void __launch_bounds__(128) greedy_advance_kernel(
   const int32_t n = blockIdx.x * blockDim.x + threadIdx.x;
   if (n == 0) counters[(k + 1) & 1] = 0;  // the next round's list
   if (n >= N) return;
-  const int32_t i0 = k * PSI_ROUND_POSITIONS;
-  const int32_t i1 = min(B + 1, i0 + PSI_ROUND_POSITIONS);
+  const int32_t i0 = round_begin(k, B, PSI_GREEDY_SHORT_ROUNDS);
+  const int32_t i1 = round_begin(k + 1, B, PSI_GREEDY_SHORT_ROUNDS);
   const int64_t row0 = (int64_t)n * (B + 1);
   int act = 1;
   if (k > 0) {
     act = active[n];
-    for (int32_t i = i0 - PSI_ROUND_POSITIONS; act && i < i0; ++i)
+    for (int32_t i = round_begin(k - 1, B, PSI_GREEDY_SHORT_ROUNDS); act && i < i0; ++i)
       if (i < B && ids[(int64_t)n * B + i] != argmax_of(partial, row0 + i, splits)) act = 0;
   }
   active[n] = act;
@@ -343,12 +343,15 @@ cudaError_t launch_greedy_early_exit(const void *logits, int64_t row_stride, psi
   int32_t *rows = reinterpret_cast<int32_t *>(ws + L.rows_off);
   int32_t *counters = reinterpret_cast<int32_t *>(ws + L.counters_off);
   int32_t *active = reinterpret_cast<int32_t *>(ws + L.active_off);
-  const int64_t grid = (int64_t)N * std::min(B + 1, PSI_ROUND_POSITIONS) * L.plan.splits;
-  if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+  if ((int64_t)N * (B + 1) * L.plan.splits > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
   cudaError_t e;
   if ((e = cudaMemsetAsync(counters, 0, 4 * sizeof(int32_t), stream)) != cudaSuccess) return e;
-  const int rounds = (B + 1 + PSI_ROUND_POSITIONS - 1) / PSI_ROUND_POSITIONS;
+  const int rounds = round_count(B, PSI_GREEDY_SHORT_ROUNDS);
   for (int k = 0; k < rounds; ++k) {
+    const int64_t grid = (int64_t)N *
+                         (round_begin(k + 1, B, PSI_GREEDY_SHORT_ROUNDS) -
+                          round_begin(k, B, PSI_GREEDY_SHORT_ROUNDS)) *
+                         L.plan.splits;
     greedy_advance_kernel<<<(N + 127) / 128, 128, 0, stream>>>(partial, L.plan.splits, ids, N, B,
                                                                k, active, rows, counters);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -11,6 +11,18 @@
 
 namespace psi {
 
+// Early-exit round schedule: `short_rounds` rounds of PSI_ROUND_POSITIONS
+// positions, then one round with the rest of the B + 1 positions.
+__host__ __device__ inline int32_t round_begin(int k, int32_t B, int short_rounds) {
+  const int32_t b = k <= short_rounds ? k * PSI_ROUND_POSITIONS : B + 1;
+  return b < B + 1 ? b : B + 1;
+}
+__host__ __device__ inline int round_count(int32_t B, int short_rounds) {
+  int k = 0;
+  while (round_begin(k, B, short_rounds) < B + 1) ++k;
+  return k;
+}
+
 // ---- greedy paths ----------------------------------------------------------
 struct ArgmaxPlan {
   int32_t splits = 1;  // CTAs per row
