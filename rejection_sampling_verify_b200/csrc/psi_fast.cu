@@ -8,22 +8,25 @@
 // "想跑 Uno：先確認官方程式需要的環境" (temperature, top-p).
 //
 // Kernels, in launch order:
-//   row_scan   Persistent CTAs stream every logit row ONCE from HBM with
-//              16-byte non-allocating loads (8 per thread in flight, double
-//              buffered in registers).  A row is read in batches of 2048
-//              vectors; inside a batch every thread uses the same reference
-//              (a lower bound of the row maximum, raised between batches), so
-//              all sums are independent of timing.  Elements within the
-//              window below the reference ("candidates", ~0.5% of a row) are
-//              masked out of the fp32 sum of exponentials; the vectors that
-//              hold them are parked in a shared-memory ring and, after the
-//              batch's barrier, split into candidates (to a per-row list in
-//              global memory) and elements that fell below the raised
-//              threshold (a 2^31 fixed-point sum).
-//   unit       One CTA per (sequence, row) unit: finishes the unit's q and p
-//              rows from their candidates (row maximum, Z, the top-p threshold
-//              and renormaliser, p's nucleus), decides the drafted token and
-//              draws the correction or bonus token over p's nucleus.
+//   round_advance  (early-exit rounds only) One thread per sequence: lists
+//              the rows and units of the next round of positions for the
+//              sequences whose drafts were all accepted so far.
+//   row_scan   Persistent CTAs stream every listed logit row ONCE from HBM
+//              with 16-byte non-allocating loads (8 per thread in flight,
+//              double buffered in registers, plus an L2 bulk prefetch).  A row
+//              is read in batches of 2048 vectors; inside a batch every
+//              thread uses the same reference (a lower bound of the row
+//              maximum, raised between batches), so all sums are independent
+//              of timing.  Elements within the window below the reference
+//              ("candidates", ~0.3% of a row) are masked out of the fp32 sum
+//              of exponentials; the vectors that hold them are parked in
+//              shared memory and, at the row's end, split into candidates
+//              (to a per-row list in global memory) and elements that fell
+//              below the final threshold (a 2^31 fixed-point sum).
+//   unit       One CTA of two warps per (sequence, row) unit: finishes the
+//              unit's p and q rows from their candidates (row maximum, Z, the
+//              top-p threshold and renormaliser), decides the drafted token
+//              and draws the correction or bonus token over p's nucleus.
 //   row_scan / unit, second pass   Rows whose window held less than top_p of
 //              the mass (rescanned with a wider window) or whose candidates
 //              overflowed (rescanned with the exact maximum known).
@@ -109,20 +112,7 @@ __device__ __forceinline__ T warp_sum_any(T v) {
   return v;
 }
 
-// Block-wide reductions (fixed order), broadcast to every thread.
-template <typename T, int W>
-__device__ __forceinline__ T block_sum_all(T v, T *scratch) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  v = warp_sum_any(v);
-  __syncthreads();
-  if (lane == 0) scratch[warp] = v;
-  __syncthreads();
-  T r = T(0);
-#pragma unroll
-  for (int w = 0; w < W; ++w) r += scratch[w];
-  return r;
-}
-
+// Block-wide maximum, broadcast to every thread.
 template <int W>
 __device__ __forceinline__ float block_max_all(float v, float *scratch) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -215,37 +205,10 @@ __device__ __forceinline__ uint32_t stream_vec(uint4 w, const Threshold<Bits> &t
   return any;
 }
 
-// Appends each lane's candidates (bit q of `mask`: element q of vector `w`,
-// vector index `j` in the row) to the row's list in global memory: one
-// shared-memory atomic per warp.  Every lane of the warp takes part.
-template <typename Bits>
-__device__ __forceinline__ void append_candidates(uint32_t mask, const uint4 &w, int32_t j,
-                                                  int *s_cand, uint64_t *dst) {
-  constexpr int VEC = Elem<Bits>::kVec;
-  const int lane = threadIdx.x & 31;
-  const int c = __popc(mask);
-  int incl = c;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  const int total = __shfl_sync(0xFFFFFFFFu, incl, 31);
-  if (total == 0) return;
-  int base = 0;
-  if (lane == 31) base = atomicAdd(s_cand, total);
-  int pos = __shfl_sync(0xFFFFFFFFu, base, 31) + incl - c;
-  while (mask) {
-    const int q = __ffs(mask) - 1;
-    mask &= mask - 1;
-    if (pos < kCandCap)
-      dst[pos] = ((uint64_t)vec_elem<Bits>(w, q) << 32) | (uint32_t)(j * VEC + q);
-    ++pos;
-  }
-}
-
-// Appends the candidates of two vectors per lane (masks m0, m1) with one
-// warp scan; every lane of the warp takes part.
+// Appends the candidates of two vectors per lane (masks m0, m1: bit q is
+// element q of vector w, vector index j in the row) to the row's list in
+// global memory with one warp scan and one shared-memory atomic per warp;
+// every lane of the warp takes part.
 template <typename Bits>
 __device__ __forceinline__ void append_candidates2(uint32_t m0, const uint4 &w0, int32_t j0,
                                                    uint32_t m1, const uint4 &w1, int32_t j1,
@@ -1115,12 +1078,14 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
   SampledArgs sa = fa.s;
   sa.records = fa.rec;
   const int clusters_a = (int)std::min<int64_t>(units, kListClusters);
-  e = launch_cluster_list(sa, dt, plan, 1, fa.list_a, fa.counters + 0, clusters_a, stream);
+  e = launch_cluster_list(sa, dt, plan, kClusterModeList, fa.list_a, fa.counters + 0, clusters_a,
+                          stream);
   if (e != cudaSuccess) return e;
   fast_emit_kernel<<<(fa.s.N + 127) / 128, 128, 0, stream>>>(fa);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int clusters_b = std::min(fa.s.N, kListClusters);
-  return launch_cluster_list(sa, dt, plan, 2, fa.list_b, fa.counters + 1, clusters_b, stream);
+  return launch_cluster_list(sa, dt, plan, kClusterModeSample, fa.list_b, fa.counters + 1,
+                             clusters_b, stream);
 }
 
 }  // namespace

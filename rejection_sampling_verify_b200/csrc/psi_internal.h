@@ -107,8 +107,10 @@ cudaError_t launch_sampled(const SampledArgs &a, psi_dtype dtype, const SampledP
                            const KernelEvents &ev, cudaStream_t stream);
 
 // The cluster kernel over a device-side list of units: full verify of each
-// listed unit (kModeList = 1) or only its correction/bonus draw, written to
-// out_tokens (kModeSample = 2).  `max_clusters` persistent clusters.
+// listed unit (kClusterModeList) or only its correction/bonus draw, written
+// to out_tokens (kClusterModeSample).  `max_clusters` persistent clusters.
+constexpr int kClusterModeList = 1;
+constexpr int kClusterModeSample = 2;
 cudaError_t launch_cluster_list(const SampledArgs &a, psi_dtype dtype, const SampledPlan &plan,
                                 int mode, const int32_t *list, const int32_t *count,
                                 int max_clusters, cudaStream_t stream);

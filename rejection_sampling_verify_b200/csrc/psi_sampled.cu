@@ -39,8 +39,8 @@ namespace {
 
 constexpr int kBins = 512;                         // radix bins per level (9 bits)
 constexpr int kModeGrid = 0;    // one unit per cluster, units in grid order
-constexpr int kModeList = 1;    // full verify of the units in a device list
-constexpr int kModeSample = 2;  // correction/bonus draw only, token written to the output
+// (kClusterModeList / kClusterModeSample: the list modes, see psi_internal.h)
+constexpr int kModeSample = kClusterModeSample;
 constexpr float kFixScale = 1099511627776.0f;      // 2^40
 constexpr double kFixScaleD = 1099511627776.0;     // 2^40
 constexpr double kFixInv = 1.0 / 1099511627776.0;  // 2^-40
