@@ -955,15 +955,17 @@ __global__ void __launch_bounds__(128) fast_emit_kernel(const __grid_constant__ 
   if (t == -2) a.list_b[atomicAdd(&a.counters[1], 1)] = n * (B + 1) + L;
 }
 
+// SM count of the current device (queried once per device).
 int sm_count() {
-  static int count = 0;
-  if (count == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        count <= 0)
-      count = 148;
-  }
+  static std::atomic<int> cached[PerDevice::kMax] = {};
+  const int dev = PerDevice::current();
+  const bool slot = dev >= 0 && dev < PerDevice::kMax;
+  int count = slot ? cached[dev].load(std::memory_order_relaxed) : 0;
+  if (count > 0) return count;
+  if (dev < 0 || cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      count <= 0)
+    count = 148;
+  if (slot) cached[dev].store(count, std::memory_order_relaxed);
   return count;
 }
 
@@ -1025,16 +1027,16 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
   const int64_t grid_scan = std::min<int64_t>(fa.rows, persistent);
   const int64_t grid_unit = units;
   cudaError_t e;
-  static bool configured = false;
-  if (!configured) {
-    if ((e = cudaFuncSetAttribute(row_scan_kernel<Bits>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)kScanSmem)) != cudaSuccess)
-      return e;
-    if ((e = cudaFuncSetAttribute(unit_kernel<Bits>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)sizeof(UnitShared))) != cudaSuccess)
-      return e;
-    configured = true;
-  }
+  static DeviceOnce configure;  // shared memory above 48 KB, once per device
+  e = configure([] {
+    cudaError_t err = cudaFuncSetAttribute(row_scan_kernel<Bits>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)kScanSmem);
+    if (err != cudaSuccess) return err;
+    return cudaFuncSetAttribute(unit_kernel<Bits>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)sizeof(UnitShared));
+  });
+  if (e != cudaSuccess) return e;
   // the work-list counters of this call start at zero
   if ((e = cudaMemsetAsync(fa.counters, 0, kCounters * sizeof(int32_t), stream)) != cudaSuccess)
     return e;

@@ -384,13 +384,13 @@ cudaError_t launch_tree_walk(const uint64_t *partial, int32_t splits, const int3
                              int32_t *out_path_nodes, int32_t *out_path_len,
                              int32_t *out_tokens, uint32_t *dev_status, cudaStream_t stream) {
   const size_t smem = sizeof(int32_t) * (size_t)(5 * M + 2);
-  static bool configured = false;  // opt in to >48 KB once (only large M needs it)
-  if (smem > 48 * 1024 && !configured) {
-    cudaError_t e = cudaFuncSetAttribute(tree_walk_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(5 * PSI_MAX_TREE_NODES + 2) * 4);
+  static DeviceOnce configure;  // opt in to > 48 KB once per device (only large M needs it)
+  if (smem > 48 * 1024) {
+    const cudaError_t e = configure([] {
+      return cudaFuncSetAttribute(tree_walk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)(5 * PSI_MAX_TREE_NODES + 2) * 4);
+    });
     if (e != cudaSuccess) return e;
-    configured = true;
   }
   tree_walk_kernel<<<N, kThreads, smem, stream>>>(partial, splits, node_tokens, parents, M, V,
                                                   out_path_nodes, out_path_len, out_tokens,

@@ -6,10 +6,40 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "psi_device.cuh"
 #include "psi_verify.h"
 
 namespace psi {
+
+// Host-side settings made once per device (launch attributes, device
+// queries): one flag bit per device ordinal below 64; larger ordinals repeat
+// the call every time.
+struct PerDevice {
+  static constexpr int kMax = 64;
+  static int current() {
+    int dev = 0;
+    return cudaGetDevice(&dev) == cudaSuccess ? dev : -1;
+  }
+};
+
+class DeviceOnce {
+ public:
+  // Runs f() unless it already succeeded on the current device.
+  template <typename F>
+  cudaError_t operator()(F &&f) {
+    const int dev = PerDevice::current();
+    const uint64_t bit = (dev >= 0 && dev < PerDevice::kMax) ? (1ull << dev) : 0ull;
+    if (bit && (done_.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    const cudaError_t e = f();
+    if (e == cudaSuccess && bit) done_.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+  }
+
+ private:
+  std::atomic<uint64_t> done_{0};
+};
 
 // Early-exit round schedule: `short_rounds` rounds of PSI_ROUND_POSITIONS
 // positions, then one round with the rest of the B + 1 positions.

@@ -871,14 +871,22 @@ static cudaError_t launch_cluster_kernel(const SampledArgs &a, const SampledPlan
                                          int64_t n_clusters, const KernelEvents *ev,
                                          cudaStream_t stream) {
   auto kernel = sampled_unit_kernel<Bits>;
-  static int configured_smem = 0;
-  if ((int)plan.smem > configured_smem) {
+  // the largest shared memory set so far, per device
+  static std::atomic<int> configured_smem[PerDevice::kMax] = {};
+  const int dev = PerDevice::current();
+  const bool slot = dev >= 0 && dev < PerDevice::kMax;
+  if (!slot || (int)plan.smem > configured_smem[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)plan.smem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
-    configured_smem = (int)plan.smem;
+    if (slot) {
+      int cur = configured_smem[dev].load(std::memory_order_relaxed);
+      while ((int)plan.smem > cur &&
+             !configured_smem[dev].compare_exchange_weak(cur, (int)plan.smem)) {
+      }
+    }
   }
   const int64_t grid = n_clusters * plan.cluster;
   if (grid > 0x7FFFFFFFLL || grid < 1) return cudaErrorInvalidConfiguration;
