@@ -23,7 +23,8 @@
  *
  * Conventions shared by every entry point:
  *  - All array arguments are DEVICE pointers owned by the caller.  The
- *    library allocates nothing and keeps no state between calls.
+ *    library allocates nothing and keeps no data between calls (only
+ *    per-device launch settings, made on a device's first call).
  *  - Calls are asynchronous on `stream` (NULL = the legacy default stream).
  *  - Argument errors are detected on the host before any launch and
  *    returned as a psi_status; nothing is launched in that case.

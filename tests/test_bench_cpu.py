@@ -1,0 +1,58 @@
+"""Host logic of the benchmark: the early-exit round schedule it assumes
+matches the header's constants, and its byte accounting is the per-row sum
+it claims to be."""
+import re
+
+import numpy as np
+
+import bench
+import psi_inputs
+import rejection_sampling_verify_b200 as psi
+
+CFG = psi_inputs.CONFIGS
+
+
+def _header_define(name):
+    text = open(bench.os.path.join(bench.ROOT, "include", "psi_verify.h")).read()
+    return int(re.search(rf"#define\s+{name}\s+(\d+)", text).group(1))
+
+
+def test_schedule_constants_come_from_the_header():
+    for name in ("PSI_ROUND_POSITIONS", "PSI_SAMPLED_SHORT_ROUNDS", "PSI_GREEDY_SHORT_ROUNDS",
+                 "PSI_EARLY_EXIT_MIN_N"):
+        assert getattr(psi, name) == _header_define(name)
+
+
+def test_rounds_partition_the_positions():
+    for name in ("large_batch_nucleus", "max_batch_greedy", "single_stream", "tiny"):
+        cfg = CFG[name]
+        r = bench.sampled_rounds(cfg)
+        assert r[0][0] == 0 and r[-1][1] == cfg.B + 1
+        assert all(a[1] == b[0] and a[0] < a[1] for a, b in zip(r, r[1:]))
+        if cfg.N < psi.PSI_EARLY_EXIT_MIN_N:
+            assert r == [(0, cfg.B + 1)]
+        else:
+            short = (psi.PSI_GREEDY_SHORT_ROUNDS if cfg.temperature == 0
+                     else psi.PSI_SAMPLED_SHORT_ROUNDS)
+            assert all(b - a == psi.PSI_ROUND_POSITIONS for a, b in r[:short])
+
+
+def test_rows_read_counts_rounds_up_to_the_emitting_position():
+    cfg = CFG["large_batch_nucleus"]  # rounds (0, 3), (3, 9), B = 8
+    assert bench.sampled_rounds(cfg) == [(0, 3), (3, 9)]
+    # emitting position 0..2: round 0 only = 3 AR + 3 draft rows; later: all 17
+    assert bench.rows_read(cfg, np.array([1, 3])) == 2 * 6
+    assert bench.rows_read(cfg, np.array([4, 9])) == 2 * 17
+    g = CFG["max_batch_greedy"]  # AR rows only
+    assert bench.rows_read(g, np.array([1])) == 3
+    assert bench.rows_read(g, np.array([17])) == 17
+
+
+def test_main_launch_bytes_is_the_first_round():
+    cfg = CFG["large_batch_nucleus"]
+    assert bench.main_launch_bytes(cfg) == cfg.N * 6 * cfg.V * 2
+    g = CFG["max_batch_greedy"]
+    assert bench.main_launch_bytes(g) == g.N * 3 * g.V * 2
+    t = CFG["tree_greedy"]
+    assert bench.main_launch_bytes(t) == bench.algorithmic_bytes(t)
+    assert bench.algorithmic_bytes(cfg) == 1322450944
