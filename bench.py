@@ -331,7 +331,7 @@ def run_reference(args, cfg, name):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * cfg.N / value, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_block(cfg, name, 1),
+        "config": dict(config_block(cfg, name, 1), schedule="every row (the oracle as it stands)"),
         "cpu_baseline": {"value": value, "unit": "blocks/s", "cores": 1, "kind": "oracle",
                          "sample": f"{seqs} sequences of the workload per step, single thread"},
         "e2e": {"value": value, "unit": "blocks/s", "h2d_bytes_per_step": 0,
