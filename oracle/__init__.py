@@ -12,7 +12,9 @@ Logit arrays are numpy ``float32`` (IEEE binary32 rows) or ``uint16``
 Every function here follows a passage of the method's pages; the citations
 are in ``psi_oracle.c``.  Parity status per function:
   - counter RNG, row softmax/top-p, linear sampled verify, greedy linear,
-    greedy tree: pinned by the CPU tests in ``tests/test_oracle_*.py``.
+    greedy tree: pinned by the CPU tests in ``tests/test_oracle_*.py``;
+    ``tests/test_oracle_mutants.py`` plants single mistakes in copies of
+    ``psi_oracle.c`` and requires those pins to catch every one.
 """
 from __future__ import annotations
 
@@ -59,8 +61,10 @@ _lib = None
 def _load():
     global _lib
     if _lib is None:
-        build()
-        lib = C.CDLL(_LIB_PATH)
+        # PSI_ORACLE_LIB names a prebuilt copy to load instead (the mutation
+        # check builds deliberately broken copies and runs the pins on them).
+        path = os.environ.get("PSI_ORACLE_LIB") or build()
+        lib = C.CDLL(path)
         u64, i64, i32, u32, dbl, vp = (C.c_uint64, C.c_int64, C.c_int32,
                                        C.c_uint32, C.c_double, C.c_void_p)
         lib.orc_splitmix64_mix.restype = u64

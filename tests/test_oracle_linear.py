@@ -16,6 +16,7 @@ What fixes the oracle here, other than itself:
   * the greedy rule on hand cases and as the T -> 0 limit of the sampled rule.
 """
 import json
+import math
 import os
 
 import numpy as np
@@ -145,6 +146,24 @@ def test_lossless_exact(case):
                                    err_msg=f"pos {pos}")
 
 
+@pytest.mark.parametrize("T", [1.0, 0.8])
+def test_lossless_exact_spread_residual_under_top_p(T):
+    """Top-p on both sides with a correction spread over several tokens, part
+    of them in the draft's tail that its nucleus drops: the target keeps
+    tokens 0-3, the draft mostly 5 and 6, so the residual max(0, p' - q') is
+    p' itself on 0-3 and any use of the unfiltered q shifts its ratios."""
+    ar_p = np.array([[0.25, 0.2, 0.2, 0.15, 0.1, 0.04, 0.03, 0.03],
+                     [0.1, 0.3, 0.2, 0.1, 0.1, 0.1, 0.05, 0.05]])
+    dr_p = np.array([[0.05, 0.05, 0.02, 0.02, 0.01, 0.5, 0.3, 0.05]])
+    ar = np.log(ar_p).astype(np.float32)
+    draft = np.log(dr_p).astype(np.float32)
+    top_p = 0.7
+    q_pos = _target(draft[0], T, top_p)
+    law = emission_law(ar, draft, [5], 0, T, top_p, q_pos)
+    np.testing.assert_allclose(law, _target(ar[0], T, top_p), rtol=0, atol=1e-12)
+    assert np.count_nonzero(law > 0) >= 3
+
+
 @pytest.mark.parametrize("q", [(0.5, 0.5), (0.9, 0.1), (0.2, 0.8), (1.0, 0.0)])
 def test_seventy_thirty_exact(q):
     """The pages' example: a 70/30 target must come out 70/30."""
@@ -167,6 +186,34 @@ def test_seventy_thirty_sampled():
                              ids, 1.0, 1.0, seed=3, step=0)
     freq_a = np.mean(r["tokens"][:, 0] == 0)
     assert abs(freq_a - 0.7) < 4 * np.sqrt(0.21 / n)
+
+
+def test_verify_draws_uniforms_from_the_counter():
+    """The batch verify gives sequence s at step t the counter uniforms
+    u(seed, s, t, row, purpose) (the generator is pinned by the published
+    SplitMix64 vector and the chain test): purpose 0 for the acceptance test
+    of each drafted row, purpose 1 for the draw at each row.  With those
+    uniforms passed in, the single-sequence verify must agree exactly."""
+    rng = np.random.default_rng(21)
+    N, B, V = 12, 4, 6
+    ar = rng.normal(0, 1, (N, B + 1, V)).astype(np.float32)
+    draft = (ar[:, :B] + rng.normal(0, 0.7, (N, B, V))).astype(np.float32)
+    ids = rng.integers(0, V, (N, B)).astype(np.int32)
+    seq_ids = np.arange(N, dtype=np.uint64) * 7919 + 3
+    seed = 17
+    by_step = []
+    for step in (0, 5):
+        r = oracle.verify_linear(ar, draft, ids, 1.0, 1.0, seed=seed, step=step,
+                                 seq_ids=seq_ids)
+        for n in range(N):
+            s = int(seq_ids[n])
+            ua = [oracle.uniform(seed, s, step, i, oracle.PURPOSE_ACCEPT) for i in range(B)]
+            ur = [oracle.uniform(seed, s, step, i, oracle.PURPOSE_RESID) for i in range(B + 1)]
+            one = oracle.verify_one(ar[n], draft[n], ids[n], 1.0, 1.0, ua, ur)
+            assert r["tokens"][n].tolist() == one["tokens"].tolist(), (step, n)
+            assert r["n_emitted"][n] == one["n_emitted"], (step, n)
+        by_step.append(r["tokens"])
+    assert not np.array_equal(by_step[0], by_step[1])
 
 
 # ---- statistics over RNG-driven draws ----------------------------------------
@@ -277,6 +324,21 @@ def test_top_p_keeps_ties_at_threshold():
     # crossing inside the lower tie group keeps the whole group
     assert 2 * a < 0.8
     np.testing.assert_allclose(_probs([1, 1, 0, 0], 1.0, 0.8), softmax([1.0, 1, 0, 0]), atol=1e-7)
+
+
+def test_top_p_mass_reaching_exactly_stops_there():
+    """The nucleus is the smallest set whose mass reaches top_p (>=): with
+    top_p equal to the top token's mass that token alone is kept, one ulp more
+    brings in the next.  top_p is set to that mass as double arithmetic gives
+    it (e_0 = exp(0) = 1, e_v = exp(x_v - x_0), the total summed in vocabulary
+    order); math.exp is the C library's exp."""
+    x = np.array([0.0, -1.0, -3.0], dtype=np.float32)
+    mass0 = 1.0 / ((1.0 + math.exp(-1.0)) + math.exp(-3.0))
+    p, st, margin = oracle.row_probs(x, 1.0, mass0)
+    assert st == 0 and p.tolist() == [1.0, 0.0, 0.0]
+    assert margin == 0.0  # the cut sits exactly on the boundary
+    p2 = _probs(x, 1.0, float(np.nextafter(mass0, 1.0)))
+    assert p2[0] > 0 and p2[1] > 0 and p2[2] == 0
 
 
 def test_top_p_limits():
