@@ -225,6 +225,11 @@ def verify_linear(ar, draft, ids, temperature: float, top_p: float = 1.0, seed: 
 
     ar [N, B+1, V], draft [N, B, V] (may be None when temperature == 0),
     ids int32 [N, B], seq_ids uint64-as-int64 [N] or None; CUDA tensors.
+
+    With ``out`` and a large enough ``workspace`` passed in, the call only
+    launches work on the stream, so it can be captured into a CUDA graph
+    (after one call on the device outside capture).  seed and step are then
+    fixed in the graph.
     """
     torch = _torch()
     N, B1 = ar.shape[0], ar.shape[1]
