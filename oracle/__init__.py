@@ -12,7 +12,8 @@ Logit arrays are numpy ``float32`` (IEEE binary32 rows) or ``uint16``
 Every function here follows a passage of the method's pages; the citations
 are in ``psi_oracle.c``.  Parity status per function:
   - counter RNG, row softmax/top-p, linear sampled verify, greedy linear,
-    greedy tree: pinned by the CPU tests in ``tests/test_oracle_*.py``;
+    greedy tree, sampled tree: pinned by the CPU tests in
+    ``tests/test_oracle_*.py``;
     ``tests/test_oracle_mutants.py`` plants single mistakes in copies of
     ``psi_oracle.c`` and requires those pins to catch every one.
 """
@@ -87,6 +88,14 @@ def _load():
         lib.orc_verify_tree_greedy.restype = u32
         lib.orc_verify_tree_greedy.argtypes = [vp, i64, C.c_int, vp, vp, i32,
                                                i32, i32, vp, vp, vp]
+        lib.orc_verify_tree_sampled_one.restype = u32
+        lib.orc_verify_tree_sampled_one.argtypes = [vp, i64, C.c_int, vp, vp, i32,
+                                                    i32, dbl, dbl, vp, vp, vp, vp,
+                                                    vp, vp]
+        lib.orc_verify_tree_sampled.restype = u32
+        lib.orc_verify_tree_sampled.argtypes = [vp, i64, C.c_int, vp, vp, i32, i32,
+                                                i32, dbl, dbl, u64, vp, u64, vp, vp,
+                                                vp, vp]
         _lib = lib
     return _lib
 
@@ -224,3 +233,52 @@ def verify_tree_greedy(ar, node_tokens, parents, V=None):
                                         N, M, V, _ptr(path), _ptr(plen),
                                         _ptr(toks))
     return dict(path_nodes=path, path_len=plen, tokens=toks, status=int(st))
+
+
+# ---- sampled tree ---------------------------------------------------------------
+
+def verify_tree_sampled_one(ar, node_tokens, parents, temperature, top_p, u_accept, u_resid,
+                            V=None):
+    """One tree with explicit uniforms.  ar [M+1, S]; node_tokens, parents
+    [M]; u_accept [M+1] (entry k+1 tests node k), u_resid [M+1] (by row)."""
+    ar = _contig(ar)
+    code = _dtype_code(ar)
+    M1, S = ar.shape
+    M = M1 - 1
+    V = S if V is None else V
+    tok = _contig(np.asarray(node_tokens), np.int32).reshape(M)
+    par = _contig(np.asarray(parents), np.int32).reshape(M)
+    ua = _contig(np.asarray(u_accept, dtype=np.float64))
+    ur = _contig(np.asarray(u_resid, dtype=np.float64))
+    assert ua.size >= M + 1 and ur.size >= M + 1
+    path = np.empty(max(M, 1), dtype=np.int32)
+    plen = np.empty(1, dtype=np.int32)
+    toks = np.empty(M + 1, dtype=np.int32)
+    margin = np.empty(1)
+    st = _load().orc_verify_tree_sampled_one(_ptr(ar), S, code, _ptr(tok), _ptr(par), M, V,
+                                             temperature, top_p, _ptr(ua), _ptr(ur),
+                                             _ptr(path), _ptr(plen), _ptr(toks), _ptr(margin))
+    return dict(path_nodes=path[:M], path_len=int(plen[0]), tokens=toks,
+                margin=float(margin[0]), status=int(st))
+
+
+def verify_tree_sampled(ar, node_tokens, parents, temperature, top_p, seed, step,
+                        seq_ids=None, V=None):
+    """Batch sampled tree verify with the counter RNG.  ar [N, M+1, S];
+    node_tokens, parents int32 [N, M]."""
+    ar = _contig(ar)
+    code = _dtype_code(ar)
+    N, M1, S = ar.shape
+    M = M1 - 1
+    V = S if V is None else V
+    tok = _contig(np.asarray(node_tokens), np.int32).reshape(N, M)
+    par = _contig(np.asarray(parents), np.int32).reshape(N, M)
+    sid = None if seq_ids is None else _contig(np.asarray(seq_ids), np.uint64)
+    path = np.empty((N, M), dtype=np.int32)
+    plen = np.empty(N, dtype=np.int32)
+    toks = np.empty((N, M + 1), dtype=np.int32)
+    margin = np.empty(N)
+    st = _load().orc_verify_tree_sampled(_ptr(ar), S, code, _ptr(tok), _ptr(par), N, M, V,
+                                         temperature, top_p, seed, _ptr(sid), step, _ptr(path),
+                                         _ptr(plen), _ptr(toks), _ptr(margin))
+    return dict(path_nodes=path, path_len=plen, tokens=toks, margin=margin, status=int(st))

@@ -26,6 +26,10 @@
  *    set whose mass reaches top_p, together with every token tied with the
  *    last one admitted, then renormalises; applied to p and q alike.
  *  - Greedy ties resolve to the lowest vocabulary index.
+ *  - Sampled tree (the pages give no rule): recursive rejection over each
+ *    reached node's children in index order, each child its own point-mass
+ *    proposal; node k's acceptance uses the uniform of row k+1, the final
+ *    draw the uniform of the row it is drawn from.
  */
 #include "psi_oracle.h"
 
@@ -422,5 +426,140 @@ uint32_t orc_verify_tree_greedy(const void *ar, int64_t ar_row_stride,
   free(am);
   free(matched);
   free(depth);
+  return status;
+}
+
+/* ---- sampled tree ------------------------------------------------------ */
+
+/* [P3] "Linear 與 Tree sampler" keeps several candidates per position in a
+ * finite prefix tree and verifies the tree in one pass, but gives no rule
+ * for sampled decoding.  The rule taken here is recursive rejection over
+ * each node's candidate list, the multi-candidate scheme of Miao et al.
+ * ("SpecInfer", ASPLOS 2024, multi-step speculative sampling), with every
+ * candidate taken as its own point-mass proposal so the result stays
+ * lossless for candidates that were chosen (top-k) rather than sampled:
+ * at a node with target P, candidate x is accepted with probability
+ * P'(x) = P(x) / R (R = mass not yet removed); on rejection x's mass is
+ * removed, which is max(0, P' - delta_x) renormalised.  Each round is one
+ * speculative-sampling step, so the emitted token at every node has law P.
+ *
+ * Node validity follows the greedy tree: a bad parent or token makes the
+ * node unusable (flagged, never accepted, its subtree unreachable). */
+static uint32_t tree_validate(const int32_t *tok, const int32_t *par,
+                              int32_t M, int32_t V, unsigned char *valid) {
+  uint32_t status = 0;
+  for (int32_t k = 0; k < M; ++k) {
+    valid[k] = 1;
+    if (par[k] < -1 || par[k] >= k) {
+      status |= ORC_BAD_PARENT;
+      valid[k] = 0;
+    } else if (tok[k] < 0 || tok[k] >= V) {
+      status |= ORC_BAD_TOKEN_ID;
+      valid[k] = 0;
+    }
+  }
+  return status;
+}
+
+uint32_t orc_verify_tree_sampled_one(const void *ar, int64_t ar_row_stride,
+                                     int dtype, const int32_t *node_tokens,
+                                     const int32_t *parents, int32_t M,
+                                     int32_t V, double temperature,
+                                     double top_p, const double *u_accept,
+                                     const double *u_resid,
+                                     int32_t *out_path_nodes,
+                                     int32_t *out_path_len, int32_t *out_tokens,
+                                     double *out_margin) {
+  if (out_margin) *out_margin = INFINITY;
+  if (temperature == 0.0)
+    return orc_verify_tree_greedy(ar, ar_row_stride, dtype, node_tokens,
+                                  parents, 1, M, V, out_path_nodes,
+                                  out_path_len, out_tokens);
+
+  unsigned char *valid = (unsigned char *)malloc((size_t)(M > 0 ? M : 1));
+  double *P = (double *)malloc((size_t)V * sizeof(double));
+  double *w = (double *)malloc((size_t)V * sizeof(double));
+  uint32_t status = tree_validate(node_tokens, parents, M, V, valid);
+
+  for (int32_t k = 0; k < M; ++k) out_path_nodes[k] = -1;
+  for (int32_t k = 0; k <= M; ++k) out_tokens[k] = -1;
+
+  double margin = INFINITY;
+  int32_t node = -1; /* -1 = root */
+  int32_t depth = 0;
+  int32_t token;
+  for (;;) {
+    const int32_t row = node + 1;
+    double mtop;
+    status |= orc_row_probs(row_ptr(ar, dtype, ar_row_stride, row), dtype, V,
+                            temperature, top_p, P, &mtop);
+    margin = dmin(margin, mtop);
+    memcpy(w, P, (size_t)V * sizeof(double)); /* what remains of P */
+    int32_t next = -1;
+    for (int32_t k = node + 1; k < M; ++k) {
+      if (parents[k] != node || !valid[k]) continue;
+      const int32_t x = node_tokens[k];
+      double R = 0.0;
+      for (int32_t v = 0; v < V; ++v) R += w[v];
+      const double px = w[x]; /* 0 once x was rejected at this node */
+      const double u = u_accept[k + 1];
+      if (R > 0.0) margin = dmin(margin, fabs(u - px / R));
+      if (u * R < px) {
+        next = k;
+        break;
+      }
+      w[x] = 0.0; /* remove the rejected candidate's mass */
+    }
+    if (next < 0) {
+      double total = 0.0;
+      for (int32_t v = 0; v < V; ++v) total += w[v];
+      if (total <= 0.0) memcpy(w, P, (size_t)V * sizeof(double));
+      double m2;
+      token = inverse_cdf(w, V, u_resid[row], &m2);
+      margin = dmin(margin, m2);
+      break;
+    }
+    out_path_nodes[depth] = next;
+    out_tokens[depth] = node_tokens[next];
+    ++depth;
+    node = next;
+  }
+  out_tokens[depth] = token;
+  *out_path_len = depth;
+  if (out_margin) *out_margin = margin;
+  free(valid);
+  free(P);
+  free(w);
+  return status;
+}
+
+uint32_t orc_verify_tree_sampled(const void *ar, int64_t ar_row_stride,
+                                 int dtype, const int32_t *node_tokens,
+                                 const int32_t *parents, int32_t N, int32_t M,
+                                 int32_t V, double temperature, double top_p,
+                                 uint64_t seed, const uint64_t *seq_ids,
+                                 uint64_t step, int32_t *out_path_nodes,
+                                 int32_t *out_path_len, int32_t *out_tokens,
+                                 double *out_margin) {
+  uint32_t status = 0;
+  double *u_accept = (double *)malloc((size_t)(M + 1) * sizeof(double));
+  double *u_resid = (double *)malloc((size_t)(M + 1) * sizeof(double));
+  for (int32_t n = 0; n < N; ++n) {
+    uint64_t seq = seq_ids ? seq_ids[n] : (uint64_t)n;
+    u_accept[0] = 0.0; /* the root row has no acceptance test */
+    for (int32_t j = 1; j <= M; ++j)
+      u_accept[j] = orc_uniform(seed, seq, step, (uint64_t)j,
+                                ORC_PURPOSE_ACCEPT);
+    for (int32_t j = 0; j <= M; ++j)
+      u_resid[j] = orc_uniform(seed, seq, step, (uint64_t)j, ORC_PURPOSE_RESID);
+    status |= orc_verify_tree_sampled_one(
+        row_ptr(ar, dtype, ar_row_stride, (int64_t)n * (M + 1)), ar_row_stride,
+        dtype, node_tokens + (size_t)n * M, parents + (size_t)n * M, M, V,
+        temperature, top_p, u_accept, u_resid,
+        out_path_nodes + (size_t)n * M, out_path_len + n,
+        out_tokens + (size_t)n * (M + 1), out_margin ? out_margin + n : NULL);
+  }
+  free(u_accept);
+  free(u_resid);
   return status;
 }

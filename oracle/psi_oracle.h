@@ -101,6 +101,39 @@ uint32_t orc_verify_tree_greedy(const void *ar, int64_t ar_row_stride,
                                 int32_t V, int32_t *out_path_nodes,
                                 int32_t *out_path_len, int32_t *out_tokens);
 
+/* Sampled tree verify of one sequence with explicitly supplied uniforms.
+ * Tree layout as orc_verify_tree_greedy for one sequence.  At each reached
+ * node the children (ascending index) are tried in turn: child k, token x,
+ * is accepted iff u_accept[k+1] * R < P(x), where P is the node row's
+ * tempered (top-p cut) distribution and R the mass of P not yet removed;
+ * a rejected child's token is removed from P.  An accepted child becomes the
+ * next node; when no child is accepted (or the node is a leaf) the last
+ * token is the inverse-CDF draw from what remains of P with u_resid[row].
+ * u_accept[M+1] (entry 0 unused), u_resid[M+1].  temperature == 0 selects the
+ * greedy tree rule.  out_margin as in orc_verify_one.  Returns status bits. */
+uint32_t orc_verify_tree_sampled_one(const void *ar, int64_t ar_row_stride,
+                                     int dtype, const int32_t *node_tokens,
+                                     const int32_t *parents, int32_t M,
+                                     int32_t V, double temperature,
+                                     double top_p, const double *u_accept,
+                                     const double *u_resid,
+                                     int32_t *out_path_nodes,
+                                     int32_t *out_path_len, int32_t *out_tokens,
+                                     double *out_margin);
+
+/* Batch sampled tree verify with the counter RNG: node k's acceptance
+ * uniform is U(seed, seq, step, k+1, ACCEPT), the draw at row j uses
+ * U(seed, seq, step, j, RESID); seq = seq_ids ? seq_ids[n] : n.
+ * out_margin [N] may be NULL.  Returns OR of status bits. */
+uint32_t orc_verify_tree_sampled(const void *ar, int64_t ar_row_stride,
+                                 int dtype, const int32_t *node_tokens,
+                                 const int32_t *parents, int32_t N, int32_t M,
+                                 int32_t V, double temperature, double top_p,
+                                 uint64_t seed, const uint64_t *seq_ids,
+                                 uint64_t step, int32_t *out_path_nodes,
+                                 int32_t *out_path_len, int32_t *out_tokens,
+                                 double *out_margin);
+
 /* Index of the largest logit in a row (lowest index among equals). */
 int32_t orc_row_argmax(const void *row, int dtype, int32_t V,
                        uint32_t *status);

@@ -4,8 +4,9 @@ Each mutant is ``oracle/psi_oracle.c`` with ONE plausible mistake planted in a
 copy: a dropped term, a flipped sign or comparison, a wrong row, index or
 uniform, transposed operands, a filter applied to one side only.  Every copy
 is compiled into a temporary library and the oracle's pin tests
-(``tests/test_oracle_rng.py``, ``test_oracle_linear.py``,
-``test_oracle_tree.py``) run against it in a subprocess; each mutant must make
+(``tests/test_oracle_rng.py``, ``test_oracle_tree.py``,
+``test_oracle_tree_sampled.py``, ``test_oracle_linear.py``) run against it in a
+subprocess; each mutant must make
 at least one pin fail.  The unmodified source, built the same way, must pass
 them all, so a failure is the mutant's doing and not the harness's.
 
@@ -24,7 +25,8 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "psi_oracle.c")
 PINS = [os.path.join("tests", f) for f in
-        ("test_oracle_rng.py", "test_oracle_linear.py", "test_oracle_tree.py")]
+        ("test_oracle_rng.py", "test_oracle_tree.py", "test_oracle_tree_sampled.py",
+         "test_oracle_linear.py")]  # the slow statistics last: most mutants fail sooner
 
 # (name, text in psi_oracle.c, the same text with the mistake planted)
 MUTANTS = [
@@ -35,8 +37,9 @@ MUTANTS = [
     ("hash_drops_step", "  h = orc_splitmix64_mix(h ^ step);", "  h = orc_splitmix64_mix(h);"),
     ("uniform_low_bits", "(double)(h >> 40) / 16777216.0",
      "(double)(h & 0xFFFFFFull) / 16777216.0"),
-    ("verify_ignores_seq_ids", "    uint64_t seq = seq_ids ? seq_ids[n] : (uint64_t)n;",
-     "    uint64_t seq = (uint64_t)n;"),
+    ("verify_ignores_seq_ids",
+     "    uint64_t seq = seq_ids ? seq_ids[n] : (uint64_t)n;\n    for (int32_t i = 0; i < B; ++i)",
+     "    uint64_t seq = (uint64_t)n;\n    for (int32_t i = 0; i < B; ++i)"),
     ("verify_ignores_step",
      "      u_accept[i] = orc_uniform(seed, seq, step, (uint64_t)i,",
      "      u_accept[i] = orc_uniform(seed, seq, 0, (uint64_t)i,"),
@@ -111,14 +114,38 @@ MUTANTS = [
     ("greedy_emits_bonus_row", "  out_tokens[L] = am[L];", "  out_tokens[L] = am[B];"),
     # ---- greedy tree
     ("tree_compares_own_row", "      int32_t parent_row = pk + 1;", "      int32_t parent_row = k + 1;"),
-    ("tree_ignores_parent_match", "      int parent_ok = (pk == -1) || matched[pk];",
-     "      int parent_ok = 1;"),
+    # (matching under an unmatched parent is not planted: the walk back from
+    # such a node would write outside the path buffer)
+    ("tree_only_root_children_match", "      int parent_ok = (pk == -1) || matched[pk];",
+     "      int parent_ok = (pk == -1);"),
     ("tree_depth_ties_to_last", "        if (depth[k] > best_depth) {",
      "        if (depth[k] >= best_depth) {"),
     ("tree_next_token_from_root", "    toks[best_depth] = am[best + 1];",
      "    toks[best_depth] = am[0];"),
     ("tree_self_parent_not_flagged", "      if (pk < -1 || pk >= k) {",
      "      if (pk < -1 || pk > k) {"),
+    # ---- sampled tree: recursive rejection over each node's children
+    ("stree_accept_not_renormalised", "      if (u * R < px) {", "      if (u < px) {"),
+    ("stree_rejected_mass_kept", "      w[x] = 0.0; /* remove the rejected candidate's mass */",
+     "      /* the rejected candidate's mass is kept */"),
+    ("stree_accept_uses_parent_row_uniform", "      const double u = u_accept[k + 1];",
+     "      const double u = u_accept[node + 1];"),
+    ("stree_draw_ignores_removed_mass", "      token = inverse_cdf(w, V, u_resid[row], &m2);",
+     "      token = inverse_cdf(P, V, u_resid[row], &m2);"),
+    ("stree_draw_uses_root_uniform", "      token = inverse_cdf(w, V, u_resid[row], &m2);",
+     "      token = inverse_cdf(w, V, u_resid[0], &m2);"),
+    ("stree_children_in_reverse", "    for (int32_t k = node + 1; k < M; ++k) {\n      if (parents[k] != node",
+     "    for (int32_t k = M - 1; k > node; --k) {\n      if (parents[k] != node"),
+    ("stree_batch_accept_row_offset",
+     "      u_accept[j] = orc_uniform(seed, seq, step, (uint64_t)j,",
+     "      u_accept[j] = orc_uniform(seed, seq, step, (uint64_t)(j - 1),"),
+    ("stree_batch_ignores_seq_ids",
+     "    uint64_t seq = seq_ids ? seq_ids[n] : (uint64_t)n;\n    u_accept[0] = 0.0;",
+     "    uint64_t seq = (uint64_t)n;\n    u_accept[0] = 0.0;"),
+    ("stree_emits_node_index", "    out_tokens[depth] = node_tokens[next];",
+     "    out_tokens[depth] = next;"),
+    ("stree_bad_parent_not_flagged", "      status |= ORC_BAD_PARENT;\n      valid[k] = 0;",
+     "      valid[k] = 0;"),
     # ---- malformed input flags
     ("posinf_not_flagged", "return isnan(x) || (isinf(x) && x > 0);", "return isnan(x);"),
     ("neginf_flagged", "return isnan(x) || (isinf(x) && x > 0);",
