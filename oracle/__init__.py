@@ -75,27 +75,27 @@ def _load():
         lib.orc_uniform.restype = dbl
         lib.orc_uniform.argtypes = [u64] * 5
         lib.orc_row_probs.restype = u32
-        lib.orc_row_probs.argtypes = [vp, C.c_int, i32, dbl, dbl, vp, vp]
+        lib.orc_row_probs.argtypes = [vp, C.c_int, i32, dbl, i32, dbl, vp, vp]
         lib.orc_row_argmax.restype = i32
         lib.orc_row_argmax.argtypes = [vp, C.c_int, i32, vp]
         lib.orc_verify_one.restype = u32
         lib.orc_verify_one.argtypes = [vp, i64, vp, i64, C.c_int, vp, i32, i32,
-                                       dbl, dbl, vp, vp, vp, vp, vp, vp, vp]
+                                       dbl, i32, dbl, vp, vp, vp, vp, vp, vp, vp]
         lib.orc_verify_linear.restype = u32
         lib.orc_verify_linear.argtypes = [vp, i64, vp, i64, C.c_int, vp, i32,
-                                          i32, i32, dbl, dbl, u64, vp, u64, vp,
-                                          vp, vp, vp, vp]
+                                          i32, i32, dbl, i32, dbl, u64, vp, u64,
+                                          vp, vp, vp, vp, vp]
         lib.orc_verify_tree_greedy.restype = u32
         lib.orc_verify_tree_greedy.argtypes = [vp, i64, C.c_int, vp, vp, i32,
                                                i32, i32, vp, vp, vp]
         lib.orc_verify_tree_sampled_one.restype = u32
         lib.orc_verify_tree_sampled_one.argtypes = [vp, i64, C.c_int, vp, vp, i32,
-                                                    i32, dbl, dbl, vp, vp, vp, vp,
-                                                    vp, vp]
+                                                    i32, dbl, i32, dbl, vp, vp, vp,
+                                                    vp, vp, vp]
         lib.orc_verify_tree_sampled.restype = u32
         lib.orc_verify_tree_sampled.argtypes = [vp, i64, C.c_int, vp, vp, i32, i32,
-                                                i32, dbl, dbl, u64, vp, u64, vp, vp,
-                                                vp, vp]
+                                                i32, dbl, i32, dbl, u64, vp, u64, vp,
+                                                vp, vp, vp]
         _lib = lib
     return _lib
 
@@ -142,13 +142,13 @@ def uniforms(seed: int, seq_ids, step: int, n_rows: int, purpose: int) -> np.nda
 
 # ---- single rows -----------------------------------------------------------
 
-def row_probs(row: np.ndarray, temperature: float, top_p: float = 1.0):
+def row_probs(row: np.ndarray, temperature: float, top_p: float = 1.0, top_k: int = 0):
     """(probabilities float64[V], status bits, top-p margin) of one row."""
     row = _contig(row)
     V = row.shape[-1]
     out = np.empty(V, dtype=np.float64)
     margin = np.empty(1, dtype=np.float64)
-    st = _load().orc_row_probs(_ptr(row), _dtype_code(row), V, temperature,
+    st = _load().orc_row_probs(_ptr(row), _dtype_code(row), V, temperature, int(top_k),
                                top_p, _ptr(out), _ptr(margin))
     return out, int(st), float(margin[0])
 
@@ -162,7 +162,7 @@ def row_argmax(row: np.ndarray) -> int:
 
 # ---- linear verify ----------------------------------------------------------
 
-def verify_one(ar, draft, ids, temperature, top_p, u_accept, u_resid, V=None):
+def verify_one(ar, draft, ids, temperature, top_p, u_accept, u_resid, V=None, top_k=0):
     """One sequence with explicit uniforms.  ar [B+1, S], draft [B, S]."""
     ar = _contig(ar)
     code = _dtype_code(ar)
@@ -183,14 +183,14 @@ def verify_one(ar, draft, ids, temperature, top_p, u_accept, u_resid, V=None):
     margin = np.empty(1)
     st = _load().orc_verify_one(
         _ptr(ar), S, _ptr(draft), draft.shape[-1] if draft is not None else S,
-        code, _ptr(ids), B, V, temperature, top_p, _ptr(u_accept),
+        code, _ptr(ids), B, V, temperature, int(top_k), top_p, _ptr(u_accept),
         _ptr(u_resid), _ptr(tokens), _ptr(n), _ptr(p), _ptr(q), _ptr(margin))
     return dict(tokens=tokens, n_emitted=int(n[0]), p_draft=p, q_draft=q,
                 margin=float(margin[0]), status=int(st))
 
 
 def verify_linear(ar, draft, ids, temperature, top_p, seed, step, seq_ids=None,
-                  V=None):
+                  V=None, top_k=0):
     """Batch verify with the counter RNG.  ar [N, B+1, S], draft [N, B, S]."""
     ar = _contig(ar)
     code = _dtype_code(ar)
@@ -209,7 +209,7 @@ def verify_linear(ar, draft, ids, temperature, top_p, seed, step, seq_ids=None,
     margin = np.empty(N)
     st = _load().orc_verify_linear(
         _ptr(ar), S, _ptr(draft), draft.shape[-1] if draft is not None else S,
-        code, _ptr(ids), N, B, V, temperature, top_p, seed, _ptr(sid), step,
+        code, _ptr(ids), N, B, V, temperature, int(top_k), top_p, seed, _ptr(sid), step,
         _ptr(tokens), _ptr(n_em), _ptr(p), _ptr(q), _ptr(margin))
     return dict(tokens=tokens, n_emitted=n_em, p_draft=p, q_draft=q,
                 margin=margin, status=int(st))
@@ -238,7 +238,7 @@ def verify_tree_greedy(ar, node_tokens, parents, V=None):
 # ---- sampled tree ---------------------------------------------------------------
 
 def verify_tree_sampled_one(ar, node_tokens, parents, temperature, top_p, u_accept, u_resid,
-                            V=None):
+                            V=None, top_k=0):
     """One tree with explicit uniforms.  ar [M+1, S]; node_tokens, parents
     [M]; u_accept [M+1] (entry k+1 tests node k), u_resid [M+1] (by row)."""
     ar = _contig(ar)
@@ -256,14 +256,15 @@ def verify_tree_sampled_one(ar, node_tokens, parents, temperature, top_p, u_acce
     toks = np.empty(M + 1, dtype=np.int32)
     margin = np.empty(1)
     st = _load().orc_verify_tree_sampled_one(_ptr(ar), S, code, _ptr(tok), _ptr(par), M, V,
-                                             temperature, top_p, _ptr(ua), _ptr(ur),
+                                             temperature, int(top_k), top_p, _ptr(ua),
+                                             _ptr(ur),
                                              _ptr(path), _ptr(plen), _ptr(toks), _ptr(margin))
     return dict(path_nodes=path[:M], path_len=int(plen[0]), tokens=toks,
                 margin=float(margin[0]), status=int(st))
 
 
 def verify_tree_sampled(ar, node_tokens, parents, temperature, top_p, seed, step,
-                        seq_ids=None, V=None):
+                        seq_ids=None, V=None, top_k=0):
     """Batch sampled tree verify with the counter RNG.  ar [N, M+1, S];
     node_tokens, parents int32 [N, M]."""
     ar = _contig(ar)
@@ -279,6 +280,7 @@ def verify_tree_sampled(ar, node_tokens, parents, temperature, top_p, seed, step
     toks = np.empty((N, M + 1), dtype=np.int32)
     margin = np.empty(N)
     st = _load().orc_verify_tree_sampled(_ptr(ar), S, code, _ptr(tok), _ptr(par), N, M, V,
-                                         temperature, top_p, seed, _ptr(sid), step, _ptr(path),
+                                         temperature, int(top_k), top_p, seed, _ptr(sid), step,
+                                         _ptr(path),
                                          _ptr(plen), _ptr(toks), _ptr(margin))
     return dict(path_nodes=path, path_len=plen, tokens=toks, margin=margin, status=int(st))

@@ -25,6 +25,10 @@
  *  - Top-p keeps, after temperature, the smallest descending-probability
  *    set whose mass reaches top_p, together with every token tied with the
  *    last one admitted, then renormalises; applied to p and q alike.
+ *  - Top-k (run card: "top-k／top-p") is taken after temperature and before
+ *    top-p: every token whose probability is at least the k-th largest stays
+ *    (ties with the k-th included), renormalised; top-p then cuts that
+ *    distribution.  k = 0 or k >= V means off; applied to p and q alike.
  *  - Greedy ties resolve to the lowest vocabulary index.
  *  - Sampled tree (the pages give no rule): recursive rejection over each
  *    reached node's children in index order, each child its own point-mass
@@ -101,8 +105,8 @@ static int by_prob_desc(const void *a, const void *b) {
 }
 
 uint32_t orc_row_probs(const void *row, int dtype, int32_t V,
-                       double temperature, double top_p, double *out_prob,
-                       double *out_topp_margin) {
+                       double temperature, int32_t top_k, double top_p,
+                       double *out_prob, double *out_topp_margin) {
   uint32_t status = 0;
   if (out_topp_margin) *out_topp_margin = INFINITY;
 
@@ -128,6 +132,24 @@ uint32_t orc_row_probs(const void *row, int dtype, int32_t V,
     total += e;
   }
   for (int32_t v = 0; v < V; ++v) out_prob[v] /= total;
+
+  if (top_k > 0 && top_k < V) {
+    /* Top-k: the k-th largest probability is the threshold; ties with it
+     * stay.  Then renormalise. */
+    prob_id *sorted = (prob_id *)malloc((size_t)V * sizeof(prob_id));
+    for (int32_t v = 0; v < V; ++v) {
+      sorted[v].prob = out_prob[v];
+      sorted[v].id = v;
+    }
+    qsort(sorted, (size_t)V, sizeof(prob_id), by_prob_desc);
+    const double kth = sorted[top_k - 1].prob;
+    free(sorted);
+    double kept = 0.0;
+    for (int32_t v = 0; v < V; ++v)
+      if (out_prob[v] >= kth) kept += out_prob[v];
+    for (int32_t v = 0; v < V; ++v)
+      out_prob[v] = (out_prob[v] >= kth) ? out_prob[v] / kept : 0.0;
+  }
 
   if (top_p < 1.0) {
     /* Nucleus: sort, find the first prefix whose mass reaches top_p. */
@@ -231,7 +253,7 @@ static uint32_t verify_greedy_one(const void *ar, int64_t ar_row_stride,
 uint32_t orc_verify_one(const void *ar, int64_t ar_row_stride,
                         const void *draft, int64_t draft_row_stride,
                         int dtype, const int32_t *ids, int32_t B, int32_t V,
-                        double temperature, double top_p,
+                        double temperature, int32_t top_k, double top_p,
                         const double *u_accept, const double *u_resid,
                         int32_t *out_tokens, int32_t *out_n, double *out_p,
                         double *out_q, double *out_margin) {
@@ -253,9 +275,9 @@ uint32_t orc_verify_one(const void *ar, int64_t ar_row_stride,
    * step 3: the frozen AR scores the whole block in one pass). */
   for (int32_t i = 0; i < B; ++i) {
     status |= orc_row_probs(row_ptr(ar, dtype, ar_row_stride, i), dtype, V,
-                            temperature, top_p, p, &mp[i]);
+                            temperature, top_k, top_p, p, &mp[i]);
     status |= orc_row_probs(row_ptr(draft, dtype, draft_row_stride, i), dtype,
-                            V, temperature, top_p, q, &mq[i]);
+                            V, temperature, top_k, top_p, q, &mq[i]);
     int32_t x = ids[i];
     if (x >= 0 && x < V) {
       px[i] = p[x];
@@ -270,7 +292,7 @@ uint32_t orc_verify_one(const void *ar, int64_t ar_row_stride,
   }
   /* The bonus row is read too; its top-p margin matters only if used. */
   status |= orc_row_probs(row_ptr(ar, dtype, ar_row_stride, B), dtype, V,
-                          temperature, top_p, p, &mp[B]);
+                          temperature, top_k, top_p, p, &mp[B]);
 
   /* Longest accepted prefix: accept x_i while u_i < p_i(x_i)/q_i(x_i)
    * ([P1] "Psi-Spec이 한 스텝에서 하는 일"; [P3] walkthrough step 3). */
@@ -293,9 +315,9 @@ uint32_t orc_verify_one(const void *ar, int64_t ar_row_stride,
   int32_t token;
   if (L < B) {
     orc_row_probs(row_ptr(ar, dtype, ar_row_stride, L), dtype, V, temperature,
-                  top_p, p, NULL);
+                  top_k, top_p, p, NULL);
     orc_row_probs(row_ptr(draft, dtype, draft_row_stride, L), dtype, V,
-                  temperature, top_p, q, NULL);
+                  temperature, top_k, top_p, q, NULL);
     double residual_mass = 0.0;
     for (int32_t v = 0; v < V; ++v) {
       double r = p[v] - q[v];
@@ -306,7 +328,7 @@ uint32_t orc_verify_one(const void *ar, int64_t ar_row_stride,
   } else {
     margin = dmin(margin, mp[B]);
     orc_row_probs(row_ptr(ar, dtype, ar_row_stride, B), dtype, V, temperature,
-                  top_p, w, NULL);
+                  top_k, top_p, w, NULL);
   }
   token = inverse_cdf(w, V, u_resid[L], &sample_margin);
   margin = dmin(margin, sample_margin);
@@ -330,8 +352,8 @@ uint32_t orc_verify_one(const void *ar, int64_t ar_row_stride,
 uint32_t orc_verify_linear(const void *ar, int64_t ar_row_stride,
                            const void *draft, int64_t draft_row_stride,
                            int dtype, const int32_t *ids, int32_t N, int32_t B,
-                           int32_t V, double temperature, double top_p,
-                           uint64_t seed, const uint64_t *seq_ids,
+                           int32_t V, double temperature, int32_t top_k,
+                           double top_p, uint64_t seed, const uint64_t *seq_ids,
                            uint64_t step, int32_t *out_tokens,
                            int32_t *out_n_emitted, double *out_p_draft,
                            double *out_q_draft, double *out_margin) {
@@ -351,7 +373,7 @@ uint32_t orc_verify_linear(const void *ar, int64_t ar_row_stride,
                              : NULL;
     status |= orc_verify_one(
         ar_n, ar_row_stride, dr_n, draft_row_stride, dtype, ids + (size_t)n * B,
-        B, V, temperature, top_p, u_accept, u_resid,
+        B, V, temperature, top_k, top_p, u_accept, u_resid,
         out_tokens + (size_t)n * (B + 1), out_n_emitted + n,
         out_p_draft ? out_p_draft + (size_t)n * B : NULL,
         out_q_draft ? out_q_draft + (size_t)n * B : NULL,
@@ -465,7 +487,8 @@ uint32_t orc_verify_tree_sampled_one(const void *ar, int64_t ar_row_stride,
                                      int dtype, const int32_t *node_tokens,
                                      const int32_t *parents, int32_t M,
                                      int32_t V, double temperature,
-                                     double top_p, const double *u_accept,
+                                     int32_t top_k, double top_p,
+                                     const double *u_accept,
                                      const double *u_resid,
                                      int32_t *out_path_nodes,
                                      int32_t *out_path_len, int32_t *out_tokens,
@@ -492,7 +515,7 @@ uint32_t orc_verify_tree_sampled_one(const void *ar, int64_t ar_row_stride,
     const int32_t row = node + 1;
     double mtop;
     status |= orc_row_probs(row_ptr(ar, dtype, ar_row_stride, row), dtype, V,
-                            temperature, top_p, P, &mtop);
+                            temperature, top_k, top_p, P, &mtop);
     margin = dmin(margin, mtop);
     memcpy(w, P, (size_t)V * sizeof(double)); /* what remains of P */
     int32_t next = -1;
@@ -536,8 +559,9 @@ uint32_t orc_verify_tree_sampled_one(const void *ar, int64_t ar_row_stride,
 uint32_t orc_verify_tree_sampled(const void *ar, int64_t ar_row_stride,
                                  int dtype, const int32_t *node_tokens,
                                  const int32_t *parents, int32_t N, int32_t M,
-                                 int32_t V, double temperature, double top_p,
-                                 uint64_t seed, const uint64_t *seq_ids,
+                                 int32_t V, double temperature, int32_t top_k,
+                                 double top_p, uint64_t seed,
+                                 const uint64_t *seq_ids,
                                  uint64_t step, int32_t *out_path_nodes,
                                  int32_t *out_path_len, int32_t *out_tokens,
                                  double *out_margin) {
@@ -555,7 +579,7 @@ uint32_t orc_verify_tree_sampled(const void *ar, int64_t ar_row_stride,
     status |= orc_verify_tree_sampled_one(
         row_ptr(ar, dtype, ar_row_stride, (int64_t)n * (M + 1)), ar_row_stride,
         dtype, node_tokens + (size_t)n * M, parents + (size_t)n * M, M, V,
-        temperature, top_p, u_accept, u_resid,
+        temperature, top_k, top_p, u_accept, u_resid,
         out_path_nodes + (size_t)n * M, out_path_len + n,
         out_tokens + (size_t)n * (M + 1), out_margin ? out_margin + n : NULL);
   }

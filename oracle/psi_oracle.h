@@ -57,13 +57,16 @@ uint64_t orc_counter_hash(uint64_t seed, uint64_t seq, uint64_t step,
 double orc_uniform(uint64_t seed, uint64_t seq, uint64_t step, uint64_t row,
                    uint64_t purpose);
 
-/* Temperature softmax (plus optional top-p truncation and renormalisation)
- * of one logit row, in double.  out_prob[V].  Returns status bits.
- * out_topp_margin (may be NULL) receives the distance of the cumulative mass
- * on either side of the crossing from top_p (+inf when top-p is off). */
+/* Temperature softmax of one logit row, in double, then optional top-k
+ * (top_k > 0: keep every token at or above the k-th largest probability,
+ * renormalise) and optional top-p (top_p < 1: the smallest descending set
+ * of mass >= top_p with the ties of its last token, renormalise).
+ * out_prob[V].  Returns status bits.  out_topp_margin (may be NULL) receives
+ * the distance of the cumulative mass on either side of the top-p crossing
+ * from top_p (+inf when top-p is off). */
 uint32_t orc_row_probs(const void *row, int dtype, int32_t V,
-                       double temperature, double top_p, double *out_prob,
-                       double *out_topp_margin);
+                       double temperature, int32_t top_k, double top_p,
+                       double *out_prob, double *out_topp_margin);
 
 /* Verify one sequence with explicitly supplied uniforms.
  * u_accept[B]: acceptance uniforms; u_resid[B+1]: residual/bonus uniforms
@@ -75,7 +78,7 @@ uint32_t orc_row_probs(const void *row, int dtype, int32_t V,
 uint32_t orc_verify_one(const void *ar, int64_t ar_row_stride,
                         const void *draft, int64_t draft_row_stride,
                         int dtype, const int32_t *ids, int32_t B, int32_t V,
-                        double temperature, double top_p,
+                        double temperature, int32_t top_k, double top_p,
                         const double *u_accept, const double *u_resid,
                         int32_t *out_tokens, int32_t *out_n, double *out_p,
                         double *out_q, double *out_margin);
@@ -85,8 +88,8 @@ uint32_t orc_verify_one(const void *ar, int64_t ar_row_stride,
 uint32_t orc_verify_linear(const void *ar, int64_t ar_row_stride,
                            const void *draft, int64_t draft_row_stride,
                            int dtype, const int32_t *ids, int32_t N, int32_t B,
-                           int32_t V, double temperature, double top_p,
-                           uint64_t seed, const uint64_t *seq_ids,
+                           int32_t V, double temperature, int32_t top_k,
+                           double top_p, uint64_t seed, const uint64_t *seq_ids,
                            uint64_t step, int32_t *out_tokens,
                            int32_t *out_n_emitted, double *out_p_draft,
                            double *out_q_draft, double *out_margin);
@@ -115,7 +118,8 @@ uint32_t orc_verify_tree_sampled_one(const void *ar, int64_t ar_row_stride,
                                      int dtype, const int32_t *node_tokens,
                                      const int32_t *parents, int32_t M,
                                      int32_t V, double temperature,
-                                     double top_p, const double *u_accept,
+                                     int32_t top_k, double top_p,
+                                     const double *u_accept,
                                      const double *u_resid,
                                      int32_t *out_path_nodes,
                                      int32_t *out_path_len, int32_t *out_tokens,
@@ -128,8 +132,9 @@ uint32_t orc_verify_tree_sampled_one(const void *ar, int64_t ar_row_stride,
 uint32_t orc_verify_tree_sampled(const void *ar, int64_t ar_row_stride,
                                  int dtype, const int32_t *node_tokens,
                                  const int32_t *parents, int32_t N, int32_t M,
-                                 int32_t V, double temperature, double top_p,
-                                 uint64_t seed, const uint64_t *seq_ids,
+                                 int32_t V, double temperature, int32_t top_k,
+                                 double top_p, uint64_t seed,
+                                 const uint64_t *seq_ids,
                                  uint64_t step, int32_t *out_path_nodes,
                                  int32_t *out_path_len, int32_t *out_tokens,
                                  double *out_margin);

@@ -72,7 +72,7 @@ def _sup_true(pred, iters=60):
     return hi
 
 
-def _correction_law(ar, draft, ids, pos, T, top_p, u_accept):
+def _correction_law(ar, draft, ids, pos, T, top_p, u_accept, top_k=0):
     """Law of the token emitted at `pos` when the step stops there, as a
     function of the residual uniform, measured interval by interval."""
     B, V = ar.shape[0] - 1, ar.shape[1]
@@ -80,7 +80,7 @@ def _correction_law(ar, draft, ids, pos, T, top_p, u_accept):
     def token(u2):
         ur = np.full(B + 1, 0.5)
         ur[pos] = u2
-        r = oracle.verify_one(ar, draft, ids, T, top_p, u_accept, ur)
+        r = oracle.verify_one(ar, draft, ids, T, top_p, u_accept, ur, top_k=top_k)
         assert r["n_emitted"] == pos + 1
         return int(r["tokens"][pos])
 
@@ -93,11 +93,11 @@ def _correction_law(ar, draft, ids, pos, T, top_p, u_accept):
     return law
 
 
-def emission_law(ar, draft, ids, pos, T, top_p, q_pos):
+def emission_law(ar, draft, ids, pos, T, top_p, q_pos, top_k=0):
     """P(token at pos = v | the step reached pos), drafts at pos ~ q_pos."""
     B, V = ar.shape[0] - 1, ar.shape[1]
     if pos == B:
-        return _correction_law(ar, draft, ids, pos, T, top_p, np.zeros(B))
+        return _correction_law(ar, draft, ids, pos, T, top_p, np.zeros(B), top_k)
     law = np.zeros(V)
     for x in range(V):
         if q_pos[x] == 0.0:
@@ -108,7 +108,8 @@ def emission_law(ar, draft, ids, pos, T, top_p, q_pos):
         def accepted(u):
             ua = np.zeros(B)
             ua[pos] = u
-            r = oracle.verify_one(ar, draft, ids_x, T, top_p, ua, np.full(B + 1, 0.5))
+            r = oracle.verify_one(ar, draft, ids_x, T, top_p, ua, np.full(B + 1, 0.5),
+                                  top_k=top_k)
             return r["n_emitted"] > pos + 1
 
         a = _sup_true(accepted)
@@ -116,14 +117,15 @@ def emission_law(ar, draft, ids, pos, T, top_p, q_pos):
         if a < 1.0:
             ua = np.zeros(B)
             ua[pos] = NEXT1
-            law += q_pos[x] * (1.0 - a) * _correction_law(ar, draft, ids_x, pos, T, top_p, ua)
+            law += q_pos[x] * (1.0 - a) * _correction_law(ar, draft, ids_x, pos, T, top_p, ua,
+                                                          top_k)
     return law
 
 
-def _target(row, T, top_p):
-    if top_p >= 1.0:
+def _target(row, T, top_p, top_k=0):
+    if top_p >= 1.0 and top_k == 0:
         return softmax(row.astype(np.float64) / T)
-    return oracle.row_probs(row, T, top_p)[0]
+    return oracle.row_probs(row, T, top_p, top_k)[0]  # pinned by the hand cases below
 
 
 @pytest.mark.parametrize("case", range(12))
@@ -353,6 +355,75 @@ def test_top_p_limits():
         want = np.zeros(257)
         want[[5, 77]] = 0.5
         np.testing.assert_allclose(p, want, atol=1e-15)
+
+
+# ---- top-k (run card: "top-k／top-p") ---------------------------------------------
+
+def test_top_k_hand_cases():
+    ln = np.log(np.array([0.5, 0.3, 0.15, 0.05]))
+    np.testing.assert_allclose(_probs_k(ln, 1.0, 2), [0.625, 0.375, 0, 0], atol=1e-7)
+    np.testing.assert_allclose(_probs_k(ln, 1.0, 3), [0.5 / 0.95, 0.3 / 0.95, 0.15 / 0.95, 0],
+                               atol=1e-7)
+    np.testing.assert_allclose(_probs_k(ln, 1.0, 1), [1, 0, 0, 0], atol=1e-7)
+    for k in (0, 4, 9):  # off
+        np.testing.assert_allclose(_probs_k(ln, 1.0, k), [0.5, 0.3, 0.15, 0.05], atol=1e-7)
+    # another vocabulary order, and temperature first: T = 0.5 squares
+    perm = [2, 0, 3, 1]
+    np.testing.assert_allclose(_probs_k(ln[perm], 1.0, 2), [0, 0.625, 0, 0.375], atol=1e-7)
+    np.testing.assert_allclose(_probs_k(ln, 0.5, 2), [0.25 / 0.34, 0.09 / 0.34, 0, 0], atol=1e-7)
+
+
+def test_top_k_keeps_ties_with_the_kth():
+    np.testing.assert_allclose(_probs_k([1, 1, 1, 0], 1.0, 2), [1 / 3, 1 / 3, 1 / 3, 0],
+                               atol=1e-7)
+    np.testing.assert_allclose(_probs_k([2, 1, 1, 0], 1.0, 2),
+                               softmax([2.0, 1, 1]).tolist() + [0], atol=1e-7)
+
+
+def test_top_k_comes_before_top_p():
+    # top-k 3 renormalises to (.526, .316, .158); top-p 0.82 then stops at
+    # .842 (two tokens).  top-p first would keep three (.5, .8, .95).
+    ln = np.log(np.array([0.5, 0.3, 0.15, 0.05]))
+    np.testing.assert_allclose(_probs_k(ln, 1.0, 3, 0.82), [0.625, 0.375, 0, 0], atol=1e-7)
+    np.testing.assert_allclose(_probs(ln, 1.0, 0.82), [0.5 / 0.95, 0.3 / 0.95, 0.15 / 0.95, 0],
+                               atol=1e-7)
+
+
+def _probs_k(vals, T, top_k, top_p=1.0):
+    p, st, _ = oracle.row_probs(np.asarray(vals, dtype=np.float32), T, top_p, top_k)
+    assert st == 0
+    return p
+
+
+def test_top_k_one_is_greedy_decoding():
+    """k = 1 leaves each distribution a point mass on its argmax: with the
+    draft's argmax drafted, the sampled rule is the greedy rule."""
+    rng = np.random.default_rng(15)
+    N, B, V = 50, 5, 20
+    ar = rng.normal(0, 1, (N, B + 1, V)).astype(np.float32)
+    draft = (ar[:, :B] + rng.normal(0, 0.5, (N, B, V))).astype(np.float32)
+    ids = np.argmax(draft, axis=-1).astype(np.int32)
+    s = oracle.verify_linear(ar, draft, ids, 0.9, 1.0, seed=4, step=0, top_k=1)
+    g = oracle.verify_linear(ar, None, ids, 0.0, 1.0, seed=4, step=0)
+    assert np.array_equal(s["tokens"], g["tokens"])
+    assert 1 < g["n_emitted"].mean() < B + 1
+
+
+@pytest.mark.parametrize("case", range(4))
+def test_lossless_exact_top_k(case):
+    rng = np.random.default_rng(2000 + case)
+    V, B = 6, 2
+    T = [1.0, 0.7][case % 2]
+    top_k = [2, 4][case // 2]
+    top_p = [1.0, 0.9][case % 2]
+    ar = rng.normal(0, 1.5, (B + 1, V)).astype(np.float32)
+    draft = rng.normal(0, 1.5, (B, V)).astype(np.float32)
+    ids = np.array([int(np.argmax(ar[i])) for i in range(B)], dtype=np.int32)
+    for pos in (0, 1, B):
+        q_pos = _target(draft[pos], T, top_p, top_k) if pos < B else None
+        law = emission_law(ar, draft, ids, pos, T, top_p, q_pos, top_k)
+        np.testing.assert_allclose(law, _target(ar[pos], T, top_p, top_k), rtol=0, atol=1e-12,
+                                   err_msg=f"pos {pos}")
 
 
 def test_bf16_rows_decode_exactly():

@@ -67,18 +67,34 @@ MUTANTS = [
     ("topp_not_renormalised", "(out_prob[v] >= tau) ? out_prob[v] / kept : 0.0;",
      "(out_prob[v] >= tau) ? out_prob[v] : 0.0;"),
     ("topp_not_applied_to_draft_at_acceptance",
-     "                            V, temperature, top_p, q, &mq[i]);",
-     "                            V, temperature, 1.0, q, &mq[i]);"),
+     "                            V, temperature, top_k, top_p, q, &mq[i]);",
+     "                            V, temperature, top_k, 1.0, q, &mq[i]);"),
     ("topp_not_applied_to_draft_in_residual",
      "    orc_row_probs(row_ptr(draft, dtype, draft_row_stride, L), dtype, V,\n"
-     "                  temperature, top_p, q, NULL);",
+     "                  temperature, top_k, top_p, q, NULL);",
      "    orc_row_probs(row_ptr(draft, dtype, draft_row_stride, L), dtype, V,\n"
-     "                  temperature, 1.0, q, NULL);"),
+     "                  temperature, top_k, 1.0, q, NULL);"),
     ("topp_not_applied_to_bonus",
      "    orc_row_probs(row_ptr(ar, dtype, ar_row_stride, B), dtype, V, temperature,\n"
-     "                  top_p, w, NULL);",
+     "                  top_k, top_p, w, NULL);",
      "    orc_row_probs(row_ptr(ar, dtype, ar_row_stride, B), dtype, V, temperature,\n"
-     "                  1.0, w, NULL);"),
+     "                  top_k, 1.0, w, NULL);"),
+    # ---- top-k (before top-p)
+    ("topk_drops_kth_ties", "(out_prob[v] >= kth) ? out_prob[v] / kept : 0.0;",
+     "(out_prob[v] > kth) ? out_prob[v] / kept : 0.0;"),
+    ("topk_threshold_one_late", "    const double kth = sorted[top_k - 1].prob;",
+     "    const double kth = sorted[top_k].prob;"),
+    ("topk_not_renormalised", "(out_prob[v] >= kth) ? out_prob[v] / kept : 0.0;",
+     "(out_prob[v] >= kth) ? out_prob[v] : 0.0;"),
+    ("topk_one_treated_as_off", "  if (top_k > 0 && top_k < V) {", "  if (top_k > 1 && top_k < V) {"),
+    ("topk_not_applied_to_draft_at_acceptance",
+     "                            V, temperature, top_k, top_p, q, &mq[i]);",
+     "                            V, temperature, 0, top_p, q, &mq[i]);"),
+    ("topk_not_applied_to_bonus",
+     "    orc_row_probs(row_ptr(ar, dtype, ar_row_stride, B), dtype, V, temperature,\n"
+     "                  top_k, top_p, w, NULL);",
+     "    orc_row_probs(row_ptr(ar, dtype, ar_row_stride, B), dtype, V, temperature,\n"
+     "                  0, top_p, w, NULL);"),
     # ---- acceptance test u < p(x) / q(x)
     ("accept_non_strict", "int accept = u_accept[i] * qx[i] < px[i];",
      "int accept = u_accept[i] * qx[i] <= px[i];"),
@@ -99,9 +115,9 @@ MUTANTS = [
      "    orc_row_probs(row_ptr(ar, dtype, ar_row_stride, L + 1), dtype, V, temperature,"),
     ("bonus_reads_last_draft_position",
      "    orc_row_probs(row_ptr(ar, dtype, ar_row_stride, B), dtype, V, temperature,\n"
-     "                  top_p, w, NULL);",
+     "                  top_k, top_p, w, NULL);",
      "    orc_row_probs(row_ptr(ar, dtype, ar_row_stride, B - 1), dtype, V, temperature,\n"
-     "                  top_p, w, NULL);"),
+     "                  top_k, top_p, w, NULL);"),
     ("correction_uses_first_row_uniform",
      "token = inverse_cdf(w, V, u_resid[L], &sample_margin);",
      "token = inverse_cdf(w, V, u_resid[0], &sample_margin);"),

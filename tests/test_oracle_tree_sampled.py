@@ -31,8 +31,8 @@ def _logp(rows):
         return np.log(np.asarray(rows, dtype=np.float64)).astype(np.float32)
 
 
-def _one(ar, tok, par, ua, ur, T=1.0, top_p=1.0):
-    return oracle.verify_tree_sampled_one(ar, tok, par, T, top_p, ua, ur)
+def _one(ar, tok, par, ua, ur, T=1.0, top_p=1.0, top_k=0):
+    return oracle.verify_tree_sampled_one(ar, tok, par, T, top_p, ua, ur, top_k=top_k)
 
 
 # ---- hand-worked cases ---------------------------------------------------------
@@ -117,14 +117,14 @@ def _children(par, node):
     return [k for k in range(len(par)) if par[k] == node]
 
 
-def oracle_sequence_law(ar, tok, par, T, top_p):
+def oracle_sequence_law(ar, tok, par, T, top_p, top_k=0):
     """P(emitted token sequence), integrated over the verify's uniforms with
     the oracle as a black box."""
     M, V = len(tok), ar.shape[1]
     law = {}
 
     def run(ua, ur):
-        return _one(ar, tok, par, ua, ur, T, top_p)
+        return _one(ar, tok, par, ua, ur, T, top_p, top_k)
 
     def visit(node, depth, prefix, weight, ua, ur):
         ua = ua.copy()
@@ -162,20 +162,20 @@ def oracle_sequence_law(ar, tok, par, T, top_p):
     return law
 
 
-def _target(row, T, top_p):
-    if top_p >= 1.0:
+def _target(row, T, top_p, top_k=0):
+    if top_p >= 1.0 and top_k == 0:
         return softmax(row.astype(np.float64) / T)
-    return oracle.row_probs(row, T, top_p)[0]  # top-p is pinned on its own
+    return oracle.row_probs(row, T, top_p, top_k)[0]  # top-k / top-p are pinned on their own
 
 
-def target_sequence_law(ar, tok, par, T, top_p):
+def target_sequence_law(ar, tok, par, T, top_p, top_k=0):
     """The autoregressive law the step must reproduce: at a node, token v has
     the row's target probability; it continues at the first child carrying v,
     or ends the step."""
     law = {}
 
     def visit(node, prefix, weight):
-        P = _target(ar[node + 1], T, top_p)
+        P = _target(ar[node + 1], T, top_p, top_k)
         first = {}
         for k in _children(par, node):
             first.setdefault(tok[k], k)
@@ -206,14 +206,15 @@ TREES = {
 
 
 @pytest.mark.parametrize("name", sorted(TREES))
-@pytest.mark.parametrize("T,top_p", [(1.0, 1.0), (0.7, 1.0), (1.0, 0.8)])
-def test_lossless_exact_hand_trees(name, T, top_p):
+@pytest.mark.parametrize("T,top_p,top_k", [(1.0, 1.0, 0), (0.7, 1.0, 0), (1.0, 0.8, 0),
+                                           (0.9, 1.0, 3)])
+def test_lossless_exact_hand_trees(name, T, top_p, top_k):
     par, tok = TREES[name]
     rng = np.random.default_rng(sorted(TREES).index(name))
     ar = rng.normal(0, 1.5, (len(par) + 1, 5)).astype(np.float32)
     ar[0, 4] = -np.inf  # a token the root can never emit
-    _assert_same_law(oracle_sequence_law(ar, tok, par, T, top_p),
-                     target_sequence_law(ar, tok, par, T, top_p))
+    _assert_same_law(oracle_sequence_law(ar, tok, par, T, top_p, top_k),
+                     target_sequence_law(ar, tok, par, T, top_p, top_k))
 
 
 @pytest.mark.parametrize("case", range(6))
