@@ -68,13 +68,46 @@ def hbm_peak():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
-    h = hashlib.sha256()
+def strip_c_comments(text: str) -> str:
+    """C / CUDA source as the compiler sees it: comments removed (string and
+    character literals kept whole), trailing spaces and blank lines dropped."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        else:
+            out.append(c)
+            i += 1
+    lines = [ln.rstrip() for ln in "".join(out).splitlines()]
+    return "\n".join(ln for ln in lines if ln)
+
+
+def kernel_source_files():
     files = sorted(glob.glob(os.path.join(ROOT, "rejection_sampling_verify_b200", "csrc", "*")))
-    for f in files + [os.path.join(ROOT, "include", "psi_verify.h")]:
-        with open(f, "rb") as fh:
+    return files + [os.path.join(ROOT, "include", "psi_verify.h")]
+
+
+def kernel_source_hash() -> str:
+    """First 16 hex digits of SHA-256 over the kernel sources' code (comments
+    and blank lines removed): a comment-only edit keeps it, any code change
+    does not."""
+    h = hashlib.sha256()
+    for f in kernel_source_files():
+        with open(f, encoding="utf-8") as fh:
             h.update(os.path.basename(f).encode())
-            h.update(fh.read())
+            h.update(strip_c_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -603,11 +603,11 @@ __device__ __forceinline__ uint32_t fixed31(float m) { return __float2uint_rn(m 
 // Row maximum, Z, top-p threshold tau and renormaliser Z' of row r from its
 // record and candidate list, by one warp.  The top-p threshold is the largest
 // logit key t whose suffix mass S(t) (every x with key >= t) reaches
-// top_p * Z: a binary search over the candidates' key range with fp32 partial
-// sums (a step may differ from exact arithmetic only within ~1e-7 of the
-// target), then S(tau) exactly in fixed point.  Only candidates can be at or
-// above tau when they hold at least top_p of the mass.  The global candidate
-// list stays unchanged, so a second pass may finish the row again.
+// top_p * Z: a binary search over the candidates' key range on exact 2^31
+// fixed-point sums of the masses (integer sums: independent of candidate
+// order).  Only candidates can be at or above tau when they hold at least
+// top_p of the mass.  The global candidate list stays unchanged, so a second
+// pass may finish the row again.
 template <typename Bits>
 __device__ RowFinal finish_row(const FastArgs &a, int64_t r, WarpScratch *ws) {
   const int lane = threadIdx.x & 31;

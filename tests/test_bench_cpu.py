@@ -1,7 +1,11 @@
 """Host logic of the benchmark: the early-exit round schedule it assumes
-matches the header's constants, and its byte accounting is the per-row sum
-it claims to be."""
+matches the header's constants, its byte accounting is the per-row sum it
+claims to be, and the kernel-source hash that ties a committed ncu capture
+to the code it measured ignores comments only."""
+import os
 import re
+import shutil
+import subprocess
 
 import numpy as np
 
@@ -56,3 +60,41 @@ def test_main_launch_bytes_is_the_first_round():
     t = CFG["tree_greedy"]
     assert bench.main_launch_bytes(t) == bench.algorithmic_bytes(t)
     assert bench.algorithmic_bytes(cfg) == 1322450944
+
+
+# ---- the kernel-source hash behind `traffic` ----------------------------------------
+
+def test_comment_stripping_matches_the_compiler():
+    """gcc's own comment removal (-fpreprocessed) leaves the same code, up to
+    whitespace (gcc also drops `#pragma once` from a main file)."""
+    for f in bench.kernel_source_files():
+        text = open(f, encoding="utf-8").read()
+        mine = "".join(bench.strip_c_comments(text).split()).replace("#pragmaonce", "")
+        g = subprocess.run(["gcc", "-fpreprocessed", "-dD", "-E", "-P", "-x", "c++", f],
+                           capture_output=True, text=True, check=True)
+        assert mine == "".join(g.stdout.split()), os.path.basename(f)
+
+
+def test_strip_keeps_literals_and_code():
+    src = 'a = "// not a comment"; /* gone */ b = \'/\'; // gone\nc = "x\\"y"; /*\n*/ d;'
+    out = bench.strip_c_comments(src)
+    assert '"// not a comment"' in out and "'/'" in out and '"x\\"y"' in out
+    # a block comment is one space, even across lines
+    assert "gone" not in out and out.splitlines()[-1] == 'c = "x\\"y";   d;'
+
+
+def test_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    root = tmp_path / "repo"
+    shutil.copytree(os.path.join(bench.ROOT, "rejection_sampling_verify_b200", "csrc"),
+                    root / "rejection_sampling_verify_b200" / "csrc")
+    (root / "include").mkdir()
+    shutil.copy(os.path.join(bench.ROOT, "include", "psi_verify.h"), root / "include")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    h0 = bench.kernel_source_hash()
+    assert h0 == bench.kernel_source_hash()
+    f = root / "rejection_sampling_verify_b200" / "csrc" / "psi_fast.cu"
+    text = f.read_text()
+    f.write_text("// a new comment line\n\n" + text.replace("\n", "  \n", 3) + "\n/* and a block */\n")
+    assert bench.kernel_source_hash() == h0
+    f.write_text(text.replace("kInFlight = 8", "kInFlight = 4", 1))
+    assert bench.kernel_source_hash() != h0
