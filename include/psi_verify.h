@@ -26,12 +26,16 @@
  *    library allocates nothing and keeps no data between calls (only
  *    per-device launch settings, made on a device's first call).
  *  - Calls are asynchronous on `stream` (NULL = the legacy default stream).
+ *    After a device's first call, a call only launches work on `stream`, so
+ *    it can be captured into a CUDA graph; its scalar arguments (seed, step,
+ *    sizes) are then fixed in the graph.
  *  - Argument errors are detected on the host before any launch and
  *    returned as a psi_status; nothing is launched in that case.
  *  - Data errors found on the device (an id outside [0, V), a bad parent
  *    index, a NaN or +inf logit) are OR-ed into *dev_status (a caller-owned
  *    device uint32 that the caller zeroes; NULL = not reported).  The
- *    kernels always run to completion: they never trap, spin or hang.
+ *    kernels always run to completion: they never trap, and the only waits
+ *    (for bulk copies into shared memory) give up after a time limit.
  *  - Logits are bfloat16 or float32, row-major; `*_row_stride` is the
  *    distance between consecutive rows in ELEMENTS (>= V).  Sampled rows
  *    whose start is 16-byte aligned take the streaming path, others the
@@ -61,7 +65,8 @@ typedef enum psi_status {
   PSI_ERR_UNSUPPORTED = 3, /* valid but beyond this build (e.g. V too large) */
   PSI_ERR_CUDA = 4,        /* a CUDA launch or query failed */
   PSI_ERR_WORKSPACE = 5,   /* workspace NULL or smaller than the query says */
-  PSI_ERR_TIMEOUT = 6      /* reserved: no kernel here waits on anything */
+  PSI_ERR_TIMEOUT = 6      /* reserved, not returned: a kernel's wait that
+                              gives up sets PSI_DEV_TIMEOUT instead */
 } psi_status;
 
 typedef enum psi_dtype { PSI_DTYPE_F32 = 0, PSI_DTYPE_BF16 = 1 } psi_dtype;
@@ -130,15 +135,14 @@ size_t psi_verify_linear_workspace_bytes(int32_t N, int32_t B, int32_t V,
  * out_p_draft, out_q_draft  float [N][B] or NULL: p_i(x_i), q_i(x_i) after
  *               top-p (T > 0 only; not written when T == 0).
  * Early exit (both out_p_draft and out_q_draft NULL, N >= PSI_EARLY_EXIT_MIN_N,
- *   any T): rows after a
- *   sequence's first rejection (or greedy mismatch) do not change its
- *   result, so positions are verified in rounds (PSI_ROUND_POSITIONS
- *   positions each for the first PSI_SAMPLED_SHORT_ROUNDS or
- *   PSI_GREEDY_SHORT_ROUNDS rounds, then the rest) and a sequence takes part
- *   in a round only if every draft of the earlier rounds was accepted.  Tokens and counts are the
- *   same as with every row read; the NONFINITE status bit then covers the
- *   rows that were read.  A caller passing p / q buffers (for T == 0 they
- *   are not written) gets every row read.
+ *   any T): rows after a sequence's first rejection (or greedy mismatch) do
+ *   not change its result, so positions are verified in rounds
+ *   (PSI_ROUND_POSITIONS positions each for the first PSI_SAMPLED_SHORT_ROUNDS
+ *   or PSI_GREEDY_SHORT_ROUNDS rounds, then the rest), and a sequence takes
+ *   part in a round only if every draft of the earlier rounds was accepted.
+ *   Tokens and counts are the same as with every row read; the NONFINITE
+ *   status bit then covers the rows that were read.  A caller passing p / q
+ *   buffers (for T == 0 they are not written) gets every row read.
  * Limits: 1 <= N, 1 <= B <= PSI_MAX_B, 1 <= V <= PSI_MAX_V, T >= 0 and
  *   finite, 0 < top_p <= 1.
  */

@@ -187,8 +187,10 @@ psi_status psi_verify_linear(const void *ar_logits, int64_t ar_row_stride,
   a.out_q = out_q_draft;
   a.dev_status = dev_status;
   a.records = static_cast<psi::UnitRecord *>(workspace);
-  // Streaming path when every row starts on a 16-byte boundary (TMA bulk
-  // copies); otherwise one cluster per unit with plain loads.
+  // The streaming path needs every row to start on a 16-byte boundary (its
+  // loads are 16-byte vectors); other rows go to one cluster per unit, which
+  // bulk-copies the aligned part of each row slice and loads the rest
+  // element by element.
   const bool rows_aligned = aligned_to(ar_logits, 16) && aligned_to(draft_logits, 16) &&
                             ((size_t)ar_row_stride * es) % 16 == 0 &&
                             ((size_t)draft_row_stride * es) % 16 == 0;

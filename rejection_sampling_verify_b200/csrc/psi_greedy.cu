@@ -260,7 +260,9 @@ size_t round_up256(size_t x) { return (x + 255) / 256 * 256; }
 ArgmaxPlan plan_argmax(int64_t rows, int32_t V, int elem_bytes) {
   ArgmaxPlan p;
   const int vec = 16 / elem_bytes;
-  // Aim for at least ~8 waves of CTAs over the SMs, but keep chunks >= 16 KB.
+  // Aim for about 8 waves of 4 resident CTAs on each of a B200's 148 SMs, but
+  // keep chunks >= 16 KB.  The split tunes speed only: the packed maxima make
+  // the result the same for any split.
   const int64_t want_ctas = 148LL * 8 * 4;
   int64_t splits = (want_ctas + rows - 1) / rows;
   const int64_t min_chunk = 16384 / elem_bytes;

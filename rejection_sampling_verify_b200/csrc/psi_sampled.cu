@@ -15,8 +15,9 @@
 //
 // Design.  One thread-block cluster of C CTAs handles one (sequence, row)
 // unit: AR row i with draft row i (i < B), or the bonus AR row B alone.  CTA
-// k of the cluster bulk-copies (TMA, no multicast) its 1/C slice of both rows
-// into its own shared memory ONCE; every later pass (max, sum of exponentials,
+// k of the cluster brings its 1/C slice of both rows into its own shared
+// memory ONCE (bulk copies, no multicast, when the slice starts on a 16-byte
+// boundary; element loads otherwise); every later pass (max, sum of exponentials,
 // top-p radix select, the correction / bonus draw) reads shared memory, and
 // the cluster combines per-CTA partials through distributed shared memory.
 // Each unit decides its own draft (accept or reject) redundantly in every
