@@ -426,6 +426,60 @@ def test_lossless_exact_top_k(case):
                                    err_msg=f"pos {pos}")
 
 
+# ---- near-tie margins (O14) ----------------------------------------------------------
+# The smallest distance of any decision from its threshold: each acceptance
+# ratio, the top-p crossing (both sides) of every row used, and the draw's
+# crossing (both sides).  The GPU parity tests excuse token differences only
+# below 1e-5 of it, so each term is pinned by a case where it is the smallest.
+
+def _margin(ar_p, dr_p, x, ua, ur, top_p=1.0):
+    r = oracle.verify_one(_logp(ar_p), _logp(dr_p), [x], 1.0, top_p, ua, ur)
+    return r["margin"], r
+
+
+def _logp(rows):
+    with np.errstate(divide="ignore"):
+        return np.log(np.asarray(rows, dtype=np.float64)).astype(np.float32)
+
+
+def test_margin_acceptance_ratio_and_draw():
+    ar_p = [[0.5, 0.3, 0.2], [0.6, 0.2, 0.2]]
+    dr_p = [[0.2, 0.6, 0.2]]
+    # x = 1: p/q = 0.5; u = 0.7 rejects (distance 0.2); the residual (.3, 0, 0)
+    # gives token 0, the draw at 0.5 is 0.5 from both crossings
+    m, r = _margin(ar_p, dr_p, 1, [0.7], [0.5, 0.5])
+    assert r["tokens"].tolist() == [0, -1] and abs(m - 0.2) < 1e-6
+    # u = 0.99 (distance 0.49); the draw at 0.05 is 0.05 above the lower
+    # crossing and 0.95 below the upper one
+    m, r = _margin(ar_p, dr_p, 1, [0.99], [0.05, 0.5])
+    assert r["tokens"].tolist() == [0, -1] and abs(m - 0.05) < 1e-6
+
+
+def test_margin_top_p_crossings_of_draft_and_bonus_rows():
+    # top_p = 0.52 everywhere.  AR row 0 (.4, .35, .15, .1): crossing masses
+    # .4 / .75, margin .12.  Draft (.3, .51, .1, .09): .51 / .81, margin .01.
+    # x = 1 accepted at u = .2 (ratio .741); bonus row (.7, .1, .1, .1): 0 / .7,
+    # margin .18; the bonus draw (.7 alone) is .5 from both crossings.
+    m, r = _margin([[0.4, 0.35, 0.15, 0.1], [0.7, 0.1, 0.1, 0.1]],
+                   [[0.3, 0.51, 0.1, 0.09]], 1, [0.2], [0.5, 0.5], top_p=0.52)
+    assert r["n_emitted"] == 2 and abs(m - 0.01) < 1e-6
+    # the bonus row's crossing the smallest: bonus (.515, .3, .1, .085) gives
+    # .515 / .815 (margin .005); draft (.3, .6, .05, .05): 0 / .6 (.08)
+    m, r = _margin([[0.4, 0.35, 0.15, 0.1], [0.515, 0.3, 0.1, 0.085]],
+                   [[0.3, 0.6, 0.05, 0.05]], 1, [0.1], [0.5, 0.3], top_p=0.52)
+    assert r["n_emitted"] == 2 and r["tokens"].tolist() == [1, 0] and abs(m - 0.005) < 1e-6
+
+
+def test_top_p_margin_is_two_sided():
+    ln = np.log(np.array([0.5, 0.3, 0.15, 0.05]))
+    # crossing between .5 and .8: distances .02 (below) and .28 (above)
+    _, _, m = oracle.row_probs(ln.astype(np.float32), 1.0, 0.52)
+    assert abs(m - 0.02) < 1e-6
+    _, _, m = oracle.row_probs(ln.astype(np.float32), 1.0, 0.78)
+    assert abs(m - 0.02) < 1e-6
+    assert oracle.row_probs(ln.astype(np.float32), 1.0, 1.0)[2] == np.inf
+
+
 def test_bf16_rows_decode_exactly():
     # hand-written bfloat16 bit patterns of 1, 0.5, -1, 2, 0, 3, -inf, -2
     bits = np.array([0x3F80, 0x3F00, 0xBF80, 0x4000, 0x0000, 0x4040, 0xFF80, 0xC000],

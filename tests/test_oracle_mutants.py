@@ -162,6 +162,24 @@ MUTANTS = [
      "    out_tokens[depth] = next;"),
     ("stree_bad_parent_not_flagged", "      status |= ORC_BAD_PARENT;\n      valid[k] = 0;",
      "      valid[k] = 0;"),
+    # ---- near-tie margins (the GPU parity tests excuse token differences only
+    # within them, so a margin that is too wide would hide a real mismatch)
+    ("margin_skips_acceptance_ratio",
+     "    if (qx[i] > 0.0) margin = dmin(margin, fabs(u_accept[i] - px[i] / qx[i]));",
+     "    (void)0;"),
+    ("margin_skips_the_draw", "  margin = dmin(margin, sample_margin);", "  (void)sample_margin;"),
+    ("margin_skips_draft_top_p", "    margin = dmin(margin, dmin(mp[i], mq[i]));",
+     "    margin = dmin(margin, mp[i]);"),
+    ("margin_skips_bonus_top_p", "    margin = dmin(margin, mp[B]);", "    (void)mp;"),
+    ("icdf_margin_one_side",
+     "      *margin = dmin(fabs(u - before / total), fabs(u - running / total));",
+     "      *margin = fabs(u - running / total);"),
+    ("topp_margin_one_side",
+     "      *out_topp_margin = dmin(fabs(above - top_p), fabs(kept - top_p));",
+     "      *out_topp_margin = fabs(kept - top_p);"),
+    ("stree_margin_skips_tests", "      if (R > 0.0) margin = dmin(margin, fabs(u - px / R));",
+     "      (void)0;"),
+    ("stree_margin_skips_top_p", "    margin = dmin(margin, mtop);", "    (void)mtop;"),
     # ---- malformed input flags
     ("posinf_not_flagged", "return isnan(x) || (isinf(x) && x > 0);", "return isnan(x);"),
     ("neginf_flagged", "return isnan(x) || (isinf(x) && x > 0);",

@@ -84,6 +84,16 @@ def test_leaf_root_is_a_plain_draw():
     assert r["path_len"] == 0 and r["tokens"].tolist() == [1, -1]  # 0.5, 0.8 > 0.55
 
 
+def test_margin_includes_the_node_rows_top_p_crossing():
+    # root (.515, .3, .1, .085) at top_p .52: crossing masses .515 / .815,
+    # margin .005; the only child (token 3) is cut by top-p (P = 0, distance
+    # .5 at u = .5); the draw from (.632, .368) at .3 is .3 from its crossings
+    rows = _logp([[0.515, 0.3, 0.1, 0.085], [0.25, 0.25, 0.25, 0.25]])
+    r = _one(rows, [3], [-1], [0, 0.5], [0.3, 0.5], top_p=0.52)
+    assert r["path_len"] == 0 and r["tokens"].tolist() == [0, -1]
+    assert abs(r["margin"] - 0.005) < 1e-6
+
+
 def test_zero_temperature_is_the_greedy_tree():
     rng = np.random.default_rng(4)
     ar = rng.normal(0, 1, (7, 9)).astype(np.float32)
