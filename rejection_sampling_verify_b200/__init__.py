@@ -198,6 +198,24 @@ def _ptr(t):
     return None if t is None else t.data_ptr()
 
 
+def _device_of(ref, **tensors):
+    """The CUDA device of `ref`, after checking that every other given tensor
+    is on it and that it is the current device (the library launches on the
+    current device and stream; it has no CPU path)."""
+    torch = _torch()
+    dev = ref.device
+    if dev.type != "cuda":
+        raise ValueError(f"tensors must be CUDA tensors (got {dev}): the library has no CPU path")
+    for name, t in tensors.items():
+        if t is not None and t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, the logits on {dev}")
+    cur = torch.cuda.current_device()
+    if dev.index != cur:
+        raise ValueError(f"the tensors are on {dev} but the current device is cuda:{cur}; "
+                         f"call under torch.cuda.device({dev.index})")
+    return dev
+
+
 def _stream(stream):
     torch = _torch()
     s = torch.cuda.current_stream() if stream is None else stream
@@ -245,7 +263,11 @@ def verify_linear(ar, draft, ids, temperature: float, top_p: float = 1.0, seed: 
         dr_stride = ar_stride
     if ids.dtype != torch.int32 or tuple(ids.shape) != (N, B) or not ids.is_contiguous():
         raise ValueError("ids must be a contiguous int32 [N, B] tensor")
-    dev = ar.device
+    dev = _device_of(ar, draft=None if greedy else draft, ids=ids, seq_ids=seq_ids,
+                     workspace=workspace,
+                     **({} if out is None else dict(tokens=out.tokens, n_emitted=out.n_emitted,
+                                                    p_draft=out.p_draft, q_draft=out.q_draft,
+                                                    status=out.status)))
     if out is None:
         out = LinearResult(
             torch.empty(N, B + 1, dtype=torch.int32, device=dev),
@@ -287,7 +309,10 @@ def verify_tree_greedy(ar, node_tokens, parents, workspace=None, stream=None,
     for name, t in (("node_tokens", node_tokens), ("parents", parents)):
         if t.dtype != torch.int32 or tuple(t.shape) != (N, M) or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous int32 [N, M] tensor")
-    dev = ar.device
+    dev = _device_of(ar, node_tokens=node_tokens, parents=parents, workspace=workspace,
+                     **({} if out is None else dict(path_nodes=out.path_nodes,
+                                                    path_len=out.path_len, tokens=out.tokens,
+                                                    status=out.status)))
     if out is None:
         out = TreeResult(torch.empty(N, M, dtype=torch.int32, device=dev),
                          torch.empty(N, dtype=torch.int32, device=dev),
@@ -310,7 +335,10 @@ def rng_uniforms(seed: int, n_seq: int, step: int, n_rows: int, purpose: int, se
                  device="cuda", stream=None):
     """float32 [n_seq, n_rows] of the verify step's uniforms."""
     torch = _torch()
+    if torch.device(device).type != "cuda":
+        raise ValueError(f"device must be a CUDA device (got {device}): the library has no CPU path")
     out = torch.empty(n_seq, n_rows, dtype=torch.float32, device=device)
+    _device_of(out, seq_ids=seq_ids)
     st = psi_rng_uniforms(int(seed) & (2**64 - 1), _ptr(seq_ids), n_seq, int(step) & (2**64 - 1),
                           n_rows, purpose, _ptr(out), _stream(stream))
     _check(st, "psi_rng_uniforms")

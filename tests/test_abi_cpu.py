@@ -125,3 +125,21 @@ def test_rng_rejects_bad_arguments():
     assert psi.psi_rng_uniforms(0, None, 0, 0, 4, 0, FAKE, None) == psi.PSI_ERR_INVALID_ARG
     assert psi.psi_rng_uniforms(0, None, 4, 0, 4, 0, None, None) == psi.PSI_ERR_INVALID_ARG
     assert psi.psi_rng_uniforms(0, None, 4, 0, 4, 0, FAKE + 2, None) == psi.PSI_ERR_MISALIGNED
+
+
+def test_binding_refuses_tensors_off_the_gpu():
+    """The library has no CPU path: host tensors are refused before any
+    launch (never handed to a kernel as device pointers)."""
+    import torch
+    ar = torch.zeros(2, 3, 64, dtype=torch.bfloat16)
+    draft = torch.zeros(2, 2, 64, dtype=torch.bfloat16)
+    ids = torch.zeros(2, 2, dtype=torch.int32)
+    for T in (0.7, 0.0):
+        with pytest.raises(ValueError, match="CUDA"):
+            psi.verify_linear(ar, draft, ids, T, 0.9)
+    tok = torch.zeros(2, 2, dtype=torch.int32)
+    par = torch.full((2, 2), -1, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        psi.verify_tree_greedy(ar, tok, par)
+    with pytest.raises(ValueError, match="CUDA"):
+        psi.rng_uniforms(0, 4, 0, 3, 0, device="cpu")
