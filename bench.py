@@ -288,17 +288,21 @@ def units(cfg) -> int:
 
 # ---- oracle (CPU) -------------------------------------------------------------------------
 
-def oracle_sample_rate(cfg, batch_cpu, target_seconds, rank=0):
+def oracle_sample_rate(cfg, batch_cpu, target_seconds, one=None):
     """Times the CPU oracle on a bounded sample of the workload; returns
-    (blocks/s, sequences timed, seconds)."""
+    (blocks/s, sequences timed, seconds).  `one` is the seconds one sequence
+    takes, if already known (else one sequence is timed first to size the
+    sample)."""
     import oracle
+    n_have = batch_cpu.ar.shape[0]
     if isinstance(cfg, psi_inputs.TreeConfig):
         ar = psi_inputs.to_host_logits(batch_cpu.ar)
         tok, par = batch_cpu.node_tokens.numpy(), batch_cpu.parents.numpy()
-        t0 = time.perf_counter()
-        oracle.verify_tree_greedy(ar[:1], tok[:1], par[:1])
-        one = time.perf_counter() - t0
-        n = max(1, min(cfg.N, int(target_seconds / max(one, 1e-6))))
+        if one is None:
+            t0 = time.perf_counter()
+            oracle.verify_tree_greedy(ar[:1], tok[:1], par[:1])
+            one = time.perf_counter() - t0
+        n = max(1, min(cfg.N, n_have, int(target_seconds / max(one, 1e-6))))
         t0 = time.perf_counter()
         oracle.verify_tree_greedy(ar[:n], tok[:n], par[:n])
         dt = time.perf_counter() - t0
@@ -306,11 +310,12 @@ def oracle_sample_rate(cfg, batch_cpu, target_seconds, rank=0):
     ar = psi_inputs.to_host_logits(batch_cpu.ar)
     draft = psi_inputs.to_host_logits(batch_cpu.draft) if cfg.temperature > 0 else None
     ids = batch_cpu.ids.numpy()
-    t0 = time.perf_counter()
-    oracle.verify_linear(ar[:1], None if draft is None else draft[:1], ids[:1], cfg.temperature,
-                         cfg.top_p, cfg.seed, 0)
-    one = time.perf_counter() - t0
-    n = max(1, min(cfg.N, int(target_seconds / max(one, 1e-6))))
+    if one is None:
+        t0 = time.perf_counter()
+        oracle.verify_linear(ar[:1], None if draft is None else draft[:1], ids[:1],
+                             cfg.temperature, cfg.top_p, cfg.seed, 0)
+        one = time.perf_counter() - t0
+    n = max(1, min(cfg.N, n_have, int(target_seconds / max(one, 1e-6))))
     t0 = time.perf_counter()
     oracle.verify_linear(ar[:n], None if draft is None else draft[:n], ids[:n], cfg.temperature,
                          cfg.top_p, cfg.seed, 0)
@@ -354,7 +359,7 @@ def run_reference(args, cfg, name):
     rates = []
     seqs = 0
     for s in range(args.warmup + args.steps):
-        r, n, dt = oracle_sample_rate(cfg, batch, per_step)
+        r, n, dt = oracle_sample_rate(cfg, batch, per_step, one=one)
         if s >= args.warmup:
             rates.append(r)
             seqs = n

@@ -98,3 +98,24 @@ def test_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
     assert bench.kernel_source_hash() == h0
     f.write_text(text.replace("kInFlight = 8", "kInFlight = 4", 1))
     assert bench.kernel_source_hash() != h0
+
+
+# ---- the reference arm (the oracle, on the host) -------------------------------------
+
+def test_reference_arm_prints_the_contract_line():
+    """`--impl reference` runs the oracle as it stands on the host (no GPU)
+    and prints one JSON line with the same metric, unit and config keys."""
+    import json
+    import sys
+    r = subprocess.run([sys.executable, os.path.join(bench.ROOT, "bench.py"), "--impl",
+                        "reference", "--config", "tiny", "--steps", "3", "--warmup", "1"],
+                       capture_output=True, text=True, timeout=600, cwd=bench.ROOT, check=True)
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["unit"] == "blocks/s" and line["higher_is_better"] is True
+    assert line["value"] > 0 and line["steps"] == 3 and line["warmup"] == 1
+    assert line["config"]["workload"] == "tiny"
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] == 1 and cb["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "blocks/s",
+                           "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
