@@ -198,6 +198,26 @@ def _ptr(t):
     return None if t is None else t.data_ptr()
 
 
+def _nbytes(t) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+def _check_out(name, t, dtype, shape, optional=False):
+    """A caller-supplied output buffer must match what the kernels write."""
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"out.{name} is required")
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"out.{name} must be a contiguous {dtype} tensor of shape "
+                         f"{tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+
+
+def _check_workspace(t):
+    if t is not None and not t.is_contiguous():
+        raise ValueError("workspace must be contiguous")
+
+
 def _device_of(ref, **tensors):
     """The CUDA device of `ref`, after checking that every other given tensor
     is on it and that it is the current device (the library launches on the
@@ -263,6 +283,13 @@ def verify_linear(ar, draft, ids, temperature: float, top_p: float = 1.0, seed: 
         dr_stride = ar_stride
     if ids.dtype != torch.int32 or tuple(ids.shape) != (N, B) or not ids.is_contiguous():
         raise ValueError("ids must be a contiguous int32 [N, B] tensor")
+    if out is not None:
+        _check_out("tokens", out.tokens, torch.int32, (N, B + 1))
+        _check_out("n_emitted", out.n_emitted, torch.int32, (N,))
+        _check_out("p_draft", out.p_draft, torch.float32, (N, B), optional=True)
+        _check_out("q_draft", out.q_draft, torch.float32, (N, B), optional=True)
+        _check_out("status", out.status, torch.int32, (1,))
+    _check_workspace(workspace)
     dev = _device_of(ar, draft=None if greedy else draft, ids=ids, seq_ids=seq_ids,
                      workspace=workspace,
                      **({} if out is None else dict(tokens=out.tokens, n_emitted=out.n_emitted,
@@ -278,14 +305,14 @@ def verify_linear(ar, draft, ids, temperature: float, top_p: float = 1.0, seed: 
     ws_bytes = psi_verify_linear_workspace_bytes(N, B, V, code, float(temperature), float(top_p))
     if ws_bytes == 0:  # invalid sizes: let the ABI report the precise status
         workspace = None
-    elif workspace is None or workspace.numel() < ws_bytes:
+    elif workspace is None or _nbytes(workspace) < ws_bytes:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     st = psi_verify_linear(
         _ptr(ar), ar_stride, None if greedy else _ptr(draft), dr_stride, code, _ptr(ids), N, B,
         V, float(temperature), float(top_p), int(seed) & (2**64 - 1),
         _ptr(seq_ids), int(step) & (2**64 - 1), _ptr(out.tokens), _ptr(out.n_emitted),
         _ptr(out.p_draft), _ptr(out.q_draft), _ptr(out.status), _ptr(workspace),
-        0 if workspace is None else workspace.numel(), _stream(stream))
+        _nbytes(workspace), _stream(stream))
     _check(st, "psi_verify_linear")
     return out
 
@@ -309,6 +336,12 @@ def verify_tree_greedy(ar, node_tokens, parents, workspace=None, stream=None,
     for name, t in (("node_tokens", node_tokens), ("parents", parents)):
         if t.dtype != torch.int32 or tuple(t.shape) != (N, M) or not t.is_contiguous():
             raise ValueError(f"{name} must be a contiguous int32 [N, M] tensor")
+    if out is not None:
+        _check_out("path_nodes", out.path_nodes, torch.int32, (N, M))
+        _check_out("path_len", out.path_len, torch.int32, (N,))
+        _check_out("tokens", out.tokens, torch.int32, (N, M + 1))
+        _check_out("status", out.status, torch.int32, (1,))
+    _check_workspace(workspace)
     dev = _device_of(ar, node_tokens=node_tokens, parents=parents, workspace=workspace,
                      **({} if out is None else dict(path_nodes=out.path_nodes,
                                                     path_len=out.path_len, tokens=out.tokens,
@@ -321,12 +354,12 @@ def verify_tree_greedy(ar, node_tokens, parents, workspace=None, stream=None,
     ws_bytes = psi_verify_tree_greedy_workspace_bytes(N, M, V, code)
     if ws_bytes == 0:  # invalid sizes: let the ABI report the precise status
         workspace = None
-    elif workspace is None or workspace.numel() < ws_bytes:
+    elif workspace is None or _nbytes(workspace) < ws_bytes:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     st = psi_verify_tree_greedy(_ptr(ar), stride, code, _ptr(node_tokens), _ptr(parents), N, M,
                                 V, _ptr(out.path_nodes), _ptr(out.path_len), _ptr(out.tokens),
                                 _ptr(out.status), _ptr(workspace),
-                                0 if workspace is None else workspace.numel(), _stream(stream))
+                                _nbytes(workspace), _stream(stream))
     _check(st, "psi_verify_tree_greedy")
     return out
 

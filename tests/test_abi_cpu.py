@@ -143,3 +143,31 @@ def test_binding_refuses_tensors_off_the_gpu():
         psi.verify_tree_greedy(ar, tok, par)
     with pytest.raises(ValueError, match="CUDA"):
         psi.rng_uniforms(0, 4, 0, 3, 0, device="cpu")
+
+
+def test_binding_checks_caller_output_buffers():
+    """A caller-supplied `out` must have the shapes and dtypes the kernels
+    write (checked before anything else, so a wrong buffer is never written
+    past its end)."""
+    import torch
+    N, B, V = 2, 3, 64
+    ar = torch.zeros(N, B + 1, V, dtype=torch.bfloat16)
+    draft = torch.zeros(N, B, V, dtype=torch.bfloat16)
+    ids = torch.zeros(N, B, dtype=torch.int32)
+
+    def out(tokens=(N, B + 1), n=(N,), pq=(N, B), dt=torch.int32):
+        return psi.LinearResult(torch.zeros(tokens, dtype=dt), torch.zeros(n, dtype=torch.int32),
+                                torch.zeros(pq), torch.zeros(pq), torch.zeros(1, dtype=torch.int32))
+
+    for bad in (out(tokens=(N, B)), out(n=(N + 1,)), out(pq=(N, B + 1)), out(dt=torch.int64)):
+        with pytest.raises(ValueError, match="out\\."):
+            psi.verify_linear(ar, draft, ids, 0.7, out=bad)
+    with pytest.raises(ValueError, match="CUDA"):  # well-formed buffers reach the device check
+        psi.verify_linear(ar, draft, ids, 0.7, out=out())
+    M = 4
+    tr = psi.TreeResult(torch.zeros(N, M, dtype=torch.int32), torch.zeros(N, dtype=torch.int32),
+                        torch.zeros(N, M, dtype=torch.int32), torch.zeros(1, dtype=torch.int32))
+    with pytest.raises(ValueError, match="out.tokens"):
+        psi.verify_tree_greedy(torch.zeros(N, M + 1, V, dtype=torch.bfloat16),
+                               torch.zeros(N, M, dtype=torch.int32),
+                               torch.full((N, M), -1, dtype=torch.int32), out=tr)
