@@ -171,3 +171,19 @@ def test_binding_checks_caller_output_buffers():
         psi.verify_tree_greedy(torch.zeros(N, M + 1, V, dtype=torch.bfloat16),
                                torch.zeros(N, M, dtype=torch.int32),
                                torch.full((N, M), -1, dtype=torch.int32), out=tr)
+
+
+def test_workspace_size_claims_of_the_header():
+    """The header's sizing notes: the sampled path needs about 16.4 KB per
+    logit row (N (2B + 1) rows), and the no-allocation scratch fits N <= 30
+    sequences at B = 8."""
+    for N, B in ((256, 8), (1024, 16), (64, 3)):
+        ws = psi.psi_verify_linear_workspace_bytes(N, B, 151936, psi.PSI_DTYPE_BF16, 0.7, 0.95)
+        per_row = ws / (N * (2 * B + 1))
+        assert 16384 <= per_row <= 16500, (N, B, per_row)
+    cap = psi.PSI_NOALLOC_SCRATCH_BYTES
+    at = lambda n: psi.psi_verify_linear_workspace_bytes(n, 8, 151936, psi.PSI_DTYPE_BF16, 0.7, 0.95)
+    assert at(30) <= cap < at(31)
+    # the greedy path needs far less: one packed maximum per (row, split), plus the rounds' lists
+    g = psi.psi_verify_linear_workspace_bytes(30, 8, 151936, psi.PSI_DTYPE_BF16, 0.0, 1.0)
+    assert g < at(30) // 10
