@@ -213,6 +213,16 @@ def _check_out(name, t, dtype, shape, optional=False):
                          f"{tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
 
 
+def _check_seq_ids(t, n):
+    """Sequence ids: n 64-bit integers (the kernels read them as uint64)."""
+    torch = _torch()
+    if t is None:
+        return
+    if t.dtype not in (torch.int64, torch.uint64) or tuple(t.shape) != (n,) or not t.is_contiguous():
+        raise ValueError(f"seq_ids must be a contiguous 64-bit integer tensor of shape ({n},), "
+                         f"got {t.dtype} {tuple(t.shape)}")
+
+
 def _check_workspace(t):
     if t is not None and not t.is_contiguous():
         raise ValueError("workspace must be contiguous")
@@ -283,6 +293,7 @@ def verify_linear(ar, draft, ids, temperature: float, top_p: float = 1.0, seed: 
         dr_stride = ar_stride
     if ids.dtype != torch.int32 or tuple(ids.shape) != (N, B) or not ids.is_contiguous():
         raise ValueError("ids must be a contiguous int32 [N, B] tensor")
+    _check_seq_ids(seq_ids, N)
     if out is not None:
         _check_out("tokens", out.tokens, torch.int32, (N, B + 1))
         _check_out("n_emitted", out.n_emitted, torch.int32, (N,))
@@ -370,6 +381,7 @@ def rng_uniforms(seed: int, n_seq: int, step: int, n_rows: int, purpose: int, se
     torch = _torch()
     if torch.device(device).type != "cuda":
         raise ValueError(f"device must be a CUDA device (got {device}): the library has no CPU path")
+    _check_seq_ids(seq_ids, n_seq)
     out = torch.empty(n_seq, n_rows, dtype=torch.float32, device=device)
     _device_of(out, seq_ids=seq_ids)
     st = psi_rng_uniforms(int(seed) & (2**64 - 1), _ptr(seq_ids), n_seq, int(step) & (2**64 - 1),

@@ -187,3 +187,18 @@ def test_workspace_size_claims_of_the_header():
     # the greedy path needs far less: one packed maximum per (row, split), plus the rounds' lists
     g = psi.psi_verify_linear_workspace_bytes(30, 8, 151936, psi.PSI_DTYPE_BF16, 0.0, 1.0)
     assert g < at(30) // 10
+
+
+def test_binding_checks_sequence_ids():
+    """seq_ids are read as N uint64 values: a short or 32-bit tensor is refused."""
+    import torch
+    ar = torch.zeros(2, 3, 64, dtype=torch.bfloat16)
+    draft = torch.zeros(2, 2, 64, dtype=torch.bfloat16)
+    ids = torch.zeros(2, 2, dtype=torch.int32)
+    for bad in (torch.zeros(1, dtype=torch.int64), torch.zeros(2, dtype=torch.int32)):
+        with pytest.raises(ValueError, match="seq_ids"):
+            psi.verify_linear(ar, draft, ids, 0.7, seq_ids=bad)
+        with pytest.raises(ValueError, match="seq_ids"):
+            psi.rng_uniforms(0, 2, 0, 3, 0, seq_ids=bad)
+    with pytest.raises(ValueError, match="CUDA"):  # well-formed ids reach the device check
+        psi.verify_linear(ar, draft, ids, 0.7, seq_ids=torch.zeros(2, dtype=torch.int64))
