@@ -22,6 +22,7 @@ from __future__ import annotations
 import ctypes as C
 import os
 import subprocess
+from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 
@@ -213,6 +214,36 @@ def verify_linear(ar, draft, ids, temperature, top_p, seed, step, seq_ids=None,
         _ptr(tokens), _ptr(n_em), _ptr(p), _ptr(q), _ptr(margin))
     return dict(tokens=tokens, n_emitted=n_em, p_draft=p, q_draft=q,
                 margin=margin, status=int(st))
+
+
+def verify_linear_parallel(ar, draft, ids, temperature, top_p, seed, step, seq_ids=None,
+                           V=None, top_k=0, threads=None):
+    """verify_linear over a pool of host threads: the batch is cut into
+    contiguous groups of sequences, each verified by one plain
+    ``orc_verify_linear`` call on its own rows (ctypes releases the GIL while
+    the C code runs).  Sequence n keeps its RNG key (seq_ids[n], default n),
+    so the result equals one verify_linear call over the whole batch."""
+    ar = _contig(ar)
+    N = ar.shape[0]
+    sid = (np.arange(N, dtype=np.uint64) if seq_ids is None
+           else _contig(np.asarray(seq_ids), np.uint64).reshape(N))
+    threads = max(1, min(N, threads or os.cpu_count() or 1))
+    cuts = np.linspace(0, N, min(N, 4 * threads) + 1).astype(int)
+    parts = [(a, b) for a, b in zip(cuts[:-1], cuts[1:]) if b > a]
+
+    def run(ab):
+        a, b = ab
+        return verify_linear(ar[a:b], None if draft is None else draft[a:b], np.asarray(ids)[a:b],
+                             temperature, top_p, seed, step, seq_ids=sid[a:b], V=V, top_k=top_k)
+
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        outs = list(ex.map(run, parts))
+    res = {k: np.concatenate([o[k] for o in outs]) for k in
+           ("tokens", "n_emitted", "p_draft", "q_draft", "margin")}
+    res["status"] = 0
+    for o in outs:
+        res["status"] |= o["status"]
+    return res
 
 
 # ---- greedy tree --------------------------------------------------------------

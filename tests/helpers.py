@@ -38,31 +38,35 @@ def gpu_linear(batch: psi_inputs.LinearBatch, seed: int, step: int, seq_ids=None
 def oracle_linear(batch: psi_inputs.LinearBatch, seed: int, step: int, seq_ids=None):
     ar = psi_inputs.to_host_logits(batch.ar)
     draft = None if batch.temperature == 0 else psi_inputs.to_host_logits(batch.draft)
-    return oracle.verify_linear(ar, draft, batch.ids.cpu().numpy(), batch.temperature,
-                                batch.top_p, seed, step, seq_ids=seq_ids)
+    return oracle.verify_linear_parallel(ar, draft, batch.ids.cpu().numpy(), batch.temperature,
+                                         batch.top_p, seed, step, seq_ids=seq_ids)
 
 
 def compare_linear(g, o, exact: bool = False):
-    """Returns (n_sequences, n_near_ties, n_mismatches_outside_near_ties)."""
+    """Returns (n_sequences, n_near_ties, n_bad, where_bad, n_differ): a
+    sequence is bad if its tokens or length differ outside a near tie, or if
+    p(x) or q(x) is off by more than PROB_TOL at any drafted position (near
+    tie or not)."""
     N = len(o["n_emitted"])
     near = (o["margin"] < NEAR_TIE) if not exact else np.zeros(N, bool)
-    mism = (g["n_emitted"] != o["n_emitted"]) | np.any(g["tokens"] != o["tokens"], axis=1)
-    bad = mism & ~near
+    differ = (g["n_emitted"] != o["n_emitted"]) | np.any(g["tokens"] != o["tokens"], axis=1)
+    bad = differ & ~near
     if "p_draft" in g and not exact:
         dp = np.abs(g["p_draft"] - o["p_draft"]).max(axis=1)
         dq = np.abs(g["q_draft"] - o["q_draft"]).max(axis=1)
-        bad |= ((dp > PROB_TOL) | (dq > PROB_TOL)) & ~near
-    return N, int(near.sum()), int(bad.sum()), np.nonzero(bad)[0]
+        bad |= (dp > PROB_TOL) | (dq > PROB_TOL)
+    return N, int(near.sum()), int(bad.sum()), np.nonzero(bad)[0], int(differ.sum())
 
 
-def assert_linear_parity(g, o, exact: bool = False, max_near_frac: float | None = None):
-    N, n_near, n_bad, where = compare_linear(g, o, exact)
+def assert_linear_parity(g, o, exact: bool = False, max_differ_frac: float = 0.001):
+    """Every difference is at a near tie, and the sequences that differ are at
+    most max_differ_frac of the batch.  Returns the number of near ties."""
+    N, n_near, n_bad, where, n_differ = compare_linear(g, o, exact)
     assert n_bad == 0, (f"{n_bad}/{N} sequences differ outside near ties: {where[:10]}\n"
                         f"gpu n={g['n_emitted'][where[:5]]} oracle n={o['n_emitted'][where[:5]]}\n"
                         f"gpu tok={g['tokens'][where[:2]]}\noracle tok={o['tokens'][where[:2]]}")
     assert g["status"] == o["status"], (g["status"], o["status"])
-    if max_near_frac is not None:
-        assert n_near <= max_near_frac * N, (n_near, N)
+    assert n_differ <= max_differ_frac * N, (n_differ, N)
     return n_near
 
 

@@ -108,21 +108,6 @@ def test_greedy_flags_and_neg_inf():
     assert np.array_equal(g["n_emitted"][ok], o["n_emitted"][ok])
 
 
-def test_greedy_max_batch_full_size_sampled():
-    """Full max-batch greedy workload (N=1024, B=16, V=151936), the launch
-    the benchmark times; the oracle checks a sample of sequences."""
-    cfg = CFG["max_batch_greedy"]
-    b = psi_inputs.linear_batch(cfg, device="cuda")
-    g = gpu_linear(b, cfg.seed, 0)
-    pick = np.array([0, 1, 511, 777, 1023])
-    sub = _batch(b.ar[pick].cpu(), None, b.ids[pick].cpu(), 0.0, 1.0)
-    o = oracle_linear(sub, cfg.seed, 0)
-    assert np.array_equal(g["tokens"][pick], o["tokens"])
-    assert np.array_equal(g["n_emitted"][pick], o["n_emitted"])
-    assert g["status"] == 0
-    assert g["n_emitted"].min() >= 1 and g["n_emitted"].max() <= cfg.B + 1
-
-
 # ---- greedy tree -------------------------------------------------------------------
 
 @pytest.mark.parametrize("iid", [False, True])
@@ -206,30 +191,6 @@ def test_sampled_nucleus_recipe_reduced(step):
     cfg = CFG["large_batch_nucleus"]
     b = psi_inputs.linear_batch(cfg, device="cuda", N=8, index=step)
     assert_linear_parity(gpu_linear(b, cfg.seed, step), oracle_linear(b, cfg.seed, step))
-
-
-def test_sampled_nucleus_full_size_sampled():
-    """Full large-batch nucleus workload (N=256, B=8, V=151936, T=0.7,
-    top-p 0.95) in the benchmark's launch; the oracle checks a sample of
-    sequences one by one, properties hold for all."""
-    cfg = CFG["large_batch_nucleus"]
-    b = psi_inputs.linear_batch(cfg, device="cuda")
-    g = gpu_linear(b, cfg.seed, 5)
-    pick = np.array([0, 37, 128, 255])
-    sub = _batch(b.ar[pick].cpu(), b.draft[pick].cpu(), b.ids[pick].cpu(), cfg.temperature,
-                 cfg.top_p)
-    o = oracle_linear(sub, cfg.seed, 5, seq_ids=pick.astype(np.uint64))
-    gs = {k: (v[pick] if isinstance(v, np.ndarray) else v) for k, v in g.items()}
-    gs["status"] = 0
-    assert_linear_parity(gs, o)
-    assert g["status"] == 0
-    n = g["n_emitted"]
-    assert n.min() >= 1 and n.max() <= cfg.B + 1
-    col = np.arange(cfg.B + 1)[None, :]
-    assert np.all((g["tokens"] >= 0) == (col < n[:, None]))
-    assert g["tokens"].max() < cfg.V
-    assert np.all((g["p_draft"] >= 0) & (g["p_draft"] <= 1 + 1e-6))
-    assert np.all((g["q_draft"] >= 0) & (g["q_draft"] <= 1 + 1e-6))
 
 
 @pytest.mark.parametrize("V", [1, 2, 33, 1000, 12289, 65537, 151936])
