@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the batch size (smaller profiling cases)")
+    ap.add_argument("--max-repeats", type=int, default=200,
+                    help="most timed passes of K steps (passes continue until ~0.5 s)")
     return ap.parse_args()
 
 
@@ -288,11 +290,12 @@ def units(cfg) -> int:
 
 # ---- oracle (CPU) -------------------------------------------------------------------------
 
-def oracle_sample_rate(cfg, batch_cpu, target_seconds, one=None):
+def oracle_sample_rate(cfg, batch_cpu, target_seconds, one=None, threads=1):
     """Times the CPU oracle on a bounded sample of the workload; returns
     (blocks/s, sequences timed, seconds).  `one` is the seconds one sequence
-    takes, if already known (else one sequence is timed first to size the
-    sample)."""
+    takes on one thread, if already known (else one sequence is timed first
+    to size the sample).  threads > 1 runs the oracle's thread pool over
+    sequences (oracle.verify_linear_parallel)."""
     import oracle
     n_have = batch_cpu.ar.shape[0]
     if isinstance(cfg, psi_inputs.TreeConfig):
@@ -315,12 +318,25 @@ def oracle_sample_rate(cfg, batch_cpu, target_seconds, one=None):
         oracle.verify_linear(ar[:1], None if draft is None else draft[:1], ids[:1],
                              cfg.temperature, cfg.top_p, cfg.seed, 0)
         one = time.perf_counter() - t0
-    n = max(1, min(cfg.N, n_have, int(target_seconds / max(one, 1e-6))))
+    n = max(1, min(cfg.N, n_have, int(threads * target_seconds / max(one, 1e-6))))
+    if threads > 1:  # whole rounds of the pool
+        n = max(1, min(n_have, (n // threads) * threads or threads))
     t0 = time.perf_counter()
-    oracle.verify_linear(ar[:n], None if draft is None else draft[:n], ids[:n], cfg.temperature,
-                         cfg.top_p, cfg.seed, 0)
+    if threads > 1:
+        oracle.verify_linear_parallel(ar[:n], None if draft is None else draft[:n], ids[:n],
+                                      cfg.temperature, cfg.top_p, cfg.seed, 0, threads=threads)
+    else:
+        oracle.verify_linear(ar[:n], None if draft is None else draft[:n], ids[:n],
+                             cfg.temperature, cfg.top_p, cfg.seed, 0)
     dt = time.perf_counter() - t0
     return n / dt, n, dt
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
 
 def sample_inputs(cfg, n):
@@ -347,31 +363,38 @@ def config_block(cfg, name, world):
 
 
 def run_reference(args, cfg, name):
-    """The reference arm: the CPU oracle as it stands, single thread, each
-    step a bounded sample of the workload (whole run ~2 minutes)."""
+    """The reference arm: the CPU oracle as it stands, on a pool of the host's
+    cores (one plain oracle call per group of sequences), each step a bounded
+    sample of the workload (whole run ~2 minutes).  ms_per_step is the time a
+    step's sample actually took."""
     if int(os.environ.get("RANK", "0")) != 0:
         return 0
+    cores = host_cores()
     per_step = max(0.2, 120.0 / max(1, args.steps + args.warmup))
     probe = make_inputs(cfg, "cpu", 0) if cfg.N * cfg.V < 4e6 else sample_inputs(cfg, 1)
     _, _, one = oracle_sample_rate(cfg, probe, 0.0)
-    n_seq = max(1, min(cfg.N, int(per_step / max(one, 1e-6))))
+    n_seq = max(1, min(cfg.N, cores * max(1, int(per_step / max(one, 1e-6)))))
     batch = probe if n_seq <= (probe.ar.shape[0]) else sample_inputs(cfg, n_seq)
-    rates = []
+    rates, times = [], []
     seqs = 0
     for s in range(args.warmup + args.steps):
-        r, n, dt = oracle_sample_rate(cfg, batch, per_step, one=one)
+        r, n, dt = oracle_sample_rate(cfg, batch, per_step, one=one, threads=cores)
         if s >= args.warmup:
             rates.append(r)
+            times.append(dt)
             seqs = n
     value = float(statistics.median(rates))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "blocks/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1000.0 * cfg.N / value, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": 1000.0 * float(statistics.median(times)),
+        "sequences_per_step": seqs,
+        "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": dict(config_block(cfg, name, 1), schedule="every row (the oracle as it stands)"),
-        "cpu_baseline": {"value": value, "unit": "blocks/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{seqs} sequences of the workload per step, single thread"},
+        "cpu_baseline": {"value": value, "unit": "blocks/s", "cores": cores, "kind": "oracle",
+                         "sample": (f"{seqs} of the {cfg.N} sequences of the workload per step, "
+                                    f"on a pool of {cores} host threads")},
         "e2e": {"value": value, "unit": "blocks/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -417,27 +440,41 @@ def main():
         call_verify(psi, cfg, batch, w, seq_ids, ws, out)
     torch.cuda.synchronize()
 
-    # timed region: K steps, main-kernel events recorded per step
+    # timed region: K steps, bracketed by a barrier and a synchronize, main-kernel
+    # events recorded per step; repeated so that the clock record spans at
+    # least ~0.5 s (the per-step time reported is the median over the repeats)
     K = args.steps
-    ev_main = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(K)]
-    for a, b in ev_main:  # torch creates the CUDA events lazily, on first record
-        a.record(stream)
-        b.record(stream)
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(pg)
+    # the same number of passes on every rank (each pass has its own barriers)
+    est = max_over_ranks(max(step_ms_estimate(psi, cfg, batch, seq_ids, ws, out, stream), 1e-3),
+                         pg, dev)
+    repeats = max(1, min(args.max_repeats, math.ceil(500.0 / (est * K))))
+    ev_main = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(K)] for _ in range(repeats)]
+    for rep in ev_main:  # torch creates the CUDA events lazily, on first record
+        for a, b in rep:
+            a.record(stream)
+            b.record(stream)
+    spans = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(repeats)]
     torch.cuda.synchronize()
+    elapsed = []
     with ClockSampler(dev) as clocks:
-        start.record(stream)
-        for k in range(K):
-            psi.psi_profile_main_kernel(ev_main[k][0].cuda_event, ev_main[k][1].cuda_event)
-            call_verify(psi, cfg, batch, args.warmup + k, seq_ids, ws, out)
-        stop.record(stream)
-        psi.psi_profile_main_kernel(None, None)
-        torch.cuda.synchronize()
-    barrier(pg)
-    elapsed_ms = max_over_ranks(start.elapsed_time(stop), pg, dev)
-    main_ms = statistics.mean(a.elapsed_time(b) for a, b in ev_main)
+        for rep in range(repeats):
+            barrier(pg)
+            torch.cuda.synchronize()
+            start, stop = spans[rep]
+            start.record(stream)
+            for k in range(K):
+                psi.psi_profile_main_kernel(ev_main[rep][k][0].cuda_event,
+                                            ev_main[rep][k][1].cuda_event)
+                call_verify(psi, cfg, batch, args.warmup + rep * K + k, seq_ids, ws, out)
+            stop.record(stream)
+            psi.psi_profile_main_kernel(None, None)
+            torch.cuda.synchronize()
+            barrier(pg)
+            elapsed.append(max_over_ranks(start.elapsed_time(stop), pg, dev))
+    elapsed_ms = float(statistics.median(elapsed))
+    main_ms = statistics.mean(a.elapsed_time(b) for rep in ev_main for a, b in rep)
     status = int(out.status.item()) & 0xFFFFFFFF
     if status:
         print(f"warning: device status bits {status:#x}", file=sys.stderr)
@@ -464,10 +501,16 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        bc = make_inputs(cfg, "cpu", 0) if cfg.N * cfg.V < 4e6 else cpu_copy(batch, cfg)
-        r, n, dt = oracle_sample_rate(cfg, bc, args.cpu_seconds)
-        cpu = {"value": r, "unit": "blocks/s", "cores": 1, "kind": "oracle",
-               "sample": f"{n} of the {cfg.N} sequences of one step ({dt:.1f} s, single thread)"}
+        cores = host_cores()
+        bc = make_inputs(cfg, "cpu", 0) if cfg.N * cfg.V < 4e6 else cpu_copy(batch, cfg, 4 * cores)
+        r1, n1, dt1 = oracle_sample_rate(cfg, bc, args.cpu_seconds / 2)
+        rp, npool, dtp = oracle_sample_rate(cfg, bc, args.cpu_seconds / 2, one=dt1 / n1,
+                                            threads=cores)
+        cpu = {"value": rp, "unit": "blocks/s", "cores": cores, "kind": "oracle",
+               "sample": (f"{npool} of the {cfg.N} sequences of one step on a pool of {cores} "
+                          f"host threads ({dtp:.1f} s)"),
+               "single_thread": {"value": r1, "unit": "blocks/s", "cores": 1,
+                                 "sample": f"{n1} sequences ({dt1:.1f} s)"}}
 
     if rank == 0:
         # our kernels per call: argmax + tree walk; greedy linear: per
@@ -497,6 +540,7 @@ def main():
                          "algorithmic_bytes_per_launch": alg, "launch_ms": main_ms,
                          "traffic": profiled_traffic(kernel, name)},
             "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks.summary(),
+            "timed_repeats": repeats,
             "gpu_launches": launches_per_step * K, "device_status": status,
         }
         print(json.dumps(line), flush=True)
@@ -505,9 +549,21 @@ def main():
     return 0
 
 
-def cpu_copy(batch, cfg):
-    """Host copy of the first few sequences (enough for the oracle sample)."""
-    n = min(cfg.N, 64)
+def step_ms_estimate(psi, cfg, batch, seq_ids, ws, out, stream) -> float:
+    """Milliseconds of one verify call (three calls timed with CUDA events)."""
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for k in range(3):
+        call_verify(psi, cfg, batch, k, seq_ids, ws, out)
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / 3.0
+
+
+def cpu_copy(batch, cfg, n=64):
+    """Host copy of the first n sequences (enough for the oracle sample)."""
+    n = min(cfg.N, n)
     if isinstance(cfg, psi_inputs.TreeConfig):
         return psi_inputs.TreeBatch(batch.ar[:n].cpu(), batch.node_tokens[:n].cpu(),
                                     batch.parents[:n].cpu(), None)

@@ -169,14 +169,17 @@ psi_status psi_verify_linear(const void *ar_logits, int64_t ar_row_stride,
  * nothing is allocated at run time).  Its address is looked up once per
  * device, on the first call made with that device current; make that first
  * call before capturing the stream into a graph, since it issues a
- * runtime query besides the launches.  The scratch needs no initialisation:
+ * runtime query besides the launches.  The address is kept for the life of
+ * the process: it belongs to the device's primary context, so after that
+ * context is torn down (cudaDeviceReset) this entry point must not be used
+ * on that device again until the library is reloaded.  The scratch needs no initialisation:
  * what the verify needs zeroed it clears itself on every call.
  * Calls that overlap in time on the same device share the scratch and race:
  * the caller serialises them (one stream, or events between streams).
  * Returns PSI_ERR_UNSUPPORTED, without launching anything, when
  * psi_verify_linear_workspace_bytes for these sizes exceeds
- * PSI_NOALLOC_SCRATCH_BYTES (the sampled path needs about 16.4 KB per logit
- * row, N * (2B + 1) rows: e.g. N <= 30 at B = 8; the greedy path far less),
+ * PSI_NOALLOC_SCRATCH_BYTES (the sampled path needs about 16.5 KB per logit
+ * row, N * (2B + 1) rows: e.g. N <= 29 at B = 8; the greedy path far less),
  * and PSI_ERR_CUDA if the scratch address cannot be obtained.
  */
 #define PSI_NOALLOC_SCRATCH_BYTES 8388608u /* 8 MiB */
@@ -220,6 +223,50 @@ psi_status psi_verify_tree_greedy(const void *ar_logits, int64_t ar_row_stride,
                                   int32_t *out_path_len, int32_t *out_tokens,
                                   uint32_t *dev_status, void *workspace,
                                   size_t workspace_bytes, psi_stream_t stream);
+
+/* Workspace needed by psi_verify_tree_sampled (bytes, a multiple of 256; 0 on
+ * invalid sizes).  The workspace needs no initialisation. */
+size_t psi_verify_tree_sampled_workspace_bytes(int32_t N, int32_t M, int32_t V,
+                                               psi_dtype dtype, float temperature,
+                                               float top_p);
+
+/*
+ * psi_verify_tree_sampled - sampled (T > 0) verify of a draft tree per
+ * sequence.
+ *
+ * [P3] "Linear 與 Tree sampler" (a prefix tree of candidates verified in one
+ * pass) with the rejection rule and residual draw of [P3] "完整走一次四個
+ * Token"; the pages give no sampled tree rule, and the one taken is
+ * recursive rejection over each reached node's children (SpecInfer's
+ * multi-candidate speculative sampling, Miao et al., ASPLOS 2024), every
+ * child being a point-mass proposal:
+ *   At a node whose AR row gives the target P (softmax at temperature T,
+ *   cut to its top-p set as in psi_verify_linear), the valid children are
+ *   tried in ascending index.  Child k with token x is accepted iff
+ *   u_k * R < w(x), where w is what remains of P after the node's rejected
+ *   tokens lost their mass (a repeated token has none left), R = sum(w) and
+ *   u_k = U(seed, seq, step, k + 1, ACCEPT).  An accepted child becomes the
+ *   next node.  When no child is accepted (or the node is a leaf) the step
+ *   ends with the inverse-CDF draw, in vocabulary order, from w (from P if
+ *   nothing remains) at u' = U(seed, seq, step, j, RESID), j being that
+ *   node's row (0 = root).  Every emitted token then has the law of its
+ *   node's P (lossless).
+ * T == 0 is the greedy tree (psi_verify_tree_greedy; top_p ignored).
+ * Arguments, layouts, validity rules and outputs as psi_verify_tree_greedy,
+ * plus temperature, top_p (0 < top_p <= 1), seed, seq_ids (uint64 [N] or
+ * NULL = n) and step as in psi_verify_linear.  out_tokens holds the accepted
+ * tokens, then the drawn one, then -1.
+ * Limits: as psi_verify_tree_greedy; T >= 0 and finite.
+ */
+psi_status psi_verify_tree_sampled(const void *ar_logits, int64_t ar_row_stride,
+                                   psi_dtype dtype, const int32_t *node_tokens,
+                                   const int32_t *parents, int32_t N, int32_t M,
+                                   int32_t V, float temperature, float top_p,
+                                   uint64_t seed, const uint64_t *seq_ids,
+                                   uint64_t step, int32_t *out_path_nodes,
+                                   int32_t *out_path_len, int32_t *out_tokens,
+                                   uint32_t *dev_status, void *workspace,
+                                   size_t workspace_bytes, psi_stream_t stream);
 
 /*
  * psi_rng_uniforms - the uniforms the verify step draws, for inspection and

@@ -55,6 +55,8 @@ EXPORTED = (
     "psi_verify_linear_noalloc",
     "psi_verify_tree_greedy_workspace_bytes",
     "psi_verify_tree_greedy",
+    "psi_verify_tree_sampled_workspace_bytes",
+    "psi_verify_tree_sampled",
     "psi_rng_uniforms",
     "psi_profile_main_kernel",
     "psi_status_string",
@@ -96,6 +98,11 @@ def load_library():
     lib.psi_verify_tree_greedy.restype = C.c_int
     lib.psi_verify_tree_greedy.argtypes = [vp, i64, C.c_int, vp, vp, i32, i32, i32, vp, vp, vp,
                                            vp, vp, sz, vp]
+    lib.psi_verify_tree_sampled_workspace_bytes.restype = sz
+    lib.psi_verify_tree_sampled_workspace_bytes.argtypes = [i32, i32, i32, C.c_int, f32, f32]
+    lib.psi_verify_tree_sampled.restype = C.c_int
+    lib.psi_verify_tree_sampled.argtypes = [vp, i64, C.c_int, vp, vp, i32, i32, i32, f32, f32,
+                                            u64, vp, u64, vp, vp, vp, vp, vp, sz, vp]
     lib.psi_rng_uniforms.restype = C.c_int
     lib.psi_rng_uniforms.argtypes = [u64, vp, i32, u64, i32, u32, vp, vp]
     lib.psi_profile_main_kernel.restype = C.c_int
@@ -153,6 +160,21 @@ def psi_verify_tree_greedy(ar_logits, ar_row_stride, dtype, node_tokens, parents
     return int(load_library().psi_verify_tree_greedy(
         ar_logits, ar_row_stride, dtype, node_tokens, parents, N, M, V, out_path_nodes,
         out_path_len, out_tokens, dev_status, workspace, workspace_bytes, stream))
+
+
+def psi_verify_tree_sampled_workspace_bytes(N, M, V, dtype, temperature, top_p) -> int:
+    return int(load_library().psi_verify_tree_sampled_workspace_bytes(N, M, V, dtype,
+                                                                      temperature, top_p))
+
+
+def psi_verify_tree_sampled(ar_logits, ar_row_stride, dtype, node_tokens, parents, N, M, V,
+                            temperature, top_p, seed, seq_ids, step, out_path_nodes,
+                            out_path_len, out_tokens, dev_status, workspace, workspace_bytes,
+                            stream) -> int:
+    return int(load_library().psi_verify_tree_sampled(
+        ar_logits, ar_row_stride, dtype, node_tokens, parents, N, M, V, temperature, top_p,
+        seed, seq_ids, step, out_path_nodes, out_path_len, out_tokens, dev_status, workspace,
+        workspace_bytes, stream))
 
 
 def psi_rng_uniforms(seed, seq_ids, n_seq, step, n_rows, purpose, out, stream) -> int:
@@ -375,6 +397,53 @@ def verify_tree_greedy(ar, node_tokens, parents, workspace=None, stream=None,
     return out
 
 
+def verify_tree_sampled(ar, node_tokens, parents, temperature: float, top_p: float = 1.0,
+                        seed: int = 0, step: int = 0, seq_ids=None, workspace=None, stream=None,
+                        out: TreeResult | None = None) -> TreeResult:
+    """Sampled tree verify (recursive rejection over each reached node's
+    children).  ar [N, M+1, V]; node_tokens, parents int32 [N, M]; seq_ids
+    int64 [N] (read as uint64) or None."""
+    torch = _torch()
+    N, M1 = ar.shape[0], ar.shape[1]
+    M = M1 - 1
+    stride, V = _rows(ar, 2, "ar")
+    code = _dtype_code(ar)
+    for name, t in (("node_tokens", node_tokens), ("parents", parents)):
+        if t.dtype != torch.int32 or tuple(t.shape) != (N, M) or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous int32 [N, M] tensor")
+    if seq_ids is not None:
+        _check_seq_ids(seq_ids, N)
+    if out is not None:
+        _check_out("path_nodes", out.path_nodes, torch.int32, (N, M))
+        _check_out("path_len", out.path_len, torch.int32, (N,))
+        _check_out("tokens", out.tokens, torch.int32, (N, M + 1))
+        _check_out("status", out.status, torch.int32, (1,))
+    _check_workspace(workspace)
+    dev = _device_of(ar, node_tokens=node_tokens, parents=parents, workspace=workspace,
+                     seq_ids=seq_ids,
+                     **({} if out is None else dict(path_nodes=out.path_nodes,
+                                                    path_len=out.path_len, tokens=out.tokens,
+                                                    status=out.status)))
+    if out is None:
+        out = TreeResult(torch.empty(N, M, dtype=torch.int32, device=dev),
+                         torch.empty(N, dtype=torch.int32, device=dev),
+                         torch.empty(N, M + 1, dtype=torch.int32, device=dev),
+                         torch.zeros(1, dtype=torch.int32, device=dev))
+    ws_bytes = psi_verify_tree_sampled_workspace_bytes(N, M, V, code, float(temperature),
+                                                       float(top_p))
+    if ws_bytes == 0:  # invalid sizes: let the ABI report the precise status
+        workspace = None
+    elif workspace is None or _nbytes(workspace) < ws_bytes:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    st = psi_verify_tree_sampled(_ptr(ar), stride, code, _ptr(node_tokens), _ptr(parents), N, M,
+                                 V, float(temperature), float(top_p), int(seed) & (2**64 - 1),
+                                 _ptr(seq_ids), int(step) & (2**64 - 1), _ptr(out.path_nodes),
+                                 _ptr(out.path_len), _ptr(out.tokens), _ptr(out.status),
+                                 _ptr(workspace), _nbytes(workspace), _stream(stream))
+    _check(st, "psi_verify_tree_sampled")
+    return out
+
+
 def rng_uniforms(seed: int, n_seq: int, step: int, n_rows: int, purpose: int, seq_ids=None,
                  device="cuda", stream=None):
     """float32 [n_seq, n_rows] of the verify step's uniforms."""
@@ -392,4 +461,4 @@ def rng_uniforms(seed: int, n_seq: int, step: int, n_rows: int, purpose: int, se
 
 __all__ = [n for n in dir() if n.startswith(("psi_", "PSI_"))] + [
     "verify_linear", "verify_tree_greedy", "rng_uniforms", "LinearResult", "TreeResult",
-    "PsiError", "load_library", "EXPORTED"]
+    "PsiError", "load_library", "EXPORTED", "verify_tree_sampled"]

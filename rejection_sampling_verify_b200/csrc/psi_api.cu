@@ -252,6 +252,59 @@ psi_status psi_verify_tree_greedy(const void *ar_logits, int64_t ar_row_stride, 
   return PSI_OK;
 }
 
+size_t psi_verify_tree_sampled_workspace_bytes(int32_t N, int32_t M, int32_t V, psi_dtype dtype,
+                                               float temperature, float top_p) {
+  (void)top_p;
+  if (!(temperature >= 0.f) || !isfinite(temperature)) return 0;
+  if (temperature == 0.f) return psi_verify_tree_greedy_workspace_bytes(N, M, V, dtype);
+  if (N < 1 || M < 1 || M > PSI_MAX_TREE_NODES || V < 1 || !valid_dtype(dtype) ||
+      V > max_v(dtype))
+    return 0;
+  return round256(psi::tree_layout(N, M).total);
+}
+
+psi_status psi_verify_tree_sampled(const void *ar_logits, int64_t ar_row_stride, psi_dtype dtype,
+                                   const int32_t *node_tokens, const int32_t *parents, int32_t N,
+                                   int32_t M, int32_t V, float temperature, float top_p,
+                                   uint64_t seed, const uint64_t *seq_ids, uint64_t step,
+                                   int32_t *out_path_nodes, int32_t *out_path_len,
+                                   int32_t *out_tokens, uint32_t *dev_status, void *workspace,
+                                   size_t workspace_bytes, psi_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (!(temperature >= 0.f) || !isfinite(temperature))
+    return fail(PSI_ERR_INVALID_ARG, "temperature %g (need finite, >= 0)", (double)temperature);
+  if (temperature == 0.f)
+    return psi_verify_tree_greedy(ar_logits, ar_row_stride, dtype, node_tokens, parents, N, M, V,
+                                  out_path_nodes, out_path_len, out_tokens, dev_status,
+                                  workspace, workspace_bytes, stream_);
+  if (!valid_dtype(dtype)) return fail(PSI_ERR_INVALID_ARG, "dtype %d", (int)dtype);
+  if (N < 1 || M < 1 || M > PSI_MAX_TREE_NODES || V < 1)
+    return fail(PSI_ERR_INVALID_ARG, "sizes N=%d M=%d V=%d (need N>=1, 1<=M<=%d, V>=1)", N, M,
+                V, PSI_MAX_TREE_NODES);
+  if (V > max_v(dtype))
+    return fail(PSI_ERR_UNSUPPORTED, "V=%d above the supported %d", V, max_v(dtype));
+  if (!(top_p > 0.f && top_p <= 1.f))
+    return fail(PSI_ERR_INVALID_ARG, "top_p %g (need 0 < top_p <= 1)", (double)top_p);
+  if (!ar_logits || !node_tokens || !parents || !out_path_nodes || !out_path_len || !out_tokens)
+    return fail(PSI_ERR_INVALID_ARG, "null pointer argument");
+  if (ar_row_stride < V) return fail(PSI_ERR_INVALID_ARG, "row stride below V");
+  const size_t es = (size_t)elem_bytes(dtype);
+  if (!aligned_to(ar_logits, es) || !aligned_to(node_tokens, 4) || !aligned_to(parents, 4) ||
+      !aligned_to(out_path_nodes, 4) || !aligned_to(out_path_len, 4) ||
+      !aligned_to(out_tokens, 4) || (seq_ids && !aligned_to(seq_ids, 8)) ||
+      (dev_status && !aligned_to(dev_status, 4)))
+    return fail(PSI_ERR_MISALIGNED, "pointer not aligned to its element type");
+  const size_t need = psi_verify_tree_sampled_workspace_bytes(N, M, V, dtype, temperature, top_p);
+  if (!workspace || workspace_bytes < need || !aligned_to(workspace, 16))
+    return fail(PSI_ERR_WORKSPACE, "workspace %zu bytes, need %zu", workspace_bytes, need);
+  cudaError_t e = psi::launch_tree_sampled(ar_logits, ar_row_stride, dtype, node_tokens, parents,
+                                           N, M, V, temperature, top_p, seed, seq_ids, step,
+                                           out_path_nodes, out_path_len, out_tokens, dev_status,
+                                           workspace, g_events, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "sampled tree launch");
+  return PSI_OK;
+}
+
 psi_status psi_rng_uniforms(uint64_t seed, const uint64_t *seq_ids, int32_t n_seq, uint64_t step,
                             int32_t n_rows, uint32_t purpose, float *out, psi_stream_t stream_) {
   if (n_seq < 1 || n_rows < 1 || !out) return fail(PSI_ERR_INVALID_ARG, "n_seq/n_rows/out");

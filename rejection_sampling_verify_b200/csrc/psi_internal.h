@@ -146,31 +146,93 @@ cudaError_t launch_cluster_list(const SampledArgs &a, psi_dtype dtype, const Sam
                                 int max_clusters, cudaStream_t stream);
 
 // ---- streaming path (rows 16-byte aligned) ------------------------------------
-// Per logit row: what the row-scan kernel leaves for the unit kernel.  Every
-// element of the row is counted exactly once: in zt (at or below the
-// threshold of its batch), in zd (above it, but at or below the row's final
-// threshold) or in the row's candidate list (above the final threshold).
-struct RowRecord {
-  float ref;        // final running reference: the row maximum, unless the row holds +inf
-  int32_t n_cand;   // candidates appended (more than the capacity: overflow)
-  int32_t flags;    // kRowLost: flagged vectors were dropped (ring overflow)
-  int32_t n_parked; // vectors parked by the scan (diagnostics)
-  double zt;        // sum of exp2((x - ref) * log2(e) / T) over the unmasked elements
-  uint64_t zd;      // 2^31 * the same sum over masked elements that are not candidates
+// Each logit row is split into `slices` contiguous slices of 16-byte vectors
+// (the last one also holds the V % vector-width tail elements); the CTAs of
+// one thread-block cluster scan the slices of the same row.  Per (row, slice)
+// the scan leaves one record and a list of candidates: the elements above the
+// row's final threshold (row maximum minus the top-p window), which are
+// exactly the elements the top-p cut can keep.
+struct SliceRecord {
+  float m;         // reference of z: the slice maximum (or the known row maximum on a rescan)
+  int32_t n_cand;  // candidates written to the slice's list (more than its capacity: overflow)
+  int32_t flags;   // kRowLost: candidates were dropped (the scan's shared-memory list overflowed)
+  int32_t n_parked;// entries the scan parked before the final filter (diagnostics)
+  double z;        // sum over the slice of exp2((x - m) * log2(e) / T), every element
 };
 constexpr int32_t kRowLost = 1;
-constexpr int kCandCap = 2048;     // candidates kept per row (global workspace)
+constexpr int kCandCap = 2048;   // candidates kept per row (global workspace), split over slices
+constexpr int kMaxSlices = 2;    // slice records reserved per row (slices per row at most)
+
+// How the scan splits a row (the same for every row of a call; chosen from V
+// and the element size only, so per-row results do not depend on N).
+struct ScanGeom {
+  int32_t nvec;        // whole 16-byte vectors per row
+  int32_t tail;        // elements after them (scanned by the last slice)
+  int32_t slices;      // slices per row = CTAs per cluster
+  int32_t stages;      // shared-memory stages per slice
+  int32_t stage_vecs;  // vectors per stage (the last stage of a slice may be shorter)
+  int32_t cap;         // list capacity per slice (kCandCap / slices)
+};
+ScanGeom plan_scan(int32_t V, int elem_bytes);
 
 struct FastLayout {  // workspace carve-up of the streaming path
-  size_t rec_off, rows_off, cand_off, counters_off, list_a_off, list_b_off, wide_rows_off,
-      wide_units_off, round_rows_off, round_units_off, active_off, total;
+  size_t rec_off, srec_off, cand_off, known_off, counters_off, list_a_off, list_b_off,
+      wide_rows_off, wide_units_off, round_rows_off, round_units_off, active_off, total;
 };
 FastLayout fast_layout(int32_t N, int32_t B);
 // False when the streaming path's row indices would not fit its lists.
 bool fast_path_fits(int32_t N, int32_t B);
 
+// Everything the streaming path's kernels read.
+struct FastArgs {
+  SampledArgs s;
+  ScanGeom g;
+  int64_t rows;        // N*(B+1) AR rows followed by N*B draft rows
+  float coef;          // log2(e) / T
+  double coef64;
+  float win_narrow;    // candidate windows below the row maximum, in logit units
+  float win_wide;
+  int use_top_p;
+  int pass;            // 1: a first scan / finish; 2: a rescan of rows that failed
+  const int32_t *rlist;   // rows to scan (nullptr: every row); entries may carry kWideBit
+  const int32_t *rcount;  // their number
+  const int32_t *ulist;   // units to finish (nullptr: every unit)
+  const int32_t *ucount;  // their number
+  int32_t *active;        // [N] sequence still verifying (early-exit rounds)
+  int32_t *round_rows;    // rows of the current round
+  int32_t *round_units;   // units of the current round
+  UnitRecord *rec;     // [N*(B+1)]
+  SliceRecord *srec;   // [rows][kMaxSlices]
+  uint64_t *cand;      // [rows][kCandCap]: slice c's list at c * g.cap; (bits << 32) | index
+  float *known_max;    // [rows] row maximum found by a first pass (read by a rescan)
+  int32_t *counters;   // [0] general units, [1] sample-mode units, [2] wide rows, [3] wide units,
+                       // [4 + 2k], [5 + 2k] rows and units of round parity k
+  int32_t *list_a;     // units for the general path
+  int32_t *list_b;     // units whose draw needs the whole row
+  int32_t *wide_rows;  // rows for the second scan (| kWideBit: wide window)
+  int32_t *wide_units; // units for the second unit pass
+};
+constexpr int32_t kWideBit = int32_t(1) << 30;  // second-pass row entry: wide window
+
+// The row scan over the listed rows (or every row): slice records and
+// candidate lists.  `clusters_hint` caps the number of clusters launched.
+cudaError_t launch_row_scan(const FastArgs &fa, psi_dtype dtype, cudaStream_t stream);
+
 cudaError_t launch_sampled_fast(const SampledArgs &a, psi_dtype dtype, const SampledPlan &plan,
                                 void *workspace, const KernelEvents &ev, cudaStream_t stream);
+
+// ---- sampled tree (psi_tree.cu) -------------------------------------------------
+struct TreeLayout {  // workspace: the row scan's records and candidate lists
+  size_t srec_off, cand_off, known_off, total;
+};
+TreeLayout tree_layout(int32_t N, int32_t M);
+cudaError_t launch_tree_sampled(const void *ar, int64_t ar_stride, psi_dtype dtype,
+                                const int32_t *node_tokens, const int32_t *parents, int32_t N,
+                                int32_t M, int32_t V, float temperature, float top_p,
+                                uint64_t seed, const uint64_t *seq_ids, uint64_t step,
+                                int32_t *out_path, int32_t *out_len, int32_t *out_tokens,
+                                uint32_t *dev_status, void *workspace, const KernelEvents &ev,
+                                cudaStream_t stream);
 
 cudaError_t launch_rng_uniforms(uint64_t seed, const uint64_t *seq_ids, int32_t n_seq,
                                 uint64_t step, int32_t n_rows, uint32_t purpose, float *out,

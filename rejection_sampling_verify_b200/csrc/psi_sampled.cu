@@ -74,22 +74,22 @@ struct Xchg {
   double zhi_part[2];                  // double part (top-p only)
   unsigned long long zwin_part[2];     // fixed-point mass inside the narrow window
   unsigned long long block_sum[4][2];  // radix level, row
-  float w_part[2];                     // [0] first draw, [1] fallback draw
+  unsigned long long w_part[2];        // [0] first draw, [1] fallback draw (fixed point)
 };
 
 struct Broadcast {  // CTA-local results shared after __syncthreads
   float m[2];
   double z[2];
   float window[2];  // top-p histogram window for this row
-  float zp[2];     // normaliser after top-p
+  double zp[2];    // normaliser after top-p (Z without top-p)
   float tau[2];    // keep v iff logit >= tau (-inf: keep all)
   unsigned long long above[2];
   unsigned long long target[2];
   uint32_t prefix[2];
   int need_sample;
   int cross_rank;
-  float t_local;
-  float w_total;
+  unsigned long long t_local;
+  unsigned long long w_total;
   int use_p_only;
 };
 
@@ -252,7 +252,7 @@ __device__ void radix_crossing(int r, int level, int level_bits, bool last, uint
     bc->above[r] = run;
     bc->prefix[r] = (bc->prefix[r] << level_bits) | (uint32_t)bstar;
     if (last) {
-      bc->zp[r] = (float)((double)(run + mass_b) * kFixInv);
+      bc->zp[r] = (double)(run + mass_b) * kFixInv;
       // threshold logit: the value whose key is the full prefix
       const uint32_t key = bc->prefix[r];
       uint32_t bits;
@@ -323,7 +323,7 @@ __global__ void __launch_bounds__(kThreads) sampled_unit_kernel(SampledArgs a, S
   unsigned long long *hist = reinterpret_cast<unsigned long long *>(buf_q + (size_t)nvp * VEC);
   const int per_max = (kBins + (int)C - 1) / (int)C;
   unsigned long long *owned = hist + 2 * kBins;
-  float *chunk_sum = reinterpret_cast<float *>(owned + 2 * per_max);
+  unsigned long long *chunk_sum = owned + 2 * per_max;
 
   // ---- 1. one bulk copy per row slice into shared memory -------------------
   const bool aligned = ((reinterpret_cast<uintptr_t>(row_p + c0) & 15u) == 0) &&
@@ -415,14 +415,15 @@ __global__ void __launch_bounds__(kThreads) sampled_unit_kernel(SampledArgs a, S
     double zhi = 0.0;
     unsigned long long zwin = 0ull;
     if (!use_top_p) {
-      for (int32_t j = tid; j < nvp; j += kThreads) {
-        const uint4 w = src[j];
-        float part = 0.f;
+      // without top-p, Z normalises the whole-row draw: every exponential in
+      // double precision
+      if (m > -INFINITY)
+        for (int32_t j = tid; j < nvp; j += kThreads) {
+          const uint4 w = src[j];
 #pragma unroll
-        for (int k = 0; k < VEC; ++k)
-          part += fast_exp2(fmaf(Elem<Bits>::to_float(vec_elem<Bits>(w, k)), coef, (r == 0 ? shift_p : shift_q)));
-        zlo += part;
-      }
+          for (int k = 0; k < VEC; ++k)
+            zhi += exact_exp2(Elem<Bits>::to_float(vec_elem<Bits>(w, k)), m, coef64);
+        }
     } else {
       for (int32_t j = tid; j < nvp; j += kThreads) {
         const uint4 w = src[j];
@@ -466,7 +467,7 @@ __global__ void __launch_bounds__(kThreads) sampled_unit_kernel(SampledArgs a, S
     zw = warp_sum_t(zw);
     if (lane == 0) {
       bc.z[r] = z;
-      bc.zp[r] = (float)z;
+      bc.zp[r] = z;
       bc.tau[r] = -INFINITY;
       bc.above[r] = 0ull;
       bc.prefix[r] = 0u;
@@ -568,28 +569,28 @@ __global__ void __launch_bounds__(kThreads) sampled_unit_kernel(SampledArgs a, S
   }
 
   // ---- 5. accept / reject the drafted token (every CTA, same result) -------
-  const float inv_zp = bc.zp[0] > 0.f ? 1.f / bc.zp[0] : 0.f;
-  const float inv_zq = bc.zp[1] > 0.f ? 1.f / bc.zp[1] : 0.f;
+  const double zp_p = bc.zp[0], zp_q = bc.zp[1];
   const float tau_p = bc.tau[0], tau_q = bc.tau[1];
+  const float m_p = bc.m[0], m_q = bc.m[1];
   if (tid == 0) {
     int need = 1;
     if (has_q) {
       const int32_t x = s_x;
-      float p = 0.f, q = 0.f;
+      double p = 0.0, q = 0.0;
       const bool valid = x >= 0 && x < V;
       if (valid) {
         const float xp = Elem<Bits>::to_float(s_x_bits[0]);
         const float xq = Elem<Bits>::to_float(s_x_bits[1]);
-        if (xp >= tau_p) p = fast_exp2(fmaf(xp, coef, shift_p)) * inv_zp;
-        if (xq >= tau_q) q = fast_exp2(fmaf(xq, coef, shift_q)) * inv_zq;
+        if (xp >= tau_p && zp_p > 0.0) p = exact_exp2(xp, m_p, coef64) / zp_p;
+        if (xq >= tau_q && zp_q > 0.0) q = exact_exp2(xq, m_q, coef64) / zp_q;
       }
-      const float u = uniform24(a.seed, seq, a.step, (uint64_t)i, PSI_PURPOSE_ACCEPT);
+      const double u = uniform24(a.seed, seq, a.step, (uint64_t)i, PSI_PURPOSE_ACCEPT);
       const int accept = (u * q < p) ? 1 : 0;
       need = (mode == kModeSample) ? 1 : !accept;
       if (rank == 0 && mode != kModeSample) {
         const int64_t o = (int64_t)n * B + i;
-        if (a.out_p) a.out_p[o] = p;
-        if (a.out_q) a.out_q[o] = q;
+        if (a.out_p) a.out_p[o] = (float)p;
+        if (a.out_q) a.out_q[o] = (float)q;
         a.records[unit].accept = accept;
         if (accept) a.records[unit].token = -1;
         if (!valid && a.dev_status) atomicOr(a.dev_status, PSI_DEV_BAD_TOKEN_ID);
@@ -605,8 +606,21 @@ __global__ void __launch_bounds__(kThreads) sampled_unit_kernel(SampledArgs a, S
     atomicOr(a.dev_status, (bad ? PSI_DEV_NONFINITE : 0u) | (timed_out ? PSI_DEV_TIMEOUT : 0u));
 
   // ---- 6. correction (rejected row) or bonus (row B) draw -------------------
-  // Weights w(v) = max(0, p(v) - q(v)) or p(v); inverse CDF in vocabulary
-  // order: the first v whose running sum exceeds u' * sum(w).
+  // Weights w(v) = max(0, p(v) - q(v)) or p(v), in double precision and
+  // 2^40 fixed point (exact integer sums in any order); inverse CDF in
+  // vocabulary order: the first v whose running sum exceeds
+  // t = floor(u' * sum(w)).
+  auto weight = [&](uint32_t bp, uint32_t bq, bool p_only) -> unsigned long long {
+    const float xp = Elem<Bits>::to_float(bp);
+    if (!(xp >= tau_p) || !(zp_p > 0.0)) return 0ull;
+    double pv = exact_exp2(xp, m_p, coef64) / zp_p;
+    if (!p_only) {
+      const float xq = Elem<Bits>::to_float(bq);
+      const double qv = (xq >= tau_q && zp_q > 0.0) ? exact_exp2(xq, m_q, coef64) / zp_q : 0.0;
+      pv = pv - qv;
+    }
+    return pv > 0.0 ? __double2ull_rn(fmin(pv, 1.0) * kFixScaleD) : 0ull;
+  };
   if (bc.need_sample) {
     for (int attempt = 0; attempt < 2; ++attempt) {
       const bool p_only = bc.use_p_only != 0;
@@ -614,182 +628,105 @@ __global__ void __launch_bounds__(kThreads) sampled_unit_kernel(SampledArgs a, S
       for (int32_t j = tid; j < nvp; j += kThreads) {
         const uint4 w = vp[j];
         const uint4 u = p_only ? w : vq[j];
-        float part = 0.f;
+        unsigned long long part = 0ull;
 #pragma unroll
-        for (int k = 0; k < VEC; ++k) {
-          const float xp = Elem<Bits>::to_float(vec_elem<Bits>(w, k));
-          float pv = 0.f;
-          if (xp >= tau_p) pv = fast_exp2(fmaf(xp, coef, shift_p)) * inv_zp;
-          if (!p_only && pv > 0.f) {
-            const float xq = Elem<Bits>::to_float(vec_elem<Bits>(u, k));
-            float qv = 0.f;
-            if (xq >= tau_q) qv = fast_exp2(fmaf(xq, coef, shift_q)) * inv_zq;
-            pv = fmaxf(pv - qv, 0.f);
-          }
-          part += pv;
-        }
-        part = warp_sum(part);
+        for (int k = 0; k < VEC; ++k)
+          part += weight(vec_elem<Bits>(w, k), vec_elem<Bits>(u, k), p_only);
+        part = warp_sum_t(part);
         if (lane == 0) chunk_sum[j >> 5] = part;
       }
       __syncthreads();
       if (tid == 0) {
-        float s = 0.f;
+        unsigned long long s = 0ull;
         for (int c = 0; c < nchunks; ++c) s += chunk_sum[c];
         xc.w_part[attempt] = s;
       }
       cluster_sync();
       if (warp == 0) {
-        const float wk =
-            (uint32_t)lane < C ? dsmem_ld_f32(dsmem_map(&xc.w_part[attempt], lane)) : 0.f;
+        const unsigned long long wk =
+            (uint32_t)lane < C ? dsmem_ld_u64(dsmem_map(&xc.w_part[attempt], lane)) : 0ull;
         // inclusive prefix over ranks in rank (= vocabulary) order
-        float pre = wk;
+        unsigned long long pre = wk;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-          const float t = __shfl_up_sync(0xFFFFFFFFu, pre, o);
+          const unsigned long long t = __shfl_up_sync(0xFFFFFFFFu, pre, o);
           if (lane >= o) pre += t;
         }
-        const float total = __shfl_sync(0xFFFFFFFFu, pre, 31);
+        const unsigned long long total = __shfl_sync(0xFFFFFFFFu, pre, 31);
         if (lane == 0) bc.w_total = total;
-        if (total > 0.f) {
+        if (total > 0ull) {
           const float u2 = uniform24(a.seed, seq, a.step, (uint64_t)i, PSI_PURPOSE_RESID);
-          const float t = u2 * total;
+          const unsigned long long k = (unsigned long long)(u2 * 16777216.0f);  // u' = k / 2^24
+          const unsigned long long t = (__umul64hi(k, total) << 40) | ((k * total) >> 24);
           const unsigned hit = __ballot_sync(0xFFFFFFFFu, (uint32_t)lane < C && pre > t);
-          int kstar;
-          float before;
-          if (hit) {
-            kstar = __ffs(hit) - 1;
-          } else {  // rounding: the last rank holding positive weight
-            const unsigned pos = __ballot_sync(0xFFFFFFFFu, (uint32_t)lane < C && wk > 0.f);
-            kstar = 31 - __clz(pos);
-          }
-          before = __shfl_sync(0xFFFFFFFFu, pre - wk, kstar);
+          const int kstar = __ffs(hit) - 1;  // exact sums: t < total, so some rank hits
+          const unsigned long long before = __shfl_sync(0xFFFFFFFFu, pre - wk, kstar);
           if (lane == 0) {
-            bc.cross_rank = hit ? kstar : -1 - kstar;  // negative: take the last positive
+            bc.cross_rank = kstar;
             bc.t_local = t - before;
           }
         }
       }
       __syncthreads();
-      if (bc.w_total > 0.f || p_only) break;
+      if (bc.w_total > 0ull || p_only) break;
       // the residual vanished (q_L(x_L) was 0): draw from p_L instead
       if (tid == 0) bc.use_p_only = 1;
       __syncthreads();
     }
 
-    const int cr = bc.cross_rank;
-    const int my_rank = cr >= 0 ? cr : -1 - cr;
-    if (bc.w_total > 0.f && (int)rank == my_rank && warp == 0) {
+    if (bc.w_total > 0ull && (int)rank == bc.cross_rank && warp == 0) {
       const bool p_only = bc.use_p_only != 0;
-      const float t = bc.t_local;
-      // find the chunk
-      int cstar = -1;
-      float before = 0.f;
-      if (cr >= 0) {
-        float run = 0.f;
-        for (int c = 0; c < nchunks; ++c) {  // same order as the CTA total
-          const float nxt = run + chunk_sum[c];
-          if (nxt > t) {
-            cstar = c;
-            before = run;
+      const unsigned long long t = bc.t_local;
+      // the chunk holding the crossing (same order as the CTA total)
+      int cstar = 0;
+      unsigned long long before = 0ull;
+      for (int c = 0; c < nchunks; ++c) {
+        const unsigned long long nxt = before + chunk_sum[c];
+        if (nxt > t) {
+          cstar = c;
+          break;
+        }
+        before = nxt;
+      }
+      const int32_t j = cstar * 32 + lane;  // this lane's vector in the chunk
+      const uint4 w = vp[j];
+      const uint4 u = p_only ? w : vq[j];
+      unsigned long long wv[VEC];
+      unsigned long long part = 0ull;
+#pragma unroll
+      for (int k = 0; k < VEC; ++k) {
+        wv[k] = weight(vec_elem<Bits>(w, k), vec_elem<Bits>(u, k), p_only);
+        part += wv[k];
+      }
+      unsigned long long pre = part;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long tt = __shfl_up_sync(0xFFFFFFFFu, pre, o);
+        if (lane >= o) pre += tt;
+      }
+      const unsigned hit = __ballot_sync(0xFFFFFFFFu, before + pre > t);
+      const int l = hit ? __ffs(hit) - 1 : 31;
+      int32_t token = c0 + j * VEC;
+      if (lane == l) {
+        unsigned long long run = before + pre - part;
+        int kk = VEC - 1;
+        for (int k = 0; k < VEC; ++k) {
+          run += wv[k];
+          if (run > t) {
+            kk = k;
             break;
           }
-          run = nxt;
         }
+        token = c0 + j * VEC + kk;
       }
-      int32_t token = -1;
-      if (cstar >= 0) {
-        const int32_t j = cstar * 32 + lane;  // this lane's vector in the chunk
-        const uint4 w = vp[j];
-        const uint4 u = p_only ? w : vq[j];
-        float wv[VEC];
-        float part = 0.f;
-#pragma unroll
-        for (int k = 0; k < VEC; ++k) {
-          const float xp = Elem<Bits>::to_float(vec_elem<Bits>(w, k));
-          float pv = 0.f;
-          if (xp >= tau_p) pv = fast_exp2(fmaf(xp, coef, shift_p)) * inv_zp;
-          if (!p_only && pv > 0.f) {
-            const float xq = Elem<Bits>::to_float(vec_elem<Bits>(u, k));
-            float qv = 0.f;
-            if (xq >= tau_q) qv = fast_exp2(fmaf(xq, coef, shift_q)) * inv_zq;
-            pv = fmaxf(pv - qv, 0.f);
-          }
-          wv[k] = pv;
-          part += pv;
-        }
-        float pre = part;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const float tt = __shfl_up_sync(0xFFFFFFFFu, pre, o);
-          if (lane >= o) pre += tt;
-        }
-        int lastpos = -1;
-#pragma unroll
-        for (int k = 0; k < VEC; ++k)
-          if (wv[k] > 0.f) lastpos = k;
-        const unsigned hit = __ballot_sync(0xFFFFFFFFu, before + pre > t);
-        if (hit) {
-          const int l = __ffs(hit) - 1;
-          if (lane == l) {
-            float run = before + pre - part;
-            int kk = -1;
-#pragma unroll
-            for (int k = 0; k < VEC; ++k) {
-              run += wv[k];
-              if (kk < 0 && run > t) kk = k;
-            }
-            if (kk < 0) kk = lastpos >= 0 ? lastpos : 0;
-            token = c0 + j * VEC + kk;
-          }
-          token = __shfl_sync(0xFFFFFFFFu, token, l);
-        } else {
-          // rounding put the target past this chunk's sum: its last positive
-          const unsigned pos = __ballot_sync(0xFFFFFFFFu, lastpos >= 0);
-          if (pos) {
-            const int l = 31 - __clz(pos);
-            const int kl = __shfl_sync(0xFFFFFFFFu, lastpos, l);
-            token = c0 + (cstar * 32 + l) * VEC + kl;
-          } else {
-            cstar = -1;
-          }
-        }
-      }
-      if (cstar < 0) {
-        // last element of this CTA's slice with positive weight
-        for (int32_t j = nvp - 1 - lane; j >= 0 && token < 0; j -= 32) {
-          int kk = -1;
-          const uint4 w = vp[j];
-          const uint4 u = p_only ? w : vq[j];
-#pragma unroll
-          for (int k = 0; k < VEC; ++k) {
-            const float xp = Elem<Bits>::to_float(vec_elem<Bits>(w, k));
-            float pv = 0.f;
-            if (xp >= tau_p) pv = fast_exp2(fmaf(xp, coef, shift_p)) * inv_zp;
-            if (!p_only && pv > 0.f) {
-              const float xq = Elem<Bits>::to_float(vec_elem<Bits>(u, k));
-              float qv = 0.f;
-              if (xq >= tau_q) qv = fast_exp2(fmaf(xq, coef, shift_q)) * inv_zq;
-              pv = fmaxf(pv - qv, 0.f);
-            }
-            if (pv > 0.f) kk = k;
-          }
-          const unsigned any = __ballot_sync(0xFFFFFFFFu, kk >= 0);
-          if (any) {
-            const int l = __ffs(any) - 1;  // lowest lane = highest vector
-            const int kl = __shfl_sync(0xFFFFFFFFu, kk, l);
-            const int jl = __shfl_sync(0xFFFFFFFFu, j, l);
-            token = c0 + jl * VEC + kl;
-          }
-        }
-        if (token < 0) token = c0;
-      }
+      token = __shfl_sync(0xFFFFFFFFu, token, l);
       if (lane == 0) {
         if (mode == kModeSample) a.out_tokens[unit] = token;
         else a.records[unit].token = token;
       }
     }
   }
-  if (bc.need_sample && bc.w_total <= 0.f && rank == 0 && tid == 0) {
+  if (bc.need_sample && bc.w_total == 0ull && rank == 0 && tid == 0) {
     // no positive weight anywhere (degenerate row)
     if (mode == kModeSample) a.out_tokens[unit] = 0;
     else a.records[unit].token = 0;
@@ -842,7 +779,7 @@ bool plan_sampled(int32_t V, int elem_bytes, SampledPlan *plan) {
   plan->slice = (int32_t)S;
   plan->nvec_pad = (int32_t)nvp;
   plan->smem = (size_t)2 * nvp * 16 + sizeof(unsigned long long) * (2 * kBins + 2 * per_max) +
-               sizeof(float) * (size_t)(nvp / 32);
+               sizeof(unsigned long long) * (size_t)(nvp / 32);
   return true;
 }
 

@@ -93,6 +93,15 @@ def test_noalloc_greedy_matches_workspace_entry():
     _run_both(b, 0.0, 1.0, 0, 0)
 
 
+def test_noalloc_greedy_early_exit_rounds_match_workspace_entry():
+    """128 sequences take the greedy early-exit rounds, whose partials, row
+    lists, counters and active flags then live in the library's scratch."""
+    cfg = CFG["max_batch_greedy"]
+    b = psi_inputs.linear_batch(cfg, device="cuda", N=128, index=1)
+    assert b.ar.shape[0] >= psi.PSI_EARLY_EXIT_MIN_N
+    _run_both(b, 0.0, 1.0, 0, 0)
+
+
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     # 600 sequences of 17 rows need far more than the scratch holds (the
     # sampled path keeps a candidate list per row); nothing is launched
