@@ -363,8 +363,13 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
   cudaError_t e;
   static DeviceOnce configure;  // shared memory above 48 KB, once per device
   e = configure([] {
-    return cudaFuncSetAttribute(unit_kernel<Bits>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)sizeof(UnitShared));
+    cudaError_t err = cudaFuncSetAttribute(unit_kernel<Bits>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)sizeof(UnitShared));
+    if (err == cudaSuccess) err = prefer_max_shared(unit_kernel<Bits>);
+    if (err == cudaSuccess) err = prefer_max_shared(round_advance_kernel);
+    if (err == cudaSuccess) err = prefer_max_shared(fast_emit_kernel);
+    return err;
   });
   if (e != cudaSuccess) return e;
   // the work-list counters of this call start at zero

@@ -54,9 +54,9 @@ constexpr int kRegCand = 16;             // candidates per lane a search keeps i
 constexpr double kFix52 = 4503599627370496.0;  // 2^52
 
 struct WarpScratch {
-  uint32_t key[kCandCap];  // candidate keys (order-preserving image of the logit)
-  uint32_t idx[kCandCap];  // vocabulary indices; later the nucleus indices
-  uint64_t m[kCandCap];    // 2^52 fixed-point masses exp2((x - M) * log2(e)/T) (double);
+  uint32_t key[kFinishCap];  // candidate keys (order-preserving image of the logit)
+  uint32_t idx[kFinishCap];  // vocabulary indices; later the nucleus indices
+  uint64_t m[kFinishCap];    // 2^52 fixed-point masses exp2((x - M) * log2(e)/T) (double);
                            // later the nucleus masses, compacted; in the q row's
                            // scratch, the draw weights
 };
@@ -65,15 +65,16 @@ struct WarpScratch {
 __device__ __forceinline__ uint64_t fixed52(double m) { return __double2ull_rn(m * kFix52); }
 
 // Row maximum, Z, top-p threshold tau and renormaliser Z' of row r from its
-// slice records and candidate lists, by one warp.  M is the largest slice
-// reference and Z the slices' sums rescaled to it (double).  The candidates
-// are exactly the elements above the row's final threshold; the top-p
-// threshold is the largest logit key t whose suffix mass S(t) (every x with
-// key >= t) reaches top_p * Z: a binary search over the candidates' key range
-// on exact 2^52 fixed-point sums of the double-precision masses (integer
-// sums: independent of candidate order).  Only candidates can be at or above tau when they hold at
-// least top_p of the mass.  The candidate lists stay unchanged, so a second
-// pass may finish the row again.
+// slice records and set-aside lists, by one warp.  M is the largest slice
+// reference; the set-aside elements above the row's final threshold
+// (M - window, rounded as the scan rounds) are the candidates, the others
+// join Z with the slices' sums (rescaled to M), every mass in double
+// precision and 2^52 fixed point.  The top-p threshold is the largest logit
+// key t whose suffix mass S(t) (every x with key >= t) reaches top_p * Z: a
+// binary search over the candidates' key range on exact integer sums
+// (independent of the order of the lists).  Only candidates can be at or
+// above tau when they hold at least top_p of the mass.  The lists stay
+// unchanged, so a second pass may finish the row again.
 template <typename Bits>
 __device__ RowFinal finish_row(const FastArgs &a, int64_t r, WarpScratch *ws) {
   const int lane = threadIdx.x & 31;
@@ -88,20 +89,29 @@ __device__ RowFinal finish_row(const FastArgs &a, int64_t r, WarpScratch *ws) {
   const SliceRecord *sr = a.srec + r * kMaxSlices;
   float M = -INFINITY;
   bool lost = false;
-  int n = 0;
   for (int c = 0; c < C; ++c) {
     M = fmaxf(M, sr[c].m);
     lost |= (sr[c].flags & kRowLost) != 0 || sr[c].n_cand > a.g.cap;
-    n += sr[c].n_cand;
   }
   out.m = M;
   if (lost) {
     out.status = kFinOverflow;
     return out;
   }
-  out.n = n;
+  double Z = 0.0;
+  for (int c = 0; c < C; ++c)
+    if (sr[c].m > -INFINITY) Z += sr[c].z * exp2(((double)sr[c].m - (double)M) * a.coef64);
+  if (!(M > -INFINITY) || !(fabsf(M * a.coef) < INFINITY) || Z != Z) {
+    out.status = kFinNonfinite;
+    return out;
+  }
+  const float thr = a.use_top_p ? threshold_value<Bits>(M - sr[0].off) : INFINITY;
+  // sort the set-aside elements: candidates to the scratch, the rest to Z
+  const unsigned below = (1u << lane) - 1u;
+  int n = 0;
+  unsigned long long zin = 0ull, zrest = 0ull;
   uint32_t kmax = 0u, kmin_inv = 0u;
-  for (int c = 0, at = 0; c < C; at += sr[c].n_cand, ++c) {
+  for (int c = 0; c < C; ++c) {
     const int nc = sr[c].n_cand;
     const unsigned long long *src = reinterpret_cast<const unsigned long long *>(
         a.cand + r * (int64_t)kCandCap + (int64_t)c * a.g.cap);
@@ -115,36 +125,39 @@ __device__ RowFinal finish_row(const FastArgs &a, int64_t r, WarpScratch *ws) {
 #pragma unroll
       for (int h = 0; h < kLoadChunk; ++h) {
         const int j = base + 32 * h + lane;
-        if (j < nc) {
-          const uint32_t key = Elem<Bits>::key((uint32_t)(e[h] >> 32));
-          ws->key[at + j] = key;
-          ws->idx[at + j] = (uint32_t)e[h];
+        const uint32_t b = (uint32_t)(e[h] >> 32);
+        const float x = Elem<Bits>::to_float(b);
+        const bool live = j < nc;
+        const bool cand = live && x > thr;
+        const double mass = live ? exact_exp2d(x, M, a.coef64) : 0.0;
+        if (live && !cand && mass > 0.0) zrest += fixed52(mass);
+        const unsigned bal = __ballot_sync(0xFFFFFFFFu, cand);
+        const int d = n + __popc(bal & below);
+        if (cand && d < kFinishCap) {
+          const uint32_t key = Elem<Bits>::key(b);
+          const uint64_t m52 = fixed52(mass);
+          ws->key[d] = key;
+          ws->idx[d] = (uint32_t)e[h];
+          ws->m[d] = m52;
+          zin += m52;
           kmax = max(kmax, key);
           kmin_inv = max(kmin_inv, ~key);
         }
+        n += __popc(bal);
       }
     }
   }
-  kmax = warp_max_u32(kmax);
-  kmin_inv = warp_max_u32(kmin_inv);
-  double Z = 0.0;
-  for (int c = 0; c < C; ++c)
-    if (sr[c].m > -INFINITY) Z += sr[c].z * exp2(((double)sr[c].m - (double)M) * a.coef64);
-  if (!(M > -INFINITY) || !(fabsf(M * a.coef) < INFINITY) || Z != Z) {
-    out.status = kFinNonfinite;
+  if (n > kFinishCap) {  // more candidates than the finish holds: rescan, then the general path
+    out.status = kFinOverflow;
     return out;
   }
-  unsigned long long zin = 0ull;
-  for (int j = lane; j < n; j += 32) {
-    const uint64_t m = fixed52(
-        exact_exp2d(Elem<Bits>::to_float(key_to_bits<Bits>(ws->key[j])), M, a.coef64));
-    ws->m[j] = m;
-    zin += m;
-  }
+  out.n = n;
+  kmax = warp_max_u32(kmax);
+  kmin_inv = warp_max_u32(kmin_inv);
   zin = warp_sum_any(zin);
+  zrest = warp_sum_any(zrest);
   __syncwarp();
-  // the slices' sums hold every element that is not a candidate
-  Z += (double)zin / kFix52;
+  Z += ((double)zin + (double)zrest) / kFix52;
   out.zp = Z;
   if (!(Z < INFINITY)) {
     out.status = kFinNonfinite;

@@ -41,6 +41,17 @@ class DeviceOnce {
   std::atomic<uint64_t> done_{0};
 };
 
+// The sampled path alternates kernels of very different shared-memory needs
+// (the row scan takes nearly all of an SM's); every one of them asks for the
+// largest shared-memory carveout, so that consecutive launches never wait for
+// an SM to re-split its L1 / shared storage.
+template <typename Kernel>
+inline cudaError_t prefer_max_shared(Kernel *k) {
+  return cudaFuncSetAttribute(reinterpret_cast<const void *>(k),
+                              cudaFuncAttributePreferredSharedMemoryCarveout,
+                              (int)cudaSharedmemCarveoutMaxShared);
+}
+
 // Early-exit round schedule: `short_rounds` rounds of PSI_ROUND_POSITIONS
 // positions, then one round with the rest of the B + 1 positions.
 __host__ __device__ inline int32_t round_begin(int k, int32_t B, int short_rounds) {
@@ -147,31 +158,45 @@ cudaError_t launch_cluster_list(const SampledArgs &a, psi_dtype dtype, const Sam
 
 // ---- streaming path (rows 16-byte aligned) ------------------------------------
 // Each logit row is split into `slices` contiguous slices of 16-byte vectors
-// (the last one also holds the V % vector-width tail elements); the CTAs of
-// one thread-block cluster scan the slices of the same row.  Per (row, slice)
-// the scan leaves one record and a list of candidates: the elements above the
-// row's final threshold (row maximum minus the top-p window), which are
-// exactly the elements the top-p cut can keep.
+// (the last one also holds the V % vector-width tail elements), each scanned
+// by its own CTA.  Per (row, slice) the scan leaves one record and the list of
+// the elements it set aside: every element above the running top-p
+// threshold of its stage (and the tail elements).  The row's final threshold
+// is known only from all slices, so the finish sorts the set-aside elements
+// into candidates (above it: exactly the elements the top-p cut can keep) and
+// the rest of the sum.
 struct SliceRecord {
   float m;         // reference of z: the slice maximum (or the known row maximum on a rescan)
-  int32_t n_cand;  // candidates written to the slice's list (more than its capacity: overflow)
-  int32_t flags;   // kRowLost: candidates were dropped (the scan's shared-memory list overflowed)
-  int32_t n_parked;// entries the scan parked before the final filter (diagnostics)
-  double z;        // sum over the slice of exp2((x - m) * log2(e) / T), every element
+  int32_t n_cand;  // elements set aside into the slice's list (above its capacity: overflow)
+  int32_t flags;   // kRowLost: elements were dropped (the list overflowed)
+  float off;       // the row's top-p window below its maximum (logit units) the scan used
+  double z;        // sum over the slice's other elements of exp2((x - m) * log2(e) / T)
 };
 constexpr int32_t kRowLost = 1;
-constexpr int kCandCap = 2048;   // candidates kept per row (global workspace), split over slices
+constexpr int kCandCap = 4096;   // set-aside elements kept per row (global workspace), split over slices
+constexpr int kFinishCap = 2048; // candidates the finish holds per row
 constexpr int kMaxSlices = 2;    // slice records reserved per row (slices per row at most)
+
+// Candidate threshold in the element type: bf16 thresholds are rounded down,
+// so rounding can only add candidates.  The scan and the finish round the
+// same way.
+template <typename Bits>
+__device__ __forceinline__ float threshold_value(float thr) {
+  if constexpr (sizeof(Bits) == 2)
+    return __bfloat162float(__float2bfloat16_rd(thr));
+  else
+    return thr;
+}
 
 // How the scan splits a row (the same for every row of a call; chosen from V
 // and the element size only, so per-row results do not depend on N).
 struct ScanGeom {
   int32_t nvec;        // whole 16-byte vectors per row
   int32_t tail;        // elements after them (scanned by the last slice)
-  int32_t slices;      // slices per row = CTAs per cluster
+  int32_t slices;      // slices per row (CTAs per row)
   int32_t stages;      // shared-memory stages per slice
   int32_t stage_vecs;  // vectors per stage (the last stage of a slice may be shorter)
-  int32_t cap;         // list capacity per slice (kCandCap / slices)
+  int32_t cap;         // set-aside list capacity per slice (kCandCap / slices)
 };
 ScanGeom plan_scan(int32_t V, int elem_bytes);
 
@@ -203,7 +228,8 @@ struct FastArgs {
   int32_t *round_units;   // units of the current round
   UnitRecord *rec;     // [N*(B+1)]
   SliceRecord *srec;   // [rows][kMaxSlices]
-  uint64_t *cand;      // [rows][kCandCap]: slice c's list at c * g.cap; (bits << 32) | index
+  uint64_t *cand;      // [rows][kCandCap]: slice c's set-aside list at c * g.cap;
+                       // (bits << 32) | vocabulary index
   float *known_max;    // [rows] row maximum found by a first pass (read by a rescan)
   int32_t *counters;   // [0] general units, [1] sample-mode units, [2] wide rows, [3] wide units,
                        // [4 + 2k], [5 + 2k] rows and units of round parity k

@@ -819,6 +819,7 @@ static cudaError_t launch_cluster_kernel(const SampledArgs &a, const SampledPlan
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
+    if ((e = prefer_max_shared(kernel)) != cudaSuccess) return e;
     if (slot) {
       int cur = configured_smem[dev].load(std::memory_order_relaxed);
       while ((int)plan.smem > cur &&

@@ -10,37 +10,47 @@
 // What one scan leaves per logit row r (an AR or draft row of a listed unit),
 // the row being split into g.slices contiguous slices of 16-byte vectors:
 //   - per slice c, a record: m_c (the slice maximum; on a rescan the known row
-//     maximum) and z_c = sum over the slice of exp2((x - m_c) * log2(e) / T),
-//     summed in fp32 by a fixed thread / accumulator assignment and reduced in
-//     double in a fixed order, so it is a deterministic function of the slice;
-//   - per slice c, its candidates: every element x > thr, where thr is the
-//     row maximum minus the top-p window, rounded down to the element type.
-//     Every element the top-p cut can keep is a candidate (the window holds
-//     at least top_p of the mass, which the finish checks), and no other
-//     element is.
+//     maximum) and z_c = sum of exp2((x - m_c) * log2(e) / T) over the
+//     slice's elements that were not set aside, summed in fp32 by a fixed
+//     thread / accumulator assignment and reduced in double in a fixed order,
+//     so it is a deterministic function of the slice;
+//   - per slice c, its set-aside list: with top-p, every element above the
+//     running threshold of its stage (the reference so far minus the top-p
+//     window, rounded down to the element type), and the tail elements.  The
+//     threshold of a stage is at most the row's final one, so every element
+//     the top-p cut can keep is in the lists; the finish (psi_finish.cuh)
+//     sorts them into candidates and the rest of the sum.
 //
-// Design: one CTA per SM, clusters of g.slices CTAs; CTA `rank` of a cluster
-// scans slice `rank` of each of the cluster's rows (rows are dealt to the
-// clusters round robin).  Warp roles:
+// Design: one CTA per SM; CTAs form groups of g.slices, CTA c of a group
+// scanning slice c of each of the group's rows (rows are dealt to the groups
+// round robin; the slices of a row are independent).  Warp roles:
 //   producer  (one warp, one lane) keeps a ring of kStages shared-memory
 //             stages filled with cp.async.bulk copies (no multicast), each
 //             completing on its stage's mbarrier, and runs ahead through row
 //             ends.
-//   consumers (kConsumerWarps) load each stage once into registers and hand
-//             the buffer back at once.  Pass 1 takes each vector's maximum;
-//             the CTA's stage maximum is combined through a per-stage
-//             mbarrier.  Pass 2 runs one stage later (so that combine never
-//             stalls them): the running reference becomes the row maximum so
-//             far (every exponent <= 0), the exponentials are added to fp32
-//             accumulators (rescaled when the reference rises), and the
-//             elements above the running threshold are parked in a
-//             shared-memory list for the row.
-//   row end   (one warp) adds the V % 8 tail elements, exchanges the slice
-//             maximum with the cluster's other CTAs over DSMEM (a store into
-//             each CTA's shared memory and a remote mbarrier arrive), filters
-//             the parked elements against the row's final threshold into the
-//             slice's candidate list in global memory and writes the slice
-//             record, off the consumers' path.
+//   consumers (kConsumerWarps) load each stage once into registers.  Pass 1
+//             takes each vector's maximum; the CTA's stage maximum is
+//             combined through a per-stage mbarrier.  Pass 2 runs one stage
+//             later (so that combine never stalls them): the running
+//             reference becomes the row maximum so far (every exponent <= 0)
+//             and the exponentials are added to fp32 accumulators (rescaled
+//             when the reference rises).  With top-p, a vector holding an
+//             element above the running threshold (reference minus the
+//             window; the reference looks one stage ahead for it) is left out
+//             of the sum whole, and its bit is set in the thread's flag byte.
+//   aux       (kAuxWarps warps) take each stage after the consumers' pass
+//             2: the flagged vectors are split among them by their index u
+//             within the consumer thread; each warp queues its share, reads
+//             those vectors again from the stage buffer (32 per round),
+//             appends their elements above the threshold to the slice's
+//             set-aside list in global memory (positions from a shared
+//             counter: the list's order is free), adds their other elements
+//             to its own fp32 sums (against the consumers' reference of the
+//             stage), and hands the buffer back to the producer.  At a row
+//             end aux warp 0 sets the V % 8 tail elements aside and writes
+//             the slice record.  The consumers never wait on the aux warps:
+//             their only effect on them is how long a buffer stays out of
+//             the ring.
 // Every wait is bounded: a wait that gives up sets the CTA's abort flag, every
 // role then leaves its loop, and the kernel reports PSI_DEV_TIMEOUT.
 #include <algorithm>
@@ -52,55 +62,69 @@ namespace psi {
 namespace {
 
 constexpr int kConsumerWarps = 8;
-constexpr int kRowEndWarps = 2;  // row t is finished by row-end warp t % 2
-constexpr int kScanWarps = kConsumerWarps + 1 + kRowEndWarps;
+constexpr int kAuxWarps = 3;  // with the producer, one extra warp per SM sub-partition
+constexpr int kScanWarps = kConsumerWarps + 1 + kAuxWarps;
 constexpr int kScanThreads = kScanWarps * 32;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kProducerWarp = kConsumerWarps;
-constexpr int kRowEndWarp0 = kConsumerWarps + 1;
-constexpr int kStages = 5;
+constexpr int kAuxWarp0 = kConsumerWarps + 1;
+constexpr int kStages = 6;
 constexpr int kStageBytes = 32768;
 constexpr int kStageVecs = kStageBytes / 16;
 constexpr int kVecsPerThread = kStageVecs / kConsumerThreads;
 constexpr int kMaxSlots = 2 * kStages;  // stage-maximum slots (see the consumer loop)
-constexpr int kParkSlots = kRowEndWarps;  // rows whose set-aside vectors await a row-end warp
-constexpr int kParkCap = 1536;            // set-aside vectors per row and slice
-constexpr int kXSlots = 2 * kRowEndWarps; // slice-maximum exchange slots (see the row-end warps)
+// rows whose set-aside lists the aux warps may be filling at once: an aux
+// warp at stage q has every aux warp past stage q - kStages (the stage's full
+// arrive needs the slot handed back by all of them), so they are at most
+// kStages rows apart
+constexpr int kRowSlots = 8;
+static_assert(kRowSlots > kStages, "row slots cover the aux warps' spread");
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kDrainLimitNs = 100000000ull;
 constexpr unsigned kSleepNs = 128;  // poll interval of the sleeping waits
 
 static_assert(kStageVecs % kConsumerThreads == 0, "stage vectors per consumer thread");
 static_assert(kConsumerWarps % 4 == 0, "stage maxima are read four at a time");
+static_assert(kConsumerWarps <= 32, "queue counts are read one per lane");
 
+// Everything per ring slot belongs to the stage in that slot: the producer
+// writes the slot's row data before the stage's full arrive, the consumers
+// write their queues, reference, threshold and (last stage of a row) their
+// sums before the stage's fready arrive, and nobody writes them again before the
+// aux warps' empty arrives hand the slot back.
 struct ScanSmem {
   uint64_t full[kStages];       // stage filled (producer arrive + copy bytes)
-  uint64_t empty[kStages];      // stage read by every consumer warp
+  uint64_t fready[kStages];     // every consumer warp finished pass 2 of the stage
+  uint64_t empty[kStages];      // the aux warp is done with the stage
   uint64_t maxbar[kMaxSlots];   // every consumer warp posted its stage maximum
-  uint64_t rowbar[kParkSlots];  // every consumer warp finished the row
-  uint64_t parkfree[kParkSlots];// the row-end warp is done with the row's parked list
-  uint64_t xbar[kXSlots];       // slice maxima of a row arrived from every CTA of the cluster
-  int32_t stage_row[kStages];   // row of the stage in the slot (written before its full arrive)
+  int32_t stage_row[kStages];   // row of the stage
   float stage_off[kStages];     // the row's candidate window
   float stage_known[kStages];   // rescan: the row maximum found by the first pass
-  int32_t park_row[kParkSlots]; // row handed to the row-end warp
-  float park_off[kParkSlots];
-  double wsum[kParkSlots][kConsumerWarps];
+  float stage_ref[kStages];     // the consumers' reference for the stage
+  uint32_t stage_thr[kStages];  // the stage's threshold (Threshold::pair)
+  float stage_thrv[kStages];    // (Threshold::value)
+  double wsum[kStages][kConsumerWarps];  // last stage of a row: each warp's sum
   __align__(16) float wmax[kMaxSlots][kConsumerWarps];
-  float sref[kParkSlots];
-  float xmax[kXSlots][kMaxSlices];
-  int park_count[kParkSlots];
+  // each consumer warp's flagged vectors of the stage (index within the
+  // stage, in the warp's ballot order) and their count
+  uint16_t queue[kStages][kConsumerWarps][32 * kVecsPerThread];
+  int qcnt[kStages][kConsumerWarps];
+  // per row slot (local row t -> t % kRowSlots): every aux warp is done with
+  // the row; the length of its set-aside list; each aux warp's sum
+  uint64_t rowdone[kRowSlots];
+  int list_n[kRowSlots];
+  double asum[kRowSlots][kAuxWarps];
   int abort;
 };
 
-constexpr size_t kScanDynSmem = (size_t)kStages * kStageBytes +
-                                (size_t)kParkSlots * kParkCap * (sizeof(uint4) + sizeof(uint32_t));
+constexpr size_t kScanDynSmem = (size_t)kStages * kStageBytes;
 
 // ---- element-type helpers ----------------------------------------------------
 
 // Candidate threshold in the element type: bf16 thresholds are rounded down,
-// so rounding can only add candidates; parking and filtering use the same
-// test (x > value).  `pair` holds the threshold in both bf16 halves.
+// so rounding can only add candidates; the vector flags, the set-aside
+// lists and the finish use the same test (x > value).  `pair` holds the
+// threshold in both bf16 halves.
 struct Threshold {
   uint32_t pair;
   float value;
@@ -118,13 +142,6 @@ __device__ __forceinline__ Threshold make_threshold(float thr) {
     t.pair = __float_as_uint(thr);
     t.value = thr;
   }
-  return t;
-}
-
-__device__ __forceinline__ Threshold no_threshold() {  // nothing is above it
-  Threshold t;
-  t.pair = 0x7F807F80u;  // bf16x2 (+inf, +inf)
-  t.value = INFINITY;
   return t;
 }
 
@@ -181,25 +198,6 @@ __device__ __forceinline__ bool max_above(uint32_t m, const Threshold &t) {
     return __uint_as_float(m) > t.value;
 }
 
-// Bit q set iff element q of the vector is above the threshold.
-template <typename Bits>
-__device__ __forceinline__ uint32_t above_mask(const uint4 &w, const Threshold &t) {
-  if constexpr (sizeof(Bits) == 2) {
-    const __nv_bfloat162 t2 = *reinterpret_cast<const __nv_bfloat162 *>(&t.pair);
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-    uint32_t mask = 0u;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint32_t m = __hgt2_mask(*reinterpret_cast<const __nv_bfloat162 *>(&ws[q]), t2);
-      mask |= ((m & 1u) | ((m >> 15) & 2u)) << (2 * q);
-    }
-    return mask;
-  } else {
-    return (__uint_as_float(w.x) > t.value ? 1u : 0u) | (__uint_as_float(w.y) > t.value ? 2u : 0u) |
-           (__uint_as_float(w.z) > t.value ? 4u : 0u) | (__uint_as_float(w.w) > t.value ? 8u : 0u);
-  }
-}
-
 // Adds exp2(x * coef + shift) of every element of the vector to the packed
 // accumulators (a fixed assignment of elements to accumulator lanes: word q
 // of a bf16 vector to acc[q], f32 element pairs to acc[0] and acc[1]).
@@ -220,6 +218,37 @@ __device__ __forceinline__ void add_exps(const uint4 &w, float2 c2, float2 s2, f
     acc[0] = __fadd2_rn(acc[0], make_float2(fast_exp2(u0.x), fast_exp2(u0.y)));
     acc[1] = __fadd2_rn(acc[1], make_float2(fast_exp2(u1.x), fast_exp2(u1.y)));
   }
+}
+
+// add_exps for a vector holding an element above the threshold: those
+// elements are left out of the sum (replaced by -inf) and returned as a bit
+// mask (bit e = element e).
+template <typename Bits>
+__device__ __forceinline__ uint32_t add_exps_masked(uint4 w, const Threshold &t, float2 c2,
+                                                    float2 s2, float2 (&acc)[4]) {
+  uint32_t em = 0u;
+  if constexpr (sizeof(Bits) == 2) {
+    const __nv_bfloat162 t2 = *reinterpret_cast<const __nv_bfloat162 *>(&t.pair);
+    uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t m = __hgt2_mask(*reinterpret_cast<const __nv_bfloat162 *>(&ws[q]), t2);
+      ws[q] = (ws[q] & ~m) | (0xFF80FF80u & m);
+      em |= ((m & 1u) | ((m >> 15) & 2u)) << (2 * q);
+    }
+    w = make_uint4(ws[0], ws[1], ws[2], ws[3]);
+  } else {
+    uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (__uint_as_float(ws[q]) > t.value) {
+        em |= 1u << q;
+        ws[q] = 0xFF800000u;
+      }
+    w = make_uint4(ws[0], ws[1], ws[2], ws[3]);
+  }
+  add_exps<Bits>(w, c2, s2, acc);
+  return em;
 }
 
 // Largest value over the warp (NaN ignored), by one reduction over an
@@ -252,7 +281,7 @@ __device__ __forceinline__ int64_t scan_row(const FastArgs &a, int64_t item, flo
 
 // What the producer tells the consumers about a stage.
 struct StageMeta {
-  int32_t r;    // row
+  int slot;     // ring slot
   float off;    // candidate window of the row (logit units)
   float known;  // rescan: the row maximum found by the first pass, else -inf
 };
@@ -287,20 +316,26 @@ struct StageCursor {
   }
 };
 
+// How a role waits between tests of an mbarrier phase.
+enum class Wait {
+  kSpin,     // consumers: test again at once
+  kSleep,    // producer: sleep kSleepNs between tests, leaving issue slots to the consumers
+  kSuspend,  // aux: the hardware may suspend the warp until the phase completes
+};
+
 // Bounded wait for an mbarrier phase.  False when it gave up (the abort flag
-// is then set) or when another role already gave up.  Roles off the
-// consumers' path (producer, row end) wait with kSleep: between tests they
-// sleep, so that their polling does not take issue slots from the consumer
-// warps that share their scheduler.
-template <bool kClusterScope, bool kSleep = false>
+// is then set) or when another role already gave up.
+template <Wait kMode>
 __device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, int *abort,
                                            uint64_t limit_ns = kWaitLimitNs) {
-  if (kClusterScope ? mbar_test_cluster(bar, parity) : mbar_test(bar, parity)) return true;
+  if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (kSleep) __nanosleep(kSleepNs);
-    if (kClusterScope ? mbar_test_cluster(bar, parity) : mbar_test(bar, parity)) return true;
-    if (kSleep || (it & 15u) == 0u) {
+    if (kMode == Wait::kSleep) __nanosleep(kSleepNs);
+    const bool done =
+        kMode == Wait::kSuspend ? mbar_try_wait(bar, parity, 1000u) : mbar_test(bar, parity);
+    if (done) return true;
+    if (kMode != Wait::kSpin || (it & 15u) == 0u) {
       if (*(volatile int *)abort) return false;
       if (global_timer_ns() - t0 > limit_ns) {
         *(volatile int *)abort = 1;
@@ -319,20 +354,18 @@ __global__ void __launch_bounds__(kScanThreads, 1) row_scan_kernel(const __grid_
   constexpr int U = kVecsPerThread;
   extern __shared__ __align__(128) unsigned char scan_dsm[];
   __shared__ ScanSmem sm;
-  // set-aside vectors of a row: copies and their indices in the row
-  uint4 *park_vec = reinterpret_cast<uint4 *>(scan_dsm + (size_t)kStages * kStageBytes);
-  uint32_t *park_idx = reinterpret_cast<uint32_t *>(park_vec + (size_t)kParkSlots * kParkCap);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const ScanGeom &g = a.g;
-  const int c = C > 1 ? (int)(blockIdx.x % C) : 0;  // == %cluster_ctarank for 1-D clusters
+  const int c = C > 1 ? (int)(blockIdx.x % C) : 0;  // the slice this CTA scans
   const int64_t cl = blockIdx.x / C, n_cl = gridDim.x / C;
   const int64_t R = a.rlist ? (int64_t)*a.rcount : a.rows;
   const int64_t my_rows = R > cl ? (R - 1 - cl) / n_cl + 1 : 0;
-  if (my_rows == 0) return;  // the same for every CTA of the cluster
+  if (my_rows == 0) return;
   const int K = g.stages;
   const int64_t Q = my_rows * K;  // stages this CTA scans
   const float coef = a.coef;
+  const uint32_t stage0 = smem_addr(scan_dsm);
   SliceSpan span;
   span.vb = (int32_t)(((int64_t)c * g.nvec) / C);
   span.ve = (int32_t)(((int64_t)(c + 1) * g.nvec) / C);
@@ -341,22 +374,18 @@ __global__ void __launch_bounds__(kScanThreads, 1) row_scan_kernel(const __grid_
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&sm.full[i], 1);
-      mbar_init(&sm.empty[i], kConsumerWarps);
+      mbar_init(&sm.fready[i], kConsumerWarps);
+      mbar_init(&sm.empty[i], kAuxWarps);
     }
     for (int i = 0; i < kMaxSlots; ++i) mbar_init(&sm.maxbar[i], kConsumerWarps);
-    for (int i = 0; i < kParkSlots; ++i) {
-      mbar_init(&sm.rowbar[i], kConsumerWarps);
-      mbar_init(&sm.parkfree[i], 1);
-      sm.park_count[i] = 0;
+    for (int i = 0; i < kRowSlots; ++i) {
+      mbar_init(&sm.rowdone[i], kAuxWarps);
+      sm.list_n[i] = 0;
     }
-    for (int i = 0; i < kXSlots; ++i) mbar_init(&sm.xbar[i], C);
     sm.abort = 0;
     fence_mbar_init();
   }
-  if constexpr (C > 1)
-    cluster_sync();  // every CTA's barriers exist before any remote arrive
-  else
-    __syncthreads();
+  __syncthreads();
 
   if (warp == kProducerWarp) {
     // ---- producer: one lane issues the bulk copies
@@ -367,9 +396,9 @@ __global__ void __launch_bounds__(kScanThreads, 1) row_scan_kernel(const __grid_
       int64_t r = 0;
       float off = 0.f, known = -INFINITY;
       for (int64_t q = 0; q < Q; ++q, cur.advance(K, kStages)) {
-        // the slot's previous stage (q - kStages) has been read by every consumer
+        // the aux warp is done with the slot's previous stage (q - kStages)
         if (q >= kStages &&
-            !wait_phase<false, true>(&sm.empty[cur.slot], cur.phase ^ 1u, &sm.abort))
+            !wait_phase<Wait::kSleep>(&sm.empty[cur.slot], cur.phase ^ 1u, &sm.abort))
           break;
         if (cur.k == 0) {
           r = scan_row(a, cl + cur.t * n_cl, off);
@@ -394,129 +423,138 @@ __global__ void __launch_bounds__(kScanThreads, 1) row_scan_kernel(const __grid_
       // normal path the consumers have already waited for every one)
       for (int64_t q = issued > kStages ? issued - kStages : 0; q < issued; ++q) {
         int never = 0;
-        wait_phase<false>(&sm.full[q % kStages], (uint32_t)((q / kStages) & 1), &never,
-                          kDrainLimitNs);
+        wait_phase<Wait::kSpin>(&sm.full[q % kStages], (uint32_t)((q / kStages) & 1), &never,
+                                kDrainLimitNs);
       }
     }
     __syncwarp();
-  } else if (warp >= kRowEndWarp0) {
-    // ---- row end: tail, cluster exchange, final split, slice record.  Row-end
-    // warp e takes rows e, e + 2, ... (parking slot e).  Its exchange slots are
-    // e and e + 2 (t % 4): a CTA sends row t + 4's maximum only after it
-    // received every peer's maximum of row t + 2, which each peer sent after
-    // it had read its slot for row t.
-    const int e_warp = warp - kRowEndWarp0;
-    for (int64_t t = e_warp; t < my_rows; t += kRowEndWarps) {
-      const int s = (int)(t % kParkSlots);
-      bool ok =
-          wait_phase<false, true>(&sm.rowbar[s], (uint32_t)((t / kParkSlots) & 1), &sm.abort);
+  } else if (warp >= kAuxWarp0) {
+    // ---- aux: each warp takes the flagged vectors of its class of every
+    // stage, then hands the buffer back; aux warp 0 closes each row (tail
+    // elements, slice record) once every aux warp is done with it
+    const int aw = warp - kAuxWarp0;
+    StageCursor ac;
+    float aref = -INFINITY;  // the reference of this warp's sums
+    float2 acc[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
+    int64_t r = 0;
+    uint64_t *list = nullptr;
+    for (int64_t q = 0; q < Q; ++q, ac.advance(K, kStages)) {
+      bool ok = wait_phase<Wait::kSuspend>(&sm.fready[ac.slot], ac.phase, &sm.abort);
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
-      const int64_t r = sm.park_row[s];
-      const float off = sm.park_off[s];
-      const float ref = sm.sref[s];  // maximum over the slice's whole vectors
-      double zc = 0.0;  // the consumers' sums, relative to ref
+      const int slot = ac.slot, k = ac.k;
+      const int rs = (int)(ac.t % kRowSlots);
+      const float sref = sm.stage_ref[slot];
+      if (k == 0) {
+        r = sm.stage_row[slot];
+        list = a.cand + r * (int64_t)kCandCap + (int64_t)c * g.cap;
+        aref = sref;
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) zc += sm.wsum[s][w];
-      const int n_park = sm.park_count[s];
-      const int n = min(n_park, kParkCap);
-      const uint4 *pv = park_vec + (size_t)s * kParkCap;
-      const uint32_t *pi = park_idx + (size_t)s * kParkCap;
-      const Bits *row = scan_row_ptr<Bits>(a, r);
-      // the V % VEC elements after the last whole vector (last slice; plain loads)
-      const bool has_tail = c == C - 1 && lane < g.tail;
-      const uint32_t tbits =
-          has_tail ? (uint32_t)row[(int64_t)g.nvec * VEC + lane] : (uint32_t)Elem<Bits>::kNegInf;
-      const float tx = Elem<Bits>::to_float(tbits);
-      const float mc = fmaxf(ref, warp_max(tx));  // the slice maximum
-      float M = mc;
-      if constexpr (C > 1) {  // the row maximum, from every CTA of the cluster
-        const int s2 = (int)(t % kXSlots);
-        if (lane == 0) {
+        for (int u = 0; u < 4; ++u) acc[u] = make_float2(0.f, 0.f);
+      } else if (sref > aref) {
+        const float f = (aref == -INFINITY) ? 0.f : fast_exp2((aref - sref) * coef);
 #pragma unroll
-          for (int p = 0; p < C; ++p) {
-            dsmem_st_f32(dsmem_map(&sm.xmax[s2][c], (uint32_t)p), mc);
-            mbar_arrive_remote(dsmem_map(&sm.xbar[s2], (uint32_t)p));
+        for (int u = 0; u < 4; ++u) acc[u] = make_float2(acc[u].x * f, acc[u].y * f);
+        aref = sref;
+      }
+      if (a.use_top_p) {
+        Threshold th;
+        th.pair = sm.stage_thr[slot];
+        th.value = sm.stage_thrv[slot];
+        // the consumer warps' queues, one after the other: entry i of the
+        // stage goes to aux warp (i / 32) % kAuxWarps
+        int end[kConsumerWarps];  // running ends of the queues
+        int n = 0;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          n += sm.qcnt[slot][w];
+          end[w] = n;
+        }
+        const float shift = (aref == -INFINITY) ? 0.f : -aref * coef;
+        const float2 c2 = make_float2(coef, coef), s2 = make_float2(shift, shift);
+        const uint32_t base = stage0 + (uint32_t)slot * kStageBytes;
+        const uint32_t v0 = (uint32_t)span.v0(k);
+        for (int i = aw * 32 + lane; i - lane < n; i += kAuxWarps * 32) {
+          if (i < n) {
+            int w = 0, start = 0;
+#pragma unroll
+            for (int x = 0; x < kConsumerWarps - 1; ++x)
+              if (i >= end[x]) {
+                w = x + 1;
+                start = end[x];
+              }
+            const uint32_t j = sm.queue[slot][w][i - start];
+            const uint4 v = lds128(base + j * 16u);
+            const uint32_t em = add_exps_masked<Bits>(v, th, c2, s2, acc);
+            const int pos = atomicAdd(&sm.list_n[rs], __popc(em));
+            const uint32_t idx0 = (v0 + j) * VEC;
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) {
+              const int p = pos + __popc(em & ((1u << e) - 1u));
+              if (((em >> e) & 1u) && p < g.cap)
+                list[p] = ((uint64_t)vec_elem<Bits>(v, e) << 32) | (idx0 + (uint32_t)e);
+            }
           }
         }
-        ok = wait_phase<true, true>(&sm.xbar[s2], (uint32_t)((t / kXSlots) & 1), &sm.abort);
-        if (!__all_sync(0xFFFFFFFFu, ok)) break;
-#pragma unroll
-        for (int p = 0; p < C; ++p) M = fmaxf(M, sm.xmax[s2][p]);
       }
-      const Threshold thf = a.use_top_p ? make_threshold<Bits>(M - off) : no_threshold();
-      // the set-aside vectors (copies in shared memory) and the tail: elements
-      // above the final threshold are the slice's candidates, the others join
-      // the sum, in 2^48 fixed point relative to mc (order-free)
-      const float shc = (mc == -INFINITY) ? 0.f : -mc * coef;
-      uint64_t *dst = a.cand + r * (int64_t)kCandCap + (int64_t)c * g.cap;
-      unsigned long long tfx = 0ull;
-      int pos = 0;
-      for (int base = 0; base < n; base += 32) {
-        const int j = base + lane;
-        const uint32_t vi = j < n ? pi[j] : 0u;
-        uint4 w;
-        w.x = w.y = w.z = w.w = neg_inf_max<Bits>();
-        if (j < n) w = pv[j];
-        const uint32_t cm = above_mask<Bits>(w, thf);
+      if (k == K - 1) {  // the row's last stage
+        double zl = 0.0;
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-          const float ex = fast_exp2(fmaf(Elem<Bits>::to_float(vec_elem<Bits>(w, e)), coef, shc));
-          if (!((cm >> e) & 1u) && ex > 0.f) tfx += __float2ull_rn(ex * 281474976710656.0f);
+        for (int u = 0; u < 4; ++u) zl += (double)acc[u].x + (double)acc[u].y;
+        const double za = warp_sum_d(zl);  // relative to sref, as the consumers' sums
+        if (lane == 0) {
+          sm.asum[rs][aw] = za;
+          __threadfence_block();
+          mbar_arrive(&sm.rowdone[rs]);
         }
-        int cnt = __popc(cm), incl = cnt;
+        if (aw == 0) {  // every aux warp's list entries and sum, then the record
+          ok = wait_phase<Wait::kSuspend>(&sm.rowdone[rs], (uint32_t)((ac.t / kRowSlots) & 1),
+                                          &sm.abort);
+          if (!__all_sync(0xFFFFFFFFu, ok)) break;
+          double zc = 0.0;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-          if (lane >= o) incl += v;
+          for (int w = 0; w < kAuxWarps; ++w) zc += sm.asum[rs][w];
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) zc += sm.wsum[slot][w];
+          int n_list = sm.list_n[rs];
+          // the V % VEC elements after the last whole vector (last slice;
+          // plain loads) are all set aside: the finish sorts them with the
+          // others
+          const bool has_tail = c == C - 1 && lane < g.tail;
+          const Bits *row = scan_row_ptr<Bits>(a, r);
+          const uint32_t tbits = has_tail ? (uint32_t)row[(int64_t)g.nvec * VEC + lane]
+                                          : (uint32_t)Elem<Bits>::kNegInf;
+          const float mc = fmaxf(sref, warp_max(Elem<Bits>::to_float(tbits)));  // slice maximum
+          if (has_tail && n_list + lane < g.cap)
+            list[n_list + lane] = ((uint64_t)tbits << 32) | (uint32_t)(g.nvec * VEC + lane);
+          if (c == C - 1) n_list += g.tail;
+          __syncwarp();
+          if (lane == 0) {
+            SliceRecord rec;
+            rec.m = mc;
+            rec.n_cand = n_list;
+            rec.flags = n_list > g.cap ? kRowLost : 0;
+            rec.off = sm.stage_off[slot];
+            rec.z = (sref == -INFINITY || !(mc > sref))
+                        ? zc
+                        : zc * exp2(((double)sref - (double)mc) * a.coef64);
+            a.srec[r * kMaxSlices + c] = rec;
+            sm.list_n[rs] = 0;  // reused kRowSlots rows later
+          }
         }
-        int d = pos + incl - cnt;
-        uint32_t m = cm;
-        while (m) {
-          const int e = __ffs(m) - 1;
-          m &= m - 1;
-          if (d < g.cap) dst[d] = ((uint64_t)vec_elem<Bits>(w, e) << 32) | (vi * VEC + (uint32_t)e);
-          ++d;
-        }
-        pos += __shfl_sync(0xFFFFFFFFu, incl, 31);
-      }
-      {
-        const bool cand = has_tail && tx > thf.value;
-        const unsigned bal = __ballot_sync(0xFFFFFFFFu, cand);
-        const int d = pos + __popc(bal & ((1u << lane) - 1u));
-        if (cand && d < g.cap) dst[d] = ((uint64_t)tbits << 32) | (uint32_t)(g.nvec * VEC + lane);
-        pos += __popc(bal);
-      }
-      // every element that is not a candidate, relative to mc: the consumers'
-      // sums (rescaled if the tail holds the maximum), the tail, the rest
-      double z = (ref == -INFINITY || !(mc > ref)) ? zc : zc * exp2(((double)ref - (double)mc) * a.coef64);
-      const double et = (has_tail && !(tx > thf.value) && mc > -INFINITY)
-                            ? exp2(((double)tx - (double)mc) * a.coef64)
-                            : 0.0;
-      z += warp_sum_d(et);
-      z += (double)warp_sum_u64(tfx) * (1.0 / 281474976710656.0);
-      if (lane == 0) {
-        SliceRecord rec;
-        rec.m = mc;
-        rec.n_cand = pos;
-        rec.flags = n_park > kParkCap ? kRowLost : 0;
-        rec.n_parked = n_park;
-        rec.z = (ref == -INFINITY && mc == -INFINITY) ? 0.0 : z;
-        a.srec[r * kMaxSlices + c] = rec;
-        sm.park_count[s] = 0;
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.parkfree[s]);
+      if (lane == 0) mbar_arrive(&sm.empty[slot]);
     }
   } else {
     // ---- consumers
     const int cw = warp, ct = tid;
-    const uint32_t stage0 = smem_addr(scan_dsm);
     uint4 neg;
     neg.x = neg.y = neg.z = neg.w = neg_inf_max<Bits>();
     bool dead = false;
     // per-row state (the same in every consumer thread except the sums)
     float ref = -INFINITY, off = 0.f;
-    int64_t r = 0;
     float2 acc[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
@@ -527,53 +565,47 @@ __global__ void __launch_bounds__(kScanThreads, 1) row_scan_kernel(const __grid_
     int lms = 0;
 
     // a stage: registers <- shared memory, then the warp's maximum to the
-    // stage's maximum slot, then the buffer back to the producer.  A maximum
-    // slot is reused 2 * kStages stages later; by then every consumer warp
-    // has read the old one (the producer refilled the stage buffer in
-    // between only after every warp released it, i.e. finished pass 2 of the
-    // stage before).
+    // stage's maximum slot.  A maximum slot is reused 2 * kStages stages
+    // later; by then every consumer warp has read the old one (the stage
+    // kStages later can only be loaded once the aux warp has handed its
+    // buffer back, which it does after every warp's pass 2 of that stage).
     auto load_stage = [&](uint4(&Rv)[U], uint32_t(&Tm)[U], StageMeta &Mt) {
-      bool ok = wait_phase<false>(&sm.full[lc.slot], lc.phase, &sm.abort);
+      bool ok = wait_phase<Wait::kSpin>(&sm.full[lc.slot], lc.phase, &sm.abort);
       if (!__all_sync(0xFFFFFFFFu, ok)) {
         dead = true;
         return;
       }
       const int32_t nv = span.nv(lc.k);
       const uint32_t base = stage0 + (uint32_t)lc.slot * kStageBytes;
-      Mt.r = sm.stage_row[lc.slot];
+      Mt.slot = lc.slot;
       Mt.off = sm.stage_off[lc.slot];
       Mt.known = sm.stage_known[lc.slot];
-      uint32_t run = neg_inf_max<Bits>();
-      if (nv == kStageVecs) {
-#pragma unroll
-        for (int u = 0; u < U; ++u) Rv[u] = lds128(base + (uint32_t)(ct + u * kConsumerThreads) * 16u);
-      } else {
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int j = ct + u * kConsumerThreads;
-          Rv[u] = j < nv ? lds128(base + (uint32_t)j * 16u) : neg;
-        }
-      }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        Tm[u] = vec_max<Bits>(Rv[u]);
-        run = max_fold<Bits>(run, Tm[u]);
+        const int j = ct + u * kConsumerThreads;
+        Rv[u] = (nv == kStageVecs || j < nv) ? lds128(base + (uint32_t)j * 16u) : neg;
       }
-      const float wm = warp_max_redux(max_to_float<Bits>(run));
+#pragma unroll
+      for (int u = 0; u < U; ++u) Tm[u] = vec_max<Bits>(Rv[u]);
+      uint32_t run[U];  // the stage maximum, folded as a tree
+#pragma unroll
+      for (int u = 0; u < U; ++u) run[u] = Tm[u];
+#pragma unroll
+      for (int h = 1; h < U; h <<= 1)
+#pragma unroll
+        for (int u = 0; u + h < U; u += 2 * h) run[u] = max_fold<Bits>(run[u], run[u + h]);
+      const float wm = warp_max_redux(max_to_float<Bits>(run[0]));
       if (lane == 0) sm.wmax[lms][cw] = wm;
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&sm.maxbar[lms]);
-        mbar_arrive(&sm.empty[lc.slot]);
-      }
+      if (lane == 0) mbar_arrive(&sm.maxbar[lms]);
       lc.advance(K, kStages);
       if (++lms == kMaxSlots) lms = 0;
     };
 
-    // a stage from registers: reference, exponentials, parked elements
+    // a stage from registers: reference, exponentials, flags
     auto pass2 = [&](const uint4(&Rv)[U], const uint32_t(&Tm)[U], const StageMeta &Mt) {
       const int ms = pc.slot;
-      bool ok = wait_phase<false>(&sm.maxbar[ms], pc.phase, &sm.abort);
+      bool ok = wait_phase<Wait::kSpin>(&sm.maxbar[ms], pc.phase, &sm.abort);
       if (!__all_sync(0xFFFFFFFFu, ok)) {
         dead = true;
         return;
@@ -584,23 +616,13 @@ __global__ void __launch_bounds__(kScanThreads, 1) row_scan_kernel(const __grid_
         const float4 m4 = *reinterpret_cast<const float4 *>(&sm.wmax[ms][w]);
         smax = fmaxf(fmaxf(smax, fmaxf(m4.x, m4.y)), fmaxf(m4.z, m4.w));
       }
-      const int64_t t = pc.t;
       const int k = pc.k;
       pc.advance(K, kMaxSlots);
-      const int s = (int)(t % kParkSlots);
       if (k == 0) {  // first stage of a row
-        r = Mt.r;
         off = Mt.off;
         ref = fmaxf(smax, Mt.known);
 #pragma unroll
         for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
-        if (t >= kParkSlots) {  // the row-end warp is done with this parking slot
-          ok = wait_phase<false>(&sm.parkfree[s], (uint32_t)((t / kParkSlots - 1) & 1), &sm.abort);
-          if (!__all_sync(0xFFFFFFFFu, ok)) {
-            dead = true;
-            return;
-          }
-        }
       } else if (smax > ref) {
         const float f = (ref == -INFINITY) ? 0.f : fast_exp2((ref - smax) * coef);
 #pragma unroll
@@ -609,59 +631,66 @@ __global__ void __launch_bounds__(kScanThreads, 1) row_scan_kernel(const __grid_
       }
       const float shift = (ref == -INFINITY) ? 0.f : -ref * coef;
       const float2 c2 = make_float2(coef, coef), s2 = make_float2(shift, shift);
-      const float2 s_off = make_float2(-INFINITY, -INFINITY);
-      const Threshold th = a.use_top_p ? make_threshold<Bits>(ref - off) : no_threshold();
-      // a vector holding an element above the running threshold is left out
-      // of the fp32 sum (its shift makes every exponential 0; NaN and +inf
-      // still reach the sum) and handed to the row-end warp whole
-      uint32_t flags = 0u;
-#pragma unroll
-      for (int u = 0; u < U; ++u) flags |= (max_above<Bits>(Tm[u], th) ? 1u : 0u) << u;
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-        add_exps<Bits>(Rv[u], c2, ((flags >> u) & 1u) ? s_off : s2, acc);
-      if (__any_sync(0xFFFFFFFFu, flags != 0u)) {  // one shared atomic per warp
-        uint32_t bal[U];
-        int total = 0;
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          bal[u] = __ballot_sync(0xFFFFFFFFu, (flags >> u) & 1u);
-          total += __popc(bal[u]);
-        }
-        int base = 0;
-        if (lane == 0) base = atomicAdd(&sm.park_count[s], total);
-        int pos = __shfl_sync(0xFFFFFFFFu, base, 0);
-        uint4 *pv = park_vec + (size_t)s * kParkCap;
-        uint32_t *pi = park_idx + (size_t)s * kParkCap;
-        const int32_t v0 = span.v0(k);
-        const unsigned below = (1u << lane) - 1u;
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int d = pos + __popc(bal[u] & below);
-          if (((flags >> u) & 1u) && d < kParkCap) {
-            pv[d] = Rv[u];
-            pi[d] = (uint32_t)(v0 + ct + u * kConsumerThreads);
+      if (a.use_top_p) {
+        // the set-aside threshold looks one stage ahead within the row (every
+        // warp posted the next stage's maximum when it loaded that stage,
+        // which it did before this pass): a higher threshold flags fewer
+        // vectors
+        float thr_ref = ref;
+        if (k + 1 < K) {
+          ok = wait_phase<Wait::kSpin>(&sm.maxbar[pc.slot], pc.phase, &sm.abort);
+          if (!__all_sync(0xFFFFFFFFu, ok)) {
+            dead = true;
+            return;
           }
-          pos += __popc(bal[u]);
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; w += 4) {
+            const float4 m4 = *reinterpret_cast<const float4 *>(&sm.wmax[pc.slot][w]);
+            thr_ref = fmaxf(fmaxf(thr_ref, fmaxf(m4.x, m4.y)), fmaxf(m4.z, m4.w));
+          }
         }
+        const Threshold th = make_threshold<Bits>(thr_ref - off);
+        // a vector with an element above the threshold stays out of this sum
+        // whole; the warp queues it for the aux warps (one ballot per u)
+        uint32_t fl = 0u;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const bool f = max_above<Bits>(Tm[u], th);
+          fl |= (f ? 1u : 0u) << u;
+          add_exps<Bits>(f ? neg : Rv[u], c2, s2, acc);
+        }
+        int nq = 0;
+        if (__any_sync(0xFFFFFFFFu, fl != 0u)) {
+          uint16_t *qw = sm.queue[Mt.slot][cw];
+          const unsigned below = (1u << lane) - 1u;
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const bool f = (fl >> u) & 1u;
+            const unsigned bal = __ballot_sync(0xFFFFFFFFu, f);
+            if (f) qw[nq + __popc(bal & below)] = (uint16_t)(ct + u * kConsumerThreads);
+            nq += __popc(bal);
+          }
+        }
+        if (lane == 0) sm.qcnt[Mt.slot][cw] = nq;
+        if (ct == 0) {
+          sm.stage_thr[Mt.slot] = th.pair;
+          sm.stage_thrv[Mt.slot] = th.value;
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < U; ++u) add_exps<Bits>(Rv[u], c2, s2, acc);
       }
-      if (k == K - 1) {  // end of the row: this warp's sum, then hand the row over
+      if (ct == 0) sm.stage_ref[Mt.slot] = ref;
+      if (k == K - 1) {  // end of the row: this warp's sum
         double zl = 0.0;
 #pragma unroll
         for (int q = 0; q < 4; ++q) zl += (double)acc[q].x + (double)acc[q].y;
         const double zs = warp_sum_d(zl);
-        if (lane == 0) {
-          sm.wsum[s][cw] = zs;
-          if (cw == 0) {
-            sm.sref[s] = ref;
-            sm.park_row[s] = (int32_t)r;
-            sm.park_off[s] = off;
-          }
-        }
-        __threadfence_block();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.rowbar[s]);
+        if (lane == 0) sm.wsum[Mt.slot][cw] = zs;
       }
+      __threadfence_block();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.fready[Mt.slot]);
     };
 
     uint4 R0[U], R1[U];
@@ -679,44 +708,20 @@ __global__ void __launch_bounds__(kScanThreads, 1) row_scan_kernel(const __grid_
     }
   }
 
-  if constexpr (C > 1) cluster_sync();  // peers write into this CTA's shared memory until here
   if (tid == 0 && *(volatile int *)&sm.abort && a.s.dev_status)
     atomicOr(a.s.dev_status, PSI_DEV_TIMEOUT);
 }
 
-// Clusters that fit on the device at once (queried once per device and
-// kernel; falls back to one per C SMs).
-template <typename Bits, int C>
-int max_clusters() {
+// SM count of the current device (queried once per device).
+int scan_sm_count() {
   static std::atomic<int> cached[PerDevice::kMax] = {};
   const int dev = PerDevice::current();
   const bool slot = dev >= 0 && dev < PerDevice::kMax;
   int n = slot ? cached[dev].load(std::memory_order_relaxed) : 0;
   if (n > 0) return n;
-  int sms = 0;
-  if (dev < 0 || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      sms <= 0)
-    sms = 148;
-  n = sms / C;
-  if (C > 1) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(n * C));
-    cfg.blockDim = dim3(kScanThreads);
-    cfg.dynamicSmemBytes = kScanDynSmem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int q = 0;
-    if (cudaOccupancyMaxActiveClusters(&q, row_scan_kernel<Bits, C>, &cfg) == cudaSuccess && q > 0)
-      n = std::min(n, q);
-    else
-      (void)cudaGetLastError();
-  }
-  if (n < 1) n = 1;
+  if (dev < 0 || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      n <= 0)
+    n = 148;
   if (slot) cached[dev].store(n, std::memory_order_relaxed);
   return n;
 }
@@ -725,27 +730,17 @@ template <typename Bits, int C>
 cudaError_t launch_scan_typed(const FastArgs &fa, cudaStream_t stream) {
   static DeviceOnce configure;
   cudaError_t e = configure([] {
-    return cudaFuncSetAttribute(row_scan_kernel<Bits, C>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScanDynSmem);
+    cudaError_t err = cudaFuncSetAttribute(row_scan_kernel<Bits, C>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)kScanDynSmem);
+    if (err == cudaSuccess) err = prefer_max_shared(row_scan_kernel<Bits, C>);
+    return err;
   });
   if (e != cudaSuccess) return e;
-  const int64_t clusters = std::min<int64_t>(max_clusters<Bits, C>(), std::max<int64_t>(fa.rows, 1));
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(clusters * C));
-  cfg.blockDim = dim3(kScanThreads);
-  cfg.dynamicSmemBytes = kScanDynSmem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  if (C > 1) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-  }
-  e = cudaLaunchKernelEx(&cfg, row_scan_kernel<Bits, C>, fa);
-  if (e != cudaSuccess) return e;
+  // one CTA per SM: groups of C CTAs, each group scanning its rows' C slices
+  const int64_t groups =
+      std::min<int64_t>(std::max(1, scan_sm_count() / C), std::max<int64_t>(fa.rows, 1));
+  row_scan_kernel<Bits, C><<<(unsigned)(groups * C), kScanThreads, kScanDynSmem, stream>>>(fa);
   return cudaGetLastError();
 }
 
@@ -765,7 +760,7 @@ ScanGeom plan_scan(int32_t V, int elem_bytes) {
   const int32_t vec = 16 / elem_bytes;
   g.nvec = V / vec;
   g.tail = V - g.nvec * vec;
-  // rows of at least four stages are split over a cluster of two CTAs
+  // rows of at least four stages are split in two slices (two CTAs)
   g.slices = (int64_t)g.nvec * 16 >= 4 * (int64_t)kStageBytes ? 2 : 1;
   const int32_t per = (g.nvec + g.slices - 1) / g.slices;
   g.stages = std::max<int32_t>(1, (per + kStageVecs - 1) / kStageVecs);
