@@ -515,17 +515,18 @@ def main():
     if rank == 0:
         # our kernels per call: argmax + tree walk; greedy linear: per
         # early-exit round list building and argmax, then emit; sampled: per
-        # round list building, row scan, unit finish and their second passes,
-        # then two cluster list launches and fast_emit
+        # round list building, row scan, row finish, unit decision and their
+        # second passes, then two cluster list launches, fast_emit and the
+        # nucleus draw
         rounds = 0 if is_tree else len(sampled_rounds(cfg))
         if is_tree or (cfg.temperature == 0 and cfg.N < 64):
             launches_per_step = 2
         elif cfg.temperature == 0:  # per round: list building and argmax; then emit
             launches_per_step = 2 * rounds + 1
-        elif cfg.N < 64:  # one pass: row scan, unit, their second passes, lists, emit
-            launches_per_step = 7
+        elif cfg.N < 64:  # one pass: scan, finish, unit, their second passes, lists, emit, draw
+            launches_per_step = 10
         else:
-            launches_per_step = 5 * rounds + 3
+            launches_per_step = 7 * rounds + 4
         line = {
             "metric": METRIC, "value": value, "unit": "blocks/s", "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,

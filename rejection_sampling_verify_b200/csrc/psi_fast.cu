@@ -11,29 +11,30 @@
 //   round_advance  (early-exit rounds only) One thread per sequence: lists
 //              the rows and units of the next round of positions for the
 //              sequences whose drafts were all accepted so far.
-//   row_scan   Persistent CTAs stream every listed logit row ONCE from HBM
-//              with 16-byte non-allocating loads (8 per thread in flight,
-//              double buffered in registers, plus an L2 bulk prefetch).  A row
-//              is read in batches of 2048 vectors; inside a batch every
-//              thread uses the same reference (a lower bound of the row
-//              maximum, raised between batches), so all sums are independent
-//              of timing.  Elements within the window below the reference
-//              ("candidates", ~0.3% of a row) are masked out of the fp32 sum
-//              of exponentials; the vectors that hold them are parked in
-//              shared memory and, at the row's end, split into candidates
-//              (to a per-row list in global memory) and elements that fell
-//              below the final threshold (a 2^31 fixed-point sum).
-//   unit       One CTA of two warps per (sequence, row) unit: finishes the
-//              unit's p and q rows from their candidates (row maximum, Z, the
-//              top-p threshold and renormaliser), decides the drafted token
-//              and draws the correction or bonus token over p's nucleus.
-//   row_scan / unit, second pass   Rows whose window held less than top_p of
-//              the mass (rescanned with a wider window) or whose candidates
-//              overflowed (rescanned with the exact maximum known).
+//   row_scan   (psi_scan.cu) Streams every listed logit row once from HBM:
+//              per slice of a row, its maximum, its fp32 sum of
+//              exponentials and its set-aside list (elements above the
+//              running top-p threshold).
+//   row_finish One warp per listed row: row maximum, Z, the top-p threshold
+//              and renormaliser from the slice records and lists, exact
+//              (double masses, 2^52 fixed-point sums); the row's candidates
+//              compacted at the front of its list area.
+//   unit       One thread per (sequence, position) unit: accepts or rejects
+//              the drafted token from the two finished rows (p(x), q(x) in
+//              double); a unit whose row failed is listed for the second pass.
+//   row_scan / row_finish / unit, second pass   Rows whose window held less
+//              than top_p of the mass (rescanned with a wider window) or
+//              whose lists overflowed (rescanned with the exact maximum
+//              known).
 //   (cluster kernel, list mode)  Units the second pass could not settle.
-//   fast_emit  First rejected row per sequence; emitted tokens.  Without
-//              top-p the emitting row's draw needs the whole row again: it is
-//              queued for the cluster kernel in sample mode.
+//   fast_emit  First rejected position per sequence; emitted tokens; lists
+//              the position whose token is still to be drawn.
+//   draw       One warp per listed position: the correction (residual
+//              max(0, p - q)) or bonus draw over p's nucleus, inverse CDF in
+//              vocabulary order on exact integer sums.  Only the emitted
+//              position of each sequence is drawn.  Without top-p the draw
+//              needs whole rows: those positions go to the cluster kernel in
+//              sample mode.
 #include <algorithm>
 
 #include "psi_finish.cuh"
@@ -45,7 +46,7 @@ namespace {
 using namespace finish;
 
 constexpr int kListClusters = 16;
-constexpr int kCounters = 8;  // work-list counters (see FastArgs::counters)
+constexpr int kCounters = 9;  // work-list counters (see FastArgs::counters)
 // Candidate window, in log2 units below the row maximum.  The first pass uses
 // a narrow window (13 units for top_p <= 0.95, wider as top_p approaches 1);
 // the second pass the wide one.
@@ -53,218 +54,269 @@ constexpr float kWindowBaseLog2 = 13.f;
 constexpr float kWindowWideLog2 = 20.f;
 
 // ---------------------------------------------------------------------------
-// unit: one CTA of two warps per (sequence, row) unit
+// row_finish: one warp per listed row
 // ---------------------------------------------------------------------------
-struct UnitShared {
-  WarpScratch ws[2];  // warp 0: the p row, warp 1: the q row
-  RowFinal fq;
-  int need;
-};
+constexpr int kFinishWarps = 1;
 
 template <typename Bits>
-__global__ void __launch_bounds__(64) unit_kernel(const __grid_constant__ FastArgs a) {
-  extern __shared__ __align__(16) unsigned char unit_smem[];  // one UnitShared (> 48 KB)
-  UnitShared &sh = *reinterpret_cast<UnitShared *>(unit_smem);
+__global__ void __launch_bounds__(32 * kFinishWarps) row_finish_kernel(const __grid_constant__ FastArgs a) {
+  __shared__ FinScratch fsm[kFinishWarps];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t R = a.rlist ? (int64_t)*a.rcount : a.rows;
+  for (int64_t item = (int64_t)blockIdx.x * kFinishWarps + warp; item < R;
+       item += (int64_t)gridDim.x * kFinishWarps) {
+    const int64_t r = a.rlist ? (int64_t)(a.rlist[item] & ~kWideBit) : item;
+    const RowFin f = finish_row_list<Bits>(a, r, &fsm[warp]);
+    if (lane == 0) a.rfin[r] = f;
+    __syncwarp();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// unit: one thread per (sequence, position) unit: accept or reject
+// ---------------------------------------------------------------------------
+constexpr int kUnitThreads = 128;
+constexpr int32_t kTokenDraw = -3;        // rec.token: the nucleus draw kernel decides it
+constexpr int32_t kTokenWholeRow = -2;    // rec.token: a whole-row draw (no top-p)
+
+__device__ __forceinline__ RowFin empty_fin() {
+  RowFin f;
+  f.m = -INFINITY;
+  f.zp = 0.0;
+  f.tau_bits = 0u;
+  f.tau_key = 0u;
+  f.n = 0;
+  f.status = 0;
+  f.pad = 0;
+  return f;
+}
+
+template <typename Bits>
+__global__ void __launch_bounds__(kUnitThreads) unit_kernel(const __grid_constant__ FastArgs a) {
   const SampledArgs &s = a.s;
   const int32_t B = s.B, N = s.N, V = s.V;
   const int64_t n_items = a.ulist ? (int64_t)*a.ucount : (int64_t)N * (B + 1);
-  for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+  for (int64_t item = (int64_t)blockIdx.x * kUnitThreads + threadIdx.x; item < n_items;
+       item += (int64_t)gridDim.x * kUnitThreads) {
     const int64_t unit = a.ulist ? (int64_t)a.ulist[item] : item;
     const int32_t n = (int32_t)(unit / (B + 1)), i = (int32_t)(unit % (B + 1));
     const bool has_q = i < B;
     const int64_t rp_idx = unit;
     const int64_t rq_idx = (int64_t)N * (B + 1) + (int64_t)n * B + i;
-    // the two rows in parallel
-    RowFinal fp;
-    if (warp == 0) {
-      fp = finish_row<Bits>(a, rp_idx, &sh.ws[0]);
-    } else if (has_q) {
-      const RowFinal f = finish_row<Bits>(a, rq_idx, &sh.ws[1]);
-      if (lane == 0) sh.fq = f;
-    } else if (lane == 0) {
-      sh.fq.m = -INFINITY;
-      sh.fq.zp = 0.0;
-      sh.fq.tau_bits = 0u;
-      sh.fq.tau_key = 0u;
-      sh.fq.n = 0;
-      sh.fq.status = 0;
+    const RowFin fp = a.rfin[rp_idx];
+    const RowFin fq = has_q ? a.rfin[rq_idx] : empty_fin();
+    const int fail_q = fq.status & (kFinOverflow | kFinCoverage);
+    const int fail_p = fp.status & (kFinOverflow | kFinCoverage);
+    if (fail_q || fail_p) {
+      if (a.pass == 1) {  // rescan the failed rows, then finish the unit again
+        // the rescan starts from the row maximum found here, so its
+        // threshold is final from the first stage
+        if (fail_q) {
+          a.known_max[rq_idx] = fq.m;
+          a.wide_rows[atomicAdd(&a.counters[2], 1)] =
+              (int32_t)rq_idx | ((fail_q & kFinCoverage) ? kWideBit : 0);
+        }
+        if (fail_p) {
+          a.known_max[rp_idx] = fp.m;
+          a.wide_rows[atomicAdd(&a.counters[2], 1)] =
+              (int32_t)rp_idx | ((fail_p & kFinCoverage) ? kWideBit : 0);
+        }
+        a.wide_units[atomicAdd(&a.counters[3], 1)] = (int32_t)unit;
+      } else {  // the general path verifies this unit (records included)
+        a.list_a[atomicAdd(&a.counters[0], 1)] = (int32_t)unit;
+        a.rec[unit].accept = -1;  // decided at the end; a later round treats it as accepted
+      }
+      continue;
     }
-    __syncthreads();
-    if (warp == 0) {
-      const RowFinal fq = sh.fq;
-      const int fail_q = fq.status & (kFinOverflow | kFinCoverage);
-      const int fail_p = fp.status & (kFinOverflow | kFinCoverage);
-      const uint64_t seq = s.seq_ids ? s.seq_ids[n] : (uint64_t)n;
+    // ---- accept / reject the drafted token (double precision)
+    const uint64_t seq = s.seq_ids ? s.seq_ids[n] : (uint64_t)n;
+    int need = 1;
+    if (has_q) {
       const Bits *row_p = static_cast<const Bits *>(s.ar) + unit * s.ar_stride;
-      const Bits *row_q =
-          has_q ? static_cast<const Bits *>(s.draft) + ((int64_t)n * B + i) * s.draft_stride : nullptr;
-      const float tau_p = Elem<Bits>::to_float(fp.tau_bits);
-      const float tau_q = Elem<Bits>::to_float(fq.tau_bits);
-      int need = 0;
-      if (fail_q || fail_p) {
-        if (lane == 0) {
-          if (a.pass == 1) {  // rescan the failed rows, then finish the unit again
-            // the rescan starts from the row maximum found here, so its
-            // threshold is final from the first stage
-            if (fail_q) {
-              a.known_max[rq_idx] = fq.m;
-              a.wide_rows[atomicAdd(&a.counters[2], 1)] =
-                  (int32_t)rq_idx | ((fail_q & kFinCoverage) ? kWideBit : 0);
-            }
-            if (fail_p) {
-              a.known_max[rp_idx] = fp.m;
-              a.wide_rows[atomicAdd(&a.counters[2], 1)] =
-                  (int32_t)rp_idx | ((fail_p & kFinCoverage) ? kWideBit : 0);
-            }
-            a.wide_units[atomicAdd(&a.counters[3], 1)] = (int32_t)unit;
-          } else {  // the general path verifies this unit (records included)
-            a.list_a[atomicAdd(&a.counters[0], 1)] = (int32_t)unit;
-            a.rec[unit].accept = -1;  // decided at the end; a later round treats it as accepted
+      const Bits *row_q = static_cast<const Bits *>(s.draft) + ((int64_t)n * B + i) * s.draft_stride;
+      const int32_t x = s.ids[(int64_t)n * B + i];
+      double p = 0.0, q = 0.0;
+      const bool valid = x >= 0 && x < V;
+      if (valid) {
+        const float xp = Elem<Bits>::to_float(row_p[x]);
+        const float xq = Elem<Bits>::to_float(row_q[x]);
+        if (xp >= Elem<Bits>::to_float(fp.tau_bits) && fp.zp > 0.0)
+          p = exact_exp2d(xp, fp.m, a.coef64) / fp.zp;
+        if (xq >= Elem<Bits>::to_float(fq.tau_bits) && fq.zp > 0.0)
+          q = exact_exp2d(xq, fq.m, a.coef64) / fq.zp;
+      }
+      const double u = (double)uniform24(s.seed, seq, s.step, (uint64_t)i, PSI_PURPOSE_ACCEPT);
+      const int accept = (u * q < p) ? 1 : 0;
+      need = !accept;
+      if (s.out_p) s.out_p[(int64_t)n * B + i] = (float)p;
+      if (s.out_q) s.out_q[(int64_t)n * B + i] = (float)q;
+      a.rec[unit].accept = accept;
+      if (accept) a.rec[unit].token = -1;
+      if (!valid && s.dev_status) atomicOr(s.dev_status, PSI_DEV_BAD_TOKEN_ID);
+    } else {
+      a.rec[unit].accept = 1;
+    }
+    if (((fp.status | fq.status) & kFinNonfinite) && s.dev_status)
+      atomicOr(s.dev_status, PSI_DEV_NONFINITE);
+    // the correction / bonus token: drawn after the emit step, and only for
+    // the position each sequence emits
+    if (need) a.rec[unit].token = a.use_top_p ? kTokenDraw : kTokenWholeRow;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// draw: one warp per listed unit (each sequence's emitted position)
+// ---------------------------------------------------------------------------
+struct DrawScratch {  // one warp's shared memory: p's nucleus and its draw weights
+  uint32_t idx[kFinishCap];
+  unsigned long long w[kFinishCap];
+};
+
+template <typename Bits>
+__global__ void __launch_bounds__(32) draw_kernel(const __grid_constant__ FastArgs a) {
+  __shared__ DrawScratch dsm;
+  DrawScratch *ds = &dsm;
+  const int lane = threadIdx.x & 31;
+  const SampledArgs &s = a.s;
+  const int32_t B = s.B, N = s.N, V = s.V;
+  const int64_t n_items = (int64_t)a.counters[8];
+  for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const int64_t unit = (int64_t)a.list_d[item];
+    const int32_t n = (int32_t)(unit / (B + 1)), i = (int32_t)(unit % (B + 1));
+    const bool has_q = i < B;
+    const int64_t rp_idx = unit;
+    const int64_t rq_idx = (int64_t)N * (B + 1) + (int64_t)n * B + i;
+    const RowFin fp = a.rfin[rp_idx];
+    const RowFin fq = has_q ? a.rfin[rq_idx] : empty_fin();
+    const uint64_t seq = s.seq_ids ? s.seq_ids[n] : (uint64_t)n;
+    const Bits *row_q =
+        has_q ? static_cast<const Bits *>(s.draft) + ((int64_t)n * B + i) * s.draft_stride : nullptr;
+    const float tau_q = Elem<Bits>::to_float(fq.tau_bits);
+    // ---- correction / bonus draw over p's nucleus (its candidates with x >=
+    // tau, compacted at the front of the p row's area), inverse CDF in
+    // vocabulary order, exact integer sums
+    const unsigned long long *pc =
+        reinterpret_cast<const unsigned long long *>(a.cand + rp_idx * (int64_t)kCandCap);
+    const int nc = (fp.status & kFinNonfinite) ? 0 : fp.n;
+    const double inv_sp = 1.0 / (fp.zp * kFix52);  // p's nucleus mass in fixed-point units
+    const double inv_zq = fq.zp > 0.0 ? 1.0 / fq.zp : 0.0;
+    // p's nucleus with its masses (as weights) to the scratch
+    auto load_nucleus = [&]() -> int {
+      int nn = 0;
+      for (int base = 0; base < nc; base += 32 * kLoadChunk) {
+        unsigned long long e[kLoadChunk];  // loads in flight together
+#pragma unroll
+        for (int h = 0; h < kLoadChunk; ++h) {
+          const int j = base + 32 * h + lane;
+          e[h] = j < nc ? __ldcg(pc + j) : 0ull;
+        }
+        uint32_t inm = 0u;  // bit h: entry h is in the nucleus
+#pragma unroll
+        for (int h = 0; h < kLoadChunk; ++h) {
+          const int j = base + 32 * h + lane;
+          const bool in = j < nc && Elem<Bits>::key((uint32_t)(e[h] >> 32)) >= fp.tau_key;
+          inm |= (in ? 1u : 0u) << h;
+        }
+        const int cnt = __popc(inm);
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        int d = nn + incl - cnt;
+        nn += __shfl_sync(0xFFFFFFFFu, incl, 31);
+#pragma unroll
+        for (int h = 0; h < kLoadChunk; ++h)
+          if ((inm >> h) & 1u) {
+            ds->idx[d] = (uint32_t)e[h];
+            ds->w[d] = e[h] >> 32;  // the logit's bits until its mass replaces them
+            ++d;
           }
+      }
+      __syncwarp();
+#pragma unroll 4
+      for (int j = lane; j < nn; j += 32)
+        ds->w[j] = fixed52(exact_exp2d(Elem<Bits>::to_float((uint32_t)ds->w[j]), fp.m, a.coef64));
+      __syncwarp();
+      return nn;
+    };
+    const int nn = load_nucleus();
+    unsigned long long W = 0ull;
+    if (has_q) {  // residual weights max(0, p - q), in double
+      for (int base = 0; base < nn; base += 32 * kQChunk) {
+        uint32_t xqb[kQChunk];  // q logits of the chunk, loads in flight together
+#pragma unroll
+        for (int c = 0; c < kQChunk; ++c) {
+          const int j = base + 32 * c + lane;
+          xqb[c] = j < nn ? (uint32_t)row_q[ds->idx[j]] : 0u;
+        }
+#pragma unroll
+        for (int c = 0; c < kQChunk; ++c) {
+          const int j = base + 32 * c + lane;
+          if (j < nn) {
+            const double pv = (double)ds->w[j] * inv_sp;
+            const float xq = Elem<Bits>::to_float(xqb[c]);
+            const double qv = xq >= tau_q ? exact_exp2d(xq, fq.m, a.coef64) * inv_zq : 0.0;
+            const unsigned long long wj = pv > qv ? fixed52(fmin(pv - qv, 1.0)) : 0ull;
+            ds->w[j] = wj;
+            W += wj;
+          }
+        }
+      }
+      W = warp_sum_any(W);
+      __syncwarp();
+      if (W == 0ull) load_nucleus();  // residual vanished: draw from p itself
+    }
+    if (W == 0ull) {
+      for (int j = lane; j < nn; j += 32) W += ds->w[j];
+      W = warp_sum_any(W);
+    }
+    int32_t token = 0;
+    if (W > 0ull) {
+      // t = floor(u' * W) exactly (u' = k / 2^24); the token is the index
+      // whose weight interval [C(x), C(x) + w_x) holds t, C(x) = weight of the
+      // entries with index < x: the largest X with C(X) <= t, by bisection
+      const float u2 = uniform24(s.seed, seq, s.step, (uint64_t)i, PSI_PURPOSE_RESID);
+      const unsigned long long k = (unsigned long long)(u2 * 16777216.0f);
+      const unsigned long long t = (__umul64hi(k, W) << 40) | ((k * W) >> 24);
+      uint32_t lo = 0u, hi = (uint32_t)V;
+      if (nn <= 32 * kRegCand) {
+        uint32_t ir[kRegCand];
+        unsigned long long wr[kRegCand];
+#pragma unroll
+        for (int c = 0; c < kRegCand; ++c) {
+          const int j = lane + 32 * c;
+          ir[c] = j < nn ? ds->idx[j] : 0xFFFFFFFFu;
+          wr[c] = j < nn ? ds->w[j] : 0ull;
+        }
+        while (hi - lo > 1u) {
+          const uint32_t mid = (lo + hi) >> 1;
+          unsigned long long cm = 0ull;
+#pragma unroll
+          for (int c = 0; c < kRegCand; ++c) cm += ir[c] < mid ? wr[c] : 0ull;
+          cm = warp_sum_any(cm);
+          if (cm > t) hi = mid;
+          else lo = mid;
         }
       } else {
-        // ---- accept / reject the drafted token (lane 0, double precision)
-        need = 1;
-        if (lane == 0) {
-          if (has_q) {
-            const int32_t x = s.ids[(int64_t)n * B + i];
-            double p = 0.0, q = 0.0;
-            const bool valid = x >= 0 && x < V;
-            if (valid) {
-              const float xp = Elem<Bits>::to_float(row_p[x]);
-              const float xq = Elem<Bits>::to_float(row_q[x]);
-              if (xp >= tau_p && fp.zp > 0.0) p = exact_exp2d(xp, fp.m, a.coef64) / fp.zp;
-              if (xq >= tau_q && fq.zp > 0.0) q = exact_exp2d(xq, fq.m, a.coef64) / fq.zp;
-            }
-            const double u = (double)uniform24(s.seed, seq, s.step, (uint64_t)i, PSI_PURPOSE_ACCEPT);
-            const int accept = (u * q < p) ? 1 : 0;
-            need = !accept;
-            if (s.out_p) s.out_p[(int64_t)n * B + i] = (float)p;
-            if (s.out_q) s.out_q[(int64_t)n * B + i] = (float)q;
-            a.rec[unit].accept = accept;
-            if (accept) a.rec[unit].token = -1;
-            if (!valid && s.dev_status) atomicOr(s.dev_status, PSI_DEV_BAD_TOKEN_ID);
-          } else {
-            a.rec[unit].accept = 1;
-          }
-          if (((fp.status | fq.status) & kFinNonfinite) && s.dev_status)
-            atomicOr(s.dev_status, PSI_DEV_NONFINITE);
-        }
-        need = __shfl_sync(0xFFFFFFFFu, need, 0);
-        if (need && !a.use_top_p) {  // the draw needs whole rows: decided after the emit step
-          if (lane == 0) a.rec[unit].token = -2;
-          need = 0;
+        while (hi - lo > 1u) {
+          const uint32_t mid = (lo + hi) >> 1;
+          unsigned long long cm = 0ull;
+          for (int j = lane; j < nn; j += 32)
+            if (ds->idx[j] < mid) cm += ds->w[j];
+          cm = warp_sum_any(cm);
+          if (cm > t) hi = mid;
+          else lo = mid;
         }
       }
-      if (need) {
-        // ---- correction / bonus draw over p's nucleus (its candidates with
-        // key >= tau), inverse CDF in vocabulary order, exact integer sums
-        WarpScratch *ws = &sh.ws[0];
-        uint64_t *wgt = sh.ws[1].m;  // draw weights (the q row's scratch is free now)
-        const int nc = (fp.status & kFinNonfinite) ? 0 : fp.n;
-        const double sp = fp.zp * kFix52;  // p's nucleus mass in fixed-point units
-        // compact the nucleus to the front, in candidate order: index in
-        // idx[], mass in m[] (reads of a group precede its writes, which land
-        // at or before the group)
-        const unsigned below = (1u << lane) - 1u;
-        int nn = 0;
-        for (int base = 0; base < nc; base += 32) {
-          const int j = base + lane;
-          const bool in = j < nc && ws->key[j] >= fp.tau_key;
-          uint32_t v = 0u;
-          uint64_t m = 0ull;
-          if (in) {
-            v = ws->idx[j];
-            m = ws->m[j];
-          }
-          const unsigned bal = __ballot_sync(0xFFFFFFFFu, in);
-          __syncwarp();
-          if (in) {
-            const int d = nn + __popc(bal & below);
-            ws->idx[d] = v;
-            ws->m[d] = m;
-          }
-          nn += __popc(bal);
-        }
-        __syncwarp();
-        int32_t token = 0;
-        for (int pass = 0; pass < 2; ++pass) {
-          const bool p_only = !has_q || pass == 1;
-          unsigned long long part = 0ull;
-          for (int base = 0; base < nn; base += 32 * kQChunk) {
-            uint32_t xqb[kQChunk];  // q logits of the chunk, loads in flight together
-#pragma unroll
-            for (int c = 0; c < kQChunk; ++c) {
-              const int j = base + 32 * c + lane;
-              xqb[c] = (!p_only && j < nn) ? (uint32_t)row_q[ws->idx[j]] : 0u;
-            }
-#pragma unroll
-            for (int c = 0; c < kQChunk; ++c) {
-              const int j = base + 32 * c + lane;
-              if (j < nn) {
-                uint64_t wj = ws->m[j];  // p alone: its masses are the weights
-                if (!p_only) {           // residual max(0, p - q), in double
-                  const double pv = (double)wj / sp;
-                  const float xq = Elem<Bits>::to_float(xqb[c]);
-                  const double qv = (xq >= tau_q && fq.zp > 0.0)
-                                        ? exact_exp2d(xq, fq.m, a.coef64) / fq.zp
-                                        : 0.0;
-                  wj = pv > qv ? fixed52(fmin(pv - qv, 1.0)) : 0ull;
-                }
-                wgt[j] = wj;
-                part += wj;
-              }
-            }
-          }
-          const unsigned long long W = warp_sum_any(part);
-          __syncwarp();
-          if (W == 0ull && !p_only) continue;  // residual vanished: draw from p itself
-          if (W > 0ull) {
-            // t = floor(u' * W) exactly (u' = k / 2^24)
-            const float u2 = uniform24(s.seed, seq, s.step, (uint64_t)i, PSI_PURPOSE_RESID);
-            const unsigned long long k = (unsigned long long)(u2 * 16777216.0f);
-            const unsigned long long t = (__umul64hi(k, W) << 40) | ((k * W) >> 24);
-            // smallest X with C(X) = (weight of entries with index < X) > t;
-            // the token is X - 1 (C(V) = W > t)
-            uint32_t lo = 0u, hi = (uint32_t)V;
-            if (nn <= 32 * kRegCand) {
-              uint32_t ir[kRegCand];
-              uint64_t wr[kRegCand];
-#pragma unroll
-              for (int c = 0; c < kRegCand; ++c) {
-                const int j = lane + 32 * c;
-                ir[c] = j < nn ? ws->idx[j] : 0xFFFFFFFFu;
-                wr[c] = j < nn ? wgt[j] : 0ull;
-              }
-              while (hi - lo > 1u) {
-                const uint32_t mid = (lo + hi) >> 1;
-                unsigned long long c = 0ull;
-#pragma unroll
-                for (int q = 0; q < kRegCand; ++q) c += ir[q] < mid ? wr[q] : 0ull;
-                c = warp_sum_any(c);
-                if (c > t) hi = mid;
-                else lo = mid;
-              }
-            } else {
-              while (hi - lo > 1u) {
-                const uint32_t mid = (lo + hi) >> 1;
-                unsigned long long c = 0ull;
-                for (int j = lane; j < nn; j += 32)
-                  if (ws->idx[j] < mid) c += wgt[j];
-                c = warp_sum_any(c);
-                if (c > t) hi = mid;
-                else lo = mid;
-              }
-            }
-            token = (int32_t)lo;
-          }
-          break;
-        }
-        if (lane == 0) a.rec[unit].token = token;
-      }
+      token = (int32_t)lo;
     }
-    __syncthreads();  // shared memory free for the next unit
+    if (lane == 0) {
+      a.rec[unit].token = token;
+      s.out_tokens[unit] = token;
+    }
+    __syncwarp();  // the scratch is reused by the warp's next unit
   }
 }
 
@@ -289,7 +341,8 @@ __global__ void __launch_bounds__(128) fast_emit_kernel(const __grid_constant__ 
   tok[L] = t;
   for (int32_t i = L + 1; i <= B; ++i) tok[i] = -1;
   s.out_n[n] = L + 1;
-  if (t == -2) a.list_b[atomicAdd(&a.counters[1], 1)] = n * (B + 1) + L;
+  if (t == kTokenWholeRow) a.list_b[atomicAdd(&a.counters[1], 1)] = n * (B + 1) + L;
+  else if (t == kTokenDraw) a.list_d[atomicAdd(&a.counters[8], 1)] = n * (B + 1) + L;
 }
 
 // SM count of the current device (queried once per device).
@@ -358,15 +411,16 @@ template <typename Bits>
 cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool early_exit,
                               const KernelEvents &ev, cudaStream_t stream) {
   const int64_t units = (int64_t)fa.s.N * (fa.s.B + 1);
-  const int64_t persistent = (int64_t)sm_count() * 2;
-  const int64_t grid_unit = units;
+  const int64_t persistent = (int64_t)sm_count() * 8;
+  const int64_t grid_unit = std::min<int64_t>((units + kUnitThreads - 1) / kUnitThreads, persistent);
+  const int64_t grid_draw = std::min<int64_t>(fa.s.N, persistent);
+  const int64_t grid_finish =
+      std::min<int64_t>((fa.rows + kFinishWarps - 1) / kFinishWarps, persistent);
   cudaError_t e;
-  static DeviceOnce configure;  // shared memory above 48 KB, once per device
+  static DeviceOnce configure;  // carveouts, once per device
   e = configure([] {
-    cudaError_t err = cudaFuncSetAttribute(unit_kernel<Bits>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)sizeof(UnitShared));
-    if (err == cudaSuccess) err = prefer_max_shared(unit_kernel<Bits>);
+    cudaError_t err = prefer_max_shared(draw_kernel<Bits>);
+    if (err == cudaSuccess) err = prefer_max_shared(row_finish_kernel<Bits>);
     if (err == cudaSuccess) err = prefer_max_shared(round_advance_kernel);
     if (err == cudaSuccess) err = prefer_max_shared(fast_emit_kernel);
     return err;
@@ -383,8 +437,9 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
         cudaSuccess)
       return err;
     if (timed && ev.after && (err = cudaEventRecord(ev.after, stream)) != cudaSuccess) return err;
-    const int64_t g = f.pass == 1 ? grid_unit : std::min<int64_t>(grid_unit, persistent);
-    unit_kernel<Bits><<<(unsigned)g, 64, sizeof(UnitShared), stream>>>(f);
+    row_finish_kernel<Bits><<<(unsigned)grid_finish, 32 * kFinishWarps, 0, stream>>>(f);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    unit_kernel<Bits><<<(unsigned)grid_unit, kUnitThreads, 0, stream>>>(f);
     return cudaGetLastError();
   };
   // the second pass over the rows and units a first pass could not settle
@@ -421,6 +476,8 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
   if (e != cudaSuccess) return e;
   fast_emit_kernel<<<(fa.s.N + 127) / 128, 128, 0, stream>>>(fa);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  draw_kernel<Bits><<<(unsigned)grid_draw, 32, 0, stream>>>(fa);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int clusters_b = std::min(fa.s.N, kListClusters);
   return launch_cluster_list(sa, dt, plan, kClusterModeSample, fa.list_b, fa.counters + 1,
                              clusters_b, stream);
@@ -441,11 +498,15 @@ FastLayout fast_layout(int32_t N, int32_t B) {
   off = align256(off + sizeof(uint64_t) * (size_t)rows * kCandCap);
   L.known_off = off;
   off = align256(off + sizeof(float) * (size_t)rows);
+  L.rfin_off = off;
+  off = align256(off + sizeof(RowFin) * (size_t)rows);
   L.counters_off = off;
   off = align256(off + sizeof(int32_t) * kCounters);
   L.list_a_off = off;
   off = align256(off + sizeof(int32_t) * (size_t)units);
   L.list_b_off = off;
+  off = align256(off + sizeof(int32_t) * (size_t)N);
+  L.list_d_off = off;
   off = align256(off + sizeof(int32_t) * (size_t)N);
   L.wide_rows_off = off;
   off = align256(off + sizeof(int32_t) * (size_t)rows);
@@ -489,9 +550,11 @@ cudaError_t launch_sampled_fast(const SampledArgs &a, psi_dtype dtype, const Sam
   fa.srec = reinterpret_cast<SliceRecord *>(ws + L.srec_off);
   fa.cand = reinterpret_cast<uint64_t *>(ws + L.cand_off);
   fa.known_max = reinterpret_cast<float *>(ws + L.known_off);
+  fa.rfin = reinterpret_cast<RowFin *>(ws + L.rfin_off);
   fa.counters = reinterpret_cast<int32_t *>(ws + L.counters_off);
   fa.list_a = reinterpret_cast<int32_t *>(ws + L.list_a_off);
   fa.list_b = reinterpret_cast<int32_t *>(ws + L.list_b_off);
+  fa.list_d = reinterpret_cast<int32_t *>(ws + L.list_d_off);
   fa.wide_rows = reinterpret_cast<int32_t *>(ws + L.wide_rows_off);
   fa.wide_units = reinterpret_cast<int32_t *>(ws + L.wide_units_off);
   fa.round_rows = reinterpret_cast<int32_t *>(ws + L.round_rows_off);

@@ -11,6 +11,21 @@
 #include "psi_internal.h"
 
 namespace psi {
+
+// A finished row, as the row_finish kernel leaves it for the unit kernel.
+// The row's candidates (x above its final threshold), as raw list entries
+// (bits << 32) | vocabulary index, are compacted in place at the front of
+// the row's set-aside area.
+struct RowFin {
+  float m;            // row maximum
+  int32_t status;     // kFin* bits
+  double zp;          // normaliser after top-p (Z without top-p)
+  uint32_t tau_bits;  // top-p threshold (raw bits): keep x >= tau
+  uint32_t tau_key;   // its order-preserving key (0 without top-p)
+  int32_t n;          // candidates at the front of the row's area
+  int32_t pad;
+};
+
 namespace finish {
 
 template <typename T>
@@ -63,6 +78,16 @@ struct WarpScratch {
 
 // A mass or weight in [0, 1] in 2^52 fixed point.
 __device__ __forceinline__ uint64_t fixed52(double m) { return __double2ull_rn(m * kFix52); }
+
+// floor(m * 2^52) of an fp32 m in [0, 1], from its bits (integer shifts
+// only): m = (2^23 + frac) * 2^(e - 150), so m * 2^52 = (2^23 + frac) << (e - 98).
+__device__ __forceinline__ uint64_t fixed52_f32(float m) {
+  const uint32_t b = __float_as_uint(m);
+  const int sh = (int)(b >> 23) - 98;
+  const uint64_t mant = (uint64_t)((b & 0x7FFFFFu) | 0x800000u);
+  if (sh <= -24) return 0ull;  // below 2^-52, zero and subnormals included
+  return sh >= 0 ? (mant << sh) : (mant >> (-sh));
+}
 
 // Row maximum, Z, top-p threshold tau and renormaliser Z' of row r from its
 // slice records and set-aside lists, by one warp.  M is the largest slice
@@ -218,6 +243,215 @@ __device__ RowFinal finish_row(const FastArgs &a, int64_t r, WarpScratch *ws) {
   out.zp = (double)s_lo / kFix52;
   out.tau_key = lo;
   out.tau_bits = key_to_bits<Bits>(lo);
+  return out;
+}
+
+
+// ---------------------------------------------------------------------------
+// The linear verify's row finish: one warp per row, results to global memory.
+// ---------------------------------------------------------------------------
+
+struct FinScratch {  // one warp's shared memory: the row's candidates
+  uint32_t key[kFinishCap];
+  unsigned long long m[kFinishCap];
+};
+
+// Largest key t in [lo, hi) whose suffix mass S(t) (every candidate with key
+// >= t) reaches `target`, by bisection on exact integer sums (order-free);
+// S(lo) = s_lo >= target.  `sum_from(mid)` is the warp's S(mid).
+template <typename SumFrom>
+__device__ __forceinline__ uint32_t suffix_bisect(uint32_t lo, uint32_t hi,
+                                                  unsigned long long target,
+                                                  unsigned long long &s_lo, SumFrom sum_from) {
+  while (hi - lo > 1u) {
+    const uint32_t mid = lo + ((hi - lo) >> 1);
+    const unsigned long long part = sum_from(mid);
+    if (part >= target) {
+      lo = mid;
+      s_lo = part;
+    } else {
+      hi = mid;
+    }
+  }
+  return lo;
+}
+
+// Row maximum, Z, top-p threshold tau and renormaliser Z' of row r, by one
+// warp, as finish_row computes them (same classification, candidate masses,
+// integer sums and bisection for tau), with two differences: the candidates
+// are also compacted in place at the front of the row's set-aside area (the
+// draw kernel reads them there), and the masses of the set-aside elements
+// below the final threshold (with top-p each under 2^-13 of the maximum's)
+// are taken in fp32, like the slices' sums that make up the rest of Z,
+// before they join Z in fixed point.  The candidates' exact masses are
+// computed after the list is sorted, in a loop of independent iterations.
+template <typename Bits>
+__device__ RowFin finish_row_list(const FastArgs &a, int64_t r, FinScratch *fs) {
+  const int lane = threadIdx.x & 31;
+  RowFin out;
+  out.m = -INFINITY;
+  out.zp = 0.0;
+  out.tau_bits = Elem<Bits>::kNegInf;
+  out.tau_key = 0u;
+  out.n = 0;
+  out.status = 0;
+  out.pad = 0;
+  const int C = a.g.slices;
+  const SliceRecord *sr = a.srec + r * kMaxSlices;
+  float M = -INFINITY;
+  bool lost = false;
+  for (int c = 0; c < C; ++c) {
+    M = fmaxf(M, sr[c].m);
+    lost |= (sr[c].flags & kRowLost) != 0 || sr[c].n_cand > a.g.cap;
+  }
+  out.m = M;
+  if (lost) {
+    out.status = kFinOverflow;
+    return out;
+  }
+  double Z = 0.0;
+  for (int c = 0; c < C; ++c)
+    if (sr[c].m > -INFINITY) Z += sr[c].z * exp2(((double)sr[c].m - (double)M) * a.coef64);
+  if (!(M > -INFINITY) || !(fabsf(M * a.coef) < INFINITY) || Z != Z) {
+    out.status = kFinNonfinite;
+    return out;
+  }
+  const float thr = a.use_top_p ? threshold_value<Bits>(M - sr[0].off) : INFINITY;
+  unsigned long long *area = reinterpret_cast<unsigned long long *>(a.cand + r * (int64_t)kCandCap);
+  int n = 0;
+  unsigned long long zin = 0ull, zrest = 0ull;
+  uint32_t kmax = 0u, kmin_inv = 0u;
+  for (int c = 0; c < C; ++c) {
+    const int nc = sr[c].n_cand;
+    const unsigned long long *src = area + (int64_t)c * a.g.cap;
+    unsigned long long e[kLoadChunk], nx[kLoadChunk];
+#pragma unroll
+    for (int h = 0; h < kLoadChunk; ++h) {
+      const int j = 32 * h + lane;
+      nx[h] = j < nc ? __ldcg(src + j) : 0ull;
+    }
+    for (int base = 0; base < nc; base += 32 * kLoadChunk) {
+#pragma unroll
+      for (int h = 0; h < kLoadChunk; ++h) e[h] = nx[h];
+      // the next chunk's loads go out before this chunk is sorted (none of
+      // them is overwritten: candidates land below base + 32 * kLoadChunk)
+#pragma unroll
+      for (int h = 0; h < kLoadChunk; ++h) {
+        const int j = base + 32 * (kLoadChunk + h) + lane;
+        nx[h] = j < nc ? __ldcg(src + j) : 0ull;
+      }
+      __syncwarp();  // every entry of the chunk is read before any is overwritten
+      // sort the chunk: the other entries' masses (fp32) join zrest at
+      // once; candidates are compacted, their masses taken afterwards
+      uint32_t cmask = 0u;  // bit h: entry h is a candidate
+#pragma unroll
+      for (int h = 0; h < kLoadChunk; ++h) {
+        const int j = base + 32 * h + lane;
+        const float x = Elem<Bits>::to_float((uint32_t)(e[h] >> 32));
+        const bool live = j < nc;
+        const bool cand = live && x > thr;
+        cmask |= (cand ? 1u : 0u) << h;
+        const float mf = (live && !cand) ? fast_exp2((x - M) * a.coef) : 0.f;  // <= 1
+        zrest += fixed52_f32(mf);
+      }
+      // this lane's candidates go to positions n + (candidates of lower
+      // lanes) + k: below every entry not yet read
+      const int cnt = __popc(cmask);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      int d = n + incl - cnt;
+      n += __shfl_sync(0xFFFFFFFFu, incl, 31);
+      while (cmask) {
+        const int h = __ffs(cmask) - 1;
+        cmask &= cmask - 1u;
+        if (d < kFinishCap) {
+          unsigned long long eh = 0ull;
+#pragma unroll
+          for (int q = 0; q < kLoadChunk; ++q) eh = q == h ? e[q] : eh;
+          const uint32_t b = (uint32_t)(eh >> 32);
+          const uint32_t key = Elem<Bits>::key(b);
+          area[d] = eh;
+          fs->key[d] = key;
+          fs->m[d] = b;  // the logit's bits until its mass replaces them
+          kmax = max(kmax, key);
+          kmin_inv = max(kmin_inv, ~key);
+        }
+        ++d;
+      }
+    }
+  }
+  // the candidates' masses, exact in double (independent iterations)
+  __syncwarp();
+  if (n <= kFinishCap) {
+#pragma unroll 4
+    for (int j = lane; j < n; j += 32) {
+      const unsigned long long m52 =
+          fixed52(exact_exp2d(Elem<Bits>::to_float((uint32_t)fs->m[j]), M, a.coef64));
+      fs->m[j] = m52;
+      zin += m52;
+    }
+  }
+  __syncwarp();
+  if (n > kFinishCap) {  // more candidates than the area holds: rescan, then the general path
+    out.status = kFinOverflow;
+    return out;
+  }
+  out.n = n;
+  kmax = warp_max_u32(kmax);
+  kmin_inv = warp_max_u32(kmin_inv);
+  zin = warp_sum_any(zin);
+  zrest = warp_sum_any(zrest);
+  __syncwarp();
+  Z += ((double)zin + (double)zrest) / kFix52;
+  out.zp = Z;
+  if (!(Z < INFINITY)) {
+    out.status = kFinNonfinite;
+    return out;
+  }
+  if (!a.use_top_p) return out;
+  const double target_d = ceil((double)a.s.top_p * Z * kFix52);
+  if (!(target_d < 9.2e18) || (double)zin < target_d) {  // (zin < 2^63)
+    out.status = kFinCoverage;
+    return out;
+  }
+  const unsigned long long target = (unsigned long long)target_d;
+  if (zin < target) {
+    out.status = kFinCoverage;
+    return out;
+  }
+  // bisection over [kmin, kmax]: S(kmin) = zin reaches the target
+  unsigned long long s_at = zin;
+  uint32_t t;
+  if (n <= 32 * kRegCand) {
+    uint32_t kr[kRegCand];  // the row's candidates in registers
+    unsigned long long mr[kRegCand];
+#pragma unroll
+    for (int c = 0; c < kRegCand; ++c) {
+      const int j = lane + 32 * c;
+      kr[c] = j < n ? fs->key[j] : 0u;
+      mr[c] = j < n ? fs->m[j] : 0ull;
+    }
+    t = suffix_bisect(~kmin_inv, kmax + 1u, target, s_at, [&](uint32_t mid) {
+      unsigned long long part = 0ull;
+#pragma unroll
+      for (int c = 0; c < kRegCand; ++c) part += kr[c] >= mid ? mr[c] : 0ull;
+      return warp_sum_any(part);
+    });
+  } else {
+    t = suffix_bisect(~kmin_inv, kmax + 1u, target, s_at, [&](uint32_t mid) {
+      unsigned long long part = 0ull;
+      for (int j = lane; j < n; j += 32)
+        if (fs->key[j] >= mid) part += fs->m[j];
+      return warp_sum_any(part);
+    });
+  }
+  out.zp = (double)s_at / kFix52;
+  out.tau_key = t;
+  out.tau_bits = key_to_bits<Bits>(t);
   return out;
 }
 

@@ -201,9 +201,11 @@ struct ScanGeom {
 ScanGeom plan_scan(int32_t V, int elem_bytes);
 
 struct FastLayout {  // workspace carve-up of the streaming path
-  size_t rec_off, srec_off, cand_off, known_off, counters_off, list_a_off, list_b_off,
+  size_t rec_off, srec_off, cand_off, known_off, rfin_off, counters_off, list_a_off, list_b_off,
+      list_d_off,
       wide_rows_off, wide_units_off, round_rows_off, round_units_off, active_off, total;
 };
+struct RowFin;  // a finished row (psi_finish.cuh)
 FastLayout fast_layout(int32_t N, int32_t B);
 // False when the streaming path's row indices would not fit its lists.
 bool fast_path_fits(int32_t N, int32_t B);
@@ -231,10 +233,12 @@ struct FastArgs {
   uint64_t *cand;      // [rows][kCandCap]: slice c's set-aside list at c * g.cap;
                        // (bits << 32) | vocabulary index
   float *known_max;    // [rows] row maximum found by a first pass (read by a rescan)
+  RowFin *rfin;        // [rows] the row finish's results (streaming linear verify)
   int32_t *counters;   // [0] general units, [1] sample-mode units, [2] wide rows, [3] wide units,
-                       // [4 + 2k], [5 + 2k] rows and units of round parity k
+                       // [4 + 2k], [5 + 2k] rows and units of round parity k, [8] draw units
   int32_t *list_a;     // units for the general path
   int32_t *list_b;     // units whose draw needs the whole row
+  int32_t *list_d;     // units whose draw is over their p row's nucleus
   int32_t *wide_rows;  // rows for the second scan (| kWideBit: wide window)
   int32_t *wide_units; // units for the second unit pass
 };

@@ -448,6 +448,7 @@ cudaError_t launch_tree_sampled(const void *ar, int64_t ar_stride, psi_dtype dty
   fa.srec = reinterpret_cast<SliceRecord *>(ws + L.srec_off);
   fa.cand = reinterpret_cast<uint64_t *>(ws + L.cand_off);
   fa.known_max = reinterpret_cast<float *>(ws + L.known_off);
+  fa.rfin = nullptr;  // the tree walk finishes its rows itself
   cudaError_t e;
   // the row scan streams 16-byte vectors; rows that do not start on a 16-byte
   // boundary are settled by the walk's exact whole-row path instead
