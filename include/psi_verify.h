@@ -158,6 +158,47 @@ psi_status psi_verify_linear(const void *ar_logits, int64_t ar_row_stride,
                              void *workspace, size_t workspace_bytes,
                              psi_stream_t stream);
 
+/* Workspace needed by psi_verify_linear_topk (bytes; the same as
+ * psi_verify_linear's for these sizes; 0 on invalid sizes). */
+size_t psi_verify_linear_topk_workspace_bytes(int32_t N, int32_t B, int32_t V,
+                                              psi_dtype dtype, float temperature,
+                                              float top_p, int32_t top_k);
+
+/*
+ * psi_verify_linear_topk - psi_verify_linear with a top-k cut.
+ *
+ * Source: the run card ("想跑 Uno：先確認官方程式需要的環境") names top-k
+ * beside top-p and temperature as sampler settings.  Reading of the order:
+ * top-k is taken on the temperature softmax first (every token whose
+ * probability is at least the k-th largest stays, ties with the k-th
+ * included), the kept mass is renormalised, and top-p then cuts that
+ * distribution as in psi_verify_linear.  It applies to p_i and q_i alike, so
+ * the acceptance test, the residual and the bonus draw all use the cut
+ * distributions.
+ *
+ * Arguments, results, layouts and limits as psi_verify_linear, plus
+ * top_k: 0 = off; top_k >= V keeps every token (also off); negative values
+ *   return PSI_ERR_INVALID_ARG.  Ignored when T == 0 (the argmax is always
+ *   kept).
+ * With top_k off the call is psi_verify_linear.  Rows whose set-aside
+ * candidates (the elements near the maximum that the streaming scan keeps)
+ * number at least k are finished from them; the other units (large k, flat
+ * rows, or rows that do not start on a 16-byte boundary) go to a slower
+ * whole-row path that reads their two rows a few more times.  Results do
+ * not depend on which path a unit takes.
+ */
+psi_status psi_verify_linear_topk(const void *ar_logits, int64_t ar_row_stride,
+                                  const void *draft_logits,
+                                  int64_t draft_row_stride, psi_dtype dtype,
+                                  const int32_t *draft_ids, int32_t N, int32_t B,
+                                  int32_t V, float temperature, float top_p,
+                                  int32_t top_k, uint64_t seed,
+                                  const uint64_t *seq_ids, uint64_t step,
+                                  int32_t *out_tokens, int32_t *out_n_emitted,
+                                  float *out_p_draft, float *out_q_draft,
+                                  uint32_t *dev_status, void *workspace,
+                                  size_t workspace_bytes, psi_stream_t stream);
+
 /*
  * psi_verify_linear_noalloc - psi_verify_linear for callers that cannot
  * allocate device memory (no counterpart on the pages: an integration

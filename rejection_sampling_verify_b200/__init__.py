@@ -53,6 +53,8 @@ EXPORTED = (
     "psi_verify_linear_workspace_bytes",
     "psi_verify_linear",
     "psi_verify_linear_noalloc",
+    "psi_verify_linear_topk_workspace_bytes",
+    "psi_verify_linear_topk",
     "psi_verify_tree_greedy_workspace_bytes",
     "psi_verify_tree_greedy",
     "psi_verify_tree_sampled_workspace_bytes",
@@ -93,6 +95,11 @@ def load_library():
     lib.psi_verify_linear_noalloc.restype = C.c_int
     lib.psi_verify_linear_noalloc.argtypes = [vp, i64, vp, i64, C.c_int, vp, i32, i32, i32, f32,
                                               f32, u64, vp, u64, vp, vp, vp, vp, vp, vp]
+    lib.psi_verify_linear_topk_workspace_bytes.restype = sz
+    lib.psi_verify_linear_topk_workspace_bytes.argtypes = [i32, i32, i32, C.c_int, f32, f32, i32]
+    lib.psi_verify_linear_topk.restype = C.c_int
+    lib.psi_verify_linear_topk.argtypes = [vp, i64, vp, i64, C.c_int, vp, i32, i32, i32, f32, f32,
+                                           i32, u64, vp, u64, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.psi_verify_tree_greedy_workspace_bytes.restype = sz
     lib.psi_verify_tree_greedy_workspace_bytes.argtypes = [i32, i32, i32, C.c_int]
     lib.psi_verify_tree_greedy.restype = C.c_int
@@ -128,6 +135,21 @@ def psi_last_error() -> str:
 def psi_verify_linear_workspace_bytes(N, B, V, dtype, temperature, top_p) -> int:
     return int(load_library().psi_verify_linear_workspace_bytes(N, B, V, dtype, temperature,
                                                                 top_p))
+
+
+def psi_verify_linear_topk_workspace_bytes(N, B, V, dtype, temperature, top_p, top_k) -> int:
+    return int(load_library().psi_verify_linear_topk_workspace_bytes(N, B, V, dtype, temperature,
+                                                                     top_p, top_k))
+
+
+def psi_verify_linear_topk(ar_logits, ar_row_stride, draft_logits, draft_row_stride, dtype,
+                           draft_ids, N, B, V, temperature, top_p, top_k, seed, seq_ids, step,
+                           out_tokens, out_n_emitted, out_p_draft, out_q_draft, dev_status,
+                           workspace, workspace_bytes, stream) -> int:
+    return int(load_library().psi_verify_linear_topk(
+        ar_logits, ar_row_stride, draft_logits, draft_row_stride, dtype, draft_ids, N, B, V,
+        temperature, top_p, top_k, seed, seq_ids, step, out_tokens, out_n_emitted, out_p_draft,
+        out_q_draft, dev_status, workspace, workspace_bytes, stream))
 
 
 def psi_verify_linear(ar_logits, ar_row_stride, draft_logits, draft_row_stride, dtype,
@@ -290,8 +312,9 @@ class LinearResult:
 
 def verify_linear(ar, draft, ids, temperature: float, top_p: float = 1.0, seed: int = 0,
                   step: int = 0, seq_ids=None, want_probs: bool = True, workspace=None,
-                  stream=None, out: LinearResult | None = None) -> LinearResult:
-    """Linear verify of a batch (see ``psi_verify_linear`` in the header).
+                  stream=None, out: LinearResult | None = None, top_k: int = 0) -> LinearResult:
+    """Linear verify of a batch (see ``psi_verify_linear`` in the header; with
+    ``top_k`` != 0, ``psi_verify_linear_topk``).
 
     ar [N, B+1, V], draft [N, B, V] (may be None when temperature == 0),
     ids int32 [N, B], seq_ids uint64-as-int64 [N] or None; CUDA tensors.
@@ -340,6 +363,15 @@ def verify_linear(ar, draft, ids, temperature: float, top_p: float = 1.0, seed: 
         workspace = None
     elif workspace is None or _nbytes(workspace) < ws_bytes:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    if top_k:
+        st = psi_verify_linear_topk(
+            _ptr(ar), ar_stride, None if greedy else _ptr(draft), dr_stride, code, _ptr(ids), N,
+            B, V, float(temperature), float(top_p), int(top_k), int(seed) & (2**64 - 1),
+            _ptr(seq_ids), int(step) & (2**64 - 1), _ptr(out.tokens), _ptr(out.n_emitted),
+            _ptr(out.p_draft), _ptr(out.q_draft), _ptr(out.status), _ptr(workspace),
+            _nbytes(workspace), _stream(stream))
+        _check(st, "psi_verify_linear_topk")
+        return out
     st = psi_verify_linear(
         _ptr(ar), ar_stride, None if greedy else _ptr(draft), dr_stride, code, _ptr(ids), N, B,
         V, float(temperature), float(top_p), int(seed) & (2**64 - 1),

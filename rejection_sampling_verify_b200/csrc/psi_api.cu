@@ -103,10 +103,10 @@ size_t psi_verify_linear_workspace_bytes(int32_t N, int32_t B, int32_t V, psi_dt
   return round256(psi::fast_layout(N, B).total);
 }
 
-psi_status psi_verify_linear(const void *ar_logits, int64_t ar_row_stride,
+static psi_status verify_linear(const void *ar_logits, int64_t ar_row_stride,
                              const void *draft_logits, int64_t draft_row_stride,
                              psi_dtype dtype, const int32_t *draft_ids, int32_t N, int32_t B,
-                             int32_t V, float temperature, float top_p, uint64_t seed,
+                             int32_t V, float temperature, float top_p, int32_t top_k, uint64_t seed,
                              const uint64_t *seq_ids, uint64_t step, int32_t *out_tokens,
                              int32_t *out_n_emitted, float *out_p_draft, float *out_q_draft,
                              uint32_t *dev_status, void *workspace, size_t workspace_bytes,
@@ -178,6 +178,7 @@ psi_status psi_verify_linear(const void *ar_logits, int64_t ar_row_stride,
   a.V = V;
   a.temperature = temperature;
   a.top_p = top_p;
+  a.top_k = (top_k > 0 && top_k < V) ? top_k : 0;  // k >= V keeps every token
   a.seed = seed;
   a.seq_ids = seq_ids;
   a.step = step;
@@ -194,12 +195,51 @@ psi_status psi_verify_linear(const void *ar_logits, int64_t ar_row_stride,
   const bool rows_aligned = aligned_to(ar_logits, 16) && aligned_to(draft_logits, 16) &&
                             ((size_t)ar_row_stride * es) % 16 == 0 &&
                             ((size_t)draft_row_stride * es) % 16 == 0;
-  if (rows_aligned && psi::fast_path_fits(N, B))
+  if (rows_aligned && psi::fast_path_fits(N, B)) {
     e = psi::launch_sampled_fast(a, dtype, plan, workspace, g_events, stream);
-  else
+  } else if (a.top_k > 0) {  // the whole-row top-k path for every unit
+    e = psi::launch_topk_units(a, dtype, nullptr, nullptr, (int64_t)N * (B + 1), stream);
+    if (e == cudaSuccess) e = psi::launch_sampled_emit(a, stream);
+  } else {
     e = psi::launch_sampled(a, dtype, plan, g_events, stream);
+  }
   if (e != cudaSuccess) return cuda_fail(e, "sampled verify launch");
   return PSI_OK;
+}
+
+psi_status psi_verify_linear(const void *ar_logits, int64_t ar_row_stride,
+                             const void *draft_logits, int64_t draft_row_stride,
+                             psi_dtype dtype, const int32_t *draft_ids, int32_t N, int32_t B,
+                             int32_t V, float temperature, float top_p, uint64_t seed,
+                             const uint64_t *seq_ids, uint64_t step, int32_t *out_tokens,
+                             int32_t *out_n_emitted, float *out_p_draft, float *out_q_draft,
+                             uint32_t *dev_status, void *workspace, size_t workspace_bytes,
+                             psi_stream_t stream) {
+  return verify_linear(ar_logits, ar_row_stride, draft_logits, draft_row_stride, dtype, draft_ids,
+                       N, B, V, temperature, top_p, 0, seed, seq_ids, step, out_tokens,
+                       out_n_emitted, out_p_draft, out_q_draft, dev_status, workspace,
+                       workspace_bytes, stream);
+}
+
+size_t psi_verify_linear_topk_workspace_bytes(int32_t N, int32_t B, int32_t V, psi_dtype dtype,
+                                              float temperature, float top_p, int32_t top_k) {
+  (void)top_k;
+  return psi_verify_linear_workspace_bytes(N, B, V, dtype, temperature, top_p);
+}
+
+psi_status psi_verify_linear_topk(const void *ar_logits, int64_t ar_row_stride,
+                                  const void *draft_logits, int64_t draft_row_stride,
+                                  psi_dtype dtype, const int32_t *draft_ids, int32_t N, int32_t B,
+                                  int32_t V, float temperature, float top_p, int32_t top_k,
+                                  uint64_t seed, const uint64_t *seq_ids, uint64_t step,
+                                  int32_t *out_tokens, int32_t *out_n_emitted, float *out_p_draft,
+                                  float *out_q_draft, uint32_t *dev_status, void *workspace,
+                                  size_t workspace_bytes, psi_stream_t stream) {
+  if (top_k < 0) return fail(PSI_ERR_INVALID_ARG, "top_k %d (need >= 0; 0 = off)", (int)top_k);
+  return verify_linear(ar_logits, ar_row_stride, draft_logits, draft_row_stride, dtype, draft_ids,
+                       N, B, V, temperature, top_p, top_k, seed, seq_ids, step, out_tokens,
+                       out_n_emitted, out_p_draft, out_q_draft, dev_status, workspace,
+                       workspace_bytes, stream);
 }
 
 size_t psi_verify_tree_greedy_workspace_bytes(int32_t N, int32_t M, int32_t V, psi_dtype dtype) {

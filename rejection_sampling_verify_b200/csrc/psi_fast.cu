@@ -46,7 +46,7 @@ namespace {
 using namespace finish;
 
 constexpr int kListClusters = 16;
-constexpr int kCounters = 9;  // work-list counters (see FastArgs::counters)
+constexpr int kCounters = 10;  // work-list counters (see FastArgs::counters)
 // Candidate window, in log2 units below the row maximum.  The first pass uses
 // a narrow window (13 units for top_p <= 0.95, wider as top_p approaches 1);
 // the second pass the wide one.
@@ -105,8 +105,15 @@ __global__ void __launch_bounds__(kUnitThreads) unit_kernel(const __grid_constan
     const int64_t rq_idx = (int64_t)N * (B + 1) + (int64_t)n * B + i;
     const RowFin fp = a.rfin[rp_idx];
     const RowFin fq = has_q ? a.rfin[rq_idx] : empty_fin();
-    const int fail_q = fq.status & (kFinOverflow | kFinCoverage);
-    const int fail_p = fp.status & (kFinOverflow | kFinCoverage);
+    const int fail_q = fq.status & (kFinOverflow | kFinCoverage | kFinTopK);
+    const int fail_p = fp.status & (kFinOverflow | kFinCoverage | kFinTopK);
+    if (a.top_k > 0 && (((fp.status | fq.status) & kFinTopK) || ((fail_q || fail_p) && a.pass == 2))) {
+      // the candidates do not hold a top-k set (or a rescan did not settle
+      // the unit): the whole-row top-k path decides it at the end
+      a.list_k[atomicAdd(&a.counters[9], 1)] = (int32_t)unit;
+      a.rec[unit].accept = -1;  // a later round treats it as accepted
+      continue;
+    }
     if (fail_q || fail_p) {
       if (a.pass == 1) {  // rescan the failed rows, then finish the unit again
         // the rescan starts from the row maximum found here, so its
@@ -160,7 +167,7 @@ __global__ void __launch_bounds__(kUnitThreads) unit_kernel(const __grid_constan
       atomicOr(s.dev_status, PSI_DEV_NONFINITE);
     // the correction / bonus token: drawn after the emit step, and only for
     // the position each sequence emits
-    if (need) a.rec[unit].token = a.use_top_p ? kTokenDraw : kTokenWholeRow;
+    if (need) a.rec[unit].token = a.use_window ? kTokenDraw : kTokenWholeRow;
   }
 }
 
@@ -470,6 +477,11 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
   const psi_dtype dt = sizeof(Bits) == 2 ? PSI_DTYPE_BF16 : PSI_DTYPE_F32;
   SampledArgs sa = fa.s;
   sa.records = fa.rec;
+  if (fa.top_k > 0) {
+    e = launch_topk_units(sa, dt, fa.list_k, fa.counters + 9,
+                          std::min<int64_t>(units, (int64_t)sm_count() * 4), stream);
+    if (e != cudaSuccess) return e;
+  }
   const int clusters_a = (int)std::min<int64_t>(units, kListClusters);
   e = launch_cluster_list(sa, dt, plan, kClusterModeList, fa.list_a, fa.counters + 0, clusters_a,
                           stream);
@@ -508,6 +520,8 @@ FastLayout fast_layout(int32_t N, int32_t B) {
   off = align256(off + sizeof(int32_t) * (size_t)N);
   L.list_d_off = off;
   off = align256(off + sizeof(int32_t) * (size_t)N);
+  L.list_k_off = off;
+  off = align256(off + sizeof(int32_t) * (size_t)units);
   L.wide_rows_off = off;
   off = align256(off + sizeof(int32_t) * (size_t)rows);
   L.wide_units_off = off;
@@ -545,6 +559,8 @@ cudaError_t launch_sampled_fast(const SampledArgs &a, psi_dtype dtype, const Sam
   fa.win_narrow = (float)(wlog2 / fa.coef64);
   fa.win_wide = (float)(kWindowWideLog2 / fa.coef64);
   fa.use_top_p = a.top_p < 1.0f ? 1 : 0;
+  fa.top_k = a.top_k;
+  fa.use_window = (fa.use_top_p || fa.top_k > 0) ? 1 : 0;
   fa.pass = 1;
   fa.rec = reinterpret_cast<UnitRecord *>(ws + L.rec_off);
   fa.srec = reinterpret_cast<SliceRecord *>(ws + L.srec_off);
@@ -555,6 +571,7 @@ cudaError_t launch_sampled_fast(const SampledArgs &a, psi_dtype dtype, const Sam
   fa.list_a = reinterpret_cast<int32_t *>(ws + L.list_a_off);
   fa.list_b = reinterpret_cast<int32_t *>(ws + L.list_b_off);
   fa.list_d = reinterpret_cast<int32_t *>(ws + L.list_d_off);
+  fa.list_k = reinterpret_cast<int32_t *>(ws + L.list_k_off);
   fa.wide_rows = reinterpret_cast<int32_t *>(ws + L.wide_rows_off);
   fa.wide_units = reinterpret_cast<int32_t *>(ws + L.wide_units_off);
   fa.round_rows = reinterpret_cast<int32_t *>(ws + L.round_rows_off);

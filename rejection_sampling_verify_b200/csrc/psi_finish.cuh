@@ -59,6 +59,7 @@ struct RowFinal {
 constexpr int kFinOverflow = 1;   // candidates lost: rescan with the exact maximum
 constexpr int kFinCoverage = 2;   // the window holds less than top_p: rescan wider
 constexpr int kFinNonfinite = 4;  // NaN / +inf logit, or no finite logit
+constexpr int kFinTopK = 8;       // the candidates do not hold the row's top-k set
 
 constexpr int kLoadChunk = 16;           // global loads per lane in flight together
 constexpr int kQChunk = 16;              // q loads per lane in flight together
@@ -316,7 +317,7 @@ __device__ RowFin finish_row_list(const FastArgs &a, int64_t r, FinScratch *fs) 
     out.status = kFinNonfinite;
     return out;
   }
-  const float thr = a.use_top_p ? threshold_value<Bits>(M - sr[0].off) : INFINITY;
+  const float thr = a.use_window ? threshold_value<Bits>(M - sr[0].off) : INFINITY;
   unsigned long long *area = reinterpret_cast<unsigned long long *>(a.cand + r * (int64_t)kCandCap);
   int n = 0;
   unsigned long long zin = 0ull, zrest = 0ull;
@@ -412,7 +413,47 @@ __device__ RowFin finish_row_list(const FastArgs &a, int64_t r, FinScratch *fs) 
     out.status = kFinNonfinite;
     return out;
   }
-  if (!a.use_top_p) return out;
+  if (!a.use_window) return out;
+  if (a.top_k > 0) {
+    // top-k: the k-th largest key among the candidates is the row's when
+    // they number at least k (every other element lies below them); else
+    // the whole-row top-k path takes the unit
+    if (n < a.top_k) {
+      out.status = kFinTopK;
+      return out;
+    }
+    const uint32_t kmin = ~kmin_inv;
+    uint32_t lo = kmin, hi = kmax + 1u;  // count(key >= lo) >= k
+    while (hi - lo > 1u) {
+      const uint32_t mid = lo + ((hi - lo) >> 1);
+      int cnt = 0;
+      for (int j = lane; j < n; j += 32) cnt += fs->key[j] >= mid ? 1 : 0;
+      cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
+      if (cnt >= a.top_k) lo = mid;
+      else hi = mid;
+    }
+    const uint32_t tk = lo;
+    unsigned long long zk = 0ull;
+    for (int j = lane; j < n; j += 32)
+      if (fs->key[j] >= tk) zk += fs->m[j];
+    zk = warp_sum_any(zk);
+    uint32_t t = tk;
+    unsigned long long s_at = zk;
+    if (a.use_top_p) {  // top-p of the renormalised top-k distribution
+      unsigned long long target = (unsigned long long)ceil((double)a.s.top_p * (double)zk);
+      if (target == 0ull) target = 1ull;
+      t = suffix_bisect(tk, kmax + 1u, target, s_at, [&](uint32_t mid) {
+        unsigned long long part = 0ull;
+        for (int j = lane; j < n; j += 32)
+          if (fs->key[j] >= mid) part += fs->m[j];
+        return warp_sum_any(part);
+      });
+    }
+    out.zp = (double)s_at / kFix52;
+    out.tau_key = t;
+    out.tau_bits = key_to_bits<Bits>(t);
+    return out;
+  }
   const double target_d = ceil((double)a.s.top_p * Z * kFix52);
   if (!(target_d < 9.2e18) || (double)zin < target_d) {  // (zin < 2^63)
     out.status = kFinCoverage;

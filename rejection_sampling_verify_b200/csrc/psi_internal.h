@@ -126,6 +126,7 @@ struct SampledArgs {
   int32_t N, B, V;
   float temperature;
   float top_p;
+  int32_t top_k;        // 0: off (else 1 <= top_k < V)
   uint64_t seed;
   const uint64_t *seq_ids;
   uint64_t step;
@@ -142,6 +143,14 @@ struct KernelEvents {
   cudaEvent_t before = nullptr;
   cudaEvent_t after = nullptr;
 };
+
+// Whole-row top-k path (psi_topk.cu): one CTA per listed unit (list and
+// count on the device), or per unit of the batch (list == nullptr), records
+// written; `max_ctas` caps the grid.
+cudaError_t launch_topk_units(const SampledArgs &a, psi_dtype dtype, const int32_t *list,
+                              const int32_t *count, int64_t max_ctas, cudaStream_t stream);
+// The emit step of the general path (records -> tokens), one thread per sequence.
+cudaError_t launch_sampled_emit(const SampledArgs &a, cudaStream_t stream);
 
 // General path: one cluster per unit for every unit, then the emit kernel.
 cudaError_t launch_sampled(const SampledArgs &a, psi_dtype dtype, const SampledPlan &plan,
@@ -202,7 +211,7 @@ ScanGeom plan_scan(int32_t V, int elem_bytes);
 
 struct FastLayout {  // workspace carve-up of the streaming path
   size_t rec_off, srec_off, cand_off, known_off, rfin_off, counters_off, list_a_off, list_b_off,
-      list_d_off,
+      list_d_off, list_k_off,
       wide_rows_off, wide_units_off, round_rows_off, round_units_off, active_off, total;
 };
 struct RowFin;  // a finished row (psi_finish.cuh)
@@ -220,6 +229,8 @@ struct FastArgs {
   float win_narrow;    // candidate windows below the row maximum, in logit units
   float win_wide;
   int use_top_p;
+  int use_window;      // top-p or top-k: the scan sets elements near the maximum aside
+  int32_t top_k;       // 0: off
   int pass;            // 1: a first scan / finish; 2: a rescan of rows that failed
   const int32_t *rlist;   // rows to scan (nullptr: every row); entries may carry kWideBit
   const int32_t *rcount;  // their number
@@ -235,10 +246,12 @@ struct FastArgs {
   float *known_max;    // [rows] row maximum found by a first pass (read by a rescan)
   RowFin *rfin;        // [rows] the row finish's results (streaming linear verify)
   int32_t *counters;   // [0] general units, [1] sample-mode units, [2] wide rows, [3] wide units,
-                       // [4 + 2k], [5 + 2k] rows and units of round parity k, [8] draw units
+                       // [4 + 2k], [5 + 2k] rows and units of round parity k, [8] draw units,
+                       // [9] whole-row top-k units
   int32_t *list_a;     // units for the general path
   int32_t *list_b;     // units whose draw needs the whole row
   int32_t *list_d;     // units whose draw is over their p row's nucleus
+  int32_t *list_k;     // units for the whole-row top-k path
   int32_t *wide_rows;  // rows for the second scan (| kWideBit: wide window)
   int32_t *wide_units; // units for the second unit pass
 };

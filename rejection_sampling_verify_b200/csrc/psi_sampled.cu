@@ -864,6 +864,12 @@ cudaError_t launch_sampled(const SampledArgs &a, psi_dtype dtype, const SampledP
   return cudaGetLastError();
 }
 
+cudaError_t launch_sampled_emit(const SampledArgs &a, cudaStream_t stream) {
+  sampled_emit_kernel<<<(a.N + 127) / 128, 128, 0, stream>>>(a.records, a.ids, a.N, a.B,
+                                                             a.out_tokens, a.out_n);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_cluster_list(const SampledArgs &a, psi_dtype dtype, const SampledPlan &plan,
                                 int mode, const int32_t *list, const int32_t *count,
                                 int max_clusters, cudaStream_t stream) {

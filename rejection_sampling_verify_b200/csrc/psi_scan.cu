@@ -458,7 +458,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) row_scan_kernel(const __grid_
         for (int u = 0; u < 4; ++u) acc[u] = make_float2(acc[u].x * f, acc[u].y * f);
         aref = sref;
       }
-      if (a.use_top_p) {
+      if (a.use_window) {
         Threshold th;
         th.pair = sm.stage_thr[slot];
         th.value = sm.stage_thrv[slot];
@@ -631,7 +631,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) row_scan_kernel(const __grid_
       }
       const float shift = (ref == -INFINITY) ? 0.f : -ref * coef;
       const float2 c2 = make_float2(coef, coef), s2 = make_float2(shift, shift);
-      if (a.use_top_p) {
+      if (a.use_window) {
         // the set-aside threshold looks one stage ahead within the row (every
         // warp posted the next stage's maximum when it loaded that stage,
         // which it did before this pass): a higher threshold flags fewer

@@ -444,6 +444,8 @@ cudaError_t launch_tree_sampled(const void *ar, int64_t ar_stride, psi_dtype dty
   if (wlog2 > 20.0) wlog2 = 20.0;
   fa.win_narrow = fa.win_wide = (float)(wlog2 / fa.coef64);
   fa.use_top_p = top_p < 1.0f ? 1 : 0;
+  fa.use_window = fa.use_top_p;
+  fa.top_k = 0;
   fa.pass = 1;
   fa.srec = reinterpret_cast<SliceRecord *>(ws + L.srec_off);
   fa.cand = reinterpret_cast<uint64_t *>(ws + L.cand_off);
