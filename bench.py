@@ -233,6 +233,10 @@ def call_verify(psi, cfg, batch, step, seq_ids, ws, out):
     """One verify step as a server calls it: tokens and counts only (no p / q
     diagnostics), which lets the sampled path read rows in early-exit rounds."""
     if isinstance(cfg, psi_inputs.TreeConfig):
+        if cfg.temperature > 0:
+            return psi.verify_tree_sampled(batch.ar, batch.node_tokens, batch.parents,
+                                           cfg.temperature, cfg.top_p, seed=cfg.seed, step=step,
+                                           workspace=ws, out=out)
         return psi.verify_tree_greedy(batch.ar, batch.node_tokens, batch.parents, workspace=ws,
                                       out=out)
     return psi.verify_linear(batch.ar, batch.draft, batch.ids, cfg.temperature, cfg.top_p,
@@ -301,13 +305,20 @@ def oracle_sample_rate(cfg, batch_cpu, target_seconds, one=None, threads=1):
     if isinstance(cfg, psi_inputs.TreeConfig):
         ar = psi_inputs.to_host_logits(batch_cpu.ar)
         tok, par = batch_cpu.node_tokens.numpy(), batch_cpu.parents.numpy()
+
+        def tree(n):
+            if cfg.temperature > 0:
+                oracle.verify_tree_sampled(ar[:n], tok[:n], par[:n], cfg.temperature, cfg.top_p,
+                                           cfg.seed, 0)
+            else:
+                oracle.verify_tree_greedy(ar[:n], tok[:n], par[:n])
         if one is None:
             t0 = time.perf_counter()
-            oracle.verify_tree_greedy(ar[:1], tok[:1], par[:1])
+            tree(1)
             one = time.perf_counter() - t0
         n = max(1, min(cfg.N, n_have, int(target_seconds / max(one, 1e-6))))
         t0 = time.perf_counter()
-        oracle.verify_tree_greedy(ar[:n], tok[:n], par[:n])
+        tree(n)
         dt = time.perf_counter() - t0
         return n / dt, n, dt
     ar = psi_inputs.to_host_logits(batch_cpu.ar)
@@ -349,7 +360,8 @@ def sample_inputs(cfg, n):
 def config_block(cfg, name, world):
     c = {"workload": name}
     if isinstance(cfg, psi_inputs.TreeConfig):
-        c.update(batch=cfg.N, tree_nodes=cfg.M, vocab=cfg.V, depth=cfg.depth, width=cfg.width)
+        c.update(batch=cfg.N, tree_nodes=cfg.M, vocab=cfg.V, depth=cfg.depth, width=cfg.width,
+                 temperature=cfg.temperature, top_p=cfg.top_p)
     else:
         c.update(batch=cfg.N, block=cfg.B, vocab=cfg.V, temperature=cfg.temperature,
                  top_p=cfg.top_p, logits_dtype=cfg.dtype,
@@ -424,7 +436,11 @@ def main():
     seq_ids = None
     if not is_tree and world > 1:
         seq_ids = torch.arange(rank * cfg.N, (rank + 1) * cfg.N, device=dev, dtype=torch.int64)
-    if is_tree:
+    if is_tree and cfg.temperature > 0:
+        ws_bytes = psi.psi_verify_tree_sampled_workspace_bytes(cfg.N, cfg.M, cfg.V,
+                                                               psi.PSI_DTYPE_BF16,
+                                                               cfg.temperature, cfg.top_p)
+    elif is_tree:
         ws_bytes = psi.psi_verify_tree_greedy_workspace_bytes(cfg.N, cfg.M, cfg.V,
                                                               psi.PSI_DTYPE_BF16)
     else:
@@ -491,8 +507,10 @@ def main():
         read = rows_read(cfg, out.n_emitted.cpu().numpy()) * cfg.V * es
     peak, peak_kind = hbm_peak()
     achieved = alg / (main_ms / 1000.0) / 1e9
-    kernel = "psi_tree_argmax" if is_tree else (
-        "psi_row_scan" if cfg.temperature > 0 else "psi_row_argmax")
+    if is_tree:
+        kernel = "psi_row_scan" if cfg.temperature > 0 else "psi_tree_argmax"
+    else:
+        kernel = "psi_row_scan" if cfg.temperature > 0 else "psi_row_argmax"
 
     # end to end through the public API with host buffers
     e2e = None
@@ -520,7 +538,7 @@ def main():
         # nucleus draw
         rounds = 0 if is_tree else len(sampled_rounds(cfg))
         if is_tree or (cfg.temperature == 0 and cfg.N < 64):
-            launches_per_step = 2
+            launches_per_step = 2  # tree: argmax + walk, or row scan + sampled walk
         elif cfg.temperature == 0:  # per round: list building and argmax; then emit
             launches_per_step = 2 * rounds + 1
         elif cfg.N < 64:  # one pass: scan, finish, unit, their second passes, lists, emit, draw

@@ -61,6 +61,8 @@ class TreeConfig:
     seed: int
     steps: int
     iid: bool = False
+    temperature: float = 0.0   # > 0: the sampled tree verify
+    top_p: float = 1.0
 
 
 CONFIGS = {
@@ -72,6 +74,9 @@ CONFIGS = {
     "max_batch_greedy": LinearConfig("max_batch_greedy", 1024, 16, V_QWEN3, "bf16",
                                      0.0, 1.0, 3, 50, "zipf", 0.6),
     "tree_greedy": TreeConfig("tree_greedy", 16, 64, V_QWEN3, 8, 4, 4, 500),
+    # the same trees and logits, verified by the sampled tree rule
+    "tree_sampled": TreeConfig("tree_sampled", 16, 64, V_QWEN3, 8, 4, 4, 500,
+                               temperature=0.7, top_p=0.95),
 }
 
 
