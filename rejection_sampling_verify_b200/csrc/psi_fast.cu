@@ -497,6 +497,25 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
 
 }  // namespace
 
+cudaError_t launch_row_finish(const FastArgs &fa, psi_dtype dtype, cudaStream_t stream) {
+  const int64_t grid = std::min<int64_t>((fa.rows + kFinishWarps - 1) / kFinishWarps,
+                                         (int64_t)sm_count() * 8);
+  if (dtype == PSI_DTYPE_BF16) {
+    static DeviceOnce configure;
+    cudaError_t e = configure([] { return prefer_max_shared(row_finish_kernel<uint16_t>); });
+    if (e != cudaSuccess) return e;
+    row_finish_kernel<uint16_t><<<(unsigned)std::max<int64_t>(grid, 1), 32 * kFinishWarps, 0,
+                                  stream>>>(fa);
+  } else {
+    static DeviceOnce configure;
+    cudaError_t e = configure([] { return prefer_max_shared(row_finish_kernel<uint32_t>); });
+    if (e != cudaSuccess) return e;
+    row_finish_kernel<uint32_t><<<(unsigned)std::max<int64_t>(grid, 1), 32 * kFinishWarps, 0,
+                                  stream>>>(fa);
+  }
+  return cudaGetLastError();
+}
+
 FastLayout fast_layout(int32_t N, int32_t B) {
   FastLayout L;
   const int64_t units = (int64_t)N * (B + 1);

@@ -261,12 +261,16 @@ constexpr int32_t kWideBit = int32_t(1) << 30;  // second-pass row entry: wide w
 // candidate lists.  `clusters_hint` caps the number of clusters launched.
 cudaError_t launch_row_scan(const FastArgs &fa, psi_dtype dtype, cudaStream_t stream);
 
+// The row finish over the listed rows (or every row): one warp per row,
+// results to fa.rfin, candidates compacted in place (psi_fast.cu).
+cudaError_t launch_row_finish(const FastArgs &fa, psi_dtype dtype, cudaStream_t stream);
+
 cudaError_t launch_sampled_fast(const SampledArgs &a, psi_dtype dtype, const SampledPlan &plan,
                                 void *workspace, const KernelEvents &ev, cudaStream_t stream);
 
 // ---- sampled tree (psi_tree.cu) -------------------------------------------------
 struct TreeLayout {  // workspace: the row scan's records and candidate lists
-  size_t srec_off, cand_off, known_off, total;
+  size_t srec_off, cand_off, known_off, rfin_off, total;
 };
 TreeLayout tree_layout(int32_t N, int32_t M);
 cudaError_t launch_tree_sampled(const void *ar, int64_t ar_stride, psi_dtype dtype,

@@ -21,11 +21,11 @@
 // node's row (0 for the root).
 //
 // Kernels: the streaming row scan over every node row (psi_scan.cu) leaves
-// each row's maximum, sum and candidates; then one CTA per tree walks the
-// path.  It finishes each visited row from its records (psi_finish.cuh:
-// exact double masses of the candidates, top-p threshold by an exact integer
-// search), evaluates the children in double precision, and draws over the
-// nucleus.  A row whose top-p set the candidate list cannot settle, and the
+// each row's maximum, sum and candidates; the row finish (psi_finish.cuh, one
+// warp per row, all rows at once) turns them into the row's maximum, top-p
+// threshold and renormaliser (exact double masses, integer searches); then
+// one CTA per tree walks the path, evaluates the children in double
+// precision, and draws over the nucleus.  A row whose top-p set the candidate list cannot settle, and the
 // draw when top-p is off (the whole vocabulary), take an exact whole-row path:
 // the CTA re-reads the row (usually from L2) with double-precision masses in
 // 2^40 fixed point (order-free integer sums).
@@ -208,9 +208,16 @@ __global__ void __launch_bounds__(kTreeThreads) tree_sampled_kernel(
     const int64_t r = (int64_t)n * (M + 1) + node + 1;
     const Bits *row = static_cast<const Bits *>(a.s.ar) + r * a.s.ar_stride;
     if (scanned) {
-      if (warp == 0) {
-        const RowFinal f = finish_row<Bits>(a, r, &sh.ws);
-        if (lane == 0) sh.fin = f;
+      if (tid == 0) {
+        const RowFin rf = a.rfin[r];
+        RowFinal f;
+        f.m = rf.m;
+        f.zp = rf.zp;
+        f.tau_bits = rf.tau_bits;
+        f.tau_key = rf.tau_key;
+        f.n = rf.n;
+        f.status = rf.status;
+        sh.fin = f;
       }
     } else {  // rows that could not be scanned: the maximum by a whole-row pass
       int32_t v0, v1;
@@ -334,29 +341,47 @@ __global__ void __launch_bounds__(kTreeThreads) tree_sampled_kernel(
       token = whole_row_draw<Bits>(row, V, fin.m, a.coef64, a.use_top_p ? tau_key : 0u,
                                    sh.removed, nrem, u2, sh);
     } else if (warp == 0) {
-      // over p's nucleus (its candidates with key >= tau): compact index and
-      // mass, remove the rejected tokens, then the integer search
+      // over p's nucleus (the row's candidates, compacted at the front of its
+      // list area by the row finish, with key >= tau): index and exact mass,
+      // remove the rejected tokens, then the integer search
       WarpScratch *ws = &sh.ws;
-      const unsigned below = (1u << lane) - 1u;
+      const unsigned long long *area =
+          reinterpret_cast<const unsigned long long *>(a.cand + r * (int64_t)kCandCap);
       int nn = 0;
-      for (int base = 0; base < fin.n; base += 32) {
-        const int j = base + lane;
-        const bool in = j < fin.n && ws->key[j] >= tau_key;
-        uint32_t v = 0u;
-        uint64_t m = 0ull;
-        if (in) {
-          v = ws->idx[j];
-          m = ws->m[j];
+      for (int base = 0; base < fin.n; base += 32 * kLoadChunk) {
+        unsigned long long e[kLoadChunk];  // loads in flight together
+#pragma unroll
+        for (int h = 0; h < kLoadChunk; ++h) {
+          const int j = base + 32 * h + lane;
+          e[h] = j < fin.n ? __ldcg(area + j) : 0ull;
         }
-        const unsigned bal = __ballot_sync(0xFFFFFFFFu, in);
-        __syncwarp();
-        if (in) {
-          const int d = nn + __popc(bal & below);
-          ws->idx[d] = v;
-          ws->m[d] = m;
+        uint32_t inm = 0u;
+#pragma unroll
+        for (int h = 0; h < kLoadChunk; ++h) {
+          const int j = base + 32 * h + lane;
+          const bool in = j < fin.n && Elem<Bits>::key((uint32_t)(e[h] >> 32)) >= tau_key;
+          inm |= (in ? 1u : 0u) << h;
         }
-        nn += __popc(bal);
+        const int cnt = __popc(inm);
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        int d = nn + incl - cnt;
+        nn += __shfl_sync(0xFFFFFFFFu, incl, 31);
+#pragma unroll
+        for (int h = 0; h < kLoadChunk; ++h)
+          if ((inm >> h) & 1u) {
+            ws->idx[d] = (uint32_t)e[h];
+            ws->m[d] = e[h] >> 32;  // the logit's bits until its mass replaces them
+            ++d;
+          }
       }
+      __syncwarp();
+      for (int j = lane; j < nn; j += 32)
+        ws->m[j] = fixed52(exact_exp2d(Elem<Bits>::to_float((uint32_t)ws->m[j]), fin.m, a.coef64));
       __syncwarp();
       int32_t tkn = 0;
       for (int attempt = 0; attempt < 2; ++attempt) {
@@ -407,6 +432,8 @@ TreeLayout tree_layout(int32_t N, int32_t M) {
   off = align(off + sizeof(uint64_t) * (size_t)rows * kCandCap);
   L.known_off = off;
   off = align(off + sizeof(float) * (size_t)rows);
+  L.rfin_off = off;
+  off = align(off + sizeof(RowFin) * (size_t)rows);
   L.total = off;
   return L;
 }
@@ -450,7 +477,7 @@ cudaError_t launch_tree_sampled(const void *ar, int64_t ar_stride, psi_dtype dty
   fa.srec = reinterpret_cast<SliceRecord *>(ws + L.srec_off);
   fa.cand = reinterpret_cast<uint64_t *>(ws + L.cand_off);
   fa.known_max = reinterpret_cast<float *>(ws + L.known_off);
-  fa.rfin = nullptr;  // the tree walk finishes its rows itself
+  fa.rfin = reinterpret_cast<RowFin *>(ws + L.rfin_off);
   cudaError_t e;
   // the row scan streams 16-byte vectors; rows that do not start on a 16-byte
   // boundary are settled by the walk's exact whole-row path instead
@@ -460,6 +487,8 @@ cudaError_t launch_tree_sampled(const void *ar, int64_t ar_stride, psi_dtype dty
     if (ev.before && (e = cudaEventRecord(ev.before, stream)) != cudaSuccess) return e;
     if ((e = launch_row_scan(fa, dtype, stream)) != cudaSuccess) return e;
     if (ev.after && (e = cudaEventRecord(ev.after, stream)) != cudaSuccess) return e;
+    // every node row finished at once (the walk reads the rows it visits)
+    if ((e = launch_row_finish(fa, dtype, stream)) != cudaSuccess) return e;
   }
   static DeviceOnce configure_bf16, configure_f32;
   const size_t smem = sizeof(TreeShared);
