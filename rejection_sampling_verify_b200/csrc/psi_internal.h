@@ -205,7 +205,8 @@ struct ScanGeom {
   int32_t slices;      // slices per row (CTAs per row)
   int32_t stages;      // shared-memory stages per slice
   int32_t stage_vecs;  // vectors per stage (the last stage of a slice may be shorter)
-  int32_t cap;         // set-aside list capacity per slice (kCandCap / slices)
+  int32_t cap;         // set-aside entries per row (kCandCap): slice 0's list from the
+                       // front of the row's area, slice 1's from its back
 };
 ScanGeom plan_scan(int32_t V, int elem_bytes);
 
@@ -241,7 +242,8 @@ struct FastArgs {
   int32_t *round_units;   // units of the current round
   UnitRecord *rec;     // [N*(B+1)]
   SliceRecord *srec;   // [rows][kMaxSlices]
-  uint64_t *cand;      // [rows][kCandCap]: slice c's set-aside list at c * g.cap;
+  uint64_t *cand;      // [rows][kCandCap]: slice 0's set-aside list at entries 0, 1, ...,
+                       // slice 1's at kCandCap - 1, kCandCap - 2, ...;
                        // (bits << 32) | vocabulary index
   float *known_max;    // [rows] row maximum found by a first pass (read by a rescan)
   RowFin *rfin;        // [rows] the row finish's results (streaming linear verify)
