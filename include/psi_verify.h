@@ -219,8 +219,8 @@ psi_status psi_verify_linear_topk(const void *ar_logits, int64_t ar_row_stride,
  * the caller serialises them (one stream, or events between streams).
  * Returns PSI_ERR_UNSUPPORTED, without launching anything, when
  * psi_verify_linear_workspace_bytes for these sizes exceeds
- * PSI_NOALLOC_SCRATCH_BYTES (the sampled path needs about 32.8 KB per logit
- * row, N * (2B + 1) rows: e.g. N <= 15 at B = 8; the greedy path far less),
+ * PSI_NOALLOC_SCRATCH_BYTES (the sampled path needs about 65.7 KB per logit
+ * row, N * (2B + 1) rows: e.g. N <= 7 at B = 8; the greedy path far less),
  * and PSI_ERR_CUDA if the scratch address cannot be obtained.
  */
 #define PSI_NOALLOC_SCRATCH_BYTES 8388608u /* 8 MiB */

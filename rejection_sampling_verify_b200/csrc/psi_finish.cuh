@@ -149,13 +149,10 @@ __device__ RowFin finish_row_list(const FastArgs &a, int64_t r, FinScratch *fs) 
   const SliceRecord *sr = a.srec + r * kMaxSlices;
   float M = -INFINITY;
   bool lost = false;
-  int n_all = 0;
   for (int c = 0; c < C; ++c) {
     M = fmaxf(M, sr[c].m);
-    lost |= (sr[c].flags & kRowLost) != 0;
-    n_all += sr[c].n_cand;
+    lost |= (sr[c].flags & kRowLost) != 0 || sr[c].n_cand > a.g.cap;
   }
-  lost |= n_all > a.g.cap;  // the two lists met in the row's area
   out.m = M;
   if (lost) {
     out.status = kFinOverflow;
@@ -175,8 +172,7 @@ __device__ RowFin finish_row_list(const FastArgs &a, int64_t r, FinScratch *fs) 
   uint32_t kmax = 0u, kmin_inv = 0u;
   for (int c = 0; c < C; ++c) {
     const int nc = sr[c].n_cand;
-    // slice 1's list fills the area from its back: read it upwards
-    const unsigned long long *src = c == 0 ? area : area + (a.g.cap - nc);
+    const unsigned long long *src = area + (int64_t)c * a.g.cap;
     unsigned long long e[kLoadChunk], nx[kLoadChunk];
 #pragma unroll
     for (int h = 0; h < kLoadChunk; ++h) {
@@ -187,7 +183,7 @@ __device__ RowFin finish_row_list(const FastArgs &a, int64_t r, FinScratch *fs) 
 #pragma unroll
       for (int h = 0; h < kLoadChunk; ++h) e[h] = nx[h];
       // the next chunk's loads go out before this chunk is sorted (none of
-      // them is overwritten: candidates land at or below the entries read)
+      // them is overwritten: candidates land below base + 32 * kLoadChunk)
 #pragma unroll
       for (int h = 0; h < kLoadChunk; ++h) {
         const int j = base + 32 * (kLoadChunk + h) + lane;
@@ -208,8 +204,7 @@ __device__ RowFin finish_row_list(const FastArgs &a, int64_t r, FinScratch *fs) 
         zrest += fixed52_f32(mf);
       }
       // this lane's candidates go to positions n + (candidates of lower
-      // lanes) + k: below every entry not yet read (at most the entries read
-      // so far precede them, and slice 1's list starts at g.cap - n1 >= n0)
+      // lanes) + k: below every entry not yet read
       const int cnt = __popc(cmask);
       int incl = cnt;
 #pragma unroll

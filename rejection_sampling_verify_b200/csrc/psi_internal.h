@@ -182,7 +182,7 @@ struct SliceRecord {
   double z;        // sum over the slice's other elements of exp2((x - m) * log2(e) / T)
 };
 constexpr int32_t kRowLost = 1;
-constexpr int kCandCap = 4096;   // set-aside elements kept per row (global workspace), split over slices
+constexpr int kCandCap = 8192;   // set-aside elements kept per row (global workspace), split over slices
 constexpr int kFinishCap = 2048; // candidates the finish holds per row
 constexpr int kMaxSlices = 2;    // slice records reserved per row (slices per row at most)
 
@@ -205,8 +205,7 @@ struct ScanGeom {
   int32_t slices;      // slices per row (CTAs per row)
   int32_t stages;      // shared-memory stages per slice
   int32_t stage_vecs;  // vectors per stage (the last stage of a slice may be shorter)
-  int32_t cap;         // set-aside entries per row (kCandCap): slice 0's list from the
-                       // front of the row's area, slice 1's from its back
+  int32_t cap;         // set-aside list capacity per slice (kCandCap / slices)
 };
 ScanGeom plan_scan(int32_t V, int elem_bytes);
 
@@ -242,8 +241,7 @@ struct FastArgs {
   int32_t *round_units;   // units of the current round
   UnitRecord *rec;     // [N*(B+1)]
   SliceRecord *srec;   // [rows][kMaxSlices]
-  uint64_t *cand;      // [rows][kCandCap]: slice 0's set-aside list at entries 0, 1, ...,
-                       // slice 1's at kCandCap - 1, kCandCap - 2, ...;
+  uint64_t *cand;      // [rows][kCandCap]: slice c's set-aside list at c * g.cap;
                        // (bits << 32) | vocabulary index
   float *known_max;    // [rows] row maximum found by a first pass (read by a rescan)
   RowFin *rfin;        // [rows] the row finish's results (streaming linear verify)

@@ -448,7 +448,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) row_scan_kernel(const __grid_
       const float sref = sm.stage_ref[slot];
       if (k == 0) {
         r = sm.stage_row[slot];
-        list = a.cand + r * (int64_t)kCandCap;
+        list = a.cand + r * (int64_t)kCandCap + (int64_t)c * g.cap;
         aref = sref;
 #pragma unroll
         for (int u = 0; u < 4; ++u) acc[u] = make_float2(0.f, 0.f);
@@ -493,8 +493,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) row_scan_kernel(const __grid_
             for (int e = 0; e < VEC; ++e) {
               const int p = pos + __popc(em & ((1u << e) - 1u));
               if (((em >> e) & 1u) && p < g.cap)
-                list[c == 0 ? p : g.cap - 1 - p] =
-                    ((uint64_t)vec_elem<Bits>(v, e) << 32) | (idx0 + (uint32_t)e);
+                list[p] = ((uint64_t)vec_elem<Bits>(v, e) << 32) | (idx0 + (uint32_t)e);
             }
           }
         }
@@ -528,8 +527,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) row_scan_kernel(const __grid_
                                           : (uint32_t)Elem<Bits>::kNegInf;
           const float mc = fmaxf(sref, warp_max(Elem<Bits>::to_float(tbits)));  // slice maximum
           if (has_tail && n_list + lane < g.cap)
-            list[c == 0 ? n_list + lane : g.cap - 1 - (n_list + lane)] =
-                ((uint64_t)tbits << 32) | (uint32_t)(g.nvec * VEC + lane);
+            list[n_list + lane] = ((uint64_t)tbits << 32) | (uint32_t)(g.nvec * VEC + lane);
           if (c == C - 1) n_list += g.tail;
           __syncwarp();
           if (lane == 0) {
@@ -767,9 +765,7 @@ ScanGeom plan_scan(int32_t V, int elem_bytes) {
   const int32_t per = (g.nvec + g.slices - 1) / g.slices;
   g.stages = std::max<int32_t>(1, (per + kStageVecs - 1) / kStageVecs);
   g.stage_vecs = std::min<int32_t>(per, kStageVecs);  // full stages, then the rest
-  // the row's set-aside area is shared: slice 0 fills it from the front,
-  // slice 1 from the back (the row is lost only when together they overflow)
-  g.cap = kCandCap;
+  g.cap = kCandCap / g.slices;
   return g;
 }
 
