@@ -415,14 +415,18 @@ __global__ void __launch_bounds__(kThreads) sampled_unit_kernel(SampledArgs a, S
     double zhi = 0.0;
     unsigned long long zwin = 0ull;
     if (!use_top_p) {
-      // without top-p, Z normalises the whole-row draw: every exponential in
-      // double precision
+      // without top-p, Z normalises the whole-row draw: fp32 exponentials,
+      // summed in fp32 per vector and in double per thread (the streaming
+      // path's Z has the same fp32 accuracy)
       if (m > -INFINITY)
         for (int32_t j = tid; j < nvp; j += kThreads) {
           const uint4 w = src[j];
+          float part = 0.f;
 #pragma unroll
           for (int k = 0; k < VEC; ++k)
-            zhi += exact_exp2(Elem<Bits>::to_float(vec_elem<Bits>(w, k)), m, coef64);
+            part += fast_exp2(fmaf(Elem<Bits>::to_float(vec_elem<Bits>(w, k)), coef,
+                                   r == 0 ? shift_p : shift_q));
+          zhi += (double)part;
         }
     } else {
       for (int32_t j = tid; j < nvp; j += kThreads) {
@@ -606,20 +610,23 @@ __global__ void __launch_bounds__(kThreads) sampled_unit_kernel(SampledArgs a, S
     atomicOr(a.dev_status, (bad ? PSI_DEV_NONFINITE : 0u) | (timed_out ? PSI_DEV_TIMEOUT : 0u));
 
   // ---- 6. correction (rejected row) or bonus (row B) draw -------------------
-  // Weights w(v) = max(0, p(v) - q(v)) or p(v), in double precision and
-  // 2^40 fixed point (exact integer sums in any order); inverse CDF in
-  // vocabulary order: the first v whose running sum exceeds
-  // t = floor(u' * sum(w)).
+  // Weights w(v) = max(0, p(v) - q(v)) or p(v), from fp32 exponentials (the
+  // draw's CDF is then within ~1e-7 of the exact one, far inside the
+  // near-tie margin), in 2^40 fixed point (exact integer sums in any
+  // order); inverse CDF in vocabulary order: the first v whose running sum
+  // exceeds t = floor(u' * sum(w)).  Every pass uses this same function.
+  const float inv_zp = zp_p > 0.0 ? (float)(1.0 / zp_p) : 0.f;
+  const float inv_zq = zp_q > 0.0 ? (float)(1.0 / zp_q) : 0.f;
   auto weight = [&](uint32_t bp, uint32_t bq, bool p_only) -> unsigned long long {
     const float xp = Elem<Bits>::to_float(bp);
     if (!(xp >= tau_p) || !(zp_p > 0.0)) return 0ull;
-    double pv = exact_exp2(xp, m_p, coef64) / zp_p;
+    float pv = fast_exp2(fmaf(xp, coef, shift_p)) * inv_zp;
     if (!p_only) {
       const float xq = Elem<Bits>::to_float(bq);
-      const double qv = (xq >= tau_q && zp_q > 0.0) ? exact_exp2(xq, m_q, coef64) / zp_q : 0.0;
+      const float qv = (xq >= tau_q) ? fast_exp2(fmaf(xq, coef, shift_q)) * inv_zq : 0.f;
       pv = pv - qv;
     }
-    return pv > 0.0 ? __double2ull_rn(fmin(pv, 1.0) * kFixScaleD) : 0ull;
+    return pv > 0.f ? __float2ull_rn(fminf(pv, 1.f) * kFixScale) : 0ull;
   };
   if (bc.need_sample) {
     for (int attempt = 0; attempt < 2; ++attempt) {
