@@ -54,21 +54,17 @@ constexpr float kWindowBaseLog2 = 13.f;
 constexpr float kWindowWideLog2 = 20.f;
 
 // ---------------------------------------------------------------------------
-// row_finish: one warp per listed row
+// row_finish: one CTA per listed row
 // ---------------------------------------------------------------------------
-constexpr int kFinishWarps = 1;
-
 template <typename Bits>
-__global__ void __launch_bounds__(32 * kFinishWarps) row_finish_kernel(const __grid_constant__ FastArgs a) {
-  __shared__ FinScratch fsm[kFinishWarps];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+__global__ void __launch_bounds__(kFinThreads) row_finish_kernel(const __grid_constant__ FastArgs a) {
+  __shared__ FinShared fsh;
   const int64_t R = a.rlist ? (int64_t)*a.rcount : a.rows;
-  for (int64_t item = (int64_t)blockIdx.x * kFinishWarps + warp; item < R;
-       item += (int64_t)gridDim.x * kFinishWarps) {
+  for (int64_t item = blockIdx.x; item < R; item += gridDim.x) {
     const int64_t r = a.rlist ? (int64_t)(a.rlist[item] & ~kWideBit) : item;
-    const RowFin f = finish_row_list<Bits>(a, r, &fsm[warp]);
-    if (lane == 0) a.rfin[r] = f;
-    __syncwarp();
+    const RowFin f = finish_row_cta<Bits>(a, r, fsh);
+    if (threadIdx.x == 0) a.rfin[r] = f;
+    __syncthreads();  // the shared lists are rewritten for the next row
   }
 }
 
@@ -421,8 +417,7 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
   const int64_t persistent = (int64_t)sm_count() * 8;
   const int64_t grid_unit = std::min<int64_t>((units + kUnitThreads - 1) / kUnitThreads, persistent);
   const int64_t grid_draw = std::min<int64_t>(fa.s.N, persistent);
-  const int64_t grid_finish =
-      std::min<int64_t>((fa.rows + kFinishWarps - 1) / kFinishWarps, persistent);
+  const int64_t grid_finish = std::min<int64_t>(fa.rows, (int64_t)sm_count() * 8);
   cudaError_t e;
   static DeviceOnce configure;  // carveouts, once per device
   e = configure([] {
@@ -444,7 +439,7 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
         cudaSuccess)
       return err;
     if (timed && ev.after && (err = cudaEventRecord(ev.after, stream)) != cudaSuccess) return err;
-    row_finish_kernel<Bits><<<(unsigned)grid_finish, 32 * kFinishWarps, 0, stream>>>(f);
+    row_finish_kernel<Bits><<<(unsigned)grid_finish, kFinThreads, 0, stream>>>(f);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     unit_kernel<Bits><<<(unsigned)grid_unit, kUnitThreads, 0, stream>>>(f);
     return cudaGetLastError();
@@ -498,20 +493,19 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
 }  // namespace
 
 cudaError_t launch_row_finish(const FastArgs &fa, psi_dtype dtype, cudaStream_t stream) {
-  const int64_t grid = std::min<int64_t>((fa.rows + kFinishWarps - 1) / kFinishWarps,
-                                         (int64_t)sm_count() * 8);
+  const int64_t grid = std::min<int64_t>(fa.rows, (int64_t)sm_count() * 8);
   if (dtype == PSI_DTYPE_BF16) {
     static DeviceOnce configure;
     cudaError_t e = configure([] { return prefer_max_shared(row_finish_kernel<uint16_t>); });
     if (e != cudaSuccess) return e;
-    row_finish_kernel<uint16_t><<<(unsigned)std::max<int64_t>(grid, 1), 32 * kFinishWarps, 0,
-                                  stream>>>(fa);
+    row_finish_kernel<uint16_t><<<(unsigned)std::max<int64_t>(grid, 1), kFinThreads, 0, stream>>>(
+        fa);
   } else {
     static DeviceOnce configure;
     cudaError_t e = configure([] { return prefer_max_shared(row_finish_kernel<uint32_t>); });
     if (e != cudaSuccess) return e;
-    row_finish_kernel<uint32_t><<<(unsigned)std::max<int64_t>(grid, 1), 32 * kFinishWarps, 0,
-                                  stream>>>(fa);
+    row_finish_kernel<uint32_t><<<(unsigned)std::max<int64_t>(grid, 1), kFinThreads, 0, stream>>>(
+        fa);
   }
   return cudaGetLastError();
 }

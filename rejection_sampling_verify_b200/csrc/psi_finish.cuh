@@ -91,52 +91,82 @@ __device__ __forceinline__ uint64_t fixed52_f32(float m) {
 }
 
 // ---------------------------------------------------------------------------
-// The linear verify's row finish: one warp per row, results to global memory.
+// The row finish: one CTA of kFinWarps warps per row, results to global
+// memory (the row_finish kernel of the linear verify and the tree walk).
 // ---------------------------------------------------------------------------
+constexpr int kFinWarps = 4;
+constexpr int kFinThreads = 32 * kFinWarps;
+constexpr int kFinChunk = 8;  // list entries per lane and chunk (loads in flight together)
 
-struct FinScratch {  // one warp's shared memory: the row's candidates
-  uint32_t key[kFinishCap];
-  unsigned long long m[kFinishCap];
+struct FinShared {
+  unsigned long long e[kFinishCap];  // the candidates' list entries (bits << 32 | index)
+  unsigned long long m[kFinishCap];  // their exact masses, 2^52 fixed point
+  unsigned long long red[kFinWarps][2];
+  uint32_t kred[kFinWarps][2];
+  unsigned long long sv[kFinWarps];  // search: the pivots' values
+  uint32_t sp[kFinWarps];            // search: the pivots
+  int n;                             // candidates found so far
 };
 
-// Largest key t in [lo, hi) whose suffix mass S(t) (every candidate with key
-// >= t) reaches `target`, by bisection on exact integer sums (order-free);
-// S(lo) = s_lo >= target.  `sum_from(mid)` is the warp's S(mid).
-template <typename SumFrom>
-__device__ __forceinline__ uint32_t suffix_bisect(uint32_t lo, uint32_t hi,
-                                                  unsigned long long target,
-                                                  unsigned long long &s_lo, SumFrom sum_from) {
+// Largest t in [lo, hi) with F(t) >= target, for F non-increasing and
+// F(lo) = f_lo >= target, by a 4-ary search: warps 1..3 each evaluate F at one
+// pivot per round (`eval(t)`: the warp's value of F(t), the same in every
+// lane).  Every thread of the CTA takes part; f_lo returns F(t).
+template <typename Eval>
+__device__ uint32_t cta_search(uint32_t lo, uint32_t hi, unsigned long long target,
+                               unsigned long long &f_lo, FinShared &sh, Eval eval) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   while (hi - lo > 1u) {
-    const uint32_t mid = lo + ((hi - lo) >> 1);
-    const unsigned long long part = sum_from(mid);
-    if (part >= target) {
-      lo = mid;
-      s_lo = part;
-    } else {
-      hi = mid;
+    if (warp >= 1) {
+      const uint32_t piv = lo + (uint32_t)(((uint64_t)(hi - lo) * (uint64_t)warp) / kFinWarps);
+      const bool valid = piv > lo;
+      const unsigned long long v = valid ? eval(piv) : 0ull;
+      if (lane == 0) {
+        sh.sv[warp] = v;
+        sh.sp[warp] = valid ? piv : 0u;
+      }
     }
+    __syncthreads();
+    uint32_t nlo = lo, nhi = hi;
+    unsigned long long nf = f_lo;
+    for (int w = 1; w < kFinWarps; ++w) {  // pivots ascend, F descends
+      const uint32_t piv = sh.sp[w];
+      if (piv == 0u || piv <= nlo) continue;
+      if (sh.sv[w] >= target) {
+        nlo = piv;
+        nf = sh.sv[w];
+      } else {
+        nhi = piv;
+        break;
+      }
+    }
+    lo = nlo;
+    hi = nhi;
+    f_lo = nf;
+    __syncthreads();  // the pivots' slots are written again next round
   }
   return lo;
 }
 
 // Row maximum, Z, top-p (and top-k) threshold tau and renormaliser Z' of
-// row r from its slice records and set-aside lists, by one warp.  M is the
+// row r from its slice records and set-aside lists, by one CTA.  M is the
 // largest slice maximum; Z is the slices' sums rescaled to M plus the
 // set-aside masses.  The set-aside elements above the row's final threshold
 // (M - window, rounded as the scan rounds) are the candidates: every element
 // the top-p cut (or a top-k cut that they hold) can keep.  Their masses are
-// exact (double precision, 2^52 fixed point) and they are compacted in place
-// at the front of the row's set-aside area, where the draws read them.  The
-// other set-aside masses (with top-p each under 2^-13 of the maximum's) are
-// taken in fp32, like the slices' sums, and join Z in fixed point; integer
-// sums keep the result independent of the lists' order.  tau is the largest
-// key t whose suffix mass S(t) (every candidate with key >= t) reaches top_p
-// * Z, found by bisection on exact integer sums; with top-k, the k-th largest
-// key t_k comes first (a count bisection) and top-p then cuts the set at or
-// above t_k, whose mass replaces Z.
+// exact (double precision, 2^52 fixed point); they are gathered in shared
+// memory and then written, compacted, to the front of the row's set-aside
+// area, where the draws read them.  The other set-aside masses (with top-p
+// each under 2^-13 of the maximum's) are taken in fp32, like the slices'
+// sums, and join Z in fixed point; integer sums keep the result independent
+// of the lists' order (and of the order in which the warps gather).  tau is
+// the largest key t whose suffix mass S(t) (every candidate with key >= t)
+// reaches top_p * Z, found by a search on exact integer sums; with top-k, the
+// k-th largest key t_k comes first (the same search on counts) and top-p
+// then cuts the set at or above t_k, whose mass replaces Z.
 template <typename Bits>
-__device__ RowFin finish_row_list(const FastArgs &a, int64_t r, FinScratch *fs) {
-  const int lane = threadIdx.x & 31;
+__device__ RowFin finish_row_cta(const FastArgs &a, int64_t r, FinShared &sh) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   RowFin out;
   out.m = -INFINITY;
   out.zp = 0.0;
@@ -149,9 +179,11 @@ __device__ RowFin finish_row_list(const FastArgs &a, int64_t r, FinScratch *fs) 
   const SliceRecord *sr = a.srec + r * kMaxSlices;
   float M = -INFINITY;
   bool lost = false;
+  int nc[kMaxSlices] = {};
   for (int c = 0; c < C; ++c) {
     M = fmaxf(M, sr[c].m);
     lost |= (sr[c].flags & kRowLost) != 0 || sr[c].n_cand > a.g.cap;
+    nc[c] = sr[c].n_cand;
   }
   out.m = M;
   if (lost) {
@@ -167,94 +199,95 @@ __device__ RowFin finish_row_list(const FastArgs &a, int64_t r, FinScratch *fs) 
   }
   const float thr = a.use_window ? threshold_value<Bits>(M - sr[0].off) : INFINITY;
   unsigned long long *area = reinterpret_cast<unsigned long long *>(a.cand + r * (int64_t)kCandCap);
-  int n = 0;
-  unsigned long long zin = 0ull, zrest = 0ull;
-  uint32_t kmax = 0u, kmin_inv = 0u;
-  for (int c = 0; c < C; ++c) {
-    const int nc = sr[c].n_cand;
+  if (tid == 0) sh.n = 0;
+  __syncthreads();
+  // ---- sort the lists: chunks of 32 * kFinChunk entries, dealt to the warps
+  constexpr int kChunkEntries = 32 * kFinChunk;
+  const int q0 = (nc[0] + kChunkEntries - 1) / kChunkEntries;
+  const int q1 = C > 1 ? (nc[1] + kChunkEntries - 1) / kChunkEntries : 0;
+  unsigned long long zrest = 0ull;
+  for (int q = warp; q < q0 + q1; q += kFinWarps) {
+    const int c = q < q0 ? 0 : 1;
+    const int base = (q < q0 ? q : q - q0) * kChunkEntries;
     const unsigned long long *src = area + (int64_t)c * a.g.cap;
-    unsigned long long e[kLoadChunk], nx[kLoadChunk];
+    unsigned long long e[kFinChunk];
 #pragma unroll
-    for (int h = 0; h < kLoadChunk; ++h) {
-      const int j = 32 * h + lane;
-      nx[h] = j < nc ? __ldcg(src + j) : 0ull;
+    for (int h = 0; h < kFinChunk; ++h) {
+      const int j = base + 32 * h + lane;
+      e[h] = j < nc[c] ? __ldcg(src + j) : 0ull;
     }
-    for (int base = 0; base < nc; base += 32 * kLoadChunk) {
+    uint32_t cmask = 0u;  // bit h: entry h is a candidate
 #pragma unroll
-      for (int h = 0; h < kLoadChunk; ++h) e[h] = nx[h];
-      // the next chunk's loads go out before this chunk is sorted (none of
-      // them is overwritten: candidates land below base + 32 * kLoadChunk)
+    for (int h = 0; h < kFinChunk; ++h) {
+      const int j = base + 32 * h + lane;
+      const float x = Elem<Bits>::to_float((uint32_t)(e[h] >> 32));
+      const bool live = j < nc[c];
+      const bool cand = live && x > thr;
+      cmask |= (cand ? 1u : 0u) << h;
+      const float mf = (live && !cand) ? fast_exp2((x - M) * a.coef) : 0.f;  // <= 1
+      zrest += fixed52_f32(mf);
+    }
+    const int cnt = __popc(cmask);
+    int incl = cnt;
 #pragma unroll
-      for (int h = 0; h < kLoadChunk; ++h) {
-        const int j = base + 32 * (kLoadChunk + h) + lane;
-        nx[h] = j < nc ? __ldcg(src + j) : 0ull;
-      }
-      __syncwarp();  // every entry of the chunk is read before any is overwritten
-      // sort the chunk: the other entries' masses (fp32) join zrest at
-      // once; candidates are compacted, their masses taken afterwards
-      uint32_t cmask = 0u;  // bit h: entry h is a candidate
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int base_d = 0;
+    if (lane == 31) base_d = atomicAdd(&sh.n, incl);
+    int d = __shfl_sync(0xFFFFFFFFu, base_d, 31) + incl - cnt;
 #pragma unroll
-      for (int h = 0; h < kLoadChunk; ++h) {
-        const int j = base + 32 * h + lane;
-        const float x = Elem<Bits>::to_float((uint32_t)(e[h] >> 32));
-        const bool live = j < nc;
-        const bool cand = live && x > thr;
-        cmask |= (cand ? 1u : 0u) << h;
-        const float mf = (live && !cand) ? fast_exp2((x - M) * a.coef) : 0.f;  // <= 1
-        zrest += fixed52_f32(mf);
-      }
-      // this lane's candidates go to positions n + (candidates of lower
-      // lanes) + k: below every entry not yet read
-      const int cnt = __popc(cmask);
-      int incl = cnt;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      int d = n + incl - cnt;
-      n += __shfl_sync(0xFFFFFFFFu, incl, 31);
-      while (cmask) {
-        const int h = __ffs(cmask) - 1;
-        cmask &= cmask - 1u;
-        if (d < kFinishCap) {
-          unsigned long long eh = 0ull;
-#pragma unroll
-          for (int q = 0; q < kLoadChunk; ++q) eh = q == h ? e[q] : eh;
-          const uint32_t b = (uint32_t)(eh >> 32);
-          const uint32_t key = Elem<Bits>::key(b);
-          area[d] = eh;
-          fs->key[d] = key;
-          fs->m[d] = b;  // the logit's bits until its mass replaces them
-          kmax = max(kmax, key);
-          kmin_inv = max(kmin_inv, ~key);
-        }
+    for (int h = 0; h < kFinChunk; ++h)
+      if ((cmask >> h) & 1u) {
+        if (d < kFinishCap) sh.e[d] = e[h];
         ++d;
       }
-    }
   }
-  // the candidates' masses, exact in double (independent iterations)
-  __syncwarp();
+  __syncthreads();
+  const int n = sh.n;
+  // ---- the candidates: exact masses, the compacted list to the area (every
+  // list entry has been read), key range
+  unsigned long long zin = 0ull;
+  uint32_t kmax = 0u, kmin_inv = 0u;
   if (n <= kFinishCap) {
-#pragma unroll 4
-    for (int j = lane; j < n; j += 32) {
-      const unsigned long long m52 =
-          fixed52(exact_exp2d(Elem<Bits>::to_float((uint32_t)fs->m[j]), M, a.coef64));
-      fs->m[j] = m52;
+    for (int j = tid; j < n; j += kFinThreads) {
+      const unsigned long long ej = sh.e[j];
+      const uint32_t b = (uint32_t)(ej >> 32);
+      const unsigned long long m52 = fixed52(exact_exp2d(Elem<Bits>::to_float(b), M, a.coef64));
+      sh.m[j] = m52;
       zin += m52;
+      area[j] = ej;
+      const uint32_t key = Elem<Bits>::key(b);
+      kmax = max(kmax, key);
+      kmin_inv = max(kmin_inv, ~key);
     }
   }
-  __syncwarp();
+  zin = warp_sum_any(zin);
+  zrest = warp_sum_any(zrest);
+  kmax = warp_max_u32(kmax);
+  kmin_inv = warp_max_u32(kmin_inv);
+  if (lane == 0) {
+    sh.red[warp][0] = zin;
+    sh.red[warp][1] = zrest;
+    sh.kred[warp][0] = kmax;
+    sh.kred[warp][1] = kmin_inv;
+  }
+  __syncthreads();
+  zin = zrest = 0ull;
+  kmax = kmin_inv = 0u;
+#pragma unroll
+  for (int w = 0; w < kFinWarps; ++w) {
+    zin += sh.red[w][0];
+    zrest += sh.red[w][1];
+    kmax = max(kmax, sh.kred[w][0]);
+    kmin_inv = max(kmin_inv, sh.kred[w][1]);
+  }
   if (n > kFinishCap) {  // more candidates than the area holds: rescan, then the general path
     out.status = kFinOverflow;
     return out;
   }
   out.n = n;
-  kmax = warp_max_u32(kmax);
-  kmin_inv = warp_max_u32(kmin_inv);
-  zin = warp_sum_any(zin);
-  zrest = warp_sum_any(zrest);
-  __syncwarp();
   Z += ((double)zin + (double)zrest) / kFix52;
   out.zp = Z;
   if (!(Z < INFINITY)) {
@@ -262,6 +295,20 @@ __device__ RowFin finish_row_list(const FastArgs &a, int64_t r, FinScratch *fs) 
     return out;
   }
   if (!a.use_window) return out;
+  const uint32_t kmin = ~kmin_inv;
+  // the warp's suffix mass (or count) at key t
+  auto mass_from = [&](uint32_t t) -> unsigned long long {
+    unsigned long long part = 0ull;
+    for (int j = lane; j < n; j += 32)
+      if (Elem<Bits>::key((uint32_t)(sh.e[j] >> 32)) >= t) part += sh.m[j];
+    return warp_sum_any(part);
+  };
+  auto count_from = [&](uint32_t t) -> unsigned long long {
+    int cnt = 0;
+    for (int j = lane; j < n; j += 32)
+      cnt += Elem<Bits>::key((uint32_t)(sh.e[j] >> 32)) >= t ? 1 : 0;
+    return (unsigned long long)__reduce_add_sync(0xFFFFFFFFu, cnt);
+  };
   if (a.top_k > 0) {
     // top-k: the k-th largest key among the candidates is the row's when
     // they number at least k (every other element lies below them); else
@@ -270,32 +317,26 @@ __device__ RowFin finish_row_list(const FastArgs &a, int64_t r, FinScratch *fs) 
       out.status = kFinTopK;
       return out;
     }
-    const uint32_t kmin = ~kmin_inv;
-    uint32_t lo = kmin, hi = kmax + 1u;  // count(key >= lo) >= k
-    while (hi - lo > 1u) {
-      const uint32_t mid = lo + ((hi - lo) >> 1);
-      int cnt = 0;
-      for (int j = lane; j < n; j += 32) cnt += fs->key[j] >= mid ? 1 : 0;
-      cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
-      if (cnt >= a.top_k) lo = mid;
-      else hi = mid;
-    }
-    const uint32_t tk = lo;
+    unsigned long long cnt_lo = (unsigned long long)n;
+    const uint32_t tk =
+        cta_search(kmin, kmax + 1u, (unsigned long long)a.top_k, cnt_lo, sh, count_from);
+    // the mass of the top-k set
     unsigned long long zk = 0ull;
-    for (int j = lane; j < n; j += 32)
-      if (fs->key[j] >= tk) zk += fs->m[j];
+    for (int j = tid; j < n; j += kFinThreads)
+      if (Elem<Bits>::key((uint32_t)(sh.e[j] >> 32)) >= tk) zk += sh.m[j];
     zk = warp_sum_any(zk);
+    __syncthreads();
+    if (lane == 0) sh.red[warp][0] = zk;
+    __syncthreads();
+    zk = 0ull;
+#pragma unroll
+    for (int w = 0; w < kFinWarps; ++w) zk += sh.red[w][0];
     uint32_t t = tk;
     unsigned long long s_at = zk;
     if (a.use_top_p) {  // top-p of the renormalised top-k distribution
       unsigned long long target = (unsigned long long)ceil((double)a.s.top_p * (double)zk);
       if (target == 0ull) target = 1ull;
-      t = suffix_bisect(tk, kmax + 1u, target, s_at, [&](uint32_t mid) {
-        unsigned long long part = 0ull;
-        for (int j = lane; j < n; j += 32)
-          if (fs->key[j] >= mid) part += fs->m[j];
-        return warp_sum_any(part);
-      });
+      t = cta_search(tk, kmax + 1u, target, s_at, sh, mass_from);
     }
     out.zp = (double)s_at / kFix52;
     out.tau_key = t;
@@ -312,32 +353,9 @@ __device__ RowFin finish_row_list(const FastArgs &a, int64_t r, FinScratch *fs) 
     out.status = kFinCoverage;
     return out;
   }
-  // bisection over [kmin, kmax]: S(kmin) = zin reaches the target
+  // search over [kmin, kmax]: S(kmin) = zin reaches the target
   unsigned long long s_at = zin;
-  uint32_t t;
-  if (n <= 32 * kRegCand) {
-    uint32_t kr[kRegCand];  // the row's candidates in registers
-    unsigned long long mr[kRegCand];
-#pragma unroll
-    for (int c = 0; c < kRegCand; ++c) {
-      const int j = lane + 32 * c;
-      kr[c] = j < n ? fs->key[j] : 0u;
-      mr[c] = j < n ? fs->m[j] : 0ull;
-    }
-    t = suffix_bisect(~kmin_inv, kmax + 1u, target, s_at, [&](uint32_t mid) {
-      unsigned long long part = 0ull;
-#pragma unroll
-      for (int c = 0; c < kRegCand; ++c) part += kr[c] >= mid ? mr[c] : 0ull;
-      return warp_sum_any(part);
-    });
-  } else {
-    t = suffix_bisect(~kmin_inv, kmax + 1u, target, s_at, [&](uint32_t mid) {
-      unsigned long long part = 0ull;
-      for (int j = lane; j < n; j += 32)
-        if (fs->key[j] >= mid) part += fs->m[j];
-      return warp_sum_any(part);
-    });
-  }
+  const uint32_t t = cta_search(kmin, kmax + 1u, target, s_at, sh, mass_from);
   out.zp = (double)s_at / kFix52;
   out.tau_key = t;
   out.tau_bits = key_to_bits<Bits>(t);
