@@ -150,6 +150,18 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with the PDL attribute
+// (launch_pdl) may start while the kernel before it on the stream finishes:
+// pdl_wait() returns once that kernel has completed and its memory writes are
+// visible (at once for a kernel launched without the attribute), and
+// pdl_trigger() lets the next kernel on the stream be launched early.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // Shared memory, mbarriers and TMA bulk copies.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {

@@ -58,6 +58,8 @@ constexpr float kWindowWideLog2 = 20.f;
 // ---------------------------------------------------------------------------
 template <typename Bits>
 __global__ void __launch_bounds__(kFinThreads) row_finish_kernel(const __grid_constant__ FastArgs a) {
+  pdl_wait();  // the previous kernel's results are visible
+  pdl_trigger();
   __shared__ FinShared fsh;
   const int64_t R = a.rlist ? (int64_t)*a.rcount : a.rows;
   for (int64_t item = blockIdx.x; item < R; item += gridDim.x) {
@@ -89,6 +91,8 @@ __device__ __forceinline__ RowFin empty_fin() {
 
 template <typename Bits>
 __global__ void __launch_bounds__(kUnitThreads) unit_kernel(const __grid_constant__ FastArgs a) {
+  pdl_wait();  // the previous kernel's results are visible
+  pdl_trigger();
   const SampledArgs &s = a.s;
   const int32_t B = s.B, N = s.N, V = s.V;
   const int64_t n_items = a.ulist ? (int64_t)*a.ucount : (int64_t)N * (B + 1);
@@ -177,6 +181,8 @@ struct DrawScratch {  // one warp's shared memory: p's nucleus and its draw weig
 
 template <typename Bits>
 __global__ void __launch_bounds__(32) draw_kernel(const __grid_constant__ FastArgs a) {
+  pdl_wait();  // the previous kernel's results are visible
+  pdl_trigger();
   __shared__ DrawScratch dsm;
   DrawScratch *ds = &dsm;
   const int lane = threadIdx.x & 31;
@@ -327,6 +333,8 @@ __global__ void __launch_bounds__(32) draw_kernel(const __grid_constant__ FastAr
 // fast_emit: one thread per sequence.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) fast_emit_kernel(const __grid_constant__ FastArgs a) {
+  pdl_wait();  // the previous kernel's results are visible
+  pdl_trigger();
   const int32_t n = blockIdx.x * blockDim.x + threadIdx.x;
   const SampledArgs &s = a.s;
   if (n >= s.N) return;
@@ -375,6 +383,8 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) round_advance_kernel(const __grid_constant__ FastArgs a,
                                                             int k) {
+  pdl_wait();  // the previous kernel's results are visible
+  pdl_trigger();
   const int32_t n = blockIdx.x * blockDim.x + threadIdx.x;
   const SampledArgs &s = a.s;
   const int32_t B = s.B, N = s.N;
@@ -439,10 +449,11 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
         cudaSuccess)
       return err;
     if (timed && ev.after && (err = cudaEventRecord(ev.after, stream)) != cudaSuccess) return err;
-    row_finish_kernel<Bits><<<(unsigned)grid_finish, kFinThreads, 0, stream>>>(f);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    unit_kernel<Bits><<<(unsigned)grid_unit, kUnitThreads, 0, stream>>>(f);
-    return cudaGetLastError();
+    if ((err = launch_pdl(row_finish_kernel<Bits>, dim3((unsigned)grid_finish), dim3(kFinThreads),
+                          0, stream, f)) != cudaSuccess)
+      return err;
+    return launch_pdl(unit_kernel<Bits>, dim3((unsigned)grid_unit), dim3(kUnitThreads), 0, stream,
+                      f);
   };
   // the second pass over the rows and units a first pass could not settle
   // (usually none: the CTAs find empty lists and exit)
@@ -458,8 +469,9 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
   } else {
     const int rounds = round_count(fa.s.B, PSI_SAMPLED_SHORT_ROUNDS);
     for (int k = 0; k < rounds; ++k) {
-      round_advance_kernel<<<(fa.s.N + 127) / 128, 128, 0, stream>>>(fa, k);
-      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      if ((e = launch_pdl(round_advance_kernel, dim3((fa.s.N + 127) / 128), dim3(128), 0, stream,
+                          fa, k)) != cudaSuccess)
+        return e;
       FastArgs f1 = fa;
       f1.rlist = fa.round_rows;
       f1.rcount = fa.counters + 4 + 2 * (k & 1);
@@ -481,10 +493,12 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
   e = launch_cluster_list(sa, dt, plan, kClusterModeList, fa.list_a, fa.counters + 0, clusters_a,
                           stream);
   if (e != cudaSuccess) return e;
-  fast_emit_kernel<<<(fa.s.N + 127) / 128, 128, 0, stream>>>(fa);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  draw_kernel<Bits><<<(unsigned)grid_draw, 32, 0, stream>>>(fa);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = launch_pdl(fast_emit_kernel, dim3((fa.s.N + 127) / 128), dim3(128), 0, stream, fa)) !=
+      cudaSuccess)
+    return e;
+  if ((e = launch_pdl(draw_kernel<Bits>, dim3((unsigned)grid_draw), dim3(32), 0, stream, fa)) !=
+      cudaSuccess)
+    return e;
   const int clusters_b = std::min(fa.s.N, kListClusters);
   return launch_cluster_list(sa, dt, plan, kClusterModeSample, fa.list_b, fa.counters + 1,
                              clusters_b, stream);
@@ -498,16 +512,15 @@ cudaError_t launch_row_finish(const FastArgs &fa, psi_dtype dtype, cudaStream_t 
     static DeviceOnce configure;
     cudaError_t e = configure([] { return prefer_max_shared(row_finish_kernel<uint16_t>); });
     if (e != cudaSuccess) return e;
-    row_finish_kernel<uint16_t><<<(unsigned)std::max<int64_t>(grid, 1), kFinThreads, 0, stream>>>(
-        fa);
+    return launch_pdl(row_finish_kernel<uint16_t>, dim3((unsigned)std::max<int64_t>(grid, 1)),
+                      dim3(kFinThreads), 0, stream, fa);
   } else {
     static DeviceOnce configure;
     cudaError_t e = configure([] { return prefer_max_shared(row_finish_kernel<uint32_t>); });
     if (e != cudaSuccess) return e;
-    row_finish_kernel<uint32_t><<<(unsigned)std::max<int64_t>(grid, 1), kFinThreads, 0, stream>>>(
-        fa);
+    return launch_pdl(row_finish_kernel<uint32_t>, dim3((unsigned)std::max<int64_t>(grid, 1)),
+                      dim3(kFinThreads), 0, stream, fa);
   }
-  return cudaGetLastError();
 }
 
 FastLayout fast_layout(int32_t N, int32_t B) {

@@ -2,6 +2,8 @@
 // (launch plans and launchers).  Not part of the public ABI.
 #pragma once
 
+#include <utility>
+
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -218,6 +220,25 @@ struct RowFin;  // a finished row (psi_finish.cuh)
 FastLayout fast_layout(int32_t N, int32_t B);
 // False when the streaming path's row indices would not fit its lists.
 bool fast_path_fits(int32_t N, int32_t B);
+
+// Launch with the programmatic-dependent-launch attribute: the kernel may
+// start while the previous kernel on the stream drains (its pdl_wait() keeps
+// it from reading that kernel's results early).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Everything the streaming path's kernels read.
 struct FastArgs {

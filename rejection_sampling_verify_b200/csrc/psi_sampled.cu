@@ -277,6 +277,8 @@ __global__ void __launch_bounds__(kThreads) sampled_unit_kernel(SampledArgs a, S
                                                                  int use_top_p, int mode,
                                                                  const int32_t *work_list,
                                                                  const int32_t *work_count) {
+  pdl_wait();  // the previous kernel's results are visible
+  pdl_trigger();
   constexpr int VEC = Elem<Bits>::kVec;
   extern __shared__ __align__(128) unsigned char dyn_smem[];
   __shared__ Xchg xc;
@@ -842,13 +844,15 @@ static cudaError_t launch_cluster_kernel(const SampledArgs &a, const SampledPlan
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = plan.smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)plan.cluster;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see launch_pdl
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t e;
   if (ev && ev->before && (e = cudaEventRecord(ev->before, stream)) != cudaSuccess) return e;
   e = cudaLaunchKernelEx(&cfg, kernel, a, plan, c.coef, c.coef64, c.w_min, c.w_narrow,

@@ -350,6 +350,8 @@ __device__ __forceinline__ bool wait_phase(uint64_t *bar, uint32_t parity, int *
 // ---------------------------------------------------------------------------
 template <typename Bits, int C>
 __global__ void __launch_bounds__(kScanThreads, 1) row_scan_kernel(const __grid_constant__ FastArgs a) {
+  pdl_wait();  // the previous kernel's results are visible
+  pdl_trigger();
   constexpr int VEC = Elem<Bits>::kVec;
   constexpr int U = kVecsPerThread;
   extern __shared__ __align__(128) unsigned char scan_dsm[];
@@ -740,8 +742,8 @@ cudaError_t launch_scan_typed(const FastArgs &fa, cudaStream_t stream) {
   // one CTA per SM: groups of C CTAs, each group scanning its rows' C slices
   const int64_t groups =
       std::min<int64_t>(std::max(1, scan_sm_count() / C), std::max<int64_t>(fa.rows, 1));
-  row_scan_kernel<Bits, C><<<(unsigned)(groups * C), kScanThreads, kScanDynSmem, stream>>>(fa);
-  return cudaGetLastError();
+  return launch_pdl(row_scan_kernel<Bits, C>, dim3((unsigned)(groups * C)), dim3(kScanThreads),
+                    kScanDynSmem, stream, fa);
 }
 
 template <typename Bits>

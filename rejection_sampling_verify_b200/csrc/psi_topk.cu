@@ -188,6 +188,8 @@ template <typename Bits>
 __global__ void __launch_bounds__(kTopkThreads) topk_unit_kernel(SampledArgs a, double coef64,
                                                                 const int32_t *list,
                                                                 const int32_t *count) {
+  pdl_wait();  // the previous kernel's results are visible
+  pdl_trigger();
   __shared__ TopkShared sh;
   const int tid = threadIdx.x;
   const int32_t B = a.B, N = a.N, V = a.V;
@@ -302,8 +304,8 @@ template <typename Bits>
 cudaError_t launch_topk_typed(const SampledArgs &a, const int32_t *list, const int32_t *count,
                               int64_t grid, cudaStream_t stream) {
   const double coef64 = 1.4426950408889634 / (double)a.temperature;
-  topk_unit_kernel<Bits><<<(unsigned)grid, kTopkThreads, 0, stream>>>(a, coef64, list, count);
-  return cudaGetLastError();
+  return launch_pdl(topk_unit_kernel<Bits>, dim3((unsigned)grid), dim3(kTopkThreads), 0, stream, a,
+                    coef64, list, count);
 }
 
 }  // namespace

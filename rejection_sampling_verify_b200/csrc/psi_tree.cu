@@ -179,6 +179,8 @@ __global__ void __launch_bounds__(kTreeThreads) tree_sampled_kernel(
     const __grid_constant__ FastArgs a, const int32_t *__restrict__ tok,
     const int32_t *__restrict__ par, int32_t M, int32_t *__restrict__ out_path,
     int32_t *__restrict__ out_len, int32_t *__restrict__ out_tokens, int scanned) {
+  pdl_wait();  // the previous kernel's results are visible
+  pdl_trigger();
   extern __shared__ __align__(16) unsigned char tree_smem[];
   TreeShared &sh = *reinterpret_cast<TreeShared *>(tree_smem);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -498,18 +500,17 @@ cudaError_t launch_tree_sampled(const void *ar, int64_t ar_stride, psi_dtype dty
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     });
     if (e != cudaSuccess) return e;
-    tree_sampled_kernel<uint16_t><<<N, kTreeThreads, smem, stream>>>(
-        fa, node_tokens, parents, M, out_path, out_len, out_tokens, scanned);
+    return launch_pdl(tree_sampled_kernel<uint16_t>, dim3(N), dim3(kTreeThreads), smem, stream, fa,
+                      node_tokens, parents, M, out_path, out_len, out_tokens, scanned);
   } else {
     e = configure_f32([smem] {
       return cudaFuncSetAttribute(tree_sampled_kernel<uint32_t>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     });
     if (e != cudaSuccess) return e;
-    tree_sampled_kernel<uint32_t><<<N, kTreeThreads, smem, stream>>>(
-        fa, node_tokens, parents, M, out_path, out_len, out_tokens, scanned);
+    return launch_pdl(tree_sampled_kernel<uint32_t>, dim3(N), dim3(kTreeThreads), smem, stream, fa,
+                      node_tokens, parents, M, out_path, out_len, out_tokens, scanned);
   }
-  return cudaGetLastError();
 }
 
 }  // namespace psi
