@@ -97,6 +97,8 @@ __global__ void __launch_bounds__(kThreads) row_argmax_kernel(
     const Bits *__restrict__ logits, int64_t row_stride, int32_t V, int32_t splits,
     int32_t chunk, uint64_t *__restrict__ partial, uint32_t *dev_status,
     const int32_t *__restrict__ rlist, const int32_t *__restrict__ rcount) {
+  pdl_wait();  // the previous kernel's results are visible
+  pdl_trigger();
   constexpr int VEC = Elem<Bits>::kVec;
   const int64_t item = blockIdx.x / splits;
   const int32_t s = blockIdx.x % splits;
@@ -166,6 +168,8 @@ __global__ void __launch_bounds__(128) greedy_emit_kernel(
     const uint64_t *__restrict__ partial, int32_t splits, const int32_t *__restrict__ ids,
     int32_t N, int32_t B, int32_t V, int32_t *__restrict__ out_tokens,
     int32_t *__restrict__ out_n, uint32_t *dev_status) {
+  pdl_wait();  // the previous kernel's results are visible
+  pdl_trigger();
   const int32_t n = blockIdx.x * blockDim.x + threadIdx.x;
   if (n >= N) return;
   const int64_t row0 = (int64_t)n * (B + 1);
@@ -192,6 +196,8 @@ __global__ void __launch_bounds__(kThreads) tree_walk_kernel(
     int32_t M, int32_t V, int32_t *__restrict__ out_path_nodes,
     int32_t *__restrict__ out_path_len, int32_t *__restrict__ out_tokens,
     uint32_t *dev_status) {
+  pdl_wait();  // the previous kernel's results are visible
+  pdl_trigger();
   extern __shared__ int32_t sm[];
   int32_t *am = sm;              // [M+1]
   int32_t *tok = am + (M + 1);   // [M]
@@ -282,15 +288,14 @@ cudaError_t launch_row_argmax(const void *logits, int64_t row_stride, psi_dtype 
                               uint64_t *partial, uint32_t *dev_status, cudaStream_t stream) {
   const int64_t grid = rows * plan.splits;
   if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+  const int32_t *no_list = nullptr;
   if (dtype == PSI_DTYPE_BF16)
-    row_argmax_kernel<uint16_t><<<(unsigned)grid, kThreads, 0, stream>>>(
-        static_cast<const uint16_t *>(logits), row_stride, V, plan.splits, plan.chunk, partial,
-        dev_status, nullptr, nullptr);
-  else
-    row_argmax_kernel<uint32_t><<<(unsigned)grid, kThreads, 0, stream>>>(
-        static_cast<const uint32_t *>(logits), row_stride, V, plan.splits, plan.chunk, partial,
-        dev_status, nullptr, nullptr);
-  return cudaGetLastError();
+    return launch_pdl(row_argmax_kernel<uint16_t>, dim3((unsigned)grid), dim3(kThreads), 0, stream,
+                      static_cast<const uint16_t *>(logits), row_stride, V, plan.splits,
+                      plan.chunk, partial, dev_status, no_list, no_list);
+  return launch_pdl(row_argmax_kernel<uint32_t>, dim3((unsigned)grid), dim3(kThreads), 0, stream,
+                    static_cast<const uint32_t *>(logits), row_stride, V, plan.splits, plan.chunk,
+                    partial, dev_status, no_list, no_list);
 }
 
 GreedyLayout greedy_layout(int32_t N, int32_t B, int32_t V, int elem_bytes) {
@@ -316,6 +321,8 @@ GreedyLayout greedy_layout(int32_t N, int32_t B, int32_t V, int elem_bytes) {
 __global__ void __launch_bounds__(128) greedy_advance_kernel(
     const uint64_t *__restrict__ partial, int32_t splits, const int32_t *__restrict__ ids,
     int32_t N, int32_t B, int k, int32_t *active, int32_t *round_rows, int32_t *counters) {
+  pdl_wait();  // the previous kernel's results are visible
+  pdl_trigger();
   const int32_t n = blockIdx.x * blockDim.x + threadIdx.x;
   if (n == 0) counters[(k + 1) & 1] = 0;  // the next round's list
   if (n >= N) return;
@@ -354,19 +361,21 @@ cudaError_t launch_greedy_early_exit(const void *logits, int64_t row_stride, psi
                          (round_begin(k + 1, B, PSI_GREEDY_SHORT_ROUNDS) -
                           round_begin(k, B, PSI_GREEDY_SHORT_ROUNDS)) *
                          L.plan.splits;
-    greedy_advance_kernel<<<(N + 127) / 128, 128, 0, stream>>>(partial, L.plan.splits, ids, N, B,
-                                                               k, active, rows, counters);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(greedy_advance_kernel, dim3((N + 127) / 128), dim3(128), 0, stream,
+                        static_cast<const uint64_t *>(partial), L.plan.splits, ids, N, B, k,
+                        active, rows, counters)) != cudaSuccess)
+      return e;
     if (k == 0 && ev.before && (e = cudaEventRecord(ev.before, stream)) != cudaSuccess) return e;
+    const int32_t *rl = rows, *rc = counters + (k & 1);
     if (dtype == PSI_DTYPE_BF16)
-      row_argmax_kernel<uint16_t><<<(unsigned)grid, kThreads, 0, stream>>>(
-          static_cast<const uint16_t *>(logits), row_stride, V, L.plan.splits, L.plan.chunk,
-          partial, dev_status, rows, counters + (k & 1));
+      e = launch_pdl(row_argmax_kernel<uint16_t>, dim3((unsigned)grid), dim3(kThreads), 0, stream,
+                     static_cast<const uint16_t *>(logits), row_stride, V, L.plan.splits,
+                     L.plan.chunk, partial, dev_status, rl, rc);
     else
-      row_argmax_kernel<uint32_t><<<(unsigned)grid, kThreads, 0, stream>>>(
-          static_cast<const uint32_t *>(logits), row_stride, V, L.plan.splits, L.plan.chunk,
-          partial, dev_status, rows, counters + (k & 1));
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      e = launch_pdl(row_argmax_kernel<uint32_t>, dim3((unsigned)grid), dim3(kThreads), 0, stream,
+                     static_cast<const uint32_t *>(logits), row_stride, V, L.plan.splits,
+                     L.plan.chunk, partial, dev_status, rl, rc);
+    if (e != cudaSuccess) return e;
     if (k == 0 && ev.after && (e = cudaEventRecord(ev.after, stream)) != cudaSuccess) return e;
   }
   return launch_greedy_emit(partial, L.plan.splits, ids, N, B, V, out_tokens, out_n, dev_status,
@@ -376,9 +385,8 @@ cudaError_t launch_greedy_early_exit(const void *logits, int64_t row_stride, psi
 cudaError_t launch_greedy_emit(const uint64_t *partial, int32_t splits, const int32_t *ids,
                                int32_t N, int32_t B, int32_t V, int32_t *out_tokens,
                                int32_t *out_n, uint32_t *dev_status, cudaStream_t stream) {
-  greedy_emit_kernel<<<(N + 127) / 128, 128, 0, stream>>>(partial, splits, ids, N, B, V,
-                                                          out_tokens, out_n, dev_status);
-  return cudaGetLastError();
+  return launch_pdl(greedy_emit_kernel, dim3((N + 127) / 128), dim3(128), 0, stream, partial,
+                    splits, ids, N, B, V, out_tokens, out_n, dev_status);
 }
 
 cudaError_t launch_tree_walk(const uint64_t *partial, int32_t splits, const int32_t *node_tokens,
@@ -394,10 +402,9 @@ cudaError_t launch_tree_walk(const uint64_t *partial, int32_t splits, const int3
     });
     if (e != cudaSuccess) return e;
   }
-  tree_walk_kernel<<<N, kThreads, smem, stream>>>(partial, splits, node_tokens, parents, M, V,
-                                                  out_path_nodes, out_path_len, out_tokens,
-                                                  dev_status);
-  return cudaGetLastError();
+  return launch_pdl(tree_walk_kernel, dim3(N), dim3(kThreads), smem, stream, partial, splits,
+                    node_tokens, parents, M, V, out_path_nodes, out_path_len, out_tokens,
+                    dev_status);
 }
 
 }  // namespace psi
