@@ -9,14 +9,17 @@
 //
 // What one scan leaves per logit row r (an AR or draft row of a listed unit),
 // the row being split into g.slices contiguous slices of 16-byte vectors:
-//   - per slice c, a record: m_c (the slice maximum; on a rescan the known row
-//     maximum) and z_c = sum of exp2((x - m_c) * log2(e) / T) over the
-//     slice's elements that were not set aside, summed in fp32 by a fixed
-//     thread / accumulator assignment and reduced in double in a fixed order,
-//     so it is a deterministic function of the slice;
+//   - per slice c, a record: m_c (the larger of the slice maximum and a known
+//     element of the row: the drafted token's logit, or on a rescan the row
+//     maximum; either way at most the row maximum) and z_c = sum of
+//     exp2((x - m_c) * log2(e) / T) over the slice's elements that were not
+//     set aside, summed in fp32 by a fixed thread / accumulator assignment
+//     and reduced in double in a fixed order, so it is a deterministic
+//     function of the slice and that known element;
 //   - per slice c, its set-aside list: with top-p, every element above the
-//     running threshold of its stage (the reference so far minus the top-p
-//     window, rounded down to the element type), and the tail elements.  The
+//     running threshold of its stage (the reference so far, which starts at
+//     the known element, minus the top-p window, rounded down to the element
+//     type), and the tail elements.  The
 //     threshold of a stage is at most the row's final one, so every element
 //     the top-p cut can keep is in the lists; the finish (psi_finish.cuh)
 //     sorts them into candidates and the rest of the sum.
@@ -99,7 +102,7 @@ struct ScanSmem {
   uint64_t maxbar[kMaxSlots];   // every consumer warp posted its stage maximum
   int32_t stage_row[kStages];   // row of the stage
   float stage_off[kStages];     // the row's candidate window
-  float stage_known[kStages];   // rescan: the row maximum found by the first pass
+  float stage_known[kStages];   // a lower bound of the row maximum (see drafted_logit)
   float stage_ref[kStages];     // the consumers' reference for the stage
   uint32_t stage_thr[kStages];  // the stage's threshold (Threshold::pair)
   float stage_thrv[kStages];    // (Threshold::value)
@@ -279,11 +282,35 @@ __device__ __forceinline__ int64_t scan_row(const FastArgs &a, int64_t item, flo
   return (int64_t)(e & ~kWideBit);
 }
 
+// A lower bound of row r's maximum known before the scan: the logit of the
+// drafted token at the row's position (AR row i < B, or draft row i), an
+// element of the row; -inf for the bonus rows and without draft ids.  A
+// sampled draft token usually lies near the top of the row, so the first
+// stages' set-aside threshold starts close to its final value.
+template <typename Bits>
+__device__ __forceinline__ float drafted_logit(const FastArgs &a, int64_t r, const Bits *row) {
+  if (!a.s.ids) return -INFINITY;
+  const int32_t B = a.s.B;
+  const int64_t nar = (int64_t)a.s.N * (B + 1);
+  int64_t n, i;
+  if (r < nar) {
+    n = r / (B + 1);
+    i = r % (B + 1);
+    if (i == B) return -INFINITY;  // the bonus row has no drafted token
+  } else {
+    n = (r - nar) / B;
+    i = (r - nar) % B;
+  }
+  const int32_t x = a.s.ids[n * B + i];
+  if (x < 0 || x >= a.s.V) return -INFINITY;
+  return Elem<Bits>::to_float((uint32_t)row[x]);
+}
+
 // What the producer tells the consumers about a stage.
 struct StageMeta {
   int slot;     // ring slot
   float off;    // candidate window of the row (logit units)
-  float known;  // rescan: the row maximum found by the first pass, else -inf
+  float known;  // a lower bound of the row maximum (rescan: the maximum itself)
 };
 
 // The vectors [vb, ve) of slice c of a row; stage k covers
@@ -406,6 +433,7 @@ __global__ void __launch_bounds__(kScanThreads, 1) row_scan_kernel(const __grid_
           r = scan_row(a, cl + cur.t * n_cl, off);
           row = scan_row_ptr<Bits>(a, r);
           known = a.pass == 2 ? a.known_max[r] : -INFINITY;
+          known = fmaxf(known, drafted_logit<Bits>(a, r, row));
         }
         sm.stage_row[cur.slot] = (int32_t)r;
         sm.stage_off[cur.slot] = off;
