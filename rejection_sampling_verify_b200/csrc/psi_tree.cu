@@ -284,40 +284,47 @@ __global__ void __launch_bounds__(kTreeThreads) tree_sampled_kernel(
       tau_key = lo;
       zp = (double)s_lo / kFix40;
     }
-    // children of the node in ascending index (warp 0, lane 0 decides)
+    // children of the node in ascending index (warp 0): every lane loads its
+    // child's logit and uniform at once, then the warp walks the children in
+    // order with the same values in every lane (the tests are sequential)
     if (warp == 0) {
       double R = 1.0;  // mass of P not yet removed
       int nrem = 0, next = -1;
       for (int32_t base = node + 1; base < M && next < 0; base += 32) {
         const int32_t k = base + lane;
         bool child = false;
+        int32_t x = 0;
         if (k < M) {
           const int32_t p = pr[k];
-          child = p == node && p < k && p >= -1 && tk[k] >= 0 && tk[k] < V;
+          x = tk[k];
+          child = p == node && p < k && p >= -1 && x >= 0 && x < V;
+        }
+        double px = 0.0, u = 0.0;
+        if (child) {
+          const uint32_t bits = (uint32_t)row[x];
+          if (Elem<Bits>::key(bits) >= tau_key && zp > 0.0)
+            px = exact_exp2d(Elem<Bits>::to_float(bits), fin.m, a.coef64) / zp;
+          u = uniform24(a.s.seed, seq, a.s.step, (uint64_t)(k + 1), PSI_PURPOSE_ACCEPT);
         }
         unsigned bal = __ballot_sync(0xFFFFFFFFu, child);
         while (bal && next < 0) {
-          const int32_t kc = base + __ffs(bal) - 1;
+          const int c = __ffs(bal) - 1;
           bal &= bal - 1;
-          if (lane == 0) {
-            const int32_t x = tk[kc];
-            const uint32_t bits = (uint32_t)row[x];
-            double px = 0.0;
-            if (Elem<Bits>::key(bits) >= tau_key && zp > 0.0)
-              px = exact_exp2d(Elem<Bits>::to_float(bits), fin.m, a.coef64) / zp;
-            const bool gone = is_removed(sh.removed, nrem, x);
-            const double u = uniform24(a.s.seed, seq, a.s.step, (uint64_t)(kc + 1),
-                                       PSI_PURPOSE_ACCEPT);
-            if (u * R < (gone ? 0.0 : px)) {
-              next = kc;
-            } else if (!gone) {
-              if (nrem < kRemovedCap) sh.removed[nrem++] = x;
-              R -= px;
+          const double pxc = __shfl_sync(0xFFFFFFFFu, px, c);
+          const double uc = __shfl_sync(0xFFFFFFFFu, u, c);
+          const int32_t xc = __shfl_sync(0xFFFFFFFFu, x, c);
+          const bool gone = is_removed(sh.removed, nrem, xc);
+          if (uc * R < (gone ? 0.0 : pxc)) {
+            next = base + c;
+          } else if (!gone) {
+            if (nrem < kRemovedCap) {
+              if (lane == 0) sh.removed[nrem] = xc;
+              ++nrem;
             }
+            R -= pxc;
+            __syncwarp();  // the removed token is visible to the next test
           }
-          next = __shfl_sync(0xFFFFFFFFu, next, 0);
         }
-        nrem = __shfl_sync(0xFFFFFFFFu, nrem, 0);
       }
       if (lane == 0) {
         sh.next = next;
