@@ -251,8 +251,10 @@ def sampled_rounds(cfg):
     import rejection_sampling_verify_b200 as psi
     if cfg.N < psi.PSI_EARLY_EXIT_MIN_N:
         return [(0, cfg.B + 1)]
-    short = psi.PSI_GREEDY_SHORT_ROUNDS if cfg.temperature == 0 else psi.PSI_SAMPLED_SHORT_ROUNDS
-    rs = psi.PSI_ROUND_POSITIONS
+    if cfg.temperature == 0:
+        short, rs = psi.PSI_GREEDY_SHORT_ROUNDS, psi.PSI_GREEDY_ROUND_POSITIONS
+    else:
+        short, rs = psi.PSI_SAMPLED_SHORT_ROUNDS, psi.PSI_SAMPLED_ROUND_POSITIONS
     begins = [min(k * rs, cfg.B + 1) for k in range(short + 1)] + [cfg.B + 1]
     return [(a, b) for a, b in zip(begins, begins[1:]) if a < b]
 
@@ -267,7 +269,8 @@ def rows_in_round(cfg, r):
 def main_launch_bytes(cfg) -> int:
     """Algorithmic bytes of one launch of the timed main kernel: the first
     round's row scan (sampled) or argmax (greedy linear) over every
-    sequence's rows of positions 0..2; the argmax of every tree row."""
+    sequence's rows of the first round's positions; the argmax of every tree
+    row."""
     if isinstance(cfg, psi_inputs.TreeConfig):
         return algorithmic_bytes(cfg)
     es = 4 if cfg.dtype == "f32" else 2

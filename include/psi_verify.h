@@ -90,10 +90,12 @@ typedef enum psi_dtype { PSI_DTYPE_F32 = 0, PSI_DTYPE_BF16 = 1 } psi_dtype;
 #define PSI_MAX_V 393216
 #define PSI_MAX_TREE_NODES 4096
 /* Early-exit rounds of the linear verify (see psi_verify_linear): the first
- * PSI_*_SHORT_ROUNDS rounds cover PSI_ROUND_POSITIONS positions each, one last
- * round covers the rest of the B + 1 positions. */
-#define PSI_ROUND_POSITIONS 3
-#define PSI_SAMPLED_SHORT_ROUNDS 1
+ * PSI_X_SHORT_ROUNDS rounds cover PSI_X_ROUND_POSITIONS positions each, one
+ * last round covers the rest of the B + 1 positions (X = SAMPLED for T > 0,
+ * GREEDY for T == 0). */
+#define PSI_SAMPLED_ROUND_POSITIONS 2
+#define PSI_SAMPLED_SHORT_ROUNDS 2
+#define PSI_GREEDY_ROUND_POSITIONS 3
 #define PSI_GREEDY_SHORT_ROUNDS 3
 /* Smallest batch that takes the early-exit rounds (smaller batches are
  * latency-bound: one pass over every row is faster). */
@@ -137,8 +139,9 @@ size_t psi_verify_linear_workspace_bytes(int32_t N, int32_t B, int32_t V,
  * Early exit (both out_p_draft and out_q_draft NULL, N >= PSI_EARLY_EXIT_MIN_N,
  *   any T): rows after a sequence's first rejection (or greedy mismatch) do
  *   not change its result, so positions are verified in rounds
- *   (PSI_ROUND_POSITIONS positions each for the first PSI_SAMPLED_SHORT_ROUNDS
- *   or PSI_GREEDY_SHORT_ROUNDS rounds, then the rest), and a sequence takes
+ *   (PSI_SAMPLED_ROUND_POSITIONS positions each for the first
+ *   PSI_SAMPLED_SHORT_ROUNDS rounds, PSI_GREEDY_ROUND_POSITIONS for the first
+ *   PSI_GREEDY_SHORT_ROUNDS, then the rest), and a sequence takes
  *   part in a round only if every draft of the earlier rounds was accepted.
  *   Tokens and counts are the same as with every row read; the NONFINITE
  *   status bit then covers the rows that were read.  A caller passing p / q

@@ -44,8 +44,9 @@ PSI_MAX_B = 32
 PSI_MAX_V = 393216
 PSI_MAX_TREE_NODES = 4096
 PSI_NOALLOC_SCRATCH_BYTES = 8 << 20
-PSI_ROUND_POSITIONS = 3
-PSI_SAMPLED_SHORT_ROUNDS = 1
+PSI_SAMPLED_ROUND_POSITIONS = 2
+PSI_GREEDY_ROUND_POSITIONS = 3
+PSI_SAMPLED_SHORT_ROUNDS = 2
 PSI_GREEDY_SHORT_ROUNDS = 3
 PSI_EARLY_EXIT_MIN_N = 64
 

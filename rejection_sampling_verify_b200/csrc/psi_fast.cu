@@ -15,7 +15,7 @@
 //              per slice of a row, its maximum, its fp32 sum of
 //              exponentials and its set-aside list (elements above the
 //              running top-p threshold).
-//   row_finish One warp per listed row: row maximum, Z, the top-p threshold
+//   row_finish One CTA of four warps per listed row: row maximum, Z, the top-p threshold
 //              and renormaliser from the slice records and lists, exact
 //              (double masses, 2^52 fixed-point sums); the row's candidates
 //              compacted at the front of its list area.
@@ -32,9 +32,11 @@
 //   draw       One warp per listed position: the correction (residual
 //              max(0, p - q)) or bonus draw over p's nucleus, inverse CDF in
 //              vocabulary order on exact integer sums.  Only the emitted
-//              position of each sequence is drawn.  Without top-p the draw
-//              needs whole rows: those positions go to the cluster kernel in
-//              sample mode.
+//              position of each sequence is drawn.
+//   whole_row_draw  Without top-p (and top-k) the draw spans the vocabulary:
+//              for rows of up to kWrMaxVocab entries, one CTA per such
+//              position, from the rows' finished maxima and normalisers;
+//              longer rows go to the cluster kernel in sample mode.
 #include <algorithm>
 
 #include "psi_finish.cuh"
@@ -330,6 +332,136 @@ __global__ void __launch_bounds__(32) draw_kernel(const __grid_constant__ FastAr
 }
 
 // ---------------------------------------------------------------------------
+// whole_row_draw: one CTA per listed position whose draw spans the whole
+// vocabulary (no top-p and no top-k): the residual max(0, p - q) or p over
+// every index, p and q from the rows' finished maxima and normalisers (the
+// same ones the decision used), fp32 exponentials in 2^40 fixed point
+// (order-free integer sums; the CDF is within ~1e-7 of the exact one),
+// inverse CDF in vocabulary order.  Each warp sums a contiguous range of
+// the vocabulary with coalesced loads; the range holding the draw's point
+// is then split over every thread of the CTA (pieces of kWrPiece), a block
+// scan finds the piece that holds it, and its thread walks the piece.
+// ---------------------------------------------------------------------------
+constexpr int kWrThreads = 512;
+constexpr int kWrWarps = kWrThreads / 32;
+constexpr int kWrPiece = 24;  // elements per thread in the final search
+constexpr int32_t kWrMaxVocab = 16384;  // longest row drawn by one CTA
+constexpr float kFix40f = 1099511627776.0f;  // 2^40
+
+template <typename Bits>
+__global__ void __launch_bounds__(kWrThreads) whole_row_draw_kernel(const __grid_constant__ FastArgs a) {
+  pdl_wait();  // the previous kernel's results are visible
+  pdl_trigger();
+  __shared__ unsigned long long wsum[kWrWarps];
+  __shared__ int32_t token_sh;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const SampledArgs &s = a.s;
+  const int32_t B = s.B, N = s.N, V = s.V;
+  const int64_t n_items = (int64_t)a.counters[1];
+  // warp w's range of the vocabulary: [w * span, (w + 1) * span)
+  const int32_t span = (V + kWrWarps - 1) / kWrWarps;
+  for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+    const int64_t unit = (int64_t)a.list_b[item];
+    const int32_t n = (int32_t)(unit / (B + 1)), i = (int32_t)(unit % (B + 1));
+    const bool has_q = i < B;
+    const RowFin fp = a.rfin[unit];
+    const RowFin fq = has_q ? a.rfin[(int64_t)N * (B + 1) + (int64_t)n * B + i] : empty_fin();
+    const uint64_t seq = s.seq_ids ? s.seq_ids[n] : (uint64_t)n;
+    const Bits *row_p = static_cast<const Bits *>(s.ar) + unit * s.ar_stride;
+    const Bits *row_q =
+        has_q ? static_cast<const Bits *>(s.draft) + ((int64_t)n * B + i) * s.draft_stride : nullptr;
+    const float shift_p = fp.m == -INFINITY ? -INFINITY : -fp.m * a.coef;
+    const float shift_q = fq.m == -INFINITY ? -INFINITY : -fq.m * a.coef;
+    const float inv_zp = fp.zp > 0.0 ? (float)(1.0 / fp.zp) : 0.f;
+    const float inv_zq = fq.zp > 0.0 ? (float)(1.0 / fq.zp) : 0.f;
+    int32_t token = 0;
+    for (int pass = has_q ? 0 : 1; pass < 2; ++pass) {
+      // explicit roundings: both searches below must see the same weights
+      auto weight = [&](int32_t v) -> unsigned long long {
+        float pv = __fmul_rn(fast_exp2(fmaf(Elem<Bits>::to_float((uint32_t)row_p[v]), a.coef, shift_p)), inv_zp);
+        if (pass == 0)
+          pv = __fmaf_rn(-fast_exp2(fmaf(Elem<Bits>::to_float((uint32_t)row_q[v]), a.coef, shift_q)), inv_zq, pv);
+        return pv > 0.f ? __float2ull_rn(__fmul_rn(fminf(pv, 1.f), kFix40f)) : 0ull;
+      };
+      const int32_t w0 = warp * span, w1 = min(V, w0 + span);
+      unsigned long long part = 0ull;
+      for (int32_t v = w0 + lane; v < w1; v += 32) part += weight(v);
+      part = warp_sum_any(part);
+      if (lane == 0) wsum[warp] = part;
+      __syncthreads();
+      unsigned long long W = 0ull;
+      for (int w = 0; w < kWrWarps; ++w) W += wsum[w];
+      __syncthreads();
+      if (W == 0ull) continue;  // no residual mass: draw from p
+      const float u2 = uniform24(s.seed, seq, s.step, (uint64_t)i, PSI_PURPOSE_RESID);
+      const unsigned long long k = (unsigned long long)(u2 * 16777216.0f);
+      const unsigned long long t = (__umul64hi(k, W) << 40) | ((k * W) >> 24);
+      // the warp whose range holds t, and the weight before that range
+      int ws = 0;
+      unsigned long long wb = 0ull;
+      for (int w = 0; w < kWrWarps; ++w) {
+        if (wb + wsum[w] > t) {
+          ws = w;
+          break;
+        }
+        wb += wsum[w];
+      }
+      if (tid == 0) token_sh = -1;
+      __syncthreads();
+      // that range split over every thread of the CTA, a chunk of
+      // kWrThreads * kWrPiece elements at a time: contiguous pieces of
+      // kWrPiece elements per thread, their loads in flight together
+      const int32_t r1 = min(V, (ws + 1) * span);
+      for (int32_t c0 = ws * span; c0 < r1; c0 += kWrThreads * kWrPiece) {
+        const int32_t q0 = min(r1, c0 + tid * kWrPiece), q1 = min(r1, q0 + kWrPiece);
+        unsigned long long wv[kWrPiece];
+        unsigned long long ps = 0ull;
+#pragma unroll
+        for (int e = 0; e < kWrPiece; ++e) {
+          wv[e] = q0 + e < q1 ? weight(q0 + e) : 0ull;
+          ps += wv[e];
+        }
+        // exclusive scan of the pieces over the CTA
+        unsigned long long incl = ps;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned long long x = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+          if (lane >= o) incl += x;
+        }
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        unsigned long long lb = wb + incl - ps, chunk = 0ull;
+        for (int w = 0; w < kWrWarps; ++w) {
+          if (w < warp) lb += wsum[w];
+          chunk += wsum[w];
+        }
+        if (lb <= t && t < lb + ps) {  // exactly one thread's piece holds t
+          unsigned long long run = lb;
+#pragma unroll
+          for (int e = 0; e < kWrPiece; ++e) {
+            run += wv[e];
+            if (run > t) {
+              token_sh = q0 + e;
+              break;
+            }
+          }
+        }
+        wb += chunk;
+        __syncthreads();
+        if (token_sh >= 0) break;
+      }
+      token = token_sh >= 0 ? token_sh : r1 - 1;  // the sums are exact: always found
+      __syncthreads();
+      break;
+    }
+    if (tid == 0) {
+      a.rec[unit].token = token;
+      s.out_tokens[unit] = token;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // fast_emit: one thread per sequence.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) fast_emit_kernel(const __grid_constant__ FastArgs a) {
@@ -374,7 +506,7 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 // ---------------------------------------------------------------------------
 // round_advance: one thread per sequence.  Early-exit rounds: round k covers
-// positions [round_begin(k), round_begin(k + 1)) of B + 1.
+// positions [sampled_round_begin(k), sampled_round_begin(k + 1)) of B + 1.
 // A sequence takes part in round k when every drafted token of the earlier
 // rounds was accepted (a unit left to the general path counts as accepted:
 // its rows are then read although a rejection may make them unused).  The
@@ -395,13 +527,13 @@ __global__ void __launch_bounds__(128) round_advance_kernel(const __grid_constan
     a.counters[5 + 2 * ((k + 1) & 1)] = 0;
   }
   if (n >= N) return;
-  const int32_t i0 = round_begin(k, B, PSI_SAMPLED_SHORT_ROUNDS);
-  const int32_t i1 = round_begin(k + 1, B, PSI_SAMPLED_SHORT_ROUNDS);
+  const int32_t i0 = sampled_round_begin(k, B);
+  const int32_t i1 = sampled_round_begin(k + 1, B);
   int act = 1;
   if (k > 0) {
     act = a.active[n];
     const UnitRecord *r = a.rec + (int64_t)n * (B + 1);
-    for (int32_t i = round_begin(k - 1, B, PSI_SAMPLED_SHORT_ROUNDS); act && i < i0; ++i)
+    for (int32_t i = sampled_round_begin(k - 1, B); act && i < i0; ++i)
       if (i < B && r[i].accept == 0) act = 0;
   }
   a.active[n] = act;
@@ -467,7 +599,8 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
     if ((e = scan_and_finish(fa, true)) != cudaSuccess) return e;
     if ((e = scan_and_finish(f2, false)) != cudaSuccess) return e;
   } else {
-    const int rounds = round_count(fa.s.B, PSI_SAMPLED_SHORT_ROUNDS);
+    const int rounds = round_count(fa.s.B, PSI_SAMPLED_SHORT_ROUNDS,
+                                   PSI_SAMPLED_ROUND_POSITIONS);
     for (int k = 0; k < rounds; ++k) {
       if ((e = launch_pdl(round_advance_kernel, dim3((fa.s.N + 127) / 128), dim3(128), 0, stream,
                           fa, k)) != cudaSuccess)
@@ -499,6 +632,14 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
   if ((e = launch_pdl(draw_kernel<Bits>, dim3((unsigned)grid_draw), dim3(32), 0, stream, fa)) !=
       cudaSuccess)
     return e;
+  // the whole-row draws (no top-p, no top-k): one CTA per draw for short
+  // rows, where a cluster's launch and synchronisation cost more than the
+  // row; a cluster per draw for long ones, which one SM reads too slowly
+  if (fa.s.V <= kWrMaxVocab) {
+    const int32_t grid_wr = std::max<int32_t>(1, std::min<int32_t>(fa.s.N, sm_count()));
+    return launch_pdl(whole_row_draw_kernel<Bits>, dim3((unsigned)grid_wr), dim3(kWrThreads), 0,
+                      stream, fa);
+  }
   const int clusters_b = std::min(fa.s.N, kListClusters);
   return launch_cluster_list(sa, dt, plan, kClusterModeSample, fa.list_b, fa.counters + 1,
                              clusters_b, stream);

@@ -301,7 +301,7 @@ cudaError_t launch_row_argmax(const void *logits, int64_t row_stride, psi_dtype 
 GreedyLayout greedy_layout(int32_t N, int32_t B, int32_t V, int elem_bytes) {
   GreedyLayout L;
   const int64_t rows = (int64_t)N * (B + 1);
-  L.plan = plan_argmax((int64_t)N * std::min(B + 1, PSI_ROUND_POSITIONS), V, elem_bytes);
+  L.plan = plan_argmax((int64_t)N * std::min(B + 1, PSI_GREEDY_ROUND_POSITIONS), V, elem_bytes);
   size_t off = 0;
   L.partial_off = off;
   off = round_up256(off + sizeof(uint64_t) * (size_t)rows * L.plan.splits);
@@ -316,8 +316,8 @@ GreedyLayout greedy_layout(int32_t N, int32_t B, int32_t V, int elem_bytes) {
 }
 
 // One thread per sequence: the AR rows of early-exit round k (positions
-// [round_begin(k), round_begin(k + 1)) of B + 1).  A sequence takes part when
-// every draft of the earlier rounds matched its row's argmax.
+// [greedy_round_begin(k), greedy_round_begin(k + 1)) of B + 1).  A sequence
+// takes part when every draft of the earlier rounds matched its row's argmax.
 __global__ void __launch_bounds__(128) greedy_advance_kernel(
     const uint64_t *__restrict__ partial, int32_t splits, const int32_t *__restrict__ ids,
     int32_t N, int32_t B, int k, int32_t *active, int32_t *round_rows, int32_t *counters) {
@@ -326,13 +326,13 @@ __global__ void __launch_bounds__(128) greedy_advance_kernel(
   const int32_t n = blockIdx.x * blockDim.x + threadIdx.x;
   if (n == 0) counters[(k + 1) & 1] = 0;  // the next round's list
   if (n >= N) return;
-  const int32_t i0 = round_begin(k, B, PSI_GREEDY_SHORT_ROUNDS);
-  const int32_t i1 = round_begin(k + 1, B, PSI_GREEDY_SHORT_ROUNDS);
+  const int32_t i0 = greedy_round_begin(k, B);
+  const int32_t i1 = greedy_round_begin(k + 1, B);
   const int64_t row0 = (int64_t)n * (B + 1);
   int act = 1;
   if (k > 0) {
     act = active[n];
-    for (int32_t i = round_begin(k - 1, B, PSI_GREEDY_SHORT_ROUNDS); act && i < i0; ++i)
+    for (int32_t i = greedy_round_begin(k - 1, B); act && i < i0; ++i)
       if (i < B && ids[(int64_t)n * B + i] != argmax_of(partial, row0 + i, splits)) act = 0;
   }
   active[n] = act;
@@ -355,11 +355,10 @@ cudaError_t launch_greedy_early_exit(const void *logits, int64_t row_stride, psi
   if ((int64_t)N * (B + 1) * L.plan.splits > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
   cudaError_t e;
   if ((e = cudaMemsetAsync(counters, 0, 4 * sizeof(int32_t), stream)) != cudaSuccess) return e;
-  const int rounds = round_count(B, PSI_GREEDY_SHORT_ROUNDS);
+  const int rounds = round_count(B, PSI_GREEDY_SHORT_ROUNDS, PSI_GREEDY_ROUND_POSITIONS);
   for (int k = 0; k < rounds; ++k) {
     const int64_t grid = (int64_t)N *
-                         (round_begin(k + 1, B, PSI_GREEDY_SHORT_ROUNDS) -
-                          round_begin(k, B, PSI_GREEDY_SHORT_ROUNDS)) *
+                         (greedy_round_begin(k + 1, B) - greedy_round_begin(k, B)) *
                          L.plan.splits;
     if ((e = launch_pdl(greedy_advance_kernel, dim3((N + 127) / 128), dim3(128), 0, stream,
                         static_cast<const uint64_t *>(partial), L.plan.splits, ids, N, B, k,

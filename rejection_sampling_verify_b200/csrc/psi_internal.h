@@ -54,16 +54,22 @@ inline cudaError_t prefer_max_shared(Kernel *k) {
                               (int)cudaSharedmemCarveoutMaxShared);
 }
 
-// Early-exit round schedule: `short_rounds` rounds of PSI_ROUND_POSITIONS
+// Early-exit round schedule: `short_rounds` rounds of `positions`
 // positions, then one round with the rest of the B + 1 positions.
-__host__ __device__ inline int32_t round_begin(int k, int32_t B, int short_rounds) {
-  const int32_t b = k <= short_rounds ? k * PSI_ROUND_POSITIONS : B + 1;
+__host__ __device__ inline int32_t round_begin(int k, int32_t B, int short_rounds, int positions) {
+  const int32_t b = k <= short_rounds ? k * positions : B + 1;
   return b < B + 1 ? b : B + 1;
 }
-__host__ __device__ inline int round_count(int32_t B, int short_rounds) {
+__host__ __device__ inline int round_count(int32_t B, int short_rounds, int positions) {
   int k = 0;
-  while (round_begin(k, B, short_rounds) < B + 1) ++k;
+  while (round_begin(k, B, short_rounds, positions) < B + 1) ++k;
   return k;
+}
+__host__ __device__ inline int32_t sampled_round_begin(int k, int32_t B) {
+  return round_begin(k, B, PSI_SAMPLED_SHORT_ROUNDS, PSI_SAMPLED_ROUND_POSITIONS);
+}
+__host__ __device__ inline int32_t greedy_round_begin(int k, int32_t B) {
+  return round_begin(k, B, PSI_GREEDY_SHORT_ROUNDS, PSI_GREEDY_ROUND_POSITIONS);
 }
 
 // ---- greedy paths ----------------------------------------------------------

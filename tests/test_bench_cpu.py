@@ -22,7 +22,8 @@ def _header_define(name):
 
 
 def test_schedule_constants_come_from_the_header():
-    for name in ("PSI_ROUND_POSITIONS", "PSI_SAMPLED_SHORT_ROUNDS", "PSI_GREEDY_SHORT_ROUNDS",
+    for name in ("PSI_SAMPLED_ROUND_POSITIONS", "PSI_GREEDY_ROUND_POSITIONS",
+                 "PSI_SAMPLED_SHORT_ROUNDS", "PSI_GREEDY_SHORT_ROUNDS",
                  "PSI_EARLY_EXIT_MIN_N"):
         assert getattr(psi, name) == _header_define(name)
 
@@ -36,17 +37,20 @@ def test_rounds_partition_the_positions():
         if cfg.N < psi.PSI_EARLY_EXIT_MIN_N:
             assert r == [(0, cfg.B + 1)]
         else:
-            short = (psi.PSI_GREEDY_SHORT_ROUNDS if cfg.temperature == 0
-                     else psi.PSI_SAMPLED_SHORT_ROUNDS)
-            assert all(b - a == psi.PSI_ROUND_POSITIONS for a, b in r[:short])
+            short, rs = ((psi.PSI_GREEDY_SHORT_ROUNDS, psi.PSI_GREEDY_ROUND_POSITIONS)
+                         if cfg.temperature == 0 else
+                         (psi.PSI_SAMPLED_SHORT_ROUNDS, psi.PSI_SAMPLED_ROUND_POSITIONS))
+            assert all(b - a == rs for a, b in r[:short])
 
 
 def test_rows_read_counts_rounds_up_to_the_emitting_position():
-    cfg = CFG["large_batch_nucleus"]  # rounds (0, 3), (3, 9), B = 8
-    assert bench.sampled_rounds(cfg) == [(0, 3), (3, 9)]
-    # emitting position 0..2: round 0 only = 3 AR + 3 draft rows; later: all 17
-    assert bench.rows_read(cfg, np.array([1, 3])) == 2 * 6
-    assert bench.rows_read(cfg, np.array([4, 9])) == 2 * 17
+    cfg = CFG["large_batch_nucleus"]  # rounds (0, 2), (2, 4), (4, 9), B = 8
+    assert bench.sampled_rounds(cfg) == [(0, 2), (2, 4), (4, 9)]
+    # emitting position 0..1: round 0 only = 2 AR + 2 draft rows; 2..3: rounds
+    # 0 and 1 = 8 rows; later: all 17
+    assert bench.rows_read(cfg, np.array([1, 2])) == 2 * 4
+    assert bench.rows_read(cfg, np.array([3, 4])) == 2 * 8
+    assert bench.rows_read(cfg, np.array([5, 9])) == 2 * 17
     g = CFG["max_batch_greedy"]  # AR rows only
     assert bench.rows_read(g, np.array([1])) == 3
     assert bench.rows_read(g, np.array([17])) == 17
@@ -54,7 +58,7 @@ def test_rows_read_counts_rounds_up_to_the_emitting_position():
 
 def test_main_launch_bytes_is_the_first_round():
     cfg = CFG["large_batch_nucleus"]
-    assert bench.main_launch_bytes(cfg) == cfg.N * 6 * cfg.V * 2
+    assert bench.main_launch_bytes(cfg) == cfg.N * 4 * cfg.V * 2
     g = CFG["max_batch_greedy"]
     assert bench.main_launch_bytes(g) == g.N * 3 * g.V * 2
     t = CFG["tree_greedy"]
