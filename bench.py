@@ -536,9 +536,9 @@ def main():
     if rank == 0:
         # our kernels per call: argmax + tree walk; greedy linear: per
         # early-exit round list building and argmax, then emit; sampled: per
-        # round list building, row scan, row finish, unit decision and their
-        # second passes, then two cluster list launches, fast_emit and the
-        # nucleus draw
+        # round list building, row scan, row finish and unit decision, then
+        # one second pass of the three, the general-path list, fast_emit, the
+        # nucleus draw and the whole-row draw
         rounds = 0 if is_tree else len(sampled_rounds(cfg))
         if is_tree or (cfg.temperature == 0 and cfg.N < 64):
             launches_per_step = 2  # tree: argmax + walk, or row scan + sampled walk
@@ -547,7 +547,7 @@ def main():
         elif cfg.N < 64:  # one pass: scan, finish, unit, their second passes, lists, emit, draw
             launches_per_step = 10
         else:
-            launches_per_step = 7 * rounds + 4
+            launches_per_step = 4 * rounds + 7
         line = {
             "metric": METRIC, "value": value, "unit": "blocks/s", "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,

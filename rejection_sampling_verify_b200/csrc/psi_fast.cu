@@ -15,8 +15,9 @@
 //              per slice of a row, its maximum, its fp32 sum of
 //              exponentials and its set-aside list (elements above the
 //              running top-p threshold).
-//   row_finish One CTA of four warps per listed row: row maximum, Z, the top-p threshold
-//              and renormaliser from the slice records and lists, exact
+//   row_finish One CTA of four warps per listed row: row maximum, Z, the
+//              top-p threshold and renormaliser from the slice records and
+//              lists, exact
 //              (double masses, 2^52 fixed-point sums); the row's candidates
 //              compacted at the front of its list area.
 //   unit       One thread per (sequence, position) unit: accepts or rejects
@@ -25,7 +26,7 @@
 //   row_scan / row_finish / unit, second pass   Rows whose window held less
 //              than top_p of the mass (rescanned with a wider window) or
 //              whose lists overflowed (rescanned with the exact maximum
-//              known).
+//              known); once, after the last round.
 //   (cluster kernel, list mode)  Units the second pass could not settle.
 //   fast_emit  First rejected position per sequence; emitted tokens; lists
 //              the position whose token is still to be drawn.
@@ -131,6 +132,7 @@ __global__ void __launch_bounds__(kUnitThreads) unit_kernel(const __grid_constan
               (int32_t)rp_idx | ((fail_p & kFinCoverage) ? kWideBit : 0);
         }
         a.wide_units[atomicAdd(&a.counters[3], 1)] = (int32_t)unit;
+        a.rec[unit].accept = -1;  // settled by the rescan; a later round treats it as accepted
       } else {  // the general path verifies this unit (records included)
         a.list_a[atomicAdd(&a.counters[0], 1)] = (int32_t)unit;
         a.rec[unit].accept = -1;  // decided at the end; a later round treats it as accepted
@@ -508,10 +510,10 @@ size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 // round_advance: one thread per sequence.  Early-exit rounds: round k covers
 // positions [sampled_round_begin(k), sampled_round_begin(k + 1)) of B + 1.
 // A sequence takes part in round k when every drafted token of the earlier
-// rounds was accepted (a unit left to the general path counts as accepted:
-// its rows are then read although a rejection may make them unused).  The
-// kernel lists the round's rows and units, and resets the lists that the
-// round's finish step and the next round fill.
+// rounds was accepted (a unit left to the second pass or the general path
+// counts as accepted: its rows are then read although a rejection may make
+// them unused).  The kernel lists the round's rows and units, and resets the
+// lists that the next round fills.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) round_advance_kernel(const __grid_constant__ FastArgs a,
                                                             int k) {
@@ -521,8 +523,6 @@ __global__ void __launch_bounds__(128) round_advance_kernel(const __grid_constan
   const SampledArgs &s = a.s;
   const int32_t B = s.B, N = s.N;
   if (n == 0) {
-    a.counters[2] = 0;  // this round's second-pass lists
-    a.counters[3] = 0;
     a.counters[4 + 2 * ((k + 1) & 1)] = 0;  // the next round's lists
     a.counters[5 + 2 * ((k + 1) & 1)] = 0;
   }
@@ -588,7 +588,9 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
                       f);
   };
   // the second pass over the rows and units a first pass could not settle
-  // (usually none: the CTAs find empty lists and exit)
+  // (usually none: the CTAs find empty lists and exit).  With early-exit
+  // rounds it runs once, after the last round: a unit left to it counts as
+  // accepted when the next round's sequences are chosen.
   FastArgs f2 = fa;
   f2.pass = 2;
   f2.rlist = fa.wide_rows;
@@ -611,8 +613,9 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
       f1.ulist = fa.round_units;
       f1.ucount = fa.counters + 5 + 2 * (k & 1);
       if ((e = scan_and_finish(f1, k == 0)) != cudaSuccess) return e;
-      if ((e = scan_and_finish(f2, false)) != cudaSuccess) return e;
     }
+    // one second pass after the last round, over every round's failures
+    if ((e = scan_and_finish(f2, false)) != cudaSuccess) return e;
   }
   const psi_dtype dt = sizeof(Bits) == 2 ? PSI_DTYPE_BF16 : PSI_DTYPE_F32;
   SampledArgs sa = fa.s;
