@@ -30,7 +30,7 @@
 //   (cluster kernel, list mode)  Units the second pass could not settle.
 //   fast_emit  First rejected position per sequence; emitted tokens; lists
 //              the position whose token is still to be drawn.
-//   draw       One warp per listed position: the correction (residual
+//   draw       One CTA per listed position: the correction (residual
 //              max(0, p - q)) or bonus draw over p's nucleus, inverse CDF in
 //              vocabulary order on exact integer sums.  Only the emitted
 //              position of each sequence is drawn.
@@ -176,23 +176,45 @@ __global__ void __launch_bounds__(kUnitThreads) unit_kernel(const __grid_constan
 }
 
 // ---------------------------------------------------------------------------
-// draw: one warp per listed unit (each sequence's emitted position)
+// draw: one CTA of kDrawWarps warps per listed unit (each sequence's emitted
+// position)
 // ---------------------------------------------------------------------------
-struct DrawScratch {  // one warp's shared memory: p's nucleus and its draw weights
+constexpr int kDrawWarps = 4;
+constexpr int kDrawThreads = kDrawWarps * 32;
+constexpr int kDrawReg = kFinishCap / kDrawThreads;  // nucleus entries a thread searches
+static_assert(kFinishCap % kDrawThreads == 0, "the nucleus fits the threads' registers");
+
+struct DrawScratch {  // the CTA's shared memory: p's nucleus and its draw weights
   uint32_t idx[kFinishCap];
   unsigned long long w[kFinishCap];
+  unsigned long long part[2][kDrawWarps];  // per-warp partial sums (two buffers)
 };
 
+// Sum over the CTA; every thread gets the total.  `buf` alternates between
+// calls so that one barrier suffices.
+__device__ __forceinline__ unsigned long long draw_block_sum(unsigned long long v,
+                                                             DrawScratch *ds, int buf) {
+  v = warp_sum_any(v);
+  if ((threadIdx.x & 31) == 0) ds->part[buf][threadIdx.x >> 5] = v;
+  __syncthreads();
+  unsigned long long t = 0ull;
+#pragma unroll
+  for (int w = 0; w < kDrawWarps; ++w) t += ds->part[buf][w];
+  return t;
+}
+
 template <typename Bits>
-__global__ void __launch_bounds__(32) draw_kernel(const __grid_constant__ FastArgs a) {
+__global__ void __launch_bounds__(kDrawThreads) draw_kernel(const __grid_constant__ FastArgs a) {
   pdl_wait();  // the previous kernel's results are visible
   pdl_trigger();
   __shared__ DrawScratch dsm;
+  __shared__ int wcnt[kDrawWarps];
   DrawScratch *ds = &dsm;
-  const int lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const SampledArgs &s = a.s;
   const int32_t B = s.B, N = s.N, V = s.V;
   const int64_t n_items = (int64_t)a.counters[8];
+  int buf = 0;  // the partial-sum buffer of the next block sum
   for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
     const int64_t unit = (int64_t)a.list_d[item];
     const int32_t n = (int32_t)(unit / (B + 1)), i = (int32_t)(unit % (B + 1));
@@ -213,20 +235,21 @@ __global__ void __launch_bounds__(32) draw_kernel(const __grid_constant__ FastAr
     const int nc = (fp.status & kFinNonfinite) ? 0 : fp.n;
     const double inv_sp = 1.0 / (fp.zp * kFix52);  // p's nucleus mass in fixed-point units
     const double inv_zq = fq.zp > 0.0 ? 1.0 / fq.zp : 0.0;
-    // p's nucleus with its masses (as weights) to the scratch
+    // p's nucleus with its masses (as weights) to the scratch, in any order
+    // (the search below sums by vocabulary index)
     auto load_nucleus = [&]() -> int {
       int nn = 0;
-      for (int base = 0; base < nc; base += 32 * kLoadChunk) {
+      for (int base = 0; base < nc; base += kDrawThreads * kLoadChunk) {
         unsigned long long e[kLoadChunk];  // loads in flight together
 #pragma unroll
         for (int h = 0; h < kLoadChunk; ++h) {
-          const int j = base + 32 * h + lane;
+          const int j = base + kDrawThreads * h + tid;
           e[h] = j < nc ? __ldcg(pc + j) : 0ull;
         }
         uint32_t inm = 0u;  // bit h: entry h is in the nucleus
 #pragma unroll
         for (int h = 0; h < kLoadChunk; ++h) {
-          const int j = base + 32 * h + lane;
+          const int j = base + kDrawThreads * h + tid;
           const bool in = j < nc && Elem<Bits>::key((uint32_t)(e[h] >> 32)) >= fp.tau_key;
           inm |= (in ? 1u : 0u) << h;
         }
@@ -237,8 +260,16 @@ __global__ void __launch_bounds__(32) draw_kernel(const __grid_constant__ FastAr
           const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
           if (lane >= o) incl += v;
         }
-        int d = nn + incl - cnt;
-        nn += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        if (lane == 31) wcnt[warp] = incl;
+        __syncthreads();
+        int before = 0, total = 0;
+#pragma unroll
+        for (int w = 0; w < kDrawWarps; ++w) {
+          before += w < warp ? wcnt[w] : 0;
+          total += wcnt[w];
+        }
+        int d = nn + before + incl - cnt;
+        nn += total;
 #pragma unroll
         for (int h = 0; h < kLoadChunk; ++h)
           if ((inm >> h) & 1u) {
@@ -246,27 +277,27 @@ __global__ void __launch_bounds__(32) draw_kernel(const __grid_constant__ FastAr
             ds->w[d] = e[h] >> 32;  // the logit's bits until its mass replaces them
             ++d;
           }
+        __syncthreads();  // wcnt is reused; the entries are complete
       }
-      __syncwarp();
 #pragma unroll 4
-      for (int j = lane; j < nn; j += 32)
+      for (int j = tid; j < nn; j += kDrawThreads)
         ds->w[j] = fixed52(exact_exp2d(Elem<Bits>::to_float((uint32_t)ds->w[j]), fp.m, a.coef64));
-      __syncwarp();
+      __syncthreads();
       return nn;
     };
     const int nn = load_nucleus();
     unsigned long long W = 0ull;
     if (has_q) {  // residual weights max(0, p - q), in double
-      for (int base = 0; base < nn; base += 32 * kQChunk) {
+      for (int base = 0; base < nn; base += kDrawThreads * kQChunk) {
         uint32_t xqb[kQChunk];  // q logits of the chunk, loads in flight together
 #pragma unroll
         for (int c = 0; c < kQChunk; ++c) {
-          const int j = base + 32 * c + lane;
+          const int j = base + kDrawThreads * c + tid;
           xqb[c] = j < nn ? (uint32_t)row_q[ds->idx[j]] : 0u;
         }
 #pragma unroll
         for (int c = 0; c < kQChunk; ++c) {
-          const int j = base + 32 * c + lane;
+          const int j = base + kDrawThreads * c + tid;
           if (j < nn) {
             const double pv = (double)ds->w[j] * inv_sp;
             const float xq = Elem<Bits>::to_float(xqb[c]);
@@ -277,13 +308,14 @@ __global__ void __launch_bounds__(32) draw_kernel(const __grid_constant__ FastAr
           }
         }
       }
-      W = warp_sum_any(W);
-      __syncwarp();
+      W = draw_block_sum(W, ds, buf);
+      buf ^= 1;
       if (W == 0ull) load_nucleus();  // residual vanished: draw from p itself
     }
     if (W == 0ull) {
-      for (int j = lane; j < nn; j += 32) W += ds->w[j];
-      W = warp_sum_any(W);
+      for (int j = tid; j < nn; j += kDrawThreads) W += ds->w[j];
+      W = draw_block_sum(W, ds, buf);
+      buf ^= 1;
     }
     int32_t token = 0;
     if (W > 0ull) {
@@ -293,43 +325,32 @@ __global__ void __launch_bounds__(32) draw_kernel(const __grid_constant__ FastAr
       const float u2 = uniform24(s.seed, seq, s.step, (uint64_t)i, PSI_PURPOSE_RESID);
       const unsigned long long k = (unsigned long long)(u2 * 16777216.0f);
       const unsigned long long t = (__umul64hi(k, W) << 40) | ((k * W) >> 24);
+      uint32_t ir[kDrawReg];
+      unsigned long long wr[kDrawReg];
+#pragma unroll
+      for (int c = 0; c < kDrawReg; ++c) {
+        const int j = tid + kDrawThreads * c;
+        ir[c] = j < nn ? ds->idx[j] : 0xFFFFFFFFu;
+        wr[c] = j < nn ? ds->w[j] : 0ull;
+      }
       uint32_t lo = 0u, hi = (uint32_t)V;
-      if (nn <= 32 * kRegCand) {
-        uint32_t ir[kRegCand];
-        unsigned long long wr[kRegCand];
+      while (hi - lo > 1u) {
+        const uint32_t mid = (lo + hi) >> 1;
+        unsigned long long cm = 0ull;
 #pragma unroll
-        for (int c = 0; c < kRegCand; ++c) {
-          const int j = lane + 32 * c;
-          ir[c] = j < nn ? ds->idx[j] : 0xFFFFFFFFu;
-          wr[c] = j < nn ? ds->w[j] : 0ull;
-        }
-        while (hi - lo > 1u) {
-          const uint32_t mid = (lo + hi) >> 1;
-          unsigned long long cm = 0ull;
-#pragma unroll
-          for (int c = 0; c < kRegCand; ++c) cm += ir[c] < mid ? wr[c] : 0ull;
-          cm = warp_sum_any(cm);
-          if (cm > t) hi = mid;
-          else lo = mid;
-        }
-      } else {
-        while (hi - lo > 1u) {
-          const uint32_t mid = (lo + hi) >> 1;
-          unsigned long long cm = 0ull;
-          for (int j = lane; j < nn; j += 32)
-            if (ds->idx[j] < mid) cm += ds->w[j];
-          cm = warp_sum_any(cm);
-          if (cm > t) hi = mid;
-          else lo = mid;
-        }
+        for (int c = 0; c < kDrawReg; ++c) cm += ir[c] < mid ? wr[c] : 0ull;
+        cm = draw_block_sum(cm, ds, buf);
+        buf ^= 1;
+        if (cm > t) hi = mid;
+        else lo = mid;
       }
       token = (int32_t)lo;
     }
-    if (lane == 0) {
+    if (tid == 0) {
       a.rec[unit].token = token;
       s.out_tokens[unit] = token;
     }
-    __syncwarp();  // the scratch is reused by the warp's next unit
+    __syncthreads();  // the scratch is reused by the CTA's next unit
   }
 }
 
@@ -632,8 +653,8 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
   if ((e = launch_pdl(fast_emit_kernel, dim3((fa.s.N + 127) / 128), dim3(128), 0, stream, fa)) !=
       cudaSuccess)
     return e;
-  if ((e = launch_pdl(draw_kernel<Bits>, dim3((unsigned)grid_draw), dim3(32), 0, stream, fa)) !=
-      cudaSuccess)
+  if ((e = launch_pdl(draw_kernel<Bits>, dim3((unsigned)grid_draw), dim3(kDrawThreads), 0,
+                      stream, fa)) != cudaSuccess)
     return e;
   // the whole-row draws (no top-p, no top-k): one CTA per draw for short
   // rows, where a cluster's launch and synchronisation cost more than the
