@@ -269,8 +269,9 @@ def rows_in_round(cfg, r):
 def main_launch_bytes(cfg) -> int:
     """Algorithmic bytes of one launch of the timed main kernel: the first
     round's row scan (sampled) or argmax (greedy linear) over every
-    sequence's rows of the first round's positions; the argmax of every tree
-    row."""
+    sequence's rows of the first round's positions; every node row of a
+    sampled tree (the greedy tree walk's bytes are counted from its matches
+    in main())."""
     if isinstance(cfg, psi_inputs.TreeConfig):
         return algorithmic_bytes(cfg)
     es = 4 if cfg.dtype == "f32" else 2
@@ -288,6 +289,21 @@ def rows_read(cfg, n_emitted) -> int:
             total += rows_in_round(cfg, r)
             if L < r[1]:
                 break
+    return total
+
+
+def tree_rows_read(argmax, node_tokens, parents) -> int:
+    """Rows the greedy tree walk reads: per tree the root's and every matched
+    node's (node k is matched when its token is its parent row's argmax and
+    its parent is matched).  argmax [N, M+1], node_tokens / parents [N, M]."""
+    total = 0
+    for am, tok, par in zip(argmax, node_tokens, parents):
+        matched = []
+        for k in range(len(tok)):
+            p = int(par[k])
+            ok = -1 <= p < k and (p < 0 or matched[p])
+            matched.append(bool(ok and int(tok[k]) == int(am[p + 1])))
+        total += 1 + sum(matched)
     return total
 
 
@@ -504,14 +520,19 @@ def main():
     alg = main_launch_bytes(cfg)
     formula = algorithmic_bytes(cfg)
     es = 4 if getattr(cfg, "dtype", "bf16") == "f32" else 2
-    if is_tree:
+    if is_tree and cfg.temperature > 0:
         read = formula
+    elif is_tree:  # the walk reads the root's and the matched nodes' rows
+        am = batch.ar.float().argmax(dim=-1).cpu().numpy()
+        read = tree_rows_read(am, batch.node_tokens.cpu().numpy(),
+                              batch.parents.cpu().numpy()) * cfg.V * es
+        alg = read  # one launch: the walk
     else:
         read = rows_read(cfg, out.n_emitted.cpu().numpy()) * cfg.V * es
     peak, peak_kind = hbm_peak()
     achieved = alg / (main_ms / 1000.0) / 1e9
     if is_tree:
-        kernel = "psi_row_scan" if cfg.temperature > 0 else "psi_tree_argmax"
+        kernel = "psi_row_scan" if cfg.temperature > 0 else "psi_tree_walk"
     else:
         kernel = "psi_row_scan" if cfg.temperature > 0 else "psi_row_argmax"
 
@@ -534,14 +555,19 @@ def main():
                                  "sample": f"{n1} sequences ({dt1:.1f} s)"}}
 
     if rank == 0:
-        # our kernels per call: argmax + tree walk; greedy linear: per
+        # our kernels per call: greedy tree: the walk; sampled tree: row
+        # scan, row finish, walk; greedy linear: argmax and emit, or per
         # early-exit round list building and argmax, then emit; sampled: per
         # round list building, row scan, row finish and unit decision, then
         # one second pass of the three, the general-path list, fast_emit, the
         # nucleus draw and the whole-row draw
         rounds = 0 if is_tree else len(sampled_rounds(cfg))
-        if is_tree or (cfg.temperature == 0 and cfg.N < 64):
-            launches_per_step = 2  # tree: argmax + walk, or row scan + sampled walk
+        if is_tree and cfg.temperature == 0:
+            launches_per_step = 1  # the level-by-level walk
+        elif is_tree:
+            launches_per_step = 3  # row scan, row finish, sampled walk
+        elif cfg.temperature == 0 and cfg.N < 64:
+            launches_per_step = 2  # argmax + emit
         elif cfg.temperature == 0:  # per round: list building and argmax; then emit
             launches_per_step = 2 * rounds + 1
         elif cfg.N < 64:  # one pass: scan, finish, unit, their second passes, lists, emit, draw

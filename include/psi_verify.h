@@ -238,7 +238,8 @@ psi_status psi_verify_linear_noalloc(const void *ar_logits, int64_t ar_row_strid
                                      float *out_q_draft, uint32_t *dev_status,
                                      psi_stream_t stream);
 
-/* Workspace needed by psi_verify_tree_greedy (bytes; 0 on invalid sizes). */
+/* Workspace needed by psi_verify_tree_greedy (bytes; 0 on invalid sizes).
+ * The walk keeps its state in shared memory: 256 bytes for any valid sizes. */
 size_t psi_verify_tree_greedy_workspace_bytes(int32_t N, int32_t M, int32_t V,
                                               psi_dtype dtype);
 
@@ -258,6 +259,9 @@ size_t psi_verify_tree_greedy_workspace_bytes(int32_t N, int32_t M, int32_t V,
  * out_path_nodes int32 [N][M]: node indices root-side first, then -1.
  * out_path_len   int32 [N]: number of accepted nodes (0..M).
  * out_tokens     int32 [N][M+1]: accepted tokens, then the bonus, then -1.
+ * Rows read: the root's and each matched node's only (level by level, one
+ * cluster of CTAs per tree); the NONFINITE status bit covers those rows.
+ * Invalid parents and token ids are flagged for every node.
  * Limits: 1 <= N, 1 <= M <= PSI_MAX_TREE_NODES, 1 <= V <= PSI_MAX_V.
  */
 psi_status psi_verify_tree_greedy(const void *ar_logits, int64_t ar_row_stride,

@@ -246,9 +246,7 @@ size_t psi_verify_tree_greedy_workspace_bytes(int32_t N, int32_t M, int32_t V, p
   if (N < 1 || M < 1 || M > PSI_MAX_TREE_NODES || V < 1 || !valid_dtype(dtype) ||
       V > max_v(dtype))
     return 0;
-  const int64_t rows = (int64_t)N * (M + 1);
-  const psi::ArgmaxPlan plan = psi::plan_argmax(rows, V, elem_bytes(dtype));
-  return round256(sizeof(uint64_t) * (size_t)rows * plan.splits);
+  return 256;  // the walk keeps its state in shared memory; any buffer will do
 }
 
 psi_status psi_verify_tree_greedy(const void *ar_logits, int64_t ar_row_stride, psi_dtype dtype,
@@ -275,19 +273,10 @@ psi_status psi_verify_tree_greedy(const void *ar_logits, int64_t ar_row_stride, 
   const size_t need = psi_verify_tree_greedy_workspace_bytes(N, M, V, dtype);
   if (!workspace || workspace_bytes < need || !aligned_to(workspace, 16))
     return fail(PSI_ERR_WORKSPACE, "workspace %zu bytes, need %zu", workspace_bytes, need);
-  const int64_t rows = (int64_t)N * (M + 1);
-  const psi::ArgmaxPlan plan = psi::plan_argmax(rows, V, (int)es);
-  uint64_t *partial = static_cast<uint64_t *>(workspace);
-  cudaError_t e;
-  if (g_events.before && (e = cudaEventRecord(g_events.before, stream)) != cudaSuccess)
-    return cuda_fail(e, "event record");
-  e = psi::launch_row_argmax(ar_logits, ar_row_stride, dtype, rows, V, plan, partial, dev_status,
-                             stream);
-  if (e != cudaSuccess) return cuda_fail(e, "row_argmax launch");
-  if (g_events.after && (e = cudaEventRecord(g_events.after, stream)) != cudaSuccess)
-    return cuda_fail(e, "event record");
-  e = psi::launch_tree_walk(partial, plan.splits, node_tokens, parents, N, M, V, out_path_nodes,
-                            out_path_len, out_tokens, dev_status, stream);
+  const cudaError_t e =
+      psi::launch_tree_walk(ar_logits, ar_row_stride, dtype, node_tokens, parents, N, M, V,
+                            out_path_nodes, out_path_len, out_tokens, dev_status, g_events,
+                            stream);
   if (e != cudaSuccess) return cuda_fail(e, "tree_walk launch");
   return PSI_OK;
 }

@@ -511,20 +511,6 @@ __global__ void __launch_bounds__(128) fast_emit_kernel(const __grid_constant__ 
   else if (t == kTokenDraw) a.list_d[atomicAdd(&a.counters[8], 1)] = n * (B + 1) + L;
 }
 
-// SM count of the current device (queried once per device).
-int sm_count() {
-  static std::atomic<int> cached[PerDevice::kMax] = {};
-  const int dev = PerDevice::current();
-  const bool slot = dev >= 0 && dev < PerDevice::kMax;
-  int count = slot ? cached[dev].load(std::memory_order_relaxed) : 0;
-  if (count > 0) return count;
-  if (dev < 0 || cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      count <= 0)
-    count = 148;
-  if (slot) cached[dev].store(count, std::memory_order_relaxed);
-  return count;
-}
-
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
 // ---------------------------------------------------------------------------
@@ -577,10 +563,10 @@ template <typename Bits>
 cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool early_exit,
                               const KernelEvents &ev, cudaStream_t stream) {
   const int64_t units = (int64_t)fa.s.N * (fa.s.B + 1);
-  const int64_t persistent = (int64_t)sm_count() * 8;
+  const int64_t persistent = (int64_t)device_sm_count() * 8;
   const int64_t grid_unit = std::min<int64_t>((units + kUnitThreads - 1) / kUnitThreads, persistent);
   const int64_t grid_draw = std::min<int64_t>(fa.s.N, persistent);
-  const int64_t grid_finish = std::min<int64_t>(fa.rows, (int64_t)sm_count() * 8);
+  const int64_t grid_finish = std::min<int64_t>(fa.rows, (int64_t)device_sm_count() * 8);
   cudaError_t e;
   static DeviceOnce configure;  // carveouts, once per device
   e = configure([] {
@@ -643,7 +629,7 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
   sa.records = fa.rec;
   if (fa.top_k > 0) {
     e = launch_topk_units(sa, dt, fa.list_k, fa.counters + 9,
-                          std::min<int64_t>(units, (int64_t)sm_count() * 4), stream);
+                          std::min<int64_t>(units, (int64_t)device_sm_count() * 4), stream);
     if (e != cudaSuccess) return e;
   }
   const int clusters_a = (int)std::min<int64_t>(units, kListClusters);
@@ -660,7 +646,7 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
   // rows, where a cluster's launch and synchronisation cost more than the
   // row; a cluster per draw for long ones, which one SM reads too slowly
   if (fa.s.V <= kWrMaxVocab) {
-    const int32_t grid_wr = std::max<int32_t>(1, std::min<int32_t>(fa.s.N, sm_count()));
+    const int32_t grid_wr = std::max<int32_t>(1, std::min<int32_t>(fa.s.N, device_sm_count()));
     return launch_pdl(whole_row_draw_kernel<Bits>, dim3((unsigned)grid_wr), dim3(kWrThreads), 0,
                       stream, fa);
   }
@@ -672,7 +658,7 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
 }  // namespace
 
 cudaError_t launch_row_finish(const FastArgs &fa, psi_dtype dtype, cudaStream_t stream) {
-  const int64_t grid = std::min<int64_t>(fa.rows, (int64_t)sm_count() * 8);
+  const int64_t grid = std::min<int64_t>(fa.rows, (int64_t)device_sm_count() * 8);
   if (dtype == PSI_DTYPE_BF16) {
     static DeviceOnce configure;
     cudaError_t e = configure([] { return prefer_max_shared(row_finish_kernel<uint16_t>); });

@@ -8,9 +8,11 @@
 //                      word.  HBM-bound: 2 bytes per bf16 logit, no exp.
 //  greedy_emit_kernel  linear rule: accept while x_i == argmax_i, emit the
 //                      argmax of the first mismatching row (or the bonus row).
-//  tree_walk_kernel    tree rule: node matched when its token is its parent
-//                      row's argmax and its parent is matched; deepest
-//                      matched node ends the path.
+//  tree_greedy_walk_kernel  tree rule: node matched when its token is its
+//                      parent row's argmax and its parent is matched;
+//                      deepest matched node ends the path.  One cluster per
+//                      tree reads only the root's and the matched nodes'
+//                      rows, level by level.
 //
 // Sources: "Uno Psi-Spec 是什麼？..." (alphalab.site), section "Linear 與 Tree
 // sampler" (tree verify); greedy linear verify is the temperature-0 case of
@@ -89,25 +91,13 @@ __device__ __forceinline__ uint32_t float_key(float v) {
     return Elem<Bits>::key(__float_as_uint(v));
 }
 
-// grid: rows * splits CTAs; CTA (item, s) covers [s*chunk, min(V, (s+1)*chunk))
-// of row `item`, or of row rlist[item] for the first *rcount items when a
-// row list is given (the other CTAs exit).
+// The packed argmax of elements [c0, c1) of row r, over the CTA (every
+// thread gets it; 0 when the range is empty); any_bad: a NaN or +inf was
+// seen.  `red` (kWarps words) is free again after the caller's next barrier.
 template <typename Bits>
-__global__ void __launch_bounds__(kThreads) row_argmax_kernel(
-    const Bits *__restrict__ logits, int64_t row_stride, int32_t V, int32_t splits,
-    int32_t chunk, uint64_t *__restrict__ partial, uint32_t *dev_status,
-    const int32_t *__restrict__ rlist, const int32_t *__restrict__ rcount) {
-  pdl_wait();  // the previous kernel's results are visible
-  pdl_trigger();
+__device__ __forceinline__ uint64_t cta_chunk_argmax(const Bits *r, int32_t c0, int32_t c1,
+                                                     uint64_t *red, bool &any_bad) {
   constexpr int VEC = Elem<Bits>::kVec;
-  const int64_t item = blockIdx.x / splits;
-  const int32_t s = blockIdx.x % splits;
-  if (rlist && item >= *rcount) return;
-  const int64_t row = rlist ? (int64_t)rlist[item] : item;
-  const Bits *r = logits + row * row_stride;
-  const int32_t c0 = s * chunk;
-  const int32_t c1 = min(V, c0 + chunk);
-
   RunMax rm;
 
   // 16-byte aligned middle part [a0, a1), scalar head and tail.
@@ -139,17 +129,37 @@ __global__ void __launch_bounds__(kThreads) row_argmax_kernel(
   if (rm.idx != 0xFFFFFFFFu) packed = pack_argmax(float_key<Bits>(rm.val), rm.idx);
   else if (c0 < c1) packed = pack_argmax(float_key<Bits>(-INFINITY), (uint32_t)c0);
   packed = warp_max_u64(packed);
-  __shared__ uint64_t red[kWarps];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (lane == 0) red[warp] = packed;
-  const bool any_bad = __syncthreads_or(rm.bad);
-  if (warp == 0) {
-    uint64_t x = lane < kWarps ? red[lane] : 0ull;
-    x = warp_max_u64(x);
-    if (lane == 0) {
-      partial[row * splits + s] = x;
-      if (any_bad && dev_status) atomicOr(dev_status, PSI_DEV_NONFINITE);
-    }
+  any_bad = __syncthreads_or(rm.bad);
+  uint64_t x = 0ull;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) x = red[w] > x ? red[w] : x;
+  return x;
+}
+
+// grid: rows * splits CTAs; CTA (item, s) covers [s*chunk, min(V, (s+1)*chunk))
+// of row `item`, or of row rlist[item] for the first *rcount items when a
+// row list is given (the other CTAs exit).
+template <typename Bits>
+__global__ void __launch_bounds__(kThreads) row_argmax_kernel(
+    const Bits *__restrict__ logits, int64_t row_stride, int32_t V, int32_t splits,
+    int32_t chunk, uint64_t *__restrict__ partial, uint32_t *dev_status,
+    const int32_t *__restrict__ rlist, const int32_t *__restrict__ rcount) {
+  pdl_wait();  // the previous kernel's results are visible
+  pdl_trigger();
+  const int64_t item = blockIdx.x / splits;
+  const int32_t s = blockIdx.x % splits;
+  if (rlist && item >= *rcount) return;
+  const int64_t row = rlist ? (int64_t)rlist[item] : item;
+  const int32_t c0 = s * chunk;
+  __shared__ uint64_t red[kWarps];
+  bool any_bad;
+  const uint64_t x = cta_chunk_argmax<Bits>(logits + row * row_stride, c0, min(V, c0 + chunk),
+                                            red, any_bad);
+  if (threadIdx.x == 0) {
+    partial[row * splits + s] = x;
+    if (any_bad && dev_status) atomicOr(dev_status, PSI_DEV_NONFINITE);
   }
 }
 
@@ -188,74 +198,129 @@ __global__ void __launch_bounds__(128) greedy_emit_kernel(
   if (bad_id && dev_status) atomicOr(dev_status, PSI_DEV_BAD_TOKEN_ID);
 }
 
-// One CTA per sequence: argmaxes and node data staged in shared memory, then
-// one thread walks the nodes in index order (parents precede children).
-__global__ void __launch_bounds__(kThreads) tree_walk_kernel(
-    const uint64_t *__restrict__ partial, int32_t splits,
-    const int32_t *__restrict__ node_tokens, const int32_t *__restrict__ parents,
-    int32_t M, int32_t V, int32_t *__restrict__ out_path_nodes,
-    int32_t *__restrict__ out_path_len, int32_t *__restrict__ out_tokens,
-    uint32_t *dev_status) {
+// Greedy tree, level by level: one cluster of C CTAs per tree (C = the
+// cluster size, 1 to 8).  Only the rows that the rule needs are read: the
+// root's and each matched node's.  A row's argmax is reduced over the
+// cluster: CTA c scans elements [c * chunk, (c + 1) * chunk) and the C CTA
+// maxima meet in distributed shared memory.  The matched children of a read
+// row are queued in index order, so every CTA of the cluster reads the same
+// rows in the same order and takes the same decisions.
+template <typename Bits>
+__global__ void __launch_bounds__(kThreads) tree_greedy_walk_kernel(
+    const Bits *__restrict__ logits, int64_t row_stride, int32_t V, int32_t chunk,
+    const int32_t *__restrict__ node_tokens, const int32_t *__restrict__ parents, int32_t M,
+    int32_t *__restrict__ out_path_nodes, int32_t *__restrict__ out_path_len,
+    int32_t *__restrict__ out_tokens, uint32_t *dev_status) {
   pdl_wait();  // the previous kernel's results are visible
   pdl_trigger();
   extern __shared__ int32_t sm[];
-  int32_t *am = sm;              // [M+1]
-  int32_t *tok = am + (M + 1);   // [M]
-  int32_t *par = tok + M;        // [M]
-  int32_t *depth = par + M;      // [M], 0 = unmatched
-  int32_t *path = depth + M;     // [M+1]
+  int32_t *par = sm;              // [M] parent; -2 for an invalid node
+  int32_t *tok = par + M;         // [M]
+  int32_t *depth = tok + M;       // [M] 0 = not matched
+  int32_t *path = depth + M;      // [M]
+  int32_t *queue = path + M;      // [M+1] rows to read, in order
+  int32_t *am = queue + (M + 1);  // [M+1] argmax of each row read
+  __shared__ uint64_t red[kWarps];
+  __shared__ uint64_t slot[2];  // this CTA's maximum of the current row (two buffers)
+  __shared__ int32_t wcnt[kWarps];
+  __shared__ uint32_t bad_nodes;
   __shared__ int32_t s_best, s_len;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t C = cluster_size(), rank = cluster_rank();
+  const int64_t n = blockIdx.x / C;
 
-  const int64_t n = blockIdx.x;
-  for (int32_t j = threadIdx.x; j <= M; j += blockDim.x)
-    am[j] = argmax_of(partial, n * (M + 1) + j, splits);
-  for (int32_t k = threadIdx.x; k < M; k += blockDim.x) {
-    tok[k] = node_tokens[n * M + k];
-    par[k] = parents[n * M + k];
+  if (tid == 0) bad_nodes = 0u;
+  __syncthreads();
+  uint32_t st = 0u;
+  for (int32_t k = tid; k < M; k += kThreads) {
+    const int32_t p = parents[n * M + k], t = node_tokens[n * M + k];
+    bool ok = true;
+    if (p < -1 || p >= k) {
+      st |= PSI_DEV_BAD_PARENT;
+      ok = false;
+    } else if (t < 0 || t >= V) {
+      st |= PSI_DEV_BAD_TOKEN_ID;
+      ok = false;
+    }
+    par[k] = ok ? p : -2;
+    tok[k] = t;
+    depth[k] = 0;
   }
+  if (st) atomicOr(&bad_nodes, st);
+  if (tid == 0) queue[0] = 0;  // the root's row
   __syncthreads();
 
-  if (threadIdx.x == 0) {
-    uint32_t status = 0;
-    int32_t best = -1, best_depth = 0;
-    for (int32_t k = 0; k < M; ++k) {
-      depth[k] = 0;
-      const int32_t p = par[k];
-      if (p < -1 || p >= k) {
-        status |= PSI_DEV_BAD_PARENT;
-        continue;
-      }
-      const int32_t t = tok[k];
-      if (t < 0 || t >= V) {
-        status |= PSI_DEV_BAD_TOKEN_ID;
-        continue;
-      }
-      const int32_t pd = (p < 0) ? 0 : depth[p];
-      if ((p < 0 || pd > 0) && t == am[p + 1]) {
-        depth[k] = pd + 1;
-        if (depth[k] > best_depth) {
-          best_depth = depth[k];
-          best = k;
-        }
-      }
+  const Bits *rows = logits + n * (int64_t)(M + 1) * row_stride;
+  const int32_t c0 = min(V, (int32_t)rank * chunk), c1 = min(V, c0 + chunk);
+  bool bad_rows = false;
+  int32_t qn = 1;  // rows queued (the same in every thread of the cluster)
+  for (int32_t qi = 0; qi < qn; ++qi) {
+    const int32_t row = queue[qi];
+    bool bad;
+    const uint64_t x = cta_chunk_argmax<Bits>(rows + row * row_stride, c0, c1, red, bad);
+    bad_rows |= bad;
+    if (tid == 0) slot[qi & 1] = x;
+    // every CTA's maximum of the row is posted; `red` and the other slot
+    // buffer are free (their readers are past this barrier)
+    cluster_sync();
+    uint64_t best = 0ull;
+    for (uint32_t c = 0; c < C; ++c) {
+      const uint64_t y = dsmem_ld_u64(dsmem_map(&slot[qi & 1], c));
+      best = y > best ? y : best;
     }
+    const int32_t a = (int32_t)(0xFFFFFFFFu - (uint32_t)best);
+    if (tid == 0) am[row] = a;
+    const int32_t pd = row == 0 ? 0 : depth[row - 1];
+    // the row's node's children whose token is the argmax: matched, queued
+    // in index order
+    for (int32_t base = 0; base < M; base += kThreads) {
+      const int32_t k = base + tid;
+      const bool hit = k < M && par[k] == row - 1 && tok[k] == a;
+      const uint32_t bal = __ballot_sync(0xFFFFFFFFu, hit);
+      if (lane == 0) wcnt[warp] = __popc(bal);
+      __syncthreads();
+      int32_t off = qn, total = 0;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        off += w < warp ? wcnt[w] : 0;
+        total += wcnt[w];
+      }
+      if (hit) {
+        depth[k] = pd + 1;
+        queue[off + __popc(bal & ((1u << lane) - 1u))] = k + 1;
+      }
+      qn += total;
+      __syncthreads();  // the queue and depths are visible; wcnt is free
+    }
+  }
+  if (tid == 0 && bad_rows && dev_status) atomicOr(dev_status, PSI_DEV_NONFINITE);
+  cluster_sync();  // no CTA leaves while another may still read its slots
+  if (rank != 0) return;
+
+  // the deepest matched node (lowest index among equals) ends the path
+  if (tid == 0) {
+    int32_t best = -1, best_depth = 0;
+    for (int32_t k = 0; k < M; ++k)
+      if (depth[k] > best_depth) {
+        best_depth = depth[k];
+        best = k;
+      }
     int32_t d = best_depth;
     for (int32_t k = best; k >= 0; k = par[k]) path[--d] = k;
     s_best = best;
     s_len = best_depth;
-    if (status && dev_status) atomicOr(dev_status, status);
+    if (bad_nodes && dev_status) atomicOr(dev_status, bad_nodes);
   }
   __syncthreads();
   const int32_t len = s_len;
-  for (int32_t k = threadIdx.x; k < M; k += blockDim.x)
-    out_path_nodes[n * M + k] = k < len ? path[k] : -1;
-  for (int32_t k = threadIdx.x; k <= M; k += blockDim.x) {
+  for (int32_t k = tid; k < M; k += kThreads) out_path_nodes[n * M + k] = k < len ? path[k] : -1;
+  for (int32_t k = tid; k <= M; k += kThreads) {
     int32_t v = -1;
     if (k < len) v = tok[path[k]];
     else if (k == len) v = am[s_best + 1];
     out_tokens[n * (M + 1) + k] = v;
   }
-  if (threadIdx.x == 0) out_path_len[n] = len;
+  if (tid == 0) out_path_len[n] = len;
 }
 
 // ---------------------------------------------------------------------------
@@ -388,22 +453,64 @@ cudaError_t launch_greedy_emit(const uint64_t *partial, int32_t splits, const in
                     splits, ids, N, B, V, out_tokens, out_n, dev_status);
 }
 
-cudaError_t launch_tree_walk(const uint64_t *partial, int32_t splits, const int32_t *node_tokens,
-                             const int32_t *parents, int32_t N, int32_t M, int32_t V,
-                             int32_t *out_path_nodes, int32_t *out_path_len,
-                             int32_t *out_tokens, uint32_t *dev_status, cudaStream_t stream) {
-  const size_t smem = sizeof(int32_t) * (size_t)(5 * M + 2);
+template <typename Bits>
+cudaError_t launch_tree_walk_typed(const Bits *logits, int64_t row_stride,
+                                   const int32_t *node_tokens, const int32_t *parents, int32_t N,
+                                   int32_t M, int32_t V, int32_t *out_path_nodes,
+                                   int32_t *out_path_len, int32_t *out_tokens,
+                                   uint32_t *dev_status, const KernelEvents &ev,
+                                   cudaStream_t stream) {
+  // the cluster spreads a tree's rows over up to 8 SMs while the trees
+  // leave SMs idle
+  int C = 8;
+  while (C > 1 && (int64_t)N * C > 2LL * device_sm_count()) C >>= 1;
+  if ((int64_t)N * C > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+  constexpr int VEC = Elem<Bits>::kVec;
+  const int32_t chunk = ((V + C - 1) / C + VEC - 1) / VEC * VEC;
+  const size_t smem = sizeof(int32_t) * (size_t)(6 * M + 2);
   static DeviceOnce configure;  // opt in to > 48 KB once per device (only large M needs it)
-  if (smem > 48 * 1024) {
-    const cudaError_t e = configure([] {
-      return cudaFuncSetAttribute(tree_walk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  (int)(5 * PSI_MAX_TREE_NODES + 2) * 4);
-    });
-    if (e != cudaSuccess) return e;
-  }
-  return launch_pdl(tree_walk_kernel, dim3(N), dim3(kThreads), smem, stream, partial, splits,
-                    node_tokens, parents, M, V, out_path_nodes, out_path_len, out_tokens,
-                    dev_status);
+  const cudaError_t ce = configure([] {
+    return cudaFuncSetAttribute(tree_greedy_walk_kernel<Bits>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)(6 * PSI_MAX_TREE_NODES + 2) * 4);
+  });
+  if (ce != cudaSuccess) return ce;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(N * C), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see launch_pdl
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaError_t e;
+  if (ev.before && (e = cudaEventRecord(ev.before, stream)) != cudaSuccess) return e;
+  e = cudaLaunchKernelEx(&cfg, tree_greedy_walk_kernel<Bits>, logits, row_stride, V, chunk,
+                         node_tokens, parents, M, out_path_nodes, out_path_len, out_tokens,
+                         dev_status);
+  if (e != cudaSuccess) return e;
+  if (ev.after && (e = cudaEventRecord(ev.after, stream)) != cudaSuccess) return e;
+  return cudaSuccess;
+}
+
+cudaError_t launch_tree_walk(const void *logits, int64_t row_stride, psi_dtype dtype,
+                             const int32_t *node_tokens, const int32_t *parents, int32_t N,
+                             int32_t M, int32_t V, int32_t *out_path_nodes,
+                             int32_t *out_path_len, int32_t *out_tokens, uint32_t *dev_status,
+                             const KernelEvents &ev, cudaStream_t stream) {
+  if (dtype == PSI_DTYPE_BF16)
+    return launch_tree_walk_typed(static_cast<const uint16_t *>(logits), row_stride, node_tokens,
+                                  parents, N, M, V, out_path_nodes, out_path_len, out_tokens,
+                                  dev_status, ev, stream);
+  return launch_tree_walk_typed(static_cast<const uint32_t *>(logits), row_stride, node_tokens,
+                                parents, N, M, V, out_path_nodes, out_path_len, out_tokens,
+                                dev_status, ev, stream);
 }
 
 }  // namespace psi

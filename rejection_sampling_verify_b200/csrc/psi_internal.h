@@ -26,6 +26,20 @@ struct PerDevice {
   }
 };
 
+// SM count of the current device (queried once per device).
+inline int device_sm_count() {
+  static std::atomic<int> cached[PerDevice::kMax] = {};
+  const int dev = PerDevice::current();
+  const bool slot = dev >= 0 && dev < PerDevice::kMax;
+  int n = slot ? cached[dev].load(std::memory_order_relaxed) : 0;
+  if (n > 0) return n;
+  if (dev < 0 || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      n <= 0)
+    n = 148;
+  if (slot) cached[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
 class DeviceOnce {
  public:
   // Runs f() unless it already succeeded on the current device.
@@ -102,10 +116,11 @@ cudaError_t launch_greedy_early_exit(const void *logits, int64_t row_stride, psi
                                      uint32_t *dev_status, const KernelEvents &ev,
                                      cudaStream_t stream);
 
-cudaError_t launch_tree_walk(const uint64_t *partial, int32_t splits, const int32_t *node_tokens,
-                             const int32_t *parents, int32_t N, int32_t M, int32_t V,
-                             int32_t *out_path_nodes, int32_t *out_path_len,
-                             int32_t *out_tokens, uint32_t *dev_status, cudaStream_t stream);
+cudaError_t launch_tree_walk(const void *logits, int64_t row_stride, psi_dtype dtype,
+                             const int32_t *node_tokens, const int32_t *parents, int32_t N,
+                             int32_t M, int32_t V, int32_t *out_path_nodes,
+                             int32_t *out_path_len, int32_t *out_tokens, uint32_t *dev_status,
+                             const KernelEvents &ev, cudaStream_t stream);
 
 // ---- sampled linear path -----------------------------------------------------
 // Per (sequence, row) record written by the unit kernel, read by the emit

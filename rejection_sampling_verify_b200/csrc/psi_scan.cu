@@ -742,20 +742,6 @@ __global__ void __launch_bounds__(kScanThreads, 1) row_scan_kernel(const __grid_
     atomicOr(a.s.dev_status, PSI_DEV_TIMEOUT);
 }
 
-// SM count of the current device (queried once per device).
-int scan_sm_count() {
-  static std::atomic<int> cached[PerDevice::kMax] = {};
-  const int dev = PerDevice::current();
-  const bool slot = dev >= 0 && dev < PerDevice::kMax;
-  int n = slot ? cached[dev].load(std::memory_order_relaxed) : 0;
-  if (n > 0) return n;
-  if (dev < 0 || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-      n <= 0)
-    n = 148;
-  if (slot) cached[dev].store(n, std::memory_order_relaxed);
-  return n;
-}
-
 template <typename Bits, int C>
 cudaError_t launch_scan_typed(const FastArgs &fa, cudaStream_t stream) {
   static DeviceOnce configure;
@@ -769,7 +755,7 @@ cudaError_t launch_scan_typed(const FastArgs &fa, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   // one CTA per SM: groups of C CTAs, each group scanning its rows' C slices
   const int64_t groups =
-      std::min<int64_t>(std::max(1, scan_sm_count() / C), std::max<int64_t>(fa.rows, 1));
+      std::min<int64_t>(std::max(1, device_sm_count() / C), std::max<int64_t>(fa.rows, 1));
   return launch_pdl(row_scan_kernel<Bits, C>, dim3((unsigned)(groups * C)), dim3(kScanThreads),
                     kScanDynSmem, stream, fa);
 }

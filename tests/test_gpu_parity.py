@@ -143,6 +143,40 @@ def test_tree_handmade_and_flags():
         assert_tree_parity(gpu_tree(tb), oracle_tree(tb))
 
 
+@pytest.mark.parametrize("N", [1, 40, 100, 200])
+def test_tree_cluster_sizes(N):
+    """The walk's cluster shrinks as the batch grows (8, 4, 2, 1 CTAs per tree
+    on 148 SMs); an odd vocabulary leaves a ragged last chunk."""
+    cfg = psi_inputs.TreeConfig(**{**CFG["tree_greedy"].__dict__, "N": N, "V": 5003})
+    tb = psi_inputs.tree_batch(cfg, device="cuda", index=N)
+    assert_tree_parity(gpu_tree(tb), oracle_tree(tb))
+
+
+def test_tree_status_covers_the_rows_read():
+    """Only the root's and the matched nodes' rows are read: a NaN in an
+    unmatched node's row leaves the status clear, one in a matched node's row
+    sets it.  Tokens and paths equal the oracle's either way."""
+    V = 6
+
+    def batch(nan_row):
+        r = torch.zeros(4, V)
+        for j, a in enumerate([1, 3, 0, 5]):
+            r[j, a] = 2.0
+        r[nan_row, 4] = float("nan")
+        # node 0 (token 1) matches the root's argmax, node 1 (token 2) does not;
+        # node 2 (token 3) is node 0's child and matches
+        return psi_inputs.TreeBatch(r[None].contiguous(), torch.tensor([[1, 2, 3]], dtype=torch.int32),
+                                    torch.tensor([[-1, -1, 0]], dtype=torch.int32), None)
+
+    for nan_row, read in ((2, False), (1, True)):
+        tb = batch(nan_row)
+        g, o = gpu_tree(tb), oracle_tree(tb)
+        for k in ("path_nodes", "path_len", "tokens"):
+            assert np.array_equal(g[k], o[k]), k
+        assert o["status"] == oracle.NONFINITE
+        assert g["status"] == (oracle.NONFINITE if read else 0), (nan_row, g["status"])
+
+
 def test_tree_large_random():
     """Many nodes (M = 2000), random valid parents, small vocabulary so that
     matches are frequent."""
