@@ -263,6 +263,10 @@ __device__ __forceinline__ void dsmem_st_f32(uint32_t cluster_addr, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_addr), "f"(v) : "memory");
 }
 
+__device__ __forceinline__ void dsmem_st_u64(uint32_t cluster_addr, uint64_t v) {
+  asm volatile("st.shared::cluster.u64 [%0], %1;" ::"r"(cluster_addr), "l"(v) : "memory");
+}
+
 // 16-byte shared-memory load.
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;

@@ -94,7 +94,8 @@ __device__ __forceinline__ uint32_t float_key(float v) {
 // The packed argmax of elements [c0, c1) of row r, over the CTA (every
 // thread gets it; 0 when the range is empty); any_bad: a NaN or +inf was
 // seen.  `red` (kWarps words) is free again after the caller's next barrier.
-template <typename Bits>
+// U: 16-byte loads in flight per thread.
+template <typename Bits, int U = 4>
 __device__ __forceinline__ uint64_t cta_chunk_argmax(const Bits *r, int32_t c0, int32_t c1,
                                                      uint64_t *red, bool &any_bad) {
   constexpr int VEC = Elem<Bits>::kVec;
@@ -110,7 +111,6 @@ __device__ __forceinline__ uint64_t cta_chunk_argmax(const Bits *r, int32_t c0, 
   for (int32_t v = c0 + threadIdx.x; v < a0; v += kThreads) scan_scalar<Bits>(r[v], v, rm);
 
   const uint4 *vp = reinterpret_cast<const uint4 *>(r + a0);
-  constexpr int U = 4;  // vectors in flight per thread
   int32_t j = threadIdx.x;
   for (; j + (U - 1) * kThreads < nvec; j += U * kThreads) {
     uint4 w[U];
@@ -205,6 +205,9 @@ __global__ void __launch_bounds__(128) greedy_emit_kernel(
 // maxima meet in distributed shared memory.  The matched children of a read
 // row are queued in index order, so every CTA of the cluster reads the same
 // rows in the same order and takes the same decisions.
+constexpr int kWalkLoads = 8;       // 16-byte loads in flight per thread of the walk
+constexpr int kWalkMaxCluster = 8;  // CTAs per tree at most
+
 template <typename Bits>
 __global__ void __launch_bounds__(kThreads) tree_greedy_walk_kernel(
     const Bits *__restrict__ logits, int64_t row_stride, int32_t V, int32_t chunk,
@@ -221,7 +224,8 @@ __global__ void __launch_bounds__(kThreads) tree_greedy_walk_kernel(
   int32_t *queue = path + M;      // [M+1] rows to read, in order
   int32_t *am = queue + (M + 1);  // [M+1] argmax of each row read
   __shared__ uint64_t red[kWarps];
-  __shared__ uint64_t slot[2];  // this CTA's maximum of the current row (two buffers)
+  // every CTA's maximum of the current row, slot[b][c] from CTA c (two buffers)
+  __shared__ uint64_t slot[2][kWalkMaxCluster];
   __shared__ int32_t wcnt[kWarps];
   __shared__ uint32_t bad_nodes;
   __shared__ int32_t s_best, s_len;
@@ -257,17 +261,15 @@ __global__ void __launch_bounds__(kThreads) tree_greedy_walk_kernel(
   for (int32_t qi = 0; qi < qn; ++qi) {
     const int32_t row = queue[qi];
     bool bad;
-    const uint64_t x = cta_chunk_argmax<Bits>(rows + row * row_stride, c0, c1, red, bad);
+    const uint64_t x =
+        cta_chunk_argmax<Bits, kWalkLoads>(rows + row * row_stride, c0, c1, red, bad);
     bad_rows |= bad;
-    if (tid == 0) slot[qi & 1] = x;
-    // every CTA's maximum of the row is posted; `red` and the other slot
-    // buffer are free (their readers are past this barrier)
+    if (tid < (int)C) dsmem_st_u64(dsmem_map(&slot[qi & 1][rank], (uint32_t)tid), x);
+    // every CTA's maximum of the row has reached every CTA; `red` and the
+    // other slot buffer are free (their readers are past this barrier)
     cluster_sync();
     uint64_t best = 0ull;
-    for (uint32_t c = 0; c < C; ++c) {
-      const uint64_t y = dsmem_ld_u64(dsmem_map(&slot[qi & 1], c));
-      best = y > best ? y : best;
-    }
+    for (uint32_t c = 0; c < C; ++c) best = slot[qi & 1][c] > best ? slot[qi & 1][c] : best;
     const int32_t a = (int32_t)(0xFFFFFFFFu - (uint32_t)best);
     if (tid == 0) am[row] = a;
     const int32_t pd = row == 0 ? 0 : depth[row - 1];
@@ -294,7 +296,7 @@ __global__ void __launch_bounds__(kThreads) tree_greedy_walk_kernel(
     }
   }
   if (tid == 0 && bad_rows && dev_status) atomicOr(dev_status, PSI_DEV_NONFINITE);
-  cluster_sync();  // no CTA leaves while another may still read its slots
+  cluster_sync();  // no CTA leaves while another may still write its slots
   if (rank != 0) return;
 
   // the deepest matched node (lowest index among equals) ends the path
@@ -462,7 +464,7 @@ cudaError_t launch_tree_walk_typed(const Bits *logits, int64_t row_stride,
                                    cudaStream_t stream) {
   // the cluster spreads a tree's rows over up to 8 SMs while the trees
   // leave SMs idle
-  int C = 8;
+  int C = kWalkMaxCluster;
   while (C > 1 && (int64_t)N * C > 2LL * device_sm_count()) C >>= 1;
   if ((int64_t)N * C > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
   constexpr int VEC = Elem<Bits>::kVec;
