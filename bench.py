@@ -559,8 +559,8 @@ def main():
         # scan, row finish, walk; greedy linear: argmax and emit, or per
         # early-exit round list building and argmax, then emit; sampled: per
         # round list building, row scan, row finish and unit decision, then
-        # one second pass of the three, the general-path list, fast_emit, the
-        # nucleus draw and the whole-row draw
+        # one second pass of the three, the general-path list, fast_emit and
+        # the draws (over the nucleus with top-p, else over the whole row)
         rounds = 0 if is_tree else len(sampled_rounds(cfg))
         if is_tree and cfg.temperature == 0:
             launches_per_step = 1  # the level-by-level walk
@@ -571,9 +571,9 @@ def main():
         elif cfg.temperature == 0:  # per round: list building and argmax; then emit
             launches_per_step = 2 * rounds + 1
         elif cfg.N < 64:  # one pass: scan, finish, unit, their second passes, lists, emit, draw
-            launches_per_step = 10
+            launches_per_step = 9
         else:
-            launches_per_step = 4 * rounds + 7
+            launches_per_step = 4 * rounds + 6
         line = {
             "metric": METRIC, "value": value, "unit": "blocks/s", "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,

@@ -37,7 +37,9 @@
 //   whole_row_draw  Without top-p (and top-k) the draw spans the vocabulary:
 //              for rows of up to kWrMaxVocab entries, one CTA per such
 //              position, from the rows' finished maxima and normalisers;
-//              longer rows go to the cluster kernel in sample mode.
+//              longer rows go to the cluster kernel in sample mode.  A call
+//              launches either the draw kernel (top-p or top-k on) or the
+//              whole-row draw, never both.
 #include <algorithm>
 
 #include "psi_finish.cuh"
@@ -639,9 +641,11 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
   if ((e = launch_pdl(fast_emit_kernel, dim3((fa.s.N + 127) / 128), dim3(128), 0, stream, fa)) !=
       cudaSuccess)
     return e;
-  if ((e = launch_pdl(draw_kernel<Bits>, dim3((unsigned)grid_draw), dim3(kDrawThreads), 0,
-                      stream, fa)) != cudaSuccess)
-    return e;
+  // a call's draws are all of one kind: over the nucleus when the window is
+  // in use (top-p or top-k), else over the whole row
+  if (fa.use_window)
+    return launch_pdl(draw_kernel<Bits>, dim3((unsigned)grid_draw), dim3(kDrawThreads), 0, stream,
+                      fa);
   // the whole-row draws (no top-p, no top-k): one CTA per draw for short
   // rows, where a cluster's launch and synchronisation cost more than the
   // row; a cluster per draw for long ones, which one SM reads too slowly
