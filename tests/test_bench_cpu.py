@@ -68,6 +68,22 @@ def test_main_launch_bytes_is_the_first_round():
 
 # ---- the kernel-source hash behind `traffic` ----------------------------------------
 
+def test_tree_rows_read_follows_the_matches():
+    """The greedy tree walk reads the root's row and each matched node's:
+    node 0 (token 1) and node 1 (token 1, a duplicate sibling) match the
+    root's argmax 1; node 2 matches node 0's row; node 3's parent row (node 1)
+    has argmax 0, not its token; node 4 hangs off the unmatched node 3; node 5
+    has an invalid parent."""
+    am = np.array([[1, 2, 0, 5, 4, 3, 0]])   # argmax of rows 0..M (row k+1 = node k)
+    tok = np.array([[1, 1, 2, 3, 4, 0]])
+    par = np.array([[-1, -1, 0, 1, 3, 7]])
+    assert bench.tree_rows_read(am, tok, par) == 1 + 3
+    # nothing matched: the root's row only; two trees add up
+    assert bench.tree_rows_read(np.array([[9, 0, 0]]), np.array([[1, 2]]), np.array([[-1, 0]])) == 1
+    assert bench.tree_rows_read(np.concatenate([am, am]), np.concatenate([tok, tok]),
+                                np.concatenate([par, par])) == 8
+
+
 def test_comment_stripping_matches_the_compiler():
     """gcc's own comment removal (-fpreprocessed) leaves the same code, up to
     whitespace (gcc also drops `#pragma once` from a main file)."""
