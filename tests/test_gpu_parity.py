@@ -177,6 +177,22 @@ def test_tree_status_covers_the_rows_read():
         assert g["status"] == (oracle.NONFINITE if read else 0), (nan_row, g["status"])
 
 
+def test_tree_max_nodes():
+    """PSI_MAX_TREE_NODES nodes per tree (the walk's largest shared-memory
+    footprint), deep random trees and a 2-token vocabulary, so that many
+    nodes match and long matched paths occur."""
+    rng = np.random.default_rng(9)
+    N, M, V = 2, psi.PSI_MAX_TREE_NODES, 2
+    par = np.array([[rng.integers(max(-1, k - 8), k) for k in range(M)] for _ in range(N)],
+                   dtype=np.int32)
+    ar = torch.tensor(rng.integers(0, 6, (N, M + 1, V)), dtype=torch.float32)
+    tok = rng.integers(0, V, (N, M)).astype(np.int32)
+    tb = psi_inputs.TreeBatch(ar, torch.tensor(tok), torch.tensor(par), None)
+    g, o = gpu_tree(tb), oracle_tree(tb)
+    assert_tree_parity(g, o)
+    assert o["path_len"].max() >= 4
+
+
 def test_tree_large_random():
     """Many nodes (M = 2000), random valid parents, small vocabulary so that
     matches are frequent."""
@@ -227,7 +243,7 @@ def test_sampled_nucleus_recipe_reduced(step):
     assert_linear_parity(gpu_linear(b, cfg.seed, step), oracle_linear(b, cfg.seed, step))
 
 
-@pytest.mark.parametrize("V", [1, 2, 33, 1000, 12289, 65537, 151936])
+@pytest.mark.parametrize("V", [1, 2, 33, 1000, 12289, 16384, 16392, 65537, 151936])
 @pytest.mark.parametrize("top_p", [1.0, 0.9])
 def test_sampled_shapes_bf16(V, top_p):
     rng = torch.Generator().manual_seed(V + int(top_p * 10))
