@@ -28,8 +28,9 @@
 //              whose lists overflowed (rescanned with the exact maximum
 //              known); once, after the last round.
 //   (cluster kernel, list mode)  Units the second pass could not settle.
-//   fast_emit  First rejected position per sequence; emitted tokens; lists
-//              the position whose token is still to be drawn.
+//   fast_emit  One warp per sequence: the first rejected position (a ballot
+//              over the positions), the emitted tokens, and the position
+//              whose token is still to be drawn, listed.
 //   draw       One CTA per listed position: the correction (residual
 //              max(0, p - q)) or bonus draw over p's nucleus, inverse CDF in
 //              vocabulary order on exact integer sums.  Only the emitted
@@ -489,28 +490,30 @@ __global__ void __launch_bounds__(kWrThreads) whole_row_draw_kernel(const __grid
 // ---------------------------------------------------------------------------
 // fast_emit: one thread per sequence.
 // ---------------------------------------------------------------------------
+static_assert(PSI_MAX_B <= 32, "fast_emit: one lane per drafted position");
+
 __global__ void __launch_bounds__(128) fast_emit_kernel(const __grid_constant__ FastArgs a) {
   pdl_wait();  // the previous kernel's results are visible
   pdl_trigger();
-  const int32_t n = blockIdx.x * blockDim.x + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int64_t n = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;  // one warp per sequence
   const SampledArgs &s = a.s;
   if (n >= s.N) return;
-  const int32_t B = s.B;
-  const UnitRecord *r = a.rec + (int64_t)n * (B + 1);
-  int32_t L = B;
-  for (int32_t i = 0; i < B; ++i)
-    if (!r[i].accept) {
-      L = i;
-      break;
-    }
-  int32_t *tok = s.out_tokens + (int64_t)n * (B + 1);
-  for (int32_t i = 0; i < L; ++i) tok[i] = s.ids[(int64_t)n * B + i];
+  const int32_t B = s.B;  // <= 32: lane i holds position i
+  const UnitRecord *r = a.rec + n * (B + 1);
+  // the first rejected position (positions past it may hold records of an
+  // earlier call: only the lowest rejection counts, and every position
+  // before it was decided in this call)
+  const uint32_t rej = __ballot_sync(0xFFFFFFFFu, lane < B && !r[lane].accept);
+  const int32_t L = rej ? __ffs(rej) - 1 : B;
   const int32_t t = r[L].token;
-  tok[L] = t;
-  for (int32_t i = L + 1; i <= B; ++i) tok[i] = -1;
-  s.out_n[n] = L + 1;
-  if (t == kTokenWholeRow) a.list_b[atomicAdd(&a.counters[1], 1)] = n * (B + 1) + L;
-  else if (t == kTokenDraw) a.list_d[atomicAdd(&a.counters[8], 1)] = n * (B + 1) + L;
+  int32_t *tok = s.out_tokens + n * (B + 1);
+  for (int32_t i = lane; i <= B; i += 32) tok[i] = i < L ? s.ids[n * B + i] : (i == L ? t : -1);
+  if (lane == 0) {
+    s.out_n[n] = L + 1;
+    if (t == kTokenWholeRow) a.list_b[atomicAdd(&a.counters[1], 1)] = (int32_t)(n * (B + 1) + L);
+    else if (t == kTokenDraw) a.list_d[atomicAdd(&a.counters[8], 1)] = (int32_t)(n * (B + 1) + L);
+  }
 }
 
 size_t align256(size_t x) { return (x + 255) / 256 * 256; }
@@ -638,7 +641,7 @@ cudaError_t launch_fast_typed(const FastArgs &fa, const SampledPlan &plan, bool 
   e = launch_cluster_list(sa, dt, plan, kClusterModeList, fa.list_a, fa.counters + 0, clusters_a,
                           stream);
   if (e != cudaSuccess) return e;
-  if ((e = launch_pdl(fast_emit_kernel, dim3((fa.s.N + 127) / 128), dim3(128), 0, stream, fa)) !=
+  if ((e = launch_pdl(fast_emit_kernel, dim3((fa.s.N + 3) / 4), dim3(128), 0, stream, fa)) !=
       cudaSuccess)
     return e;
   // a call's draws are all of one kind: over the nucleus when the window is

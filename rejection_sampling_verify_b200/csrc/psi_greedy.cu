@@ -173,29 +173,37 @@ __device__ __forceinline__ int32_t argmax_of(const uint64_t *partial, int64_t ro
   return (int32_t)(0xFFFFFFFFu - (uint32_t)best);
 }
 
-// One thread per sequence.
+// One warp per sequence, lane i at position i.
+static_assert(PSI_MAX_B <= 32, "one lane per drafted position");
 __global__ void __launch_bounds__(128) greedy_emit_kernel(
     const uint64_t *__restrict__ partial, int32_t splits, const int32_t *__restrict__ ids,
     int32_t N, int32_t B, int32_t V, int32_t *__restrict__ out_tokens,
     int32_t *__restrict__ out_n, uint32_t *dev_status) {
   pdl_wait();  // the previous kernel's results are visible
   pdl_trigger();
-  const int32_t n = blockIdx.x * blockDim.x + threadIdx.x;
+  const int lane = threadIdx.x & 31;
+  const int64_t n = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (n >= N) return;
-  const int64_t row0 = (int64_t)n * (B + 1);
-  int32_t L = B;
-  bool bad_id = false;
-  for (int32_t i = 0; i < B; ++i) {
-    const int32_t x = ids[(int64_t)n * B + i];
-    bad_id |= (x < 0 || x >= V);
-    if (L == B && x != argmax_of(partial, row0 + i, splits)) L = i;
+  const int64_t row0 = n * (B + 1);
+  bool bad_id = false, mismatch = false;
+  if (lane < B) {
+    const int32_t x = ids[n * B + lane];
+    bad_id = x < 0 || x >= V;
+    // with early exit the rows past a sequence's first mismatch were not
+    // read in this call: only the lowest mismatch counts, and every row
+    // before it was read
+    mismatch = x != argmax_of(partial, row0 + lane, splits);
   }
-  int32_t *tok = out_tokens + (int64_t)n * (B + 1);
-  for (int32_t i = 0; i < L; ++i) tok[i] = ids[(int64_t)n * B + i];
-  tok[L] = argmax_of(partial, row0 + L, splits);
-  for (int32_t i = L + 1; i <= B; ++i) tok[i] = -1;
-  out_n[n] = L + 1;
-  if (bad_id && dev_status) atomicOr(dev_status, PSI_DEV_BAD_TOKEN_ID);
+  const uint32_t mm = __ballot_sync(0xFFFFFFFFu, mismatch);
+  const int32_t L = mm ? __ffs(mm) - 1 : B;
+  const int32_t am = argmax_of(partial, row0 + L, splits);
+  int32_t *tok = out_tokens + n * (B + 1);
+  for (int32_t i = lane; i <= B; i += 32) tok[i] = i < L ? ids[n * B + i] : (i == L ? am : -1);
+  const bool any_bad = __any_sync(0xFFFFFFFFu, bad_id);
+  if (lane == 0) {
+    out_n[n] = L + 1;
+    if (any_bad && dev_status) atomicOr(dev_status, PSI_DEV_BAD_TOKEN_ID);
+  }
 }
 
 // Greedy tree, level by level: one cluster of C CTAs per tree (C = the
@@ -451,7 +459,7 @@ cudaError_t launch_greedy_early_exit(const void *logits, int64_t row_stride, psi
 cudaError_t launch_greedy_emit(const uint64_t *partial, int32_t splits, const int32_t *ids,
                                int32_t N, int32_t B, int32_t V, int32_t *out_tokens,
                                int32_t *out_n, uint32_t *dev_status, cudaStream_t stream) {
-  return launch_pdl(greedy_emit_kernel, dim3((N + 127) / 128), dim3(128), 0, stream, partial,
+  return launch_pdl(greedy_emit_kernel, dim3((N + 3) / 4), dim3(128), 0, stream, partial,
                     splits, ids, N, B, V, out_tokens, out_n, dev_status);
 }
 
